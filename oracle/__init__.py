@@ -1,0 +1,197 @@
+"""Float64 CPU oracle for grouped-query exact attention.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The CUDA library and
+its Python binding never do, and they share no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain C, float64, OpenMP over rows); this
+module only compiles it on first use and marshals numpy arrays.  Each entry point
+states the passage of the pages it follows in the C source:
+
+* ``attention``        -- the plain definition S = scale*QK^T, P = softmax(S),
+                          O = PV, L = m + ln l (FlashAttention-2 summary page,
+                          standard-attention and normalisation paragraphs), with the
+                          causal mask of that page's masking paragraph and the
+                          grouping of the Ultralytics GQA glossary, "How GQA works".
+* ``attention_rows``   -- the same, for a list of (b, h, i) rows only.
+* ``attention_keyrange`` / ``combine`` -- split-KV partials and their
+                          log-sum-exp weighted combine.
+* ``attention_tiled``  -- the per-step normalised (form 1) and deferred
+                          normalisation (form 2) online-softmax forms.
+
+Every function takes float32 numpy arrays (bf16 and fp32 values widen exactly)
+and returns float64 arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import pathlib
+import subprocess
+
+import numpy as np
+
+_HERE = pathlib.Path(__file__).resolve().parent
+_SRC = _HERE / "oracle.c"
+_LIB_PATH = _HERE / "liboracle.so"
+_lib = None
+
+FLAWS = {
+    "none": 0,
+    "strided_heads": 1,
+    "drop_diagonal": 2,
+    "top_left_causal": 3,
+    "no_scale": 4,
+    "lse_no_max": 5,
+    "fa1_no_rescale": 6,
+    "swap_kv": 7,
+}
+
+
+def build(force: bool = False) -> pathlib.Path:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, OpenMP)."""
+    if force or not _LIB_PATH.exists() or _LIB_PATH.stat().st_mtime < _SRC.stat().st_mtime:
+        tmp = _LIB_PATH.with_suffix(f".so.tmp{os.getpid()}")
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", str(_SRC),
+               "-o", str(tmp), "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(str(_LIB_PATH))
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        Dbl = ctypes.c_double
+        lib.oracle_attention.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, P, I]
+        lib.oracle_attention_rows.argtypes = [P, P, P, I, I, I, I, I, I, Dbl, I, P, I, P, P,
+                                              P, I]
+        lib.oracle_attention_keyrange.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, I,
+                                                  I, I]
+        lib.oracle_combine.argtypes = [I, I, P, P, P, P]
+        lib.oracle_combine.restype = None
+        lib.oracle_attention_tiled.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, I, I,
+                                               I]
+        lib.oracle_set_flaw.argtypes = [I]
+        lib.oracle_set_flaw.restype = None
+        lib.oracle_get_flaw.restype = I
+        lib.oracle_max_threads.restype = I
+        for name in ("oracle_attention", "oracle_attention_rows", "oracle_attention_keyrange",
+                     "oracle_attention_tiled"):
+            getattr(lib, name).restype = I
+        _lib = lib
+    return _lib
+
+
+def _f32(a) -> np.ndarray:
+    if hasattr(a, "detach"):  # torch tensor: widen bf16/fp16 exactly to float32
+        a = a.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dims(q, k, cu):
+    """(B, Hq, Hkv, Sq, Sk, D) from dense [B,S,H,D] or packed [total,H,D] arrays."""
+    if cu is None:
+        if q.ndim != 4 or k.ndim != 4:
+            raise ValueError("dense inputs are [B, S, H, D]")
+        B, Sq, Hq, D = q.shape
+        _, Sk, Hkv, _ = k.shape
+    else:
+        if q.ndim != 3 or k.ndim != 3:
+            raise ValueError("packed inputs are [total, H, D]")
+        B = len(cu) - 1
+        _, Hq, D = q.shape
+        _, Hkv, _ = k.shape
+        Sq = Sk = int(np.max(np.diff(cu))) if B > 0 else 0
+    return B, Hq, Hkv, Sq, Sk, D
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def set_flaw(name: str) -> None:
+    """Plant one deliberate mistake (pin-strength tests only); 'none' clears it."""
+    _load().oracle_set_flaw(FLAWS[name])
+
+
+def attention(q, k, v, *, scale: float, causal: bool, cu_seqlens=None, threads: int = 0):
+    """Full forward.  Returns (O float64 like q, L float64 [B,Hq,Sq] or [Hq,total])."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    B, Hq, Hkv, Sq, Sk, D = _dims(q, k, cu)
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((Hq, q.shape[0]) if cu is not None else (B, Hq, Sq), dtype=np.float64)
+    rc = _load().oracle_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv,
+                                  Sq, Sk, D, float(scale), int(bool(causal)),
+                                  None if cu is None else _ptr(cu), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention: bad arguments")
+    return o, lse
+
+
+def attention_rows(q, k, v, rows, *, scale: float, causal: bool, cu_seqlens=None,
+                   threads: int = 0):
+    """O and L for selected rows; rows is an int array [n, 3] of (b, h, i)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    B, Hq, Hkv, Sq, Sk, D = _dims(q, k, cu)
+    rows = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 3)
+    n = rows.shape[0]
+    o = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    rc = _load().oracle_attention_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk, D,
+                                       float(scale), int(bool(causal)),
+                                       None if cu is None else _ptr(cu), n, _ptr(rows),
+                                       _ptr(o), _ptr(lse), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_rows: bad arguments")
+    return o, lse
+
+
+def attention_keyrange(q, k, v, j0: int, j1: int, *, scale: float, causal: bool,
+                       threads: int = 0):
+    """Split-KV partial over keys [j0, j1) of a dense problem: (O_s, L_s)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, Hq, Hkv, Sq, Sk, D = _dims(q, k, None)
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    rc = _load().oracle_attention_keyrange(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
+                                           Hq, Hkv, Sq, Sk, D, float(scale),
+                                           int(bool(causal)), int(j0), int(j1), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_keyrange: bad arguments")
+    return o, lse
+
+
+def combine(Os, Ls):
+    """Log-sum-exp combine of one row's partials: Os [n, D], Ls [n] -> (O [D], L)."""
+    Os = np.ascontiguousarray(Os, dtype=np.float64)
+    Ls = np.ascontiguousarray(Ls, dtype=np.float64)
+    n, D = Os.shape
+    O = np.zeros((D,), dtype=np.float64)
+    L = np.zeros((1,), dtype=np.float64)
+    _load().oracle_combine(n, D, _ptr(Os), _ptr(Ls), _ptr(O), _ptr(L))
+    return O, float(L[0])
+
+
+def attention_tiled(q, k, v, *, scale: float, causal: bool, Bm: int, Bn: int, form: int):
+    """Online-softmax forward in float64 with Bm x Bn blocks (form 1 or 2)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, Hq, Hkv, Sq, Sk, D = _dims(q, k, None)
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    rc = _load().oracle_attention_tiled(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
+                                        Hkv, Sq, Sk, D, float(scale), int(bool(causal)),
+                                        int(Bm), int(Bn), int(form))
+    if rc != 0:
+        raise ValueError("oracle_attention_tiled: bad arguments")
+    return o, lse

@@ -1,0 +1,471 @@
+/*
+ * Float64 reference ("the oracle") for exact scaled-dot-product attention with
+ * grouped-query heads.
+ *
+ * TEST INFRASTRUCTURE ONLY.  The test suite, the smoke check and the benchmark's
+ * CPU-baseline leg call this code; the CUDA library never does, and the two share
+ * no source, header, table or helper.
+ *
+ * What it computes (plain definition, no blocking or fusion):
+ *   FlashAttention-2 summary page (azimuth.plus), paragraph on standard attention:
+ *     S = Q K^T, P = row-wise softmax(S), O = P V, with S and P materialised.
+ *   The scale multiplies the logits inside the softmax (S = scale * Q K^T).
+ *   Same page, deferred-normalisation paragraph: the per-row log-sum-exp
+ *     L = m + log(l) is the statistic written out next to O.
+ *   Same page, causal-masking paragraph: every entry above the diagonal is -inf,
+ *     the diagonal itself is kept.
+ *   Ultralytics glossary "Grouped Query Attention (GQA)", section "How GQA works":
+ *     Hq query heads share Hkv key/value heads in contiguous groups of G = Hq/Hkv
+ *     (the printed repeat_interleave(G, dim=1) equivalence gives query head h the
+ *     key/value head h / G).
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   - causal alignment for Sq != Sk is bottom-right: key j is visible to query i
+ *     iff j <= i + (Sk - Sq); a decode row (Sq = 1) therefore sees every key;
+ *   - a row with no visible key has O = 0 and L = -inf;
+ *   - L uses the natural logarithm of the scaled logits;
+ *   - split-KV partials cut the keys into contiguous ranges; a partial is the
+ *     attention restricted to its range (normalised), with its own L; the combine
+ *     is L = M + ln sum_s exp(L_s - M), O = sum_s exp(L_s - L) O_s.
+ *
+ * Layouts (all contiguous, row-major):
+ *   dense:  q [B, Sq, Hq, D], k and v [B, Sk, Hkv, D]; o like q; lse [B, Hq, Sq]
+ *   varlen: cu_seqlens int32[B+1]; q [total, Hq, D], k and v [total, Hkv, D];
+ *           sequence b owns rows cu[b]..cu[b+1]-1 of all three (self-attention,
+ *           Sq = Sk = its length); o like q; lse [Hq, total]
+ * Inputs are float32 (bf16 and fp32 values widen to float64 exactly); every
+ * arithmetic step is float64.
+ *
+ * Return value of every entry point: 0 on success, -1 on bad arguments.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------- */
+/* Deliberate-mistake switch.  Only the pin-strength tests set it: each value
+ * plants one plausible bug so that a test can show the pins catch it.        */
+enum {
+    FLAW_NONE = 0,
+    FLAW_STRIDED_HEADS = 1,   /* kv head = h % Hkv instead of h / G            */
+    FLAW_DROP_DIAGONAL = 2,   /* causal mask also hides the diagonal           */
+    FLAW_TOP_LEFT_CAUSAL = 3, /* causal alignment j <= i instead of bottom-right */
+    FLAW_NO_SCALE = 4,        /* scale left out of the logits                 */
+    FLAW_LSE_NO_MAX = 5,      /* L = log(l) without adding the max back        */
+    FLAW_FA1_NO_RESCALE = 6,  /* tiled FA-1 form drops exp(m_old - m_new)      */
+    FLAW_SWAP_KV = 7,         /* uses K where V belongs in O = P V             */
+};
+static int g_flaw = FLAW_NONE;
+void oracle_set_flaw(int flaw) { g_flaw = flaw; }
+int oracle_get_flaw(void) { return g_flaw; }
+
+/* ------------------------------------------------------------------------- */
+/* Shape of one attention problem as seen by a single (sequence, query head). */
+typedef struct {
+    const float* q;   /* first element of query row 0 of this head            */
+    const float* k;   /* first element of key row 0 of this head's kv head     */
+    const float* v;
+    size_t q_stride;  /* elements between consecutive query rows               */
+    size_t kv_stride; /* elements between consecutive key / value rows         */
+    int Sq, Sk, D;
+    double scale;
+    int causal;
+} head_view;
+
+/* Grouped-query mapping: query head h reads key/value head h / G. */
+static int kv_head_of(int h, int Hq, int Hkv)
+{
+    if (g_flaw == FLAW_STRIDED_HEADS) return h % Hkv;
+    return h / (Hq / Hkv);
+}
+
+/* Causal visibility of key j to query i (bottom-right aligned). */
+static int key_visible(int i, int j, int Sq, int Sk, int causal)
+{
+    if (!causal) return 1;
+    if (g_flaw == FLAW_TOP_LEFT_CAUSAL) return j <= i;
+    if (g_flaw == FLAW_DROP_DIAGONAL) return j < i + (Sk - Sq);
+    return j <= i + (Sk - Sq);
+}
+
+static double dot(const float* a, const float* b, int D)
+{
+    double acc = 0.0;
+    for (int d = 0; d < D; ++d) acc += (double)a[d] * (double)b[d];
+    return acc;
+}
+
+/*
+ * One query row i, restricted to keys [j0, j1): materialises the score row
+ * S[i, j0:j1] and the probability row P[i, j0:j1] in `row` (length >= Sk),
+ * then O[i, :] = P[i, :] V and L_i = m_i + ln(l_i).
+ */
+static void attend_row(const head_view* hv, int i, int j0, int j1, double* row,
+                       double* o_out, double* lse_out)
+{
+    const float* qi = hv->q + (size_t)i * hv->q_stride;
+    const double scale = (g_flaw == FLAW_NO_SCALE) ? 1.0 : hv->scale;
+    double m = -INFINITY;
+    for (int j = j0; j < j1; ++j) {
+        if (key_visible(i, j, hv->Sq, hv->Sk, hv->causal)) {
+            row[j] = scale * dot(qi, hv->k + (size_t)j * hv->kv_stride, hv->D);
+            if (row[j] > m) m = row[j];
+        } else {
+            row[j] = -INFINITY;
+        }
+    }
+    if (m == -INFINITY) { /* no visible key */
+        for (int d = 0; d < hv->D; ++d) o_out[d] = 0.0;
+        *lse_out = -INFINITY;
+        return;
+    }
+    double l = 0.0;
+    for (int j = j0; j < j1; ++j) {
+        row[j] = (row[j] == -INFINITY) ? 0.0 : exp(row[j] - m);
+        l += row[j];
+    }
+    for (int j = j0; j < j1; ++j) row[j] /= l; /* row now holds P[i, j] */
+    const float* vsrc = (g_flaw == FLAW_SWAP_KV) ? hv->k : hv->v;
+    for (int d = 0; d < hv->D; ++d) {
+        double acc = 0.0;
+        for (int j = j0; j < j1; ++j)
+            if (row[j] != 0.0) acc += row[j] * (double)vsrc[(size_t)j * hv->kv_stride + d];
+        o_out[d] = acc;
+    }
+    *lse_out = (g_flaw == FLAW_LSE_NO_MAX) ? log(l) : m + log(l);
+}
+
+/* Build the view of (sequence b, query head h). */
+static head_view make_view(const float* q, const float* k, const float* v, int B, int Hq,
+                           int Hkv, int Sq, int Sk, int D, double scale, int causal,
+                           const int32_t* cu, int b, int h, size_t* q_row0, size_t* lse_off,
+                           size_t* lse_step)
+{
+    head_view hv;
+    const int kvh = kv_head_of(h, Hq, Hkv);
+    size_t qrow0, krow0;
+    int sq, sk;
+    if (cu) {
+        qrow0 = (size_t)cu[b];
+        krow0 = (size_t)cu[b];
+        sq = sk = cu[b + 1] - cu[b];
+        *lse_off = (size_t)h * (size_t)cu[B] + (size_t)cu[b];
+    } else {
+        qrow0 = (size_t)b * Sq;
+        krow0 = (size_t)b * Sk;
+        sq = Sq;
+        sk = Sk;
+        *lse_off = ((size_t)b * Hq + h) * (size_t)Sq;
+    }
+    *lse_step = 1;
+    *q_row0 = qrow0;
+    hv.q = q + (qrow0 * Hq + h) * (size_t)D;
+    hv.k = k + (krow0 * Hkv + kvh) * (size_t)D;
+    hv.v = v + (krow0 * Hkv + kvh) * (size_t)D;
+    hv.q_stride = (size_t)Hq * D;
+    hv.kv_stride = (size_t)Hkv * D;
+    hv.Sq = sq;
+    hv.Sk = sk;
+    hv.D = D;
+    hv.scale = scale;
+    hv.causal = causal;
+    return hv;
+}
+
+static int check_args(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                      int Sq, int Sk, int D, const int32_t* cu)
+{
+    if (!q || !k || !v) return -1;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0) return -1;
+    if (Hq % Hkv != 0) return -1;
+    if (!cu && (Sq < 0 || Sk < 0)) return -1;
+    if (cu) {
+        if (cu[0] != 0) return -1;
+        for (int b = 0; b < B; ++b)
+            if (cu[b + 1] < cu[b]) return -1;
+    }
+    return 0;
+}
+
+static int max_keys(int B, int Sk, const int32_t* cu)
+{
+    if (!cu) return Sk;
+    int mx = 0;
+    for (int b = 0; b < B; ++b)
+        if (cu[b + 1] - cu[b] > mx) mx = cu[b + 1] - cu[b];
+    return mx;
+}
+
+static void set_threads(int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Full attention forward: every (sequence, head, query row).
+ * o has the layout of q; lse is [B, Hq, Sq] (dense) or [Hq, total] (varlen).
+ */
+int oracle_attention(const float* q, const float* k, const float* v, double* o, double* lse,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D, double scale, int causal,
+                     const int32_t* cu_seqlens, int nthreads)
+{
+    if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, cu_seqlens) || !o || !lse) return -1;
+    set_threads(nthreads);
+    const int kmax = max_keys(B, Sk, cu_seqlens);
+    const int nbh = B * Hq;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* row = (double*)malloc(sizeof(double) * (size_t)(kmax > 0 ? kmax : 1));
+        if (!row) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int bh = 0; bh < nbh; ++bh) {
+            if (!row) continue;
+            const int b = bh / Hq, h = bh % Hq;
+            size_t qrow0, lse_off, lse_step;
+            head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, cu_seqlens,
+                                     b, h, &qrow0, &lse_off, &lse_step);
+            for (int i = 0; i < hv.Sq; ++i) {
+                double* orow = o + ((qrow0 + (size_t)i) * Hq + h) * (size_t)D;
+                attend_row(&hv, i, 0, hv.Sk, row, orow, lse + lse_off + (size_t)i * lse_step);
+            }
+        }
+        free(row);
+    }
+    return err;
+}
+
+/*
+ * Selected rows only: rows holds n_rows triples (b, h, i).  For each, O[i, :] of
+ * query head h of sequence b goes to o_rows[r*D .. r*D+D) and L_i to lse_rows[r].
+ * Used to check outputs of problems too large to evaluate in full.
+ */
+int oracle_attention_rows(const float* q, const float* k, const float* v, int B, int Hq,
+                          int Hkv, int Sq, int Sk, int D, double scale, int causal,
+                          const int32_t* cu_seqlens, int n_rows, const int32_t* rows,
+                          double* o_rows, double* lse_rows, int nthreads)
+{
+    if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, cu_seqlens) || n_rows < 0) return -1;
+    if (n_rows > 0 && (!rows || !o_rows || !lse_rows)) return -1;
+    for (int r = 0; r < n_rows; ++r) {
+        const int b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+        if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0) return -1;
+        const int len = cu_seqlens ? cu_seqlens[b + 1] - cu_seqlens[b] : Sq;
+        if (i >= len) return -1;
+    }
+    set_threads(nthreads);
+    const int kmax = max_keys(B, Sk, cu_seqlens);
+    int err = 0;
+#pragma omp parallel
+    {
+        double* row = (double*)malloc(sizeof(double) * (size_t)(kmax > 0 ? kmax : 1));
+        if (!row) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int r = 0; r < n_rows; ++r) {
+            if (!row) continue;
+            size_t qrow0, lse_off, lse_step;
+            head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, cu_seqlens,
+                                     rows[3 * r], rows[3 * r + 1], &qrow0, &lse_off, &lse_step);
+            attend_row(&hv, rows[3 * r + 2], 0, hv.Sk, row, o_rows + (size_t)r * D,
+                       lse_rows + r);
+        }
+        free(row);
+    }
+    return err;
+}
+
+/*
+ * Attention restricted to keys [j0, j1) of a dense problem: the split-KV partial
+ * (O_s normalised over its own keys, L_s its log-sum-exp; O_s = 0 and L_s = -inf
+ * when the range holds no visible key).  Layout of o and lse as in
+ * oracle_attention.
+ */
+int oracle_attention_keyrange(const float* q, const float* k, const float* v, double* o,
+                              double* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                              double scale, int causal, int j0, int j1, int nthreads)
+{
+    if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, NULL) || !o || !lse) return -1;
+    if (j0 < 0 || j1 > Sk || j0 > j1) return -1;
+    set_threads(nthreads);
+    const int nbh = B * Hq;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* row = (double*)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+        if (!row) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int bh = 0; bh < nbh; ++bh) {
+            if (!row) continue;
+            const int b = bh / Hq, h = bh % Hq;
+            size_t qrow0, lse_off, lse_step;
+            head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, NULL, b, h,
+                                     &qrow0, &lse_off, &lse_step);
+            for (int i = 0; i < Sq; ++i)
+                attend_row(&hv, i, j0, j1, row, o + ((qrow0 + (size_t)i) * Hq + h) * (size_t)D,
+                           lse + lse_off + (size_t)i);
+        }
+        free(row);
+    }
+    return err;
+}
+
+/*
+ * Log-sum-exp weighted combine of n partial results of one row:
+ *   M = max_s L_s,  L = M + ln sum_s exp(L_s - M),  O = sum_s exp(L_s - L) O_s.
+ * Partials with L_s = -inf carry weight 0; if every L_s is -inf then O = 0 and
+ * L = -inf.  Os is [n, D].
+ */
+void oracle_combine(int n, int D, const double* Os, const double* Ls, double* O, double* L)
+{
+    double M = -INFINITY;
+    for (int s = 0; s < n; ++s)
+        if (Ls[s] > M) M = Ls[s];
+    for (int d = 0; d < D; ++d) O[d] = 0.0;
+    if (M == -INFINITY) {
+        *L = -INFINITY;
+        return;
+    }
+    double sum = 0.0;
+    for (int s = 0; s < n; ++s)
+        if (Ls[s] != -INFINITY) sum += exp(Ls[s] - M);
+    const double Lall = M + log(sum);
+    for (int s = 0; s < n; ++s) {
+        if (Ls[s] == -INFINITY) continue;
+        const double w = exp(Ls[s] - Lall);
+        for (int d = 0; d < D; ++d) O[d] += w * Os[(size_t)s * D + d];
+    }
+    *L = Lall;
+}
+
+/*
+ * The tiled (online-softmax) forms of the same forward, in float64, on a dense
+ * problem.  The outer loop walks query row blocks of Bm rows, the inner loop key
+ * blocks of Bn columns, skipping blocks that lie entirely above the causal
+ * diagonal.  Per row the running max m and sum l are updated per key block.
+ *   form 1, per-step normalised update (FlashAttention-2 summary page, first
+ *     equation of the normalisation paragraph):
+ *       O_j = diag(l_{j-1} e^{m_{j-1} - m_j} / l_j) O_{j-1}
+ *             + diag(l_j)^{-1} e^{S_j - m_j} V_j
+ *     (the page prints the carried term as diag(l_{j-1}/l_j) O_{j-1}, with the
+ *     max-shift factor left implicit; it is written out here);
+ *   form 2, deferred normalisation (second equation):
+ *       Ot_j = diag(e^{m_{j-1} - m_j}) Ot_{j-1} + e^{S_j - m_j} V_j,
+ *     one division by l at the end;
+ *   both: L = m + ln l.
+ */
+int oracle_attention_tiled(const float* q, const float* k, const float* v, double* o,
+                           double* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                           double scale, int causal, int Bm, int Bn, int form)
+{
+    if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, NULL) || !o || !lse) return -1;
+    if (Bm <= 0 || Bn <= 0 || (form != 1 && form != 2)) return -1;
+    double* m = (double*)malloc(sizeof(double) * (size_t)Bm);
+    double* l = (double*)malloc(sizeof(double) * (size_t)Bm);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)Bm * D);
+    double* sblk = (double*)malloc(sizeof(double) * (size_t)Bm * Bn);
+    if (!m || !l || !acc || !sblk) {
+        free(m); free(l); free(acc); free(sblk);
+        return -1;
+    }
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            size_t qrow0, lse_off, lse_step;
+            head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, NULL, b, h,
+                                     &qrow0, &lse_off, &lse_step);
+            for (int i0 = 0; i0 < Sq; i0 += Bm) {
+                const int bm = (Sq - i0 < Bm) ? Sq - i0 : Bm;
+                for (int r = 0; r < bm; ++r) {
+                    m[r] = -INFINITY;
+                    l[r] = 0.0;
+                    for (int d = 0; d < D; ++d) acc[(size_t)r * D + d] = 0.0;
+                }
+                for (int j0 = 0; j0 < Sk; j0 += Bn) {
+                    const int bn = (Sk - j0 < Bn) ? Sk - j0 : Bn;
+                    /* block entirely above the diagonal: every key invisible to every row */
+                    if (causal && !key_visible(i0 + bm - 1, j0, Sq, Sk, causal)) continue;
+                    for (int r = 0; r < bm; ++r) {
+                        const int i = i0 + r;
+                        const float* qi = hv.q + (size_t)i * hv.q_stride;
+                        double mblk = -INFINITY;
+                        for (int c = 0; c < bn; ++c) {
+                            const int j = j0 + c;
+                            double s = -INFINITY;
+                            if (key_visible(i, j, Sq, Sk, causal))
+                                s = scale * dot(qi, hv.k + (size_t)j * hv.kv_stride, D);
+                            sblk[(size_t)r * Bn + c] = s;
+                            if (s > mblk) mblk = s;
+                        }
+                        const double mnew = (mblk > m[r]) ? mblk : m[r];
+                        if (mnew == -INFINITY) continue; /* nothing visible yet */
+                        const double carry =
+                            (m[r] == -INFINITY) ? 0.0
+                            : (g_flaw == FLAW_FA1_NO_RESCALE && form == 1) ? 1.0
+                                                                           : exp(m[r] - mnew);
+                        double rowsum = 0.0;
+                        for (int c = 0; c < bn; ++c) {
+                            const double s = sblk[(size_t)r * Bn + c];
+                            const double p = (s == -INFINITY) ? 0.0 : exp(s - mnew);
+                            sblk[(size_t)r * Bn + c] = p;
+                            rowsum += p;
+                        }
+                        const double lnew = carry * l[r] + rowsum;
+                        double* ar = acc + (size_t)r * D;
+                        for (int d = 0; d < D; ++d) {
+                            double pv = 0.0;
+                            for (int c = 0; c < bn; ++c)
+                                pv += sblk[(size_t)r * Bn + c] *
+                                      (double)hv.v[(size_t)(j0 + c) * hv.kv_stride + d];
+                            if (form == 1) /* running O stays normalised by l_j */
+                                ar[d] = (l[r] * carry / lnew) * ar[d] + pv / lnew;
+                            else /* running O-tilde, unnormalised */
+                                ar[d] = carry * ar[d] + pv;
+                        }
+                        m[r] = mnew;
+                        l[r] = lnew;
+                    }
+                }
+                for (int r = 0; r < bm; ++r) {
+                    const int i = i0 + r;
+                    double* orow = o + ((qrow0 + (size_t)i) * Hq + h) * (size_t)D;
+                    if (m[r] == -INFINITY) {
+                        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+                        lse[lse_off + (size_t)i] = -INFINITY;
+                        continue;
+                    }
+                    for (int d = 0; d < D; ++d)
+                        orow[d] = (form == 1) ? acc[(size_t)r * D + d]
+                                              : acc[(size_t)r * D + d] / l[r];
+                    lse[lse_off + (size_t)i] = m[r] + log(l[r]);
+                }
+            }
+        }
+    free(m); free(l); free(acc); free(sblk);
+    return 0;
+}

@@ -1,0 +1,414 @@
+"""Pins of the float64 oracle against what the pages and the mathematics fix.
+
+None of these tests reruns the oracle's own formula: each compares it with a
+printed example of the pages, a library routine (torch's float64 SDPA, logsumexp),
+a 50-digit brute force, a closed form or an invariant.  The last test plants
+plausible mistakes in the oracle and checks that at least one pin catches each.
+"""
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g) * scale).numpy().astype(np.float32)
+
+
+def bshd_to_bhsd64(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).double().transpose(1, 2)
+
+
+def sdpa_ref(q, k, v, scale, causal, bottom_right=False):
+    """torch float64 SDPA on [B,S,H,D] numpy inputs; returns O [B,S,H,D] and L [B,H,S]."""
+    qt, kt, vt = bshd_to_bhsd64(q), bshd_to_bhsd64(k), bshd_to_bhsd64(v)
+    G = qt.shape[1] // kt.shape[1]
+    mask = None
+    is_causal = causal
+    if causal and bottom_right:
+        Sq, Sk = qt.shape[2], kt.shape[2]
+        mask = torch.ones(Sq, Sk, dtype=torch.bool).tril(diagonal=Sk - Sq)
+        is_causal = False
+    o = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, is_causal=is_causal,
+                                       scale=scale, enable_gqa=True)
+    kf = kt.repeat_interleave(G, dim=1)
+    s = scale * qt @ kf.transpose(-1, -2)
+    if causal:
+        Sq, Sk = s.shape[-2:]
+        vis = torch.ones(Sq, Sk, dtype=torch.bool)
+        vis = vis.tril(diagonal=Sk - Sq) if bottom_right else vis.tril()
+        s = s.masked_fill(~vis, float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    return o.transpose(1, 2).numpy(), lse.numpy()
+
+
+# ---------------------------------------------------------------------------------
+# The page's worked example
+
+def test_glossary_example_gqa_equals_repeat_interleaved_mha():
+    gold = json.load(open(os.path.join(GOLDEN, "gqa_glossary_example.json")))
+    w = W.TINY
+    assert [w.B, w.Hq, w.Sq, w.D] == gold["q_shape_bhsd"]
+    assert [w.B, w.Hkv, w.Sk, w.D] == gold["kv_shape_bhsd"]
+    q, k, v = W.make_qkv(w)
+    # the recipe reproduces the page's draws: torch.manual_seed(0) then randn in order
+    torch.manual_seed(gold["seed"])
+    q_page = torch.randn(*gold["q_shape_bhsd"])
+    k_page = torch.randn(*gold["kv_shape_bhsd"])
+    assert torch.equal(q.transpose(1, 2), q_page)
+    assert torch.equal(k.transpose(1, 2), k_page)
+    scale = 1.0 / math.sqrt(64)
+    o, lse = oracle.attention(q, k, v, scale=scale, causal=gold["causal"])
+    assert list(o.transpose(0, 2, 1, 3).shape) == gold["printed_output_shape"]
+    G = gold["group"]
+    o_mha, lse_mha = oracle.attention(q, k.repeat_interleave(G, dim=2),
+                                      v.repeat_interleave(G, dim=2), scale=scale,
+                                      causal=gold["causal"])
+    # same arithmetic on the same operands: identical, hence allclose(atol=1e-6) True
+    assert np.array_equal(o, o_mha) and np.array_equal(lse, lse_mha)
+    assert np.allclose(o, o_mha, atol=gold["printed_allclose_atol"]) == \
+        gold["printed_same_as_copied_heads"]
+    assert W.kv_values_per_token(w.Hkv, w.D) == \
+        gold["printed_cached_values_per_token_per_layer_gqa"]
+    assert W.kv_values_per_token(w.Hq, w.D) == \
+        gold["printed_cached_values_per_token_per_layer_mha"]
+    # and the page's own library call agrees with the oracle in float64
+    o_ref, lse_ref = sdpa_ref(q.numpy(), k.numpy(), v.numpy(), scale, True)
+    assert np.max(np.abs(o - o_ref)) < 1e-13
+    assert np.max(np.abs(lse - lse_ref)) < 1e-13
+
+
+def test_kv_cache_arithmetic_of_the_pages():
+    gold = json.load(open(os.path.join(GOLDEN, "kv_cache_arithmetic.json")))
+    ll = gold["llama31_8b"]
+    per_tok = W.kv_cache_bytes(1, 1, ll["kv_heads"], ll["head_dim"], ll["bytes_per_value"],
+                               ll["layers"])
+    assert per_tok == ll["bytes_per_token_gqa"] == 128 * 1024
+    assert W.kv_cache_bytes(1, 131072, ll["kv_heads"], ll["head_dim"], 2, ll["layers"]) == \
+        ll["bytes_at_131072_tokens_gqa"] == 16 * 2**30
+    assert W.kv_cache_bytes(1, 1, ll["q_heads"], ll["head_dim"], 2, ll["layers"]) == \
+        ll["bytes_per_token_mha"]
+    assert W.kv_cache_bytes(1, 131072, ll["q_heads"], ll["head_dim"], 2, ll["layers"]) == \
+        ll["bytes_at_131072_tokens_mha"]
+    g = gold["grouping_48_12"]
+    red = 1 - W.kv_cache_bytes(1, 1, g["kv_heads"], 64) / W.kv_cache_bytes(1, 1, g["q_heads"], 64)
+    assert round(100 * red) == g["reduction_percent"]
+
+
+def test_flop_accounting_counts_visible_pairs():
+    for Sq, Sk in [(1, 7), (5, 5), (4, 9), (9, 4), (16, 16)]:
+        brute = sum(1 for i in range(Sq) for j in range(Sk) if j <= i + Sk - Sq)
+        assert W.causal_pairs(Sq, Sk) == brute
+    assert W.causal_pairs(8192, 8192) == 8192 * 8193 // 2
+    assert W.attention_flops(2, 3, 5, 7, 8, False) == 4 * 8 * 5 * 7 * 2 * 3
+
+
+# ---------------------------------------------------------------------------------
+# Library routine: torch float64 scaled_dot_product_attention(enable_gqa=True)
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal", [
+    (2, 8, 2, 33, 33, 16, True),
+    (2, 8, 2, 33, 33, 16, False),
+    (1, 6, 3, 17, 40, 8, False),
+    (1, 4, 1, 12, 12, 32, True),     # MQA limit (one group)
+    (1, 4, 4, 12, 12, 32, True),     # MHA limit (G = 1)
+    (3, 12, 4, 20, 31, 24, True),    # Sq < Sk, bottom-right mask given explicitly
+    (1, 4, 2, 25, 9, 8, True),       # Sq > Sk: leading rows see no key
+])
+def test_matches_torch_sdpa_float64(B, Hq, Hkv, Sq, Sk, D, causal):
+    q = rnd((B, Sq, Hq, D), 11)
+    k = rnd((B, Sk, Hkv, D), 12)
+    v = rnd((B, Sk, Hkv, D), 13)
+    scale = 0.37
+    o, lse = oracle.attention(q, k, v, scale=scale, causal=causal)
+    bottom_right = causal and Sq != Sk
+    o_ref, lse_ref = sdpa_ref(q, k, v, scale, causal, bottom_right=bottom_right)
+    if causal and Sq > Sk:
+        dead = Sq - Sk  # rows with no visible key: O = 0, L = -inf (SDPA gives NaN)
+        assert np.all(o[:, :dead] == 0) and np.all(np.isneginf(lse[:, :, :dead]))
+        o, o_ref = o[:, dead:], o_ref[:, dead:]
+        lse, lse_ref = lse[:, :, dead:], lse_ref[:, :, dead:]
+    assert np.max(np.abs(o - o_ref)) < 1e-12
+    assert np.max(np.abs(lse - lse_ref)) < 1e-12
+
+
+def test_decode_row_sees_every_key():
+    """Sq = 1 under the bottom-right causal reading equals the unmasked result."""
+    q = rnd((3, 1, 8, 16), 21)
+    k = rnd((3, 50, 2, 16), 22)
+    v = rnd((3, 50, 2, 16), 23)
+    a = oracle.attention(q, k, v, scale=0.25, causal=True)
+    b = oracle.attention(q, k, v, scale=0.25, causal=False)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    o_ref, lse_ref = sdpa_ref(q, k, v, 0.25, False)
+    assert np.max(np.abs(a[0] - o_ref)) < 1e-12
+
+
+# ---------------------------------------------------------------------------------
+# Softmax properties, read through V = identity (then O = P)
+
+@pytest.mark.parametrize("causal,Sq,Sk", [(False, 9, 9), (True, 9, 9), (True, 5, 11)])
+def test_probabilities_are_a_distribution(causal, Sq, Sk):
+    Hq, Hkv = 4, 2
+    q = rnd((1, Sq, Hq, Sk), 31, 2.0)
+    k = rnd((1, Sk, Hkv, Sk), 32, 2.0)
+    eye = np.broadcast_to(np.eye(Sk, dtype=np.float32)[:, None, :], (Sk, Hkv, Sk))
+    v = np.ascontiguousarray(eye[None])
+    P, _ = oracle.attention(q, k, v, scale=0.5, causal=causal)  # [1, Sq, Hq, Sk] == P
+    assert np.all(P >= 0)
+    assert np.max(np.abs(P.sum(-1) - 1.0)) < 1e-12
+    if causal:
+        for i in range(Sq):
+            hidden = np.arange(Sk) > i + Sk - Sq
+            assert np.all(P[0, i, :, hidden] == 0.0)
+            assert np.all(P[0, i, :, ~hidden] > 0.0)
+
+
+# ---------------------------------------------------------------------------------
+# Exact values: 50-digit brute force of the definition on tiny problems
+
+def brute_force(q, k, v, scale, causal):
+    mpmath.mp.dps = 50
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    G = Hq // Hkv
+    O = np.zeros(q.shape)
+    L = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            c = h // G
+            for i in range(Sq):
+                vis = [j for j in range(Sk) if not causal or j <= i + Sk - Sq]
+                s = [mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(float(q[b, i, h, d])) *
+                                                     mpmath.mpf(float(k[b, j, c, d]))
+                                                     for d in range(D)) for j in vis]
+                e = [mpmath.exp(x) for x in s]
+                z = mpmath.fsum(e)
+                for d in range(D):
+                    O[b, i, h, d] = float(mpmath.fsum(e[t] * mpmath.mpf(float(v[b, j, c, d]))
+                                                      for t, j in enumerate(vis)) / z)
+                L[b, h, i] = float(mpmath.log(z))
+    return O, L
+
+
+@pytest.mark.parametrize("causal,Sq,Sk", [(True, 4, 4), (False, 3, 5), (True, 2, 6)])
+def test_brute_force_50_digits(causal, Sq, Sk):
+    q = rnd((2, Sq, 4, 3), 41, 3.0)  # large logits: exercises the max shift
+    k = rnd((2, Sk, 2, 3), 42, 3.0)
+    v = rnd((2, Sk, 2, 3), 43)
+    o, lse = oracle.attention(q, k, v, scale=1.3, causal=causal)
+    o_bf, lse_bf = brute_force(q, k, v, 1.3, causal)
+    assert np.max(np.abs(o - o_bf)) < 1e-13
+    assert np.max(np.abs(lse - lse_bf)) < 1e-13
+
+
+# ---------------------------------------------------------------------------------
+# Closed forms
+
+def test_single_key_returns_its_value():
+    q = rnd((2, 3, 4, 8), 51)
+    k = rnd((2, 1, 2, 8), 52)
+    v = rnd((2, 1, 2, 8), 53)
+    o, lse = oracle.attention(q, k, v, scale=0.7, causal=False)
+    for h in range(4):
+        np.testing.assert_array_equal(o[:, :, h, :], np.broadcast_to(v[:, 0:1, h // 2, :], (2, 3, 8)))
+        expect = 0.7 * np.einsum("bid,bd->bi", q[:, :, h, :].astype(np.float64),
+                                 k[:, 0, h // 2, :].astype(np.float64))
+        assert np.max(np.abs(lse[:, h, :] - expect)) < 1e-12
+
+
+def test_equal_keys_average_the_visible_values():
+    Sq = Sk = 7
+    q = rnd((1, Sq, 2, 5), 61)
+    k1 = rnd((1, 1, 1, 5), 62)
+    k = np.ascontiguousarray(np.repeat(k1, Sk, axis=1))
+    v = rnd((1, Sk, 1, 5), 63)
+    o, lse = oracle.attention(q, k, v, scale=0.9, causal=True)
+    for i in range(Sq):
+        mean = v[0, : i + 1, 0, :].astype(np.float64).mean(0)
+        for h in range(2):
+            assert np.max(np.abs(o[0, i, h] - mean)) < 1e-13
+            s0 = 0.9 * float(np.dot(q[0, i, h].astype(np.float64), k1[0, 0, 0].astype(np.float64)))
+            assert abs(lse[0, h, i] - (s0 + math.log(i + 1))) < 1e-12
+
+
+def test_zero_query_gives_uniform_average_and_log_count():
+    q = np.zeros((1, 6, 2, 4), np.float32)
+    k = rnd((1, 6, 1, 4), 71)
+    v = rnd((1, 6, 1, 4), 72)
+    o, lse = oracle.attention(q, k, v, scale=0.5, causal=True)
+    for i in range(6):
+        assert np.max(np.abs(o[0, i, 0] - v[0, : i + 1, 0].astype(np.float64).mean(0))) < 1e-14
+        assert abs(lse[0, 0, i] - math.log(i + 1)) < 1e-14
+    # causal row 0 attends to key 0 only
+    np.testing.assert_array_equal(o[0, 0, 1], v[0, 0, 0].astype(np.float64))
+
+
+# ---------------------------------------------------------------------------------
+# Invariants
+
+def test_key_permutation_invariance_when_unmasked():
+    q = rnd((2, 5, 4, 8), 81)
+    k = rnd((2, 13, 2, 8), 82)
+    v = rnd((2, 13, 2, 8), 83)
+    perm = np.random.default_rng(0).permutation(13)
+    a = oracle.attention(q, k, v, scale=0.3, causal=False)
+    b = oracle.attention(q, np.ascontiguousarray(k[:, perm]), np.ascontiguousarray(v[:, perm]),
+                         scale=0.3, causal=False)
+    assert np.max(np.abs(a[0] - b[0])) < 1e-13 and np.max(np.abs(a[1] - b[1])) < 1e-13
+
+
+def test_key_shift_leaves_probabilities_and_shifts_lse():
+    """k_j -> k_j + u adds scale*q_i.u to every logit of row i."""
+    # dyadic values with few bits, so that k + u is exact in float32
+    q = np.round(rnd((1, 6, 2, 4), 91) * 8) / 8
+    k = np.round(rnd((1, 6, 1, 4), 92) * 8) / 8
+    v = rnd((1, 6, 1, 4), 93)
+    u = np.array([0.5, -0.25, 1.0, 0.125], np.float32)
+    a = oracle.attention(q, k, v, scale=0.5, causal=True)
+    b = oracle.attention(q, np.ascontiguousarray(k + u), v, scale=0.5, causal=True)
+    assert np.max(np.abs(a[0] - b[0])) < 1e-12
+    shift = 0.5 * np.einsum("ihd,d->hi", q[0].astype(np.float64), u.astype(np.float64))
+    assert np.max(np.abs(b[1][0] - a[1][0] - shift)) < 1e-12
+
+
+def test_value_linearity_and_scale_folding():
+    q = rnd((1, 7, 4, 8), 101)
+    k = rnd((1, 9, 2, 8), 102)
+    v1 = rnd((1, 9, 2, 8), 103)
+    v2 = rnd((1, 9, 2, 8), 104)
+    o1, _ = oracle.attention(q, k, v1, scale=0.4, causal=True)
+    o2, _ = oracle.attention(q, k, v2, scale=0.4, causal=True)
+    o12, _ = oracle.attention(q, k, np.ascontiguousarray(v1.astype(np.float64) + v2).astype(np.float32),
+                              scale=0.4, causal=True)
+    assert np.max(np.abs(o12 - (o1 + o2))) < 1e-6  # v1 + v2 rounds to float32
+    a = oracle.attention(q, k, v1, scale=0.5, causal=True)
+    b = oracle.attention(np.ascontiguousarray(q * 2), k, v1, scale=0.25, causal=True)
+    assert np.max(np.abs(a[0] - b[0])) < 1e-13 and np.max(np.abs(a[1] - b[1])) < 1e-13
+
+
+def test_varlen_equals_per_sequence_problems():
+    lengths = [5, 1, 12, 7]
+    cu = W.cu_seqlens_of(lengths).numpy()
+    total = int(cu[-1])
+    q = rnd((total, 8, 16), 111)
+    k = rnd((total, 2, 16), 112)
+    v = rnd((total, 2, 16), 113)
+    o, lse = oracle.attention(q, k, v, scale=0.25, causal=True, cu_seqlens=cu)
+    assert lse.shape == (8, total)
+    for b, L in enumerate(lengths):
+        s0 = cu[b]
+        ob, lb = oracle.attention(q[None, s0:s0 + L], k[None, s0:s0 + L], v[None, s0:s0 + L],
+                                  scale=0.25, causal=True)
+        np.testing.assert_array_equal(o[s0:s0 + L], ob[0])
+        np.testing.assert_array_equal(lse[:, s0:s0 + L], lb[0])
+
+
+def test_rows_entry_point_matches_full():
+    q = rnd((2, 10, 8, 16), 121)
+    k = rnd((2, 14, 2, 16), 122)
+    v = rnd((2, 14, 2, 16), 123)
+    o, lse = oracle.attention(q, k, v, scale=0.25, causal=True)
+    rows = np.array([[0, 0, 0], [1, 7, 9], [0, 3, 4], [1, 2, 0]])
+    orow, lrow = oracle.attention_rows(q, k, v, rows, scale=0.25, causal=True)
+    for r, (b, h, i) in enumerate(rows):
+        np.testing.assert_array_equal(orow[r], o[b, i, h])
+        assert lrow[r] == lse[b, h, i]
+
+
+# ---------------------------------------------------------------------------------
+# Online softmax: "exactly identical, no approximation"
+
+@pytest.mark.parametrize("Bm,Bn", [(1, 1), (3, 3), (16, 64), (64, 16), (7, 5)])
+@pytest.mark.parametrize("form", [1, 2])
+@pytest.mark.parametrize("causal,Sq,Sk", [(True, 37, 37), (False, 20, 45), (True, 9, 40)])
+def test_tiled_forms_equal_full_matrix(Bm, Bn, form, causal, Sq, Sk):
+    q = rnd((1, Sq, 4, 8), 131, 3.0)  # large logits so the running max moves
+    k = rnd((1, Sk, 2, 8), 132, 3.0)
+    v = rnd((1, Sk, 2, 8), 133)
+    full = oracle.attention(q, k, v, scale=0.5, causal=causal)
+    tiled = oracle.attention_tiled(q, k, v, scale=0.5, causal=causal, Bm=Bm, Bn=Bn, form=form)
+    assert np.max(np.abs(full[0] - tiled[0])) < 1e-12
+    assert np.max(np.abs(full[1] - tiled[1])) < 1e-12
+
+
+# ---------------------------------------------------------------------------------
+# Split-KV: contiguous ranges of whole key blocks, log-sum-exp combine
+
+def split_ranges(Sk, n, Bn):
+    nblk = -(-Sk // Bn)
+    n = min(n, nblk)
+    per = -(-nblk // n)
+    return [(min(s * per * Bn, Sk), min((s + 1) * per * Bn, Sk)) for s in range(n)]
+
+
+@pytest.mark.parametrize("n", [1, 2, 4, 8, 1000])
+@pytest.mark.parametrize("causal,Sq,Sk", [(False, 1, 300), (True, 1, 300), (True, 24, 24)])
+def test_split_combine_equals_full(n, causal, Sq, Sk):
+    q = rnd((2, Sq, 4, 8), 141, 2.0)
+    k = rnd((2, Sk, 2, 8), 142, 2.0)
+    v = rnd((2, Sk, 2, 8), 143)
+    Bn = 16
+    o, lse = oracle.attention(q, k, v, scale=0.5, causal=causal)
+    parts = [oracle.attention_keyrange(q, k, v, a, b, scale=0.5, causal=causal)
+             for a, b in split_ranges(Sk, n, Bn)]
+    for bb in range(2):
+        for h in range(4):
+            for i in range(Sq):
+                Os = np.stack([p[0][bb, i, h] for p in parts])
+                Ls = np.array([p[1][bb, h, i] for p in parts])
+                O, L = oracle.combine(Os, Ls)
+                assert np.max(np.abs(O - o[bb, i, h])) < 1e-12
+                assert abs(L - lse[bb, h, i]) < 1e-12
+
+
+def test_combine_of_empty_partials():
+    O, L = oracle.combine(np.zeros((3, 4)), np.full(3, -np.inf))
+    assert np.all(O == 0) and L == -np.inf
+    O, L = oracle.combine(np.array([[1.0, 2.0], [9.0, 9.0]]), np.array([0.5, -np.inf]))
+    np.testing.assert_array_equal(O, [1.0, 2.0])
+    assert L == 0.5
+
+
+# ---------------------------------------------------------------------------------
+# Pin strength: every planted mistake is caught by at least one pin above
+
+PIN_BATTERY = [
+    lambda: test_glossary_example_gqa_equals_repeat_interleaved_mha(),
+    lambda: test_matches_torch_sdpa_float64(2, 8, 2, 33, 33, 16, True),
+    lambda: test_matches_torch_sdpa_float64(3, 12, 4, 20, 31, 24, True),
+    lambda: test_decode_row_sees_every_key(),
+    lambda: test_brute_force_50_digits(True, 4, 4),
+    lambda: test_tiled_forms_equal_full_matrix(7, 5, 1, True, 37, 37),
+    lambda: test_equal_keys_average_the_visible_values(),
+]
+
+
+def battery_passes():
+    for pin in PIN_BATTERY:
+        try:
+            pin()
+        except AssertionError:
+            return False
+    return True
+
+
+@pytest.mark.parametrize("flaw", [f for f in oracle.FLAWS if f != "none"])
+def test_each_planted_mistake_is_caught(flaw):
+    try:
+        oracle.set_flaw(flaw)
+        assert not battery_passes(), f"planted mistake '{flaw}' slipped through every pin"
+    finally:
+        oracle.set_flaw("none")
+    assert battery_passes()

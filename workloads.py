@@ -1,0 +1,195 @@
+"""Seeded synthetic inputs for grouped-query attention, and work accounting.
+
+This module is shared by the tests, the benchmark and the smoke check.  It holds
+no attention arithmetic: it only draws inputs and counts bytes and flops.
+
+Recipe (the same for every workload):
+* a ``torch.Generator`` on the target device, seeded with the workload's seed;
+* q, k, v drawn in that order with ``randn`` in the logical [B, H, S, D] order of
+  the Ultralytics GQA glossary example (``torch.manual_seed(0)`` then
+  ``randn(1, 8, 16, 64)``, ``randn(1, 2, 16, 64)`` twice), in float32;
+* cast to the workload dtype (bf16 rounds to nearest even);
+* a "stress" variant multiplies q by 4 after the cast (exact in bf16);
+* permuted to the library layout [B, S, H, D] (contiguous), as FlashAttention's
+  ``flash_attn_func`` expects (StructBERT/FlashAttention page, section 2.2).
+
+Variable-length batches draw their lengths with ``randint(lo, hi + 1, (n,))`` from
+their own seed, then q, k, v for the packed [total, H, D] tensors.
+
+Decode KV caches too large to draw on the host are drawn on the device, one
+batch element at a time, each from its own seed ``seed * 1_000_003 + b``, so any
+element can be redrawn alone.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Sq: int
+    Sk: int
+    D: int
+    dtype: str          # "f32" or "bf16"
+    causal: bool
+    seed: int
+    q_mult: float = 1.0  # 4.0 for the large-logit stress variant
+    pack_gqa: int = 1
+    num_splits: int = 1
+    varlen: dict = field(default_factory=dict)  # {"n": 32, "lo": 128, "hi": 8192}
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+
+# The five workloads of the headline measurement; sizes as the pages' examples.
+TINY = Workload("tiny_gqa_causal", B=1, Hq=8, Hkv=2, Sq=16, Sk=16, D=64, dtype="f32",
+                causal=True, seed=0)
+ENCODER = Workload("encoder_b64_h48kv12_s512_d64", B=64, Hq=48, Hkv=12, Sq=512, Sk=512,
+                   D=64, dtype="bf16", causal=False, seed=1)
+LLAMA = Workload("llama8b_prefill_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8192, Sk=8192,
+                 D=128, dtype="bf16", causal=True, seed=2)
+LLAMA_STRESS = Workload("llama8b_prefill_b4_s8192_causal_qx4", B=4, Hq=32, Hkv=8, Sq=8192,
+                        Sk=8192, D=128, dtype="bf16", causal=True, seed=3, q_mult=4.0)
+DECODE_BATCHES = (1, 16, 64, 128, 256)
+DECODE_SPLITS = (1, 2, 4, 8)
+
+
+def decode(B: int, num_splits: int = 1, pack_gqa: int = 1) -> Workload:
+    return Workload(f"decode_b{B}_sk32768_n{num_splits}_pack{pack_gqa}", B=B, Hq=32, Hkv=8,
+                    Sq=1, Sk=32768, D=128, dtype="bf16", causal=False, seed=4,
+                    pack_gqa=pack_gqa, num_splits=num_splits)
+
+
+VARLEN = Workload("varlen32_len128to8192_causal", B=32, Hq=32, Hkv=8, Sq=0, Sk=0, D=128,
+                  dtype="bf16", causal=True, seed=5,
+                  varlen={"n": 32, "lo": 128, "hi": 8192})
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def make_qkv(w: Workload, device="cpu", *, B=None, Sq=None, Sk=None):
+    """Dense q [B,Sq,Hq,D], k/v [B,Sk,Hkv,D] for workload w (shape overrides allowed)."""
+    B = w.B if B is None else B
+    Sq = w.Sq if Sq is None else Sq
+    Sk = w.Sk if Sk is None else Sk
+    g = _gen(device, w.seed)
+    q = torch.randn(B, w.Hq, Sq, w.D, generator=g, device=device)
+    k = torch.randn(B, w.Hkv, Sk, w.D, generator=g, device=device)
+    v = torch.randn(B, w.Hkv, Sk, w.D, generator=g, device=device)
+    q, k, v = (t.to(w.torch_dtype) for t in (q, k, v))
+    if w.q_mult != 1.0:
+        q = q * w.q_mult
+    return tuple(t.transpose(1, 2).contiguous() for t in (q, k, v))
+
+
+def varlen_lengths(w: Workload, n=None, lo=None, hi=None) -> torch.Tensor:
+    n = w.varlen["n"] if n is None else n
+    lo = w.varlen["lo"] if lo is None else lo
+    hi = w.varlen["hi"] if hi is None else hi
+    g = _gen("cpu", w.seed)
+    return torch.randint(lo, hi + 1, (n,), generator=g, dtype=torch.int64)
+
+
+def cu_seqlens_of(lengths) -> torch.Tensor:
+    lengths = torch.as_tensor(lengths, dtype=torch.int64)
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(lengths, 0)
+    return cu.to(torch.int32)
+
+
+def make_varlen(w: Workload, device="cpu", lengths=None):
+    """Packed q [total,Hq,D], k/v [total,Hkv,D] and int32 cu_seqlens (host)."""
+    if lengths is None:
+        lengths = varlen_lengths(w)
+    cu = cu_seqlens_of(lengths)
+    total = int(cu[-1])
+    g = _gen(device, w.seed + 1000)
+    q = torch.randn(total, w.Hq, w.D, generator=g, device=device).to(w.torch_dtype)
+    k = torch.randn(total, w.Hkv, w.D, generator=g, device=device).to(w.torch_dtype)
+    v = torch.randn(total, w.Hkv, w.D, generator=g, device=device).to(w.torch_dtype)
+    if w.q_mult != 1.0:
+        q = q * w.q_mult
+    return q, k, v, cu
+
+
+def make_decode_q(w: Workload, device="cpu"):
+    g = _gen(device, w.seed)
+    q = torch.randn(w.B, w.Hq, 1, w.D, generator=g, device=device).to(w.torch_dtype)
+    return q.transpose(1, 2).contiguous()
+
+
+def make_decode_kv_one(w: Workload, b: int, device="cpu"):
+    """K and V [Sk, Hkv, D] of batch element b, from its own seed."""
+    g = _gen(device, w.seed * 1_000_003 + b)
+    k = torch.randn(w.Hkv, w.Sk, w.D, generator=g, device=device).to(w.torch_dtype)
+    v = torch.randn(w.Hkv, w.Sk, w.D, generator=g, device=device).to(w.torch_dtype)
+    return k.transpose(0, 1).contiguous(), v.transpose(0, 1).contiguous()
+
+
+def fill_decode_kv(w: Workload, k_out: torch.Tensor, v_out: torch.Tensor) -> None:
+    """Fill preallocated k/v [B,Sk,Hkv,D] element by element (on their device)."""
+    for b in range(k_out.shape[0]):
+        kb, vb = make_decode_kv_one(w, b, device=k_out.device)
+        k_out[b].copy_(kb)
+        v_out[b].copy_(vb)
+
+
+# ----------------------------------------------------------------------------------
+# Work accounting (the benchmark's denominators)
+
+def causal_pairs(Sq: int, Sk: int) -> int:
+    """Number of visible (i, j) pairs under the bottom-right causal mask j <= i + Sk - Sq."""
+    off = Sk - Sq
+    return sum(min(max(i + off + 1, 0), Sk) for i in range(Sq))
+
+
+def attention_flops(B: int, Hq: int, Sq: int, Sk: int, D: int, causal: bool) -> int:
+    """4*D flops per visible (query, key) pair per head: 2*D for QK^T, 2*D for PV."""
+    pairs = causal_pairs(Sq, Sk) if causal else Sq * Sk
+    return 4 * D * pairs * B * Hq
+
+
+def varlen_flops(lengths, Hq: int, D: int, causal: bool) -> int:
+    return sum(attention_flops(1, Hq, int(L), int(L), D, causal) for L in lengths)
+
+
+def kv_values_per_token(Hkv: int, D: int, layers: int = 1) -> int:
+    """Cached key and value elements per token: 2 * Hkv * D per layer."""
+    return 2 * Hkv * D * layers
+
+
+def kv_cache_bytes(batch: int, seq: int, Hkv: int, D: int, bytes_per_elt: int = 2,
+                   layers: int = 1) -> int:
+    """KV memory = 2 x batch x seq x head_dim x kv_heads (x bytes x layers)."""
+    return 2 * batch * seq * D * Hkv * bytes_per_elt * layers
+
+
+def decode_bytes(B: int, Hq: int, Hkv: int, Sk: int, D: int, elt: int = 2) -> int:
+    """Algorithmic HBM bytes of one decode step: K and V once, q, O (elt) and L (fp32)."""
+    return kv_cache_bytes(B, Sk, Hkv, D, elt) + 2 * B * Hq * D * elt + 4 * B * Hq
+
+
+def prefill_min_bytes(B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int, elt: int = 2):
+    """q, k, v read once, O written once (elt bytes), L written (fp32)."""
+    return elt * D * (2 * B * Sq * Hq + 2 * B * Sk * Hkv) + 4 * B * Hq * Sq
