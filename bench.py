@@ -1,0 +1,505 @@
+"""Benchmark of the B200 grouped-query attention forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one forward pass (gqa_attn_fwd through the C ABI) over one batch of the
+workload, with the inputs already resident in HBM.  The default workload is the
+encoder-shaped GQA batch (B=64, Hq=48, Hkv=12, S=512, D=64, bf16, non-causal);
+others: llama (B=4, Hq=32, Hkv=8, S=8192, D=128, causal), llama_stress (q x 4),
+decode_b{1,16,64,128,256} (Sq=1, Sk=32768, split-KV), varlen (32 packed causal
+sequences of 128..8192 tokens).  Prefill workloads report TFLOP/s, decode GB/s.
+
+Under torchrun every rank runs its own copy of the workload (independent batches,
+no collective on the data path: weak scaling); the time is the max over ranks.
+``--impl reference`` times the float64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import math
+import os
+import pathlib
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = pathlib.Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "GQA attn fwd TFLOP/s (prefill) & KV-read GB/s (decode), % roofline, 1×B200"
+L2_BYTES = 126 * 2**20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["exact_attention_gqa_b200/csrc/" + f for f in
+                  ("sm100_ptx.cuh", "prefill_sm100.cuh", "decode.cuh", "gqa_attn.cu")]
+
+
+# ----------------------------------------------------------------------------- helpers
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update((ROOT / f).read_bytes())
+    return h.hexdigest()[:12]
+
+
+def load_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if still current."""
+    f = ROOT / "profiles" / "dram_traffic.txt"
+    if not f.exists():
+        return None
+    src = kernel_source_hash()
+    for line in f.read_text().splitlines():
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload \
+                and parts[1] == kernel and parts[2] == src:
+            return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        out_dir = ROOT / "gpurun_out"
+        out_dir.mkdir(exist_ok=True)
+        self.path = out_dir / f"clocks_rank{os.environ.get('RANK', '0')}.csv"
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not self.path.exists():
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        rows = []
+        for line in self.path.read_text().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [r for r in rows if r[2] > 300.0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3][1:5])
+                          if v.lower() in ("active", "1")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(loaded)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Largest value of x over all ranks (the slowest rank decides the time)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- workloads
+def workload_by_name(name: str):
+    if name == "encoder":
+        return W.ENCODER
+    if name == "llama":
+        return W.LLAMA
+    if name == "llama_stress":
+        return W.LLAMA_STRESS
+    if name == "varlen":
+        return W.VARLEN
+    if name.startswith("decode_b"):
+        return W.decode(int(name[len("decode_b"):]), num_splits=0)
+    raise SystemExit(f"unknown workload {name}")
+
+
+class Case:
+    """Device tensors, the work accounting and a zero-argument step for one workload."""
+
+    def __init__(self, w: W.Workload, device, rank: int):
+        import exact_attention_gqa_b200 as G
+        self.G = G
+        self.w = w
+        self.device = device
+        self.decode = w.Sq == 1
+        self.varlen = bool(w.varlen)
+        if self.decode:
+            q = W.make_decode_q(w, device=device)
+            # rotate several KV copies when one is not larger than L2
+            kv_bytes = W.kv_cache_bytes(w.B, w.Sk, w.Hkv, w.D)
+            n_copies = 1 if kv_bytes > 2 * L2_BYTES else 3
+            self.kv = []
+            for c in range(n_copies):
+                k = torch.empty(w.B, w.Sk, w.Hkv, w.D, dtype=torch.bfloat16, device=device)
+                v = torch.empty_like(k)
+                W.fill_decode_kv(w, k, v)
+                self.kv.append((k, v))
+            self.q = q
+            rc, kern, splits, pack = G.gqa_attn_plan(w.B, w.Hq, w.Hkv, 1, w.Sk, w.D,
+                                                     num_splits=w.num_splits,
+                                                     pack_gqa=w.pack_gqa)
+            self.splits, self.pack = splits, pack
+            self.bytes = W.decode_bytes(w.B, w.Hq, w.Hkv, w.Sk, w.D)
+            self.flops = W.attention_flops(w.B, w.Hq, 1, w.Sk, w.D, False)
+            self.units, self.unit = self.bytes / 1e9, "GB/s"
+            self.launches_per_step = 2 if splits > 1 else 1
+            self.kernel = "decode_split_sm100"
+        elif self.varlen:
+            lengths = W.varlen_lengths(w)
+            q, k, v, cu = W.make_varlen(w, device=device, lengths=lengths)
+            self.q, self.kv, self.cu = q, [(k, v)], cu.to(device)
+            self.max_len = int(lengths.max())
+            self.lengths = lengths
+            self.flops = W.varlen_flops(lengths.tolist(), w.Hq, w.D, True)
+            self.units, self.unit = self.flops / 1e12, "TFLOP/s"
+            self.launches_per_step = 1
+            self.kernel = "prefill_fwd_sm100"
+            self.splits, self.pack = 1, 1
+        else:
+            q, k, v = W.make_qkv(w, device=device)
+            self.q, self.kv = q, [(k, v)]
+            self.flops = W.attention_flops(w.B, w.Hq, w.Sq, w.Sk, w.D, w.causal)
+            self.units, self.unit = self.flops / 1e12, "TFLOP/s"
+            self.launches_per_step = 1
+            self.kernel = "prefill_fwd_sm100"
+            rc, kern, self.splits, self.pack = G.gqa_attn_plan(w.B, w.Hq, w.Hkv, w.Sq, w.Sk,
+                                                               w.D, causal=w.causal,
+                                                               pack_gqa=w.pack_gqa)
+        self.out = torch.empty_like(self.q)
+        if self.varlen:
+            self.lse = torch.empty(w.Hq, self.q.shape[0], dtype=torch.float32, device=device)
+        else:
+            self.lse = torch.empty(self.q.shape[0], w.Hq, self.q.shape[1], dtype=torch.float32,
+                                   device=device)
+        self.i = 0
+
+    def in_bytes(self):
+        k, v = self.kv[0]
+        return self.q.numel() * 2 + k.numel() * 2 + v.numel() * 2
+
+    def out_bytes(self):
+        return self.out.numel() * 2 + self.lse.numel() * 4
+
+    def step(self):
+        k, v = self.kv[self.i % len(self.kv)]
+        self.i += 1
+        w = self.w
+        kw = dict(causal=w.causal, out=self.out, lse=self.lse, pack_gqa=w.pack_gqa)
+        if self.decode:
+            kw["num_splits"] = w.num_splits
+        if self.varlen:
+            kw.update(cu_seqlens=self.cu, max_seqlen=self.max_len)
+        self.G.gqa_attn(self.q, k, v, **kw)
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
+    """Time the float64 oracle on a bounded sample of workload w.
+
+    Prefill: random query rows (b, h, i), doubling the count until target_s of CPU
+    work; returns TFLOP/s of the sampled rows.  Decode: whole batch elements (all
+    heads over the 32768-key cache); returns GB/s of their KV.
+    Returns (value, sample description, threads used, seconds).
+    """
+    import oracle
+    rng = np.random.default_rng(seed)
+    cores = oracle.max_threads()
+    if w.Sq == 1:
+        k, v = W.make_decode_kv_one(w, 0)
+        q = W.make_decode_q(W.decode(1))
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.attention(q, k[None], v[None], scale=w.scale, causal=False)
+            el += time.perf_counter() - t0
+            n += 1
+        gb = n * W.decode_bytes(1, w.Hq, w.Hkv, w.Sk, w.D) / 1e9
+        return gb / el, f"{n} x one batch element (all {w.Hq} heads, Sk={w.Sk})", cores, el
+    if w.varlen:
+        lengths = W.varlen_lengths(w)
+        q, k, v, cu = W.make_varlen(w, lengths=lengths)
+        cu = cu.numpy()
+        lens = [int(x) for x in lengths]
+
+        def rows_of(n):
+            b = rng.integers(0, len(lens), n)
+            i = np.array([rng.integers(0, lens[x]) for x in b])
+            return np.stack([b, rng.integers(0, w.Hq, n), i], axis=1).astype(np.int32)
+
+        def flops(rows):
+            return int(sum(4 * w.D * (i + 1) for _, _, i in rows))
+    else:
+        q, k, v = W.make_qkv(w)
+        cu = None
+
+        def rows_of(n):
+            return np.stack([rng.integers(0, w.B, n), rng.integers(0, w.Hq, n),
+                             rng.integers(0, w.Sq, n)], axis=1).astype(np.int32)
+
+        def flops(rows):
+            if not w.causal:
+                return len(rows) * 4 * w.D * w.Sk
+            return int(sum(4 * w.D * min(w.Sk, i + w.Sk - w.Sq + 1) for _, _, i in rows))
+    n, el, done, nrows = 64, 0.0, 0, 0
+    while el < target_s and el < max_s:
+        rows = rows_of(n)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, rows, scale=w.scale, causal=w.causal, cu_seqlens=cu)
+        el += time.perf_counter() - t0
+        done += flops(rows)
+        nrows += n
+        n = min(n * 2, 1 << 16)
+    return done / 1e12 / el, f"{nrows} random query rows (b, h, i) of the workload", cores, el
+
+
+# ----------------------------------------------------------------------------- arms
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = workload_by_name(args.workload)
+    unit = "GB/s" if w.Sq == 1 else "TFLOP/s"
+    per_step = []
+    desc, cores = "", 0
+    for s in range(args.warmup + args.steps):
+        v, desc, cores, el = oracle_sample(w, target_s=2.0, max_s=6.0, seed=s)
+        if s >= args.warmup:
+            per_step.append((v, el))
+    value = statistics.median(v for v, _ in per_step)
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(e for _, e in per_step),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {desc}"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import exact_attention_gqa_b200 as G
+    from exact_attention_gqa_b200 import build
+    build.build()
+    device = torch.device("cuda", local)
+    w = workload_by_name(args.workload)
+    case = Case(w, device, rank)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(args.warmup, 3)):
+        case.step()
+    torch.cuda.synchronize()
+    # calibrate the step count so the timed region lasts about 2 s unless given
+    if args.steps <= 0:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(5):
+            case.step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / 5
+        steps = int(max(20, min(20000, 2000.0 / max(ms, 1e-3))))
+        steps = int(max_over_ranks(steps, world))
+    else:
+        steps = args.steps
+    # ---- device-timed region: inputs resident, K steps
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        torch.cuda.synchronize()
+        barrier(world)
+        ev0.record(stream)
+        for _ in range(steps):
+            case.step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    ms_step = ms_total / steps
+    value = case.units * world / (ms_step / 1e3)
+    if rank != 0:
+        # the other ranks take part in the e2e timing below, then exit
+        pass
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(3, min(steps, 20))
+    k0, v0 = case.kv[0]
+    hq = torch.empty(case.q.shape, dtype=case.q.dtype, pin_memory=True).copy_(case.q)
+    hk = torch.empty(k0.shape, dtype=k0.dtype, pin_memory=True).copy_(k0)
+    hv = torch.empty(v0.shape, dtype=v0.dtype, pin_memory=True).copy_(v0)
+    ho = torch.empty(case.out.shape, dtype=case.out.dtype, pin_memory=True)
+    hl = torch.empty(case.lse.shape, dtype=case.lse.dtype, pin_memory=True)
+    dq, dk, dv = torch.empty_like(case.q), torch.empty_like(k0), torch.empty_like(v0)
+    cu_h = case.cu.cpu().pin_memory() if case.varlen else None
+    dcu = torch.empty_like(case.cu) if case.varlen else None
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        kw = dict(causal=w.causal, out=case.out, lse=case.lse, pack_gqa=w.pack_gqa)
+        if case.decode:
+            kw["num_splits"] = w.num_splits
+        if case.varlen:
+            dcu.copy_(cu_h, non_blocking=True)
+            kw.update(cu_seqlens=dcu, max_seqlen=case.max_len)
+        G.gqa_attn(dq, dk, dv, **kw)
+        ho.copy_(case.out, non_blocking=True)
+        hl.copy_(case.lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = hq.numel() * hq.element_size() + hk.numel() * 2 + hv.numel() * 2 + \
+        (cu_h.numel() * 4 if cu_h is not None else 0)
+    d2h = ho.numel() * 2 + hl.numel() * 4
+    err = G.gqa_attn_get_device_error()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    # ---- roofline of the dominant kernel
+    peaks, peak_kind = load_peaks()
+    kernel_ms = ms_step  # one launch per step (decode: split kernel + combine)
+    if case.decode:
+        achieved = case.bytes / (kernel_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = case.flops / (kernel_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_kind} ({'hbm_gbs' if case.decode else 'bf16_tflops'}, burst)"
+    roof["kernel"] = case.kernel
+    tr = load_traffic(w.name, case.kernel)
+    roof["traffic"] = tr
+    if tr is not None:
+        roof["traffic_per_algorithmic"] = tr / (case.bytes if case.decode else
+                                                W.prefill_min_bytes(w.B, w.Hq, w.Hkv, w.Sq,
+                                                                    w.Sk, w.D))
+    # ---- CPU baseline (oracle on a bounded sample, rank 0, N=1 only)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v_cpu, desc, cores, el = oracle_sample(w, target_s=args.cpu_seconds, max_s=30.0)
+        cpu = {"value": v_cpu, "unit": case.unit, "cores": cores, "kind": "oracle",
+               "sample": f"{desc}; {el:.1f} s of float64 CPU work"}
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Sk": w.Sk,
+           "D": w.D, "causal": w.causal, "pack_gqa": case.pack, "num_splits": case.splits,
+           "per_rank": "independent copy of the workload on every rank",
+           "l2": ("inputs larger than L2 (%.0f MB per step)" % (case.in_bytes() / 1e6)
+                  if case.in_bytes() > L2_BYTES or len(case.kv) > 1 else "inputs fit in L2"),
+           "kv_copies_rotated": len(case.kv)}
+    if case.varlen:
+        cfg["total_tokens"] = int(case.q.shape[0])
+    line = {"metric": METRIC, "value": value, "unit": case.unit, "n_gpus": world,
+            "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) bf16)", "config": cfg, "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": steps * case.launches_per_step,
+            "clocks": clocks.summary(), "device_error": err,
+            "kernel_source": kernel_source_hash(), "library": G.library_path()}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0: about 2 s)")
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="encoder")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        if args.steps <= 0:
+            args.steps = 3
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,165 @@
+"""Exact grouped-query attention forward for B200 (sm_100a).
+
+The computation runs in hand-written CUDA kernels behind the C ABI of
+``include/gqa_attn.h`` (``libgqa_attn.so``).  This module marshals torch
+tensors into that ABI: it checks dtypes, devices and layouts, allocates the
+outputs (and the split-KV workspace) with torch, passes raw pointers and the
+current CUDA stream, and raises on a non-zero status.  There is no fallback:
+without the built library or a CUDA tensor every call raises.
+
+    out, lse = gqa_attn(q, k, v, causal=True)
+
+Layouts follow FlashAttention's ``flash_attn_func`` ([batch, seq, heads, dim]):
+q [B, Sq, Hq, D], k/v [B, Sk, Hkv, D] -> out [B, Sq, Hq, D], lse [B, Hq, Sq];
+packed variable length: q [total, Hq, D], k/v [total, Hkv, D], cu_seqlens
+int32 [B + 1] -> out [total, Hq, D], lse [Hq, total].
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+from . import _capi
+from ._capi import GqaError, STATUS, STATUS_CODE, strerror
+
+__all__ = ["gqa_attn", "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
+           "gqa_attn_workspace_bytes", "gqa_attn_set_workspace", "gqa_attn_get_device_error",
+           "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path"]
+
+KERNEL_NAMES = {0: "none", 1: "prefill_sm100", 2: "decode_splitkv", 3: "zero_fill"}
+
+
+def library_path() -> str:
+    return str(_capi.LIB_PATH)
+
+
+def _stream_handle(torch, device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+# ------------------------------------------------------------------ raw C-ABI calls
+def gqa_attn_fwd(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Sq, Sk, D, scale, causal,
+                 num_splits, pack_gqa, cu_seqlens_ptr, stream) -> int:
+    """Direct call of the C entry point (pointers as ints or c_void_p); returns the status."""
+    return _capi.load().gqa_attn_fwd(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Sq, Sk,
+                                     D, scale, causal, num_splits, pack_gqa, cu_seqlens_ptr,
+                                     stream)
+
+
+def gqa_attn_fwd_f32(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Sq, Sk, D, scale, causal,
+                     num_splits, pack_gqa, cu_seqlens_ptr, stream) -> int:
+    return _capi.load().gqa_attn_fwd_f32(q_ptr, k_ptr, v_ptr, out_ptr, lse_ptr, B, Hq, Hkv, Sq,
+                                         Sk, D, scale, causal, num_splits, pack_gqa,
+                                         cu_seqlens_ptr, stream)
+
+
+def gqa_attn_workspace_bytes(B, Hq, Sq, D, num_splits) -> int:
+    return int(_capi.load().gqa_attn_workspace_bytes(B, Hq, Sq, D, num_splits))
+
+
+def gqa_attn_set_workspace(ptr, nbytes) -> int:
+    return _capi.load().gqa_attn_set_workspace(ptr, nbytes)
+
+
+def gqa_attn_plan(B, Hq, Hkv, Sq, Sk, D, scale=None, causal=False, num_splits=1, pack_gqa=-1,
+                  varlen=False):
+    """(status, kernel name, effective num_splits, effective pack_gqa)."""
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    kern, spl, pk = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    rc = _capi.load().gqa_attn_plan(B, Hq, Hkv, Sq, Sk, D, scale, int(bool(causal)), num_splits,
+                                    pack_gqa, int(bool(varlen)), ctypes.byref(kern),
+                                    ctypes.byref(spl), ctypes.byref(pk))
+    return rc, KERNEL_NAMES.get(kern.value, kern.value), spl.value, pk.value
+
+
+def gqa_attn_get_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    rc = _capi.load().gqa_attn_get_device_error(ctypes.byref(code), stream)
+    if rc != 0:
+        raise GqaError("gqa_attn_get_device_error", rc)
+    return code.value
+
+
+# ------------------------------------------------------------------ torch front end
+_ws = {}  # device index -> torch buffer registered as the split-KV workspace
+
+
+def _workspace(torch, device, nbytes):
+    if nbytes == 0:
+        return
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    buf = _ws.get(idx)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws[idx] = buf
+    rc = gqa_attn_set_workspace(ctypes.c_void_p(buf.data_ptr()), buf.numel())
+    if rc != 0:
+        raise GqaError("gqa_attn_set_workspace", rc)
+
+
+def gqa_attn(q, k, v, *, causal: bool = False, scale: float | None = None,
+             num_splits: int = 1, pack_gqa: int = -1, cu_seqlens=None, max_seqlen=None,
+             out=None, lse=None):
+    """Exact attention forward with grouped-query heads on the current CUDA stream.
+
+    Returns (out, lse).  bf16 inputs run the sm_100a kernels, fp32 inputs the fp32
+    path.  ``scale`` defaults to 1/sqrt(D) (FlashAttention's softmax_scale=None).
+    """
+    import torch
+
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("gqa_attn needs CUDA tensors (there is no CPU path)")
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("q, k, v must all be bf16 or all fp32")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    varlen = cu_seqlens is not None
+    if varlen:
+        if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+            raise ValueError("packed inputs are q [total, Hq, D], k/v [total, Hkv, D]")
+        total, Hq, D = q.shape
+        Hkv = k.shape[1]
+        if k.shape[0] != total:
+            raise ValueError("q and k/v must hold the same packed rows")
+        cu = cu_seqlens
+        if not cu.is_cuda or cu.dtype != torch.int32:
+            raise ValueError("cu_seqlens must be a CUDA int32 tensor")
+        B = cu.numel() - 1
+        if max_seqlen is None:
+            max_seqlen = int((cu[1:] - cu[:-1]).max().item()) if B > 0 else 0
+        Sq, Sk = int(max_seqlen), int(total)
+        lse_shape = (Hq, total)
+    else:
+        if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+            raise ValueError("dense inputs are q [B, Sq, Hq, D], k/v [B, Sk, Hkv, D]")
+        B, Sq, Hq, D = q.shape
+        _, Sk, Hkv, _ = k.shape
+        cu = None
+        lse_shape = (B, Hq, Sq)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    stream = _stream_handle(torch, q.device)
+    if q.dtype == torch.bfloat16:
+        rc, _, splits, _ = gqa_attn_plan(B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
+                                         pack_gqa, varlen)
+        if rc == 0 and splits > 1:
+            _workspace(torch, q.device, gqa_attn_workspace_bytes(B, Hq, Sq, D, splits))
+        rc = gqa_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk,
+                          D, scale, int(bool(causal)), num_splits, pack_gqa, _ptr(cu), stream)
+        if rc != 0:
+            raise GqaError("gqa_attn_fwd", rc)
+    else:
+        rc = gqa_attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq,
+                              Sk, D, scale, int(bool(causal)), num_splits, pack_gqa, _ptr(cu),
+                              stream)
+        if rc != 0:
+            raise GqaError("gqa_attn_fwd_f32", rc)
+    return out, lse

@@ -1,0 +1,374 @@
+// Split-KV decode (one query position against a long KV cache) and the
+// log-sum-exp weighted combine of its partial results.
+//
+// Decode reads every key and value once and does ~4 flops per byte, so it is
+// bound by HBM bandwidth.  The kernel therefore streams K/V blocks through a
+// TMA + mbarrier ring (one producer warp, four consumer warps), spreads the cache
+// over many CTAs (batch x KV-head unit x split), and keeps the arithmetic small
+// enough never to limit the stream: per 16 keys a consumer warp issues 16
+// ldmatrix and 32 warp-level bf16 MMAs (m16n8k16, fp32 accumulate) for
+// S = q K^T and O += P V, with P kept in registers between the two.
+//
+// The split-KV knob is the num_splits parameter of the GQA batch-size guide
+// (parameter table and flash_attn_func example).  Its combine follows from the
+// online softmax being exact and associative (FlashAttention-2 summary page,
+// streaming softmax and L = m + log l): with per-split normalised O_s and L_s,
+// L = M + ln sum_s exp(L_s - M) and O = sum_s exp(L_s - L) O_s.
+// Splits are contiguous ranges of whole 64-key blocks.
+//
+// pack_gqa = 1 puts the query heads of one KV head (up to 16) in the rows of
+// one CTA so that K/V are read once per group; pack_gqa = 0 gives every query
+// head its own CTA (the group's CTAs then share K/V through L2).
+#pragma once
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+
+struct DecodeParams {
+    const __nv_bfloat16* q;  // [B, 1, Hq, D]
+    __nv_bfloat16* out;      // [B, 1, Hq, D]
+    float* lse;              // [B, Hq, 1]
+    float* part_o;           // [B, Hq, n, D] fp32 (n > 1)
+    float* part_l;           // [B, Hq, n]    fp32 (n > 1)
+    int B, Hq, Hkv, Sk, G;
+    int rows;                // query heads per CTA (1..16)
+    int units_per_kv;        // ceil(G / rows)
+    int n_splits;
+    int blocks_per_split;    // 64-key blocks per split
+    float scale_log2;
+};
+
+template <int HD>
+struct DecodeCfg {
+    static constexpr int BN = 64;                  // keys per stage
+    static constexpr int ATOMS = HD / 64;
+    static constexpr int ATOM = BN * 128;          // bytes of one 64-key x 64-dim atom
+    static constexpr int TILE = BN * HD * 2;       // bytes of K (or V) per stage
+    static constexpr int STAGES = (HD == 128) ? 3 : 6;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = STAGES * TILE;
+    static constexpr int OFF_BAR = 2 * STAGES * TILE;
+    static constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
+    static constexpr int MERGE_BYTES = 4 * 16 * (HD + 2) * 4;  // per-warp partials
+    static constexpr int SMEM_BYTES =
+        (OFF_MISC + 16 > MERGE_BYTES ? OFF_MISC + 16 : MERGE_BYTES) + 1024;
+    static constexpr int THREADS = 160;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                          uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulate
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte offset of the 16-byte chunk holding dims [8c, 8c+8) of row `row` in a
+// 128B-swizzled [rows x 64 dims] atom written by TMA.
+__device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
+    return uint32_t(row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+template <int HD>
+__global__ void __launch_bounds__(160, 2)
+    decode_split_sm100(const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+    using C = DecodeCfg<HD>;
+    constexpr int ST = C::STAGES;
+    constexpr int KSTEPS = HD / 16;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* bar_empty = bar_full + ST;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC);
+
+    const int split = blockIdx.x;
+    const int unit = blockIdx.y;  // kv head * units_per_kv + head chunk
+    const int b = blockIdx.z;
+    const int kvh = unit / p.units_per_kv;
+    const int h0 = kvh * p.G + (unit - kvh * p.units_per_kv) * p.rows;
+    const int rows = min(p.rows, kvh * p.G + p.G - h0);
+    const int nblk_total = (p.Sk + C::BN - 1) / C::BN;
+    const int blk0 = split * p.blocks_per_split;
+    const int blk1 = min(blk0 + p.blocks_per_split, nblk_total);
+    const int nblk = max(blk1 - blk0, 0);
+    const int key_end = min(blk1 * C::BN, p.Sk);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(bar_full + s, 1);
+            mbar_init(bar_empty + s, 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // per-warp online-softmax state: rows g = lane/4 and g + 8
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_part[2] = {0.f, 0.f};
+    float o[KSTEPS * 2][4];
+#pragma unroll
+    for (int t = 0; t < KSTEPS * 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[t][e] = 0.f;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            int c = 0;
+            for (; c < nblk; ++c) {
+                const int s = c % ST;
+                if (!mbar_wait(bar_empty + s, ((c / ST) & 1) ^ 1, abort_flag)) break;
+                mbar_arrive_expect_tx(bar_full + s, 2 * C::TILE);
+                const int z = b * p.Sk + (blk0 + c) * C::BN;
+#pragma unroll
+                for (int a = 0; a < C::ATOMS; ++a) {
+                    tma_load_3d(smem + C::OFF_K + s * C::TILE + a * C::ATOM, &tm_k, bar_full + s,
+                                a * 64, kvh, z);
+                    tma_load_3d(smem + C::OFF_V + s * C::TILE + a * C::ATOM, &tm_v, bar_full + s,
+                                a * 64, kvh, z);
+                }
+            }
+            // every issued copy lands before the CTA may reuse or release the memory
+            for (int s = 0; s < ST; ++s) {
+                const int u = c / ST + (s < c % ST ? 1 : 0);
+                if (u > 0) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!mbar_try_wait(bar_full + s, (u - 1) & 1))
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                            raise_device_error(kDevWaitTimeout);
+                            break;
+                        }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ consumers
+        const float sl2 = p.scale_log2;
+        const int g = lane >> 2;      // row (query head offset) of c0/c1, +8 for c2/c3
+        const int qd = (lane & 3) * 2;  // column pair within an 8-wide tile
+        // q as the A operand of m16n8k16 (rows >= `rows` are zero)
+        uint32_t qa[KSTEPS][4];
+        {
+            const uint32_t* qrow0 = reinterpret_cast<const uint32_t*>(
+                p.q + (size_t(b) * p.Hq + h0 + g) * HD);
+            const uint32_t* qrow1 = reinterpret_cast<const uint32_t*>(
+                p.q + (size_t(b) * p.Hq + h0 + g + 8) * HD);
+            const bool v0 = g < rows, v1 = g + 8 < rows;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                qa[kk][0] = v0 ? __ldg(qrow0 + (kk * 16 + qd) / 2) : 0u;
+                qa[kk][1] = v1 ? __ldg(qrow1 + (kk * 16 + qd) / 2) : 0u;
+                qa[kk][2] = v0 ? __ldg(qrow0 + (kk * 16 + 8 + qd) / 2) : 0u;
+                qa[kk][3] = v1 ? __ldg(qrow1 + (kk * 16 + 8 + qd) / 2) : 0u;
+            }
+        }
+        const uint32_t sK0 = smem_u32(smem + C::OFF_K);
+        const uint32_t sV0 = smem_u32(smem + C::OFF_V);
+        // ldmatrix row addresses: lane provides row (lane & 7) of matrix (lane >> 3)
+        const int mat = lane >> 3, mrow = lane & 7;
+        // QK: matrices (keys +0/+8) x (dim chunk +0/+1): key = 16w + (mat>>1)*8 + mrow
+        const int key_qk = warp * 16 + (mat >> 1) * 8 + mrow;
+        const int chunk_qk = mat & 1;
+        // PV (trans): matrices (keys +0/+8) x (dim chunk +0/+1): key = 16w + (mat&1)*8 + mrow
+        const int key_pv = warp * 16 + (mat & 1) * 8 + mrow;
+        const int chunk_pv = mat >> 1;
+        for (int c = 0; c < nblk; ++c) {
+            const int s = c % ST;
+            if (!mbar_wait_warp(bar_full + s, (c / ST) & 1, abort_flag)) break;
+            const uint32_t sK = sK0 + s * C::TILE;
+            const uint32_t sV = sV0 + s * C::TILE;
+            float sc[2][4];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[t][e] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                const int chunk = kk * 2 + chunk_qk;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(sK + (chunk >> 3) * C::ATOM + sw128_off(key_qk, chunk), b0, b1, b2, b3);
+                mma_bf16_16816(sc[0], qa[kk], b0, b1);
+                mma_bf16_16816(sc[1], qa[kk], b2, b3);
+            }
+            // mask keys past the end of this split / of the cache
+            const int kbase = (blk0 + c) * C::BN + warp * 16 + qd;
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (kbase + t * 8 + (e & 1) >= key_end) sc[t][e] = -INFINITY;
+            // online softmax (rows g and g + 8), quad reduction of the block max
+            float alpha[2];
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                float mx = fmaxf(fmaxf(sc[0][2 * hr], sc[0][2 * hr + 1]),
+                                 fmaxf(sc[1][2 * hr], sc[1][2 * hr + 1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float mb = mx * sl2;
+                alpha[hr] = 1.f;
+                if (mb > m_run[hr] + 8.0f) {
+                    alpha[hr] = ex2_approx(m_run[hr] - mb);
+                    m_run[hr] = mb;
+                }
+            }
+            uint32_t pa[4];
+            {
+                float pr[2][4];
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int hr = e >> 1;
+                        const float mu = (m_run[hr] == -INFINITY) ? 0.f : m_run[hr];
+                        pr[t][e] = ex2_approx(fmaf(sc[t][e], sl2, -mu));
+                    }
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr)
+                    l_part[hr] = l_part[hr] * alpha[hr] + pr[0][2 * hr] + pr[0][2 * hr + 1] +
+                                 pr[1][2 * hr] + pr[1][2 * hr + 1];
+                pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+                pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+                pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+                pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+            }
+            if (alpha[0] != 1.f || alpha[1] != 1.f) {
+#pragma unroll
+                for (int t = 0; t < KSTEPS * 2; ++t) {
+                    o[t][0] *= alpha[0];
+                    o[t][1] *= alpha[0];
+                    o[t][2] *= alpha[1];
+                    o[t][3] *= alpha[1];
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < KSTEPS; ++nt) {
+                const int chunk = nt * 2 + chunk_pv;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(sV + (chunk >> 3) * C::ATOM + sw128_off(key_pv, chunk), b0, b1, b2, b3);
+                mma_bf16_16816(o[2 * nt], pa, b0, b1);
+                mma_bf16_16816(o[2 * nt + 1], pa, b2, b3);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_empty + s);
+        }
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            l_part[hr] += __shfl_xor_sync(0xffffffffu, l_part[hr], 1);
+            l_part[hr] += __shfl_xor_sync(0xffffffffu, l_part[hr], 2);
+        }
+    }
+    __syncthreads();  // every stage consumed, every copy landed: reuse smem for the merge
+
+    // ---------------------------------------------------------------- merge warps
+    float* mo = reinterpret_cast<float*>(smem);           // [4][16][HD]
+    float* mm = mo + 4 * 16 * HD;                          // [4][16]
+    float* ml = mm + 4 * 16;                               // [4][16]
+    if (warp < 4) {
+        const int g = lane >> 2, qd = (lane & 3) * 2;
+#pragma unroll
+        for (int nt = 0; nt < KSTEPS * 2; ++nt) {
+            float* r0 = mo + (warp * 16 + g) * HD + nt * 8 + qd;
+            float* r1 = mo + (warp * 16 + g + 8) * HD + nt * 8 + qd;
+            r0[0] = o[nt][0];
+            r0[1] = o[nt][1];
+            r1[0] = o[nt][2];
+            r1[1] = o[nt][3];
+        }
+        if ((lane & 3) == 0) {
+            mm[warp * 16 + g] = m_run[0];
+            mm[warp * 16 + g + 8] = m_run[1];
+            ml[warp * 16 + g] = l_part[0];
+            ml[warp * 16 + g + 8] = l_part[1];
+        }
+    }
+    __syncthreads();
+    if (*abort_flag) return;
+    for (int idx = threadIdx.x; idx < rows * HD; idx += blockDim.x) {
+        const int r = idx / HD, d = idx - r * HD;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * 16 + r]);
+        const float Mu = (M == -INFINITY) ? 0.f : M;
+        float acc = 0.f, l = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float f = ex2_approx(mm[w * 16 + r] - Mu);
+            acc += f * mo[(w * 16 + r) * HD + d];
+            l += f * ml[w * 16 + r];
+        }
+        const int h = h0 + r;
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const float L = (l > 0.f) ? (Mu + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (p.n_splits == 1) {
+            p.out[(size_t(b) * p.Hq + h) * HD + d] = __float2bfloat16_rn(acc * inv_l);
+            if (d == 0) p.lse[size_t(b) * p.Hq + h] = L;
+        } else {
+            const size_t base = (size_t(b) * p.Hq + h) * p.n_splits + split;
+            p.part_o[base * HD + d] = acc * inv_l;
+            if (d == 0) p.part_l[base] = L;
+        }
+    }
+}
+
+// One warp per (batch, query head): O = sum_s exp(L_s - L) O_s, L = logsumexp(L_s).
+template <int HD>
+__global__ void __launch_bounds__(128)
+    splitkv_combine(const float* __restrict__ part_o, const float* __restrict__ part_l,
+                    __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int rows_bh,
+                    int n) {
+    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= rows_bh) return;
+    const float* Ls = part_l + size_t(w) * n;
+    float M = -INFINITY;
+    for (int s = lane; s < n; s += 32) M = fmaxf(M, Ls[s]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    constexpr int PER = HD / 32;
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    float L = -INFINITY;
+    if (M != -INFINITY) {
+        float sum = 0.f;
+        for (int s = lane; s < n; s += 32) sum += (Ls[s] == -INFINITY) ? 0.f : expf(Ls[s] - M);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        L = M + logf(sum);
+        for (int s = 0; s < n; ++s) {
+            const float ls = Ls[s];
+            if (ls == -INFINITY) continue;
+            const float wgt = expf(ls - L);
+            const float* os = part_o + (size_t(w) * n + s) * HD;
+#pragma unroll
+            for (int e = 0; e < PER; ++e) acc[e] += wgt * os[lane + 32 * e];
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) out[size_t(w) * HD + lane + 32 * e] = __float2bfloat16_rn(acc[e]);
+    if (lane == 0) lse[w] = L;
+}
+
+}  // namespace gqa

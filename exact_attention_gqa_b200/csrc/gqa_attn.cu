@@ -1,0 +1,421 @@
+// Host side of the C ABI declared in include/gqa_attn.h: argument checks, the
+// choice of kernel and knobs, TMA descriptor encoding and the launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gqa_attn.h"
+#include "sm100_ptx.cuh"
+#include "prefill_sm100.cuh"
+#include "decode.cuh"
+#include "simt_f32.cuh"
+
+namespace {
+
+using gqa::DecodeCfg;
+using gqa::DecodeParams;
+using gqa::F32Params;
+using gqa::PrefillCfg;
+using gqa::PrefillParams;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxSplits = 256;
+
+enum Kernel { kNone = 0, kPrefill = 1, kDecode = 2, kZeroFill = 3 };
+
+struct Workspace {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+};
+Workspace g_ws;
+std::mutex g_mu;
+
+// ---------------------------------------------------------------------------- device
+struct DeviceInfo {
+    int ok = 0;       // 1 when the device is sm_100
+    int sms = 0;
+    int attrs_set = 0;
+};
+DeviceInfo g_dev[64];
+
+int device_info(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQA_ERR_CUDA;
+    DeviceInfo& d = g_dev[dev];
+    if (d.sms == 0) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        d.ok = (major == 10 && minor == 0);
+        d.sms = sms;
+    }
+    *out = &d;
+    return d.ok ? GQA_OK : GQA_ERR_UNSUPPORTED;
+}
+
+// ---------------------------------------------------------------------------- TMA
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 view [rows, heads, D] with a {64, box_h, box_rows} box, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int heads, int D, int box_h,
+              int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(heads), cuuint64_t(rows)};
+    cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(heads) * D * 2};
+    cuuint32_t box[3] = {64u, cuuint32_t(box_h), cuuint32_t(box_rows)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------- plan
+struct Plan {
+    int kernel = kNone;
+    int splits = 1;
+    int pack = 0;
+    int decode_rows = 1;
+    int decode_units = 1;
+    int blocks_per_split = 0;
+};
+
+int check_shape(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int num_splits,
+                int pack_gqa, bool varlen, bool is_f32) {
+    if (B < 0 || Sq < 0 || Sk < 0 || Hq <= 0 || Hkv <= 0) return GQA_ERR_SHAPE;
+    if (Hq % Hkv != 0) return GQA_ERR_SHAPE;
+    if (is_f32) {
+        if (D < 1 || D > 256) return GQA_ERR_HEADDIM;
+    } else if (D != 64 && D != 128) {
+        return GQA_ERR_HEADDIM;
+    }
+    if (!(std::isfinite(scale) && scale > 0.f)) return GQA_ERR_SCALE;
+    if (pack_gqa < -1 || pack_gqa > 1) return GQA_ERR_UNSUPPORTED;
+    if (num_splits < 0 || num_splits > kMaxSplits) return GQA_ERR_SPLITS;
+    if (num_splits > 1 && (is_f32 || varlen || Sq != 1)) return GQA_ERR_SPLITS;
+    // index ranges: rows * heads * D must stay addressable with 32-bit row indices
+    const long long rows_q = varlen ? 0 : (long long)B * Sq;
+    const long long rows_k = varlen ? 0 : (long long)B * Sk;
+    if (rows_q > INT32_MAX || rows_k > INT32_MAX) return GQA_ERR_SHAPE;
+    return GQA_OK;
+}
+
+void make_plan(Plan* pl, int B, int Hq, int Hkv, int Sq, int Sk, int num_splits, int pack_gqa,
+               bool varlen, int sms) {
+    const int G = Hq / Hkv;
+    *pl = Plan();
+    if (B == 0 || Sq == 0) return;
+    if (!varlen && Sk == 0) {
+        pl->kernel = kZeroFill;
+        return;
+    }
+    if (!varlen && Sq == 1) {
+        pl->kernel = kDecode;
+        pl->pack = (pack_gqa < 0) ? (G > 1 ? 1 : 0) : pack_gqa;
+        pl->decode_rows = pl->pack ? (G < 16 ? G : 16) : 1;
+        pl->decode_units = (G + pl->decode_rows - 1) / pl->decode_rows;
+        const int nblk = (Sk + DecodeCfg<128>::BN - 1) / DecodeCfg<128>::BN;
+        int n = num_splits;
+        if (n == 0) {
+            // enough CTAs for two per SM, splits of at least four 64-key blocks
+            const long long ctas = (long long)B * Hkv * pl->decode_units;
+            const long long want = (2LL * sms + ctas - 1) / ctas;
+            n = int(want < 1 ? 1 : (want > 64 ? 64 : want));
+            const int max_by_len = nblk / 4 > 0 ? nblk / 4 : 1;
+            if (n > max_by_len) n = max_by_len;
+        }
+        if (n > nblk) n = nblk;
+        if (n < 1) n = 1;
+        pl->blocks_per_split = (nblk + n - 1) / n;
+        n = (nblk + pl->blocks_per_split - 1) / pl->blocks_per_split;  // drop empty splits
+        pl->splits = n;
+        return;
+    }
+    pl->kernel = kPrefill;
+    pl->splits = 1;
+    const bool can_pack = G > 1 && (128 % G == 0);
+    pl->pack = (pack_gqa < 0) ? (can_pack ? 1 : 0) : (pack_gqa == 1 && can_pack ? 1 : 0);
+}
+
+size_t ws_bytes(int B, int Hq, int Sq, int D, int n) {
+    if (n <= 1) return 0;
+    const size_t rows = size_t(B) * Hq * Sq * n;
+    const size_t o = rows * D * 4;
+    return ((o + 255) / 256) * 256 + rows * 4;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+template <int HD>
+int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                   int Hq, int Hkv, int Sq, int Sk, float scale, int causal, int pack,
+                   const int* cu, int sms, cudaStream_t stream) {
+    using C = PrefillCfg<HD>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(gqa::prefill_fwd_sm100<HD>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        attr_done = true;
+    }
+    const int G = Hq / Hkv;
+    PrefillParams p;
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.cu_seqlens = cu;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sq = Sq;
+    p.Sk = Sk;
+    p.G = G;
+    p.pack = pack;
+    p.sub_pos = pack ? 128 / G : 128;
+    p.n_mblk = (Sq + 2 * p.sub_pos - 1) / (2 * p.sub_pos);
+    p.n_hu = pack ? Hkv : Hq;
+    const long long units = (long long)p.n_mblk * B * p.n_hu;
+    if (units > INT32_MAX) return GQA_ERR_SHAPE;
+    p.n_units = int(units);
+    p.causal = causal ? 1 : 0;
+    p.scale_log2 = scale * kLog2e;
+    // Row extents of the 3-D views: exactly the rows the caller allocated
+    // (packed variable length: Sk carries the packed row count).
+    const long long rows_q = cu ? (long long)Sk : (long long)B * Sq;
+    const long long rows_k = cu ? (long long)Sk : (long long)B * Sk;
+    p.total_rows = cu ? Sk : 0;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) ||
+        !make_map(&tk, k, rows_k, Hkv, HD, 1, C::BN) ||
+        !make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN))
+        return GQA_ERR_CUDA;
+    const int grid = p.n_units < sms ? p.n_units : sms;
+    gqa::prefill_fwd_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+template <int HD>
+int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                  int Hq, int Hkv, int Sk, float scale, const Plan& pl, cudaStream_t stream) {
+    using C = DecodeCfg<HD>;
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(gqa::decode_split_sm100<HD>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        attr_done = true;
+    }
+    DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sk = Sk;
+    p.G = Hq / Hkv;
+    p.rows = pl.decode_rows;
+    p.units_per_kv = pl.decode_units;
+    p.n_splits = pl.splits;
+    p.blocks_per_split = pl.blocks_per_split;
+    p.scale_log2 = scale * kLog2e;
+    p.part_o = nullptr;
+    p.part_l = nullptr;
+    if (pl.splits > 1) {
+        const size_t need = ws_bytes(B, Hq, 1, HD, pl.splits);
+        if (!g_ws.ptr || g_ws.bytes < need) return GQA_ERR_WORKSPACE;
+        const size_t o_bytes = size_t(B) * Hq * pl.splits * HD * 4;
+        p.part_o = static_cast<float*>(g_ws.ptr);
+        p.part_l = reinterpret_cast<float*>(static_cast<char*>(g_ws.ptr) +
+                                            ((o_bytes + 255) / 256) * 256);
+    }
+    CUtensorMap tk, tv;
+    const long long rows = (long long)B * Sk;
+    if (!make_map(&tk, k, rows, Hkv, HD, 1, C::BN) || !make_map(&tv, v, rows, Hkv, HD, 1, C::BN))
+        return GQA_ERR_CUDA;
+    dim3 grid(pl.splits, Hkv * pl.decode_units, B);
+    gqa::decode_split_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+    if (pl.splits > 1) {
+        const int rows_bh = B * Hq;
+        const int blocks = (rows_bh + 3) / 4;
+        gqa::splitkv_combine<HD><<<blocks, 128, 0, stream>>>(
+            p.part_o, p.part_l, p.out, lse, rows_bh, pl.splits);
+        if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+    }
+    return GQA_OK;
+}
+
+int fwd_common(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+               int Hkv, int Sq, int Sk, int D, float scale, int causal, int num_splits,
+               int pack_gqa, const int* cu, cudaStream_t stream, bool is_f32) {
+    const bool varlen = cu != nullptr;
+    int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, num_splits, pack_gqa, varlen, is_f32);
+    if (rc != GQA_OK) return rc;
+    if (B == 0 || Sq == 0 || (varlen && Sk == 0)) return GQA_OK;  // nothing to compute
+    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || (cu && !aligned(cu, 4)))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+
+    if (is_f32) {
+        if (!varlen && Sk == 0) {
+            gqa::fill_no_keys<float><<<256, 256, 0, stream>>>(
+                static_cast<float*>(out), (long long)B * Sq * Hq * D, lse, (long long)B * Hq * Sq);
+            return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+        }
+        F32Params p;
+        p.q = static_cast<const float*>(q);
+        p.k = static_cast<const float*>(k);
+        p.v = static_cast<const float*>(v);
+        p.out = static_cast<float*>(out);
+        p.lse = lse;
+        p.cu_seqlens = cu;
+        p.B = B;
+        p.Hq = Hq;
+        p.Hkv = Hkv;
+        p.Sq = Sq;
+        p.Sk = Sk;
+        p.D = D;
+        p.G = Hq / Hkv;
+        p.causal = causal ? 1 : 0;
+        p.scale = scale;
+        p.total_rows = varlen ? Sk : 0;
+        p.n_rows = varlen ? (long long)Sk * Hq : (long long)B * Sq * Hq;
+        const long long blocks = (p.n_rows + 3) / 4;
+        if (blocks > INT32_MAX) return GQA_ERR_SHAPE;
+        gqa::attn_fwd_f32_simt<<<unsigned(blocks), 128, 0, stream>>>(p);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
+
+    Plan pl;
+    make_plan(&pl, B, Hq, Hkv, Sq, Sk, num_splits, pack_gqa, varlen, dev->sms);
+    switch (pl.kernel) {
+        case kNone:
+            return GQA_OK;
+        case kZeroFill:
+            gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
+                static_cast<__nv_bfloat16*>(out), (long long)B * Sq * Hq * D, lse,
+                (long long)B * Hq * Sq);
+            return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+        case kDecode:
+            return D == 128 ? launch_decode<128>(q, k, v, out, lse, B, Hq, Hkv, Sk, scale, pl,
+                                                 stream)
+                            : launch_decode<64>(q, k, v, out, lse, B, Hq, Hkv, Sk, scale, pl,
+                                                stream);
+        default:
+            return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale,
+                                                  causal, pl.pack, cu, dev->sms, stream)
+                            : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale,
+                                                 causal, pl.pack, cu, dev->sms, stream);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                 int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                 int num_splits, int pack_gqa, const int* cu_seqlens, cudaStream_t stream) {
+    return fwd_common(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
+                      pack_gqa, cu_seqlens, stream, false);
+}
+
+int gqa_attn_fwd_f32(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                     int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                     int num_splits, int pack_gqa, const int* cu_seqlens, cudaStream_t stream) {
+    return fwd_common(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
+                      pack_gqa, cu_seqlens, stream, true);
+}
+
+size_t gqa_attn_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits) {
+    if (B <= 0 || Hq <= 0 || Sq <= 0 || D <= 0 || num_splits <= 1) return 0;
+    return ws_bytes(B, Hq, Sq, D, num_splits);
+}
+
+int gqa_attn_set_workspace(void* dev_ptr, size_t bytes) {
+    if (dev_ptr && !aligned(dev_ptr, 16)) return GQA_ERR_ALIGN;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_ws.ptr = bytes ? dev_ptr : nullptr;
+    g_ws.bytes = dev_ptr ? bytes : 0;
+    return GQA_OK;
+}
+
+int gqa_attn_plan(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                  int num_splits, int pack_gqa, int varlen, int* kernel, int* splits, int* pack) {
+    (void)causal;
+    int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, num_splits, pack_gqa, varlen != 0, false);
+    if (rc != GQA_OK) return rc;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    const int sms = (dev && dev->sms > 0) ? dev->sms : 148;
+    Plan pl;
+    make_plan(&pl, B, Hq, Hkv, Sq, Sk, num_splits, pack_gqa, varlen != 0, sms);
+    if (kernel) *kernel = pl.kernel;
+    if (splits) *splits = pl.splits;
+    if (pack) *pack = pl.pack;
+    return rc;
+}
+
+int gqa_attn_get_device_error(int* host_code, cudaStream_t stream) {
+    if (!host_code) return GQA_ERR_NULL;
+    int code = 0;
+    if (cudaMemcpyFromSymbolAsync(&code, gqa::g_device_error, sizeof(int), 0,
+                                  cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GQA_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(gqa::g_device_error, &zero, sizeof(int), 0,
+                                cudaMemcpyHostToDevice, stream) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GQA_ERR_CUDA;
+    *host_code = code;
+    return GQA_OK;
+}
+
+const char* gqa_attn_strerror(int code) {
+    switch (code) {
+        case GQA_OK: return "success";
+        case GQA_ERR_NULL: return "a required pointer is NULL";
+        case GQA_ERR_SHAPE: return "invalid shape (negative size, Hq % Hkv != 0, or varlen Sq != Sk)";
+        case GQA_ERR_HEADDIM: return "unsupported head dimension";
+        case GQA_ERR_ALIGN: return "pointer not aligned (tensors 16 bytes, lse 4 bytes)";
+        case GQA_ERR_SPLITS: return "invalid num_splits for this shape";
+        case GQA_ERR_WORKSPACE: return "split-KV workspace missing or too small";
+        case GQA_ERR_SCALE: return "scale must be finite and positive";
+        case GQA_ERR_CUDA: return "CUDA runtime or launch failure";
+        case GQA_ERR_UNSUPPORTED: return "unsupported device or pack_gqa value";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,488 @@
+// Prefill forward of exact grouped-query attention on sm_100a.
+//
+// What it computes: O = softmax(scale * Q K^T [+ causal mask]) V per query head,
+// with the per-row log-sum-exp L written out (FlashAttention-2 summary page:
+// tiled online softmax, deferred 1/l normalisation, L = m + log l; causal
+// paragraph: blocks above the diagonal skipped, the mask applied only where the
+// diagonal crosses a block).  Query head h reads key/value head h / G
+// (Ultralytics GQA glossary, "How GQA works").
+//
+// Work unit ("CTA tile"): 256 query rows that share one key/value head, split
+// in two sub-tiles of 128 rows that ping-pong on the tensor core:
+//   pack_gqa = 1: rows are (position, head) pairs, 128/G positions x the G query
+//                 heads of one KV head per sub-tile, so K/V are streamed once
+//                 for the whole group (GQA batch-size guide, PackGQA items 1-3);
+//   pack_gqa = 0: rows are 128 consecutive positions of one query head.
+// Work units are spread over a persistent grid, longest first for causal and
+// variable-length batches (sequence-dimension parallelism, FlashAttention-2
+// summary page; attention balancing, Raptor-T abstract).
+//
+// Roles inside the CTA (320 threads):
+//   warps 0-3  softmax for sub-tile 0 (one thread = one row = one TMEM lane)
+//   warps 4-7  softmax for sub-tile 1
+//   warp 8     tcgen05.mma issuer (one thread), owns the TMEM allocation
+//   warp 9     TMA producer (one thread): Q once per tile, K/V blocks in a ring
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D)
+// O1 [256+D, 256+2D); P_i (bf16, 64 columns) overwrites the first half of S_i
+// after the softmax has read S_i into registers.
+//
+// Online softmax in the log2 domain: s2 = s * scale * log2(e).  The running
+// max used for the exponentials is only raised when a block's max exceeds it by
+// more than 8 (a factor 256), so O is rescaled rarely; since O and l always
+// share the same reference max, O / l and L = m + log l are unchanged.
+#pragma once
+#include "sm100_ptx.cuh"
+
+namespace gqa {
+
+struct PrefillParams {
+    __nv_bfloat16* out;      // [rows, Hq, D]
+    float* lse;              // [B, Hq, Sq] or [Hq, total]
+    const int* cu_seqlens;   // device int32[B+1] or nullptr
+    int B, Hq, Hkv, Sq, Sk;  // varlen: Sq = maximum sequence length, Sk = total_rows
+    int total_rows;          // varlen: packed rows of q, k, v (cu_seqlens[B])
+    int G;
+    int pack;
+    int sub_pos;             // positions per 128-row sub-tile: 128 / G (pack) or 128
+    int n_mblk;              // CTA tiles along the positions of the longest sequence
+    int n_hu;                // head units: Hkv (pack) or Hq
+    int n_units;             // n_mblk * B * n_hu
+    int causal;
+    float scale_log2;        // scale * log2(e)
+};
+
+template <int HD>
+struct PrefillCfg {
+    static constexpr int BM = 128;                // rows per sub-tile
+    static constexpr int BN = 128;                // keys per K/V block
+    static constexpr int ATOMS = HD / 64;         // 128-byte swizzle atoms along D
+    static constexpr int ATOM_Q = BM * 128;       // bytes of one Q atom
+    static constexpr int ATOM_KV = BN * 128;      // bytes of one K or V atom
+    static constexpr int Q_SUB = BM * HD * 2;     // bytes of one Q sub-tile
+    static constexpr int KV_TILE = BN * HD * 2;   // bytes of one K or V block
+    static constexpr int STAGES = (HD == 128) ? 2 : 4;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + 2 * Q_SUB;
+    static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
+    static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
+    static constexpr int NUM_BARS = 2 + 4 * STAGES + 6 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int THREADS = 320;
+    __device__ static constexpr uint32_t s_col(int i) { return uint32_t(i) * 128u; }
+    __device__ static constexpr uint32_t o_col(int i) { return 256u + uint32_t(i) * HD; }
+    static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+};
+
+struct TileInfo {
+    int b, hu, m;
+    int q_row0, k_row0;   // first row of this sequence in the [rows, H, D] views
+    int sq, sk;           // lengths of this sequence
+    int p0[2];            // first position of each sub-tile
+    int nblk[2];          // K/V blocks each sub-tile visits (0: nothing to compute)
+    int valid[2];         // sub-tile holds at least one real query row
+    int full_blk[2];      // blocks [0, full_blk) need no mask for any row
+};
+
+template <int BN>
+__device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
+    TileInfo ti;
+    const int per_m = p.B * p.n_hu;
+    ti.m = p.n_mblk - 1 - t / per_m;
+    const int r = t - (t / per_m) * per_m;
+    ti.b = r / p.n_hu;
+    ti.hu = r - ti.b * p.n_hu;
+    if (p.cu_seqlens) {
+        const int a = __ldg(p.cu_seqlens + ti.b), e = __ldg(p.cu_seqlens + ti.b + 1);
+        ti.q_row0 = ti.k_row0 = a;
+        ti.sq = ti.sk = e - a;
+    } else {
+        ti.q_row0 = ti.b * p.Sq;
+        ti.k_row0 = ti.b * p.Sk;
+        ti.sq = p.Sq;
+        ti.sk = p.Sk;
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int p0 = ti.m * 2 * p.sub_pos + i * p.sub_pos;
+        ti.p0[i] = p0;
+        ti.valid[i] = p0 < ti.sq;
+        const int last = min(p0 + p.sub_pos - 1, ti.sq - 1);
+        int lim = p.causal ? min(ti.sk, last + ti.sk - ti.sq + 1) : ti.sk;
+        ti.nblk[i] = (ti.valid[i] && lim > 0) ? (lim + BN - 1) / BN : 0;
+        int first_lim = p.causal ? min(ti.sk, p0 + ti.sk - ti.sq + 1) : ti.sk;
+        ti.full_blk[i] = first_lim > 0 ? first_lim / BN : 0;
+    }
+    return ti;
+}
+
+// Wait that ignores the abort flag (used to drain in-flight copies before exit).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            raise_device_error(kDevWaitTimeout);
+            return;
+        }
+    }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(320, 1)
+    prefill_fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+    using C = PrefillCfg<HD>;
+    constexpr int BN = C::BN;
+    constexpr int ST = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* bar_q_full = bars + 0;
+    uint64_t* bar_q_empty = bars + 1;
+    uint64_t* bar_k_full = bars + 2;
+    uint64_t* bar_k_empty = bar_k_full + ST;
+    uint64_t* bar_v_full = bar_k_empty + ST;
+    uint64_t* bar_v_empty = bar_v_full + ST;
+    uint64_t* bar_s_full = bar_v_empty + ST;  // [2]
+    uint64_t* bar_p_full = bar_s_full + 2;    // [2]
+    uint64_t* bar_o_full = bar_p_full + 2;    // [2]
+    uint64_t* bar_drain = bar_o_full + 2;     // MMA completion before exit
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_empty, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(bar_k_full + s, 1);
+            mbar_init(bar_k_empty + s, 1);
+            mbar_init(bar_v_full + s, 1);
+            mbar_init(bar_v_empty + s, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_s_full + i, 1);
+            mbar_init(bar_p_full + i, 128);
+            mbar_init(bar_o_full + i, 1);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            uint8_t* sQ = smem + C::OFF_Q;
+            uint8_t* sK = smem + C::OFF_K;
+            uint8_t* sV = smem + C::OFF_V;
+            int qc = 0, kc = 0, vc = 0;
+            for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
+                const TileInfo ti = decode_tile<BN>(p, t);
+                const int n = max(ti.nblk[0], ti.nblk[1]);
+                if (n == 0) continue;
+                if (!mbar_wait(bar_q_empty, (qc & 1) ^ 1, abort_flag)) goto producer_done;
+                mbar_arrive_expect_tx(bar_q_full,
+                                      uint32_t(((ti.nblk[0] > 0) + (ti.nblk[1] > 0)) * C::Q_SUB));
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (ti.nblk[i] == 0) continue;
+                    const int y = p.pack ? ti.hu * p.G : ti.hu;
+                    const int z = ti.q_row0 + ti.p0[i];
+#pragma unroll
+                    for (int a = 0; a < C::ATOMS; ++a)
+                        tma_load_3d(sQ + i * C::Q_SUB + a * C::ATOM_Q, &tm_q, bar_q_full, a * 64,
+                                    y, z);
+                }
+                ++qc;
+                const int kvh = p.pack ? ti.hu : ti.hu / p.G;
+                for (int j = 0; j < n; ++j) {
+                    const int z = ti.k_row0 + j * BN;
+                    {
+                        const int s = kc % ST;
+                        if (!mbar_wait(bar_k_empty + s, ((kc / ST) & 1) ^ 1, abort_flag))
+                            goto producer_done;
+                        mbar_arrive_expect_tx(bar_k_full + s, C::KV_TILE);
+#pragma unroll
+                        for (int a = 0; a < C::ATOMS; ++a)
+                            tma_load_3d(sK + s * C::KV_TILE + a * C::ATOM_KV, &tm_k,
+                                        bar_k_full + s, a * 64, kvh, z);
+                        ++kc;
+                    }
+                    {
+                        const int s = vc % ST;
+                        if (!mbar_wait(bar_v_empty + s, ((vc / ST) & 1) ^ 1, abort_flag))
+                            goto producer_done;
+                        mbar_arrive_expect_tx(bar_v_full + s, C::KV_TILE);
+#pragma unroll
+                        for (int a = 0; a < C::ATOMS; ++a)
+                            tma_load_3d(sV + s * C::KV_TILE + a * C::ATOM_KV, &tm_v,
+                                        bar_v_full + s, a * 64, kvh, z);
+                        ++vc;
+                    }
+                }
+            }
+        producer_done:
+            // Every copy this thread issued has landed before the CTA may exit.
+            if (qc > 0) drain_wait(bar_q_full, (qc - 1) & 1);
+            for (int s = 0; s < ST; ++s) {
+                const int uk = kc / ST + (s < kc % ST ? 1 : 0);  // loads issued into stage s
+                if (uk > 0) drain_wait(bar_k_full + s, (uk - 1) & 1);
+                const int uv = vc / ST + (s < vc % ST ? 1 : 0);
+                if (uv > 0) drain_wait(bar_v_full + s, (uv - 1) & 1);
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, 0, 0);
+            constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, 0, 1);
+            const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+            const uint32_t sK = smem_u32(smem + C::OFF_K);
+            const uint32_t sV = smem_u32(smem + C::OFF_V);
+            int qc = 0, kc = 0, vc = 0;
+            uint32_t p_phase[2] = {0, 0};
+            auto issue_s = [&](int i, int stage) {
+                const uint32_t qa = sQ + i * C::Q_SUB;
+                const uint32_t ka = sK + stage * C::KV_TILE;
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::ATOM_Q + (kk & 3) * 32;
+                    const uint32_t offk = (kk >> 2) * C::ATOM_KV + (kk & 3) * 32;
+                    umma_ss(tmem + C::s_col(i), sw128_desc(qa + off, 16, 1024),
+                            sw128_desc(ka + offk, 16, 1024), idesc_s, kk > 0);
+                }
+            };
+            auto issue_pv = [&](int i, int stage, bool accumulate) {
+                const uint32_t va = sV + stage * C::KV_TILE;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_ts(tmem + C::o_col(i), tmem + C::s_col(i) + kk * 8,
+                            sw128_desc(va + kk * 16 * 128, C::ATOM_KV, 1024), idesc_o,
+                            (accumulate || kk > 0) ? 1u : 0u);
+            };
+            for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
+                const TileInfo ti = decode_tile<BN>(p, t);
+                const int n = max(ti.nblk[0], ti.nblk[1]);
+                if (n == 0) continue;
+                if (!mbar_wait(bar_q_full, qc & 1, abort_flag)) goto mma_done;
+                ++qc;
+                {
+                    const int s = kc % ST;
+                    if (!mbar_wait(bar_k_full + s, (kc / ST) & 1, abort_flag)) goto mma_done;
+                    tc_fence_after();
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        if (ti.nblk[i] > 0) {
+                            issue_s(i, s);
+                            umma_commit(bar_s_full + i);
+                        }
+                    umma_commit(bar_k_empty + s);
+                    ++kc;
+                }
+                for (int j = 0; j < n; ++j) {
+                    const int sv = vc % ST;
+                    if (!mbar_wait(bar_v_full + sv, (vc / ST) & 1, abort_flag)) goto mma_done;
+                    tc_fence_after();
+                    int sk_next = -1;
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        if (j >= ti.nblk[i]) continue;
+                        if (!mbar_wait(bar_p_full + i, p_phase[i], abort_flag)) goto mma_done;
+                        p_phase[i] ^= 1;
+                        tc_fence_after();
+                        issue_pv(i, sv, j > 0);
+                        if (j + 1 == ti.nblk[i]) umma_commit(bar_o_full + i);
+                        if (j + 1 < ti.nblk[i]) {
+                            if (sk_next < 0) {
+                                sk_next = kc % ST;
+                                if (!mbar_wait(bar_k_full + sk_next, (kc / ST) & 1, abort_flag))
+                                    goto mma_done;
+                                tc_fence_after();
+                            }
+                            issue_s(i, sk_next);
+                            umma_commit(bar_s_full + i);
+                        }
+                    }
+                    umma_commit(bar_v_empty + sv);
+                    ++vc;
+                    if (sk_next >= 0) {
+                        umma_commit(bar_k_empty + sk_next);
+                        ++kc;
+                    }
+                }
+                umma_commit(bar_q_empty);
+            }
+        mma_done:
+            // Wait until every MMA issued by this thread has completed.
+            umma_commit(bar_drain);
+            drain_wait(bar_drain, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warps
+        const int i = warp >> 2;                       // sub-tile
+        const int r = ((warp & 3) << 5) + lane;        // row within the sub-tile
+        const uint32_t lane_base = uint32_t((warp & 3) << 5) << 16;
+        const uint32_t tS = tmem + lane_base + C::s_col(i);
+        const uint32_t tO = tmem + lane_base + C::o_col(i);
+        const float sl2 = p.scale_log2;
+        uint32_t s_phase = 0, o_phase = 0;
+        for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
+            const TileInfo ti = decode_tile<BN>(p, t);
+            // this warp's sub-tile, selected without runtime array indexing
+            const int my_valid = i ? ti.valid[1] : ti.valid[0];
+            const int my_p0 = i ? ti.p0[1] : ti.p0[0];
+            const int nb = i ? ti.nblk[1] : ti.nblk[0];
+            const int my_full = i ? ti.full_blk[1] : ti.full_blk[0];
+            if (!my_valid) continue;
+            int pos, head;
+            if (p.pack) {
+                pos = my_p0 + r / p.G;
+                head = ti.hu * p.G + (r - (r / p.G) * p.G);
+            } else {
+                pos = my_p0 + r;
+                head = ti.hu;
+            }
+            const bool row_valid = pos < ti.sq;
+            if (p.cu_seqlens && r == 0 &&
+                (ti.sq > p.Sq || ti.q_row0 + ti.sq > p.total_rows))
+                raise_device_error(kDevBadTile);
+            int key_lim = p.causal ? pos + ti.sk - ti.sq + 1 : ti.sk;
+            key_lim = min(key_lim, ti.sk);
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int j = 0; j < nb; ++j) {
+                if (!mbar_wait_warp(bar_s_full + i, s_phase, abort_flag)) goto softmax_done;
+                s_phase ^= 1;
+                tc_fence_after();
+                uint32_t sr[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+                if (j >= my_full) {
+                    const int lim = key_lim - j * BN;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (c * 32 + e >= lim) sr[c][e] = __float_as_uint(-INFINITY);
+                }
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+                const float mb = mx * sl2;
+                float alpha = 1.f;
+                if (mb > m_run + C::RESCALE_THRESHOLD) {
+                    alpha = ex2_approx(m_run - mb);
+                    m_run = mb;
+                }
+                const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+                float lsum = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_use));
+                        const float p1 =
+                            ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_use));
+                        lsum += p0 + p1;
+                        pk[e] = pack_bf16x2(p0, p1);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sr[c >> 1][(c & 1) * 16 + e] = pk[e];
+                }
+                // P (bf16 pairs) into the first 64 columns of S
+                tmem_st32(tS, sr[0]);
+                tmem_st32(tS + 32, sr[1]);
+                l_run = l_run * alpha + lsum;
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                    for (int c = 0; c < HD / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + c * 32, o);
+                        tmem_ld_wait();
+                        reg_fence(o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tO + c * 32, o);
+                    }
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(bar_p_full + i);
+            }
+            // ---------------------------------------------------------- epilogue
+            {
+                const size_t row = size_t(ti.q_row0 + pos) * p.Hq + head;
+                if (nb > 0) {
+                    if (!mbar_wait_warp(bar_o_full + i, o_phase, abort_flag)) goto softmax_done;
+                    o_phase ^= 1;
+                    tc_fence_after();
+                }
+                const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+#pragma unroll 1
+                for (int c = 0; c < HD / 32; ++c) {
+                    uint32_t o[32];
+                    if (nb > 0) {
+                        tmem_ld32(tO + c * 32, o);
+                        tmem_ld_wait();
+                        reg_fence(o);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = 0u;
+                    }
+                    if (row_valid) {
+                        uint32_t w[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                               __uint_as_float(o[2 * e + 1]) * inv_l);
+                        uint4* dst = reinterpret_cast<uint4*>(p.out + row * HD + c * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    }
+                }
+                if (row_valid) {
+                    const float L = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f
+                                                  : -INFINITY;
+                    size_t li;
+                    if (p.cu_seqlens)
+                        li = size_t(head) * p.total_rows + ti.q_row0 + pos;
+                    else
+                        li = (size_t(ti.b) * p.Hq + head) * p.Sq + pos;
+                    p.lse[li] = L;
+                }
+            }
+        }
+    softmax_done:;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 8) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace gqa

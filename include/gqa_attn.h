@@ -1,0 +1,148 @@
+/*
+ * gqa_attn.h -- C ABI of the B200 (sm_100a) exact grouped-query attention forward.
+ *
+ * Operation (every entry point computes the same definition):
+ *   for each batch element (or packed sequence) b and query head h, with
+ *   G = Hq / Hkv and key/value head c = h / G,
+ *     S[i, j] = scale * sum_d q[b, i, h, d] * k[b, j, c, d]
+ *     S[i, j] = -inf where causal and j > i + (Sk - Sq)
+ *     O[b, i, h, :] = sum_j softmax_j(S[i, :]) v[b, j, c, :]
+ *     L[b, h, i]    = ln sum_j exp(S[i, j])
+ *   Sources: FlashAttention-2 summary page (azimuth.plus) -- standard attention
+ *   S = QK^T, P = softmax(S), O = PV; tiled online softmax with running max m
+ *   and sum l, deferred normalisation, L = m + log l; causal mask (entries above
+ *   the diagonal are -inf, the diagonal is kept).  Ultralytics glossary
+ *   "Grouped Query Attention (GQA)", section "How GQA works" -- groups of Hq/Hkv
+ *   query heads share one K/V head; Hkv = 1 is MQA and Hkv = Hq is MHA.
+ *   Interface shape: flash_attn_func(q, k, v, dropout_p, softmax_scale, causal)
+ *   on [batch, seq_len, num_heads, head_dim] tensors (StructBERT/FlashAttention
+ *   page, section 2.2) and flash_attn_func(q, k, v, pack_gqa=..., num_splits=...)
+ *   (GQA batch-size guide, "Dynamic parameter tuning").
+ *   Readings where the pages are silent: causal masks are bottom-right aligned
+ *   when Sq != Sk (a single decode query sees every key); a row with no visible
+ *   key gets O = 0 and L = -inf; L is the natural log of the scaled logits.
+ *
+ * Memory and layout:
+ *   All tensor pointers are DEVICE pointers owned by the caller; the library
+ *   never allocates, frees or synchronises.  Every call is enqueued on `stream`
+ *   and returns after the enqueue (stream-ordered, no host sync inside), so a
+ *   call may be captured in a CUDA graph once its workspace is registered.
+ *   Dense:  q, out [B, Sq, Hq, D]; k, v [B, Sk, Hkv, D]; lse [B, Hq, Sq] fp32;
+ *           all contiguous row-major.
+ *   Packed variable-length (cu_seqlens != NULL): q, out [total, Hq, D];
+ *           k, v [total, Hkv, D]; lse [Hq, total]; cu_seqlens is a device int32
+ *           array [B + 1], non-decreasing, cu_seqlens[0] = 0, cu_seqlens[B] =
+ *           total; sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of q,
+ *           k and v (self-attention: its query and key lengths are its length).
+ *           The caller passes Sq = the largest sequence length (an upper bound
+ *           is accepted) and Sk = total, the number of packed rows it allocated:
+ *           TMA descriptors are sized from it, so nothing past the buffers is
+ *           read.  A sequence longer than Sq, or cu_seqlens[B] > Sk, raises
+ *           device error 2 and the offending tiles are not trusted.
+ *   Tensor pointers must be 16-byte aligned (TMA), lse 4-byte aligned.
+ *
+ * Errors: every entry point returns a gqa_status (0 = success).  Argument errors
+ *   are detected on the host before anything is enqueued.  GQA_ERR_CUDA reports
+ *   a failed launch (cudaGetLastError).  Kernels never trap: a pipeline wait that
+ *   exceeds its time limit records a device error code and the kernel returns;
+ *   read it with gqa_attn_get_device_error().
+ */
+#ifndef GQA_ATTN_H
+#define GQA_ATTN_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GQA_OK = 0,
+    GQA_ERR_NULL = -1,        /* a required pointer is NULL */
+    GQA_ERR_SHAPE = -2,       /* negative sizes, Hq % Hkv != 0, index range overflow */
+    GQA_ERR_HEADDIM = -3,     /* D not supported (bf16: 64 or 128; fp32: 1..256) */
+    GQA_ERR_ALIGN = -4,       /* tensor pointer not 16-byte aligned (lse: 4-byte) */
+    GQA_ERR_SPLITS = -5,      /* num_splits < 0, > 256, or > 1 outside dense Sq == 1 */
+    GQA_ERR_WORKSPACE = -6,   /* num_splits > 1 and the registered workspace is too small */
+    GQA_ERR_SCALE = -7,       /* scale not finite or not > 0 */
+    GQA_ERR_CUDA = -8,        /* a CUDA runtime call or a launch failed */
+    GQA_ERR_UNSUPPORTED = -9  /* device is not sm_100, or pack_gqa not in {-1, 0, 1} */
+} gqa_status;
+
+/*
+ * bf16 forward (fp32 accumulation, bf16 output, fp32 lse).
+ *   q, k, v, out : bf16 tensors as described above
+ *   lse          : fp32 log-sum-exp per (b, h, query row)
+ *   B            : batch size, or number of packed sequences when cu_seqlens != NULL
+ *   Hq, Hkv      : query heads and key/value heads (Hq % Hkv == 0)
+ *   Sq, Sk       : query and key lengths (varlen: Sq = maximum length,
+ *                  Sk = total packed rows)
+ *   D            : head dimension, 64 or 128
+ *   scale        : softmax scale (finite, > 0); 1/sqrt(D) is the usual choice
+ *   causal       : nonzero for the causal mask
+ *   num_splits   : split-KV factor for decode (dense, Sq == 1): 1 = none,
+ *                  n > 1 = n contiguous key ranges combined by log-sum-exp
+ *                  (needs a workspace, see below), 0 = chosen by the library.
+ *                  Must be 0 or 1 for every other shape.
+ *   pack_gqa     : 1 = the G query heads of a KV head share one tile (K/V read
+ *                  once per group), 0 = one query head per tile, -1 = chosen by
+ *                  the library.  Changes speed only, never the definition.
+ *   cu_seqlens   : NULL (dense) or device int32[B + 1] (packed variable length)
+ *   stream       : CUDA stream the work is enqueued on
+ */
+int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                 int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                 int num_splits, int pack_gqa, const int* cu_seqlens, cudaStream_t stream);
+
+/*
+ * fp32 forward: same parameters and layouts with fp32 q, k, v and out, computed
+ * in fp32 on CUDA cores.  D may be 1..256; num_splits must be 0 or 1; pack_gqa
+ * is accepted and ignored.
+ */
+int gqa_attn_fwd_f32(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                     int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                     int num_splits, int pack_gqa, const int* cu_seqlens, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace gqa_attn_fwd needs for a split-KV decode with the
+ * given sizes and num_splits (0 when num_splits <= 1): fp32 partial outputs
+ * [B, Hq, Sq, n, D] and partial log-sum-exps [B, Hq, Sq, n].
+ */
+size_t gqa_attn_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits);
+
+/*
+ * Register a caller-owned device buffer as the split-KV workspace of this
+ * process (borrowed, never freed by the library; NULL/0 unregisters).  Calls
+ * that run concurrently on different streams must not share one workspace.
+ * Returns GQA_ERR_ALIGN if dev_ptr is not 16-byte aligned.
+ */
+int gqa_attn_set_workspace(void* dev_ptr, size_t bytes);
+
+/*
+ * The choices gqa_attn_fwd makes for these arguments, without launching:
+ *   *kernel = 0 nothing to do, 1 sm_100a tcgen05 prefill, 2 split-KV decode,
+ *             3 zero fill (no keys);
+ *   *splits and *pack = the effective num_splits and pack_gqa.
+ * Returns the status gqa_attn_fwd would return for the argument checks that do
+ * not need pointers (shape, head dim, splits, pack, scale, device).
+ */
+int gqa_attn_plan(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                  int num_splits, int pack_gqa, int varlen, int* kernel, int* splits,
+                  int* pack);
+
+/*
+ * Read and clear the device error word on `stream` (synchronises that stream).
+ * *host_code: 0 none, 1 a pipeline wait timed out, 2 a packed sequence is longer
+ * than the Sq that was passed.
+ */
+int gqa_attn_get_device_error(int* host_code, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char* gqa_attn_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H */

@@ -1,0 +1,52 @@
+"""Tolerances and comparison helpers for the GPU-versus-oracle parity tests.
+
+bf16 path (inputs bf16, fp32 accumulation, bf16 output): max |dO| <= 1e-2,
+mean |dO| <= 1e-3, max |dL| <= 1e-3 against the unrounded float64 oracle.  An
+output element whose reference magnitude is so large that one bf16 ulp exceeds
+1e-2 (|O| >= 2) may differ by up to that ulp instead: rounding to bf16 alone
+can use half of it.  fp32 path: max |dO| <= 1e-4, max |dL| <= 1e-4.
+Rows with no visible key must give exactly O = 0 and L = -inf.
+"""
+import numpy as np
+
+BF16_MAX_ABS = 1e-2
+BF16_MEAN_ABS = 1e-3
+BF16_MAX_LSE = 1e-3
+F32_MAX_ABS = 1e-4
+F32_MAX_LSE = 1e-4
+
+
+def bf16_ulp(x):
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 7)
+
+
+def to_np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def compare(o_gpu, lse_gpu, o_ref, lse_ref, *, f32=False):
+    """Assert the tolerances; returns a dict of the observed errors."""
+    o = to_np(o_gpu) if not isinstance(o_gpu, np.ndarray) else o_gpu.astype(np.float64)
+    lse = to_np(lse_gpu) if not isinstance(lse_gpu, np.ndarray) else lse_gpu.astype(np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    lse_ref = np.asarray(lse_ref, dtype=np.float64)
+    assert o.shape == o_ref.shape, (o.shape, o_ref.shape)
+    assert lse.shape == lse_ref.shape, (lse.shape, lse_ref.shape)
+    assert np.all(np.isfinite(o)), "non-finite output"
+    dead = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), dead), "rows without visible keys differ"
+    err = np.abs(o - o_ref)
+    lerr = np.abs(lse[~dead] - lse_ref[~dead]) if np.any(~dead) else np.zeros(1)
+    stats = {"max_abs": float(err.max(initial=0.0)), "mean_abs": float(err.mean()) if err.size else 0.0,
+             "max_lse": float(lerr.max(initial=0.0))}
+    if f32:
+        assert stats["max_abs"] <= F32_MAX_ABS, stats
+        assert stats["max_lse"] <= F32_MAX_LSE, stats
+        return stats
+    allowed = np.maximum(BF16_MAX_ABS, bf16_ulp(o_ref))
+    stats["n_ulp_allowance"] = int(np.count_nonzero(err > BF16_MAX_ABS))
+    assert np.all(err <= allowed), stats
+    assert stats["mean_abs"] <= BF16_MEAN_ABS, stats
+    assert stats["max_lse"] <= BF16_MAX_LSE, stats
+    return stats

@@ -1,0 +1,121 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, and rejects bad arguments with the documented status codes before it
+touches a GPU.  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_gqa_b200 as G
+from exact_attention_gqa_b200 import _capi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _capi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gqa_attn_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(_capi.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_library_needs_no_driver_to_load():
+    out = os.popen(f"ldd {_capi.LIB_PATH}").read()
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def test_status_codes_match_header(lib):
+    text = open(HEADER).read()
+    for name, val in re.findall(r"(GQA_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", text):
+        assert G.STATUS[int(val)] == name
+        assert lib.gqa_attn_strerror(int(val)) != b"unknown status"
+
+
+FAKE = ctypes.c_void_p(0x1000)  # never dereferenced: every case fails argument checks first
+
+
+def call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=8, Hkv=2, Sq=16, Sk=16,
+         D=64, scale=0.125, causal=1, splits=1, pack=-1, cu=None, f32=False):
+    fn = lib.gqa_attn_fwd_f32 if f32 else lib.gqa_attn_fwd
+    return fn(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, splits, pack, cu, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), "GQA_ERR_NULL"),
+    (dict(lse=None), "GQA_ERR_NULL"),
+    (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
+    (dict(B=-1), "GQA_ERR_SHAPE"),
+    (dict(Sk=-3), "GQA_ERR_SHAPE"),
+    (dict(Hkv=0), "GQA_ERR_SHAPE"),
+    (dict(D=96), "GQA_ERR_HEADDIM"),
+    (dict(D=256), "GQA_ERR_HEADDIM"),
+    (dict(D=300, f32=True), "GQA_ERR_HEADDIM"),
+    (dict(scale=0.0), "GQA_ERR_SCALE"),
+    (dict(scale=float("nan")), "GQA_ERR_SCALE"),
+    (dict(scale=float("inf")), "GQA_ERR_SCALE"),
+    (dict(splits=-1), "GQA_ERR_SPLITS"),
+    (dict(splits=257, Sq=1), "GQA_ERR_SPLITS"),
+    (dict(splits=4), "GQA_ERR_SPLITS"),                   # split-KV needs Sq == 1
+    (dict(splits=2, Sq=1, f32=True), "GQA_ERR_SPLITS"),
+    (dict(pack=2), "GQA_ERR_UNSUPPORTED"),
+    (dict(q=ctypes.c_void_p(0x1008)), "GQA_ERR_ALIGN"),
+    (dict(lse=ctypes.c_void_p(0x1002)), "GQA_ERR_ALIGN"),
+])
+def test_argument_errors(lib, kw, code):
+    assert G.STATUS[call(lib, **kw)] == code
+
+
+def test_empty_problems_are_successful_noops(lib):
+    assert call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert call(lib, Sq=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert call(lib, B=0, f32=True, q=None, k=None, v=None, out=None, lse=None) == 0
+    # packed batch with no rows at all
+    assert call(lib, Sk=0, Sq=5, cu=FAKE, q=None, k=None, v=None, out=None, lse=None) == 0
+
+
+def test_workspace_accounting(lib):
+    assert lib.gqa_attn_workspace_bytes(4, 32, 1, 128, 1) == 0
+    n = lib.gqa_attn_workspace_bytes(4, 32, 1, 128, 8)
+    rows = 4 * 32 * 8
+    assert n >= rows * 128 * 4 + rows * 4
+    assert lib.gqa_attn_set_workspace(ctypes.c_void_p(0x1004), 64) == G.STATUS_CODE["GQA_ERR_ALIGN"]
+    assert lib.gqa_attn_set_workspace(None, 0) == 0
+
+
+def test_plan_choices(lib):
+    # prefill: PackGQA when the group divides the 128-row tile
+    rc, kern, splits, pack = G.gqa_attn_plan(4, 32, 8, 8192, 8192, 128, causal=True)
+    assert (kern, splits, pack) == ("prefill_sm100", 1, 1)
+    rc, kern, splits, pack = G.gqa_attn_plan(1, 6, 2, 100, 100, 64, pack_gqa=1)
+    assert kern == "prefill_sm100" and pack == 0        # G = 3 cannot pack a 128-row tile
+    rc, kern, splits, pack = G.gqa_attn_plan(1, 32, 8, 1, 32768, 128, num_splits=8)
+    assert (kern, splits, pack) == ("decode_splitkv", 8, 1)
+    rc, kern, splits, pack = G.gqa_attn_plan(1, 32, 8, 1, 100, 128, num_splits=8)
+    assert kern == "decode_splitkv" and splits == 2     # clamped to the 64-key blocks
+    rc, kern, splits, pack = G.gqa_attn_plan(1, 32, 8, 1, 32768, 128, num_splits=0)
+    assert kern == "decode_splitkv" and 1 < splits <= 64
+    rc, kern, splits, pack = G.gqa_attn_plan(2, 8, 2, 5, 0, 64)
+    assert kern == "zero_fill"
+    rc, kern, splits, pack = G.gqa_attn_plan(0, 8, 2, 5, 7, 64)
+    assert kern == "none"
+
+
+def test_python_front_end_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        G.gqa_attn(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous())
