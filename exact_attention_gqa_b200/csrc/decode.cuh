@@ -49,7 +49,7 @@ struct DecodeCfg {
     static constexpr int OFF_V = STAGES * TILE;
     static constexpr int OFF_BAR = 2 * STAGES * TILE;
     static constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
-    static constexpr int MERGE_BYTES = 4 * 16 * (HD + 2) * 4;  // per-warp partials
+    static constexpr int MERGE_BYTES = 4 * 16 * (HD + 3) * 4;  // per-warp partials
     static constexpr int SMEM_BYTES =
         (OFF_MISC + 16 > MERGE_BYTES ? OFF_MISC + 16 : MERGE_BYTES) + 1024;
     static constexpr int THREADS = 160;
@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(160, 2)
     // per-warp online-softmax state: rows g = lane/4 and g + 8
     float m_run[2] = {-INFINITY, -INFINITY};
     float l_part[2] = {0.f, 0.f};
+    float l_rnd[2] = {0.f, 0.f};
     float o[KSTEPS * 2][4];
 #pragma unroll
     for (int t = 0; t < KSTEPS * 2; ++t)
@@ -244,14 +245,20 @@ __global__ void __launch_bounds__(160, 2)
                         const float mu = (m_run[hr] == -INFINITY) ? 0.f : m_run[hr];
                         pr[t][e] = ex2_approx(fmaf(sc[t][e], sl2, -mu));
                     }
-#pragma unroll
-                for (int hr = 0; hr < 2; ++hr)
-                    l_part[hr] = l_part[hr] * alpha[hr] + pr[0][2 * hr] + pr[0][2 * hr + 1] +
-                                 pr[1][2 * hr] + pr[1][2 * hr + 1];
                 pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
                 pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
                 pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
                 pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+                // two row sums: exact p (for L) and the bf16 weights the MMA consumes
+                // (for O / l); rows g: pa[0], pa[2]; rows g + 8: pa[1], pa[3]
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr)
+                    l_part[hr] = l_part[hr] * alpha[hr] + pr[0][2 * hr] + pr[0][2 * hr + 1] +
+                                 pr[1][2 * hr] + pr[1][2 * hr + 1];
+                l_rnd[0] = l_rnd[0] * alpha[0] + bf16_lo(pa[0]) + bf16_hi(pa[0]) +
+                           bf16_lo(pa[2]) + bf16_hi(pa[2]);
+                l_rnd[1] = l_rnd[1] * alpha[1] + bf16_lo(pa[1]) + bf16_hi(pa[1]) +
+                           bf16_lo(pa[3]) + bf16_hi(pa[3]);
             }
             if (alpha[0] != 1.f || alpha[1] != 1.f) {
 #pragma unroll
@@ -277,6 +284,8 @@ __global__ void __launch_bounds__(160, 2)
         for (int hr = 0; hr < 2; ++hr) {
             l_part[hr] += __shfl_xor_sync(0xffffffffu, l_part[hr], 1);
             l_part[hr] += __shfl_xor_sync(0xffffffffu, l_part[hr], 2);
+            l_rnd[hr] += __shfl_xor_sync(0xffffffffu, l_rnd[hr], 1);
+            l_rnd[hr] += __shfl_xor_sync(0xffffffffu, l_rnd[hr], 2);
         }
     }
     __syncthreads();  // every stage consumed, every copy landed: reuse smem for the merge
@@ -284,7 +293,8 @@ __global__ void __launch_bounds__(160, 2)
     // ---------------------------------------------------------------- merge warps
     float* mo = reinterpret_cast<float*>(smem);           // [4][16][HD]
     float* mm = mo + 4 * 16 * HD;                          // [4][16]
-    float* ml = mm + 4 * 16;                               // [4][16]
+    float* ml = mm + 4 * 16;                               // [4][16] exact sums
+    float* mr = ml + 4 * 16;                               // [4][16] bf16-weight sums
     if (warp < 4) {
         const int g = lane >> 2, qd = (lane & 3) * 2;
 #pragma unroll
@@ -301,6 +311,8 @@ __global__ void __launch_bounds__(160, 2)
             mm[warp * 16 + g + 8] = m_run[1];
             ml[warp * 16 + g] = l_part[0];
             ml[warp * 16 + g + 8] = l_part[1];
+            mr[warp * 16 + g] = l_rnd[0];
+            mr[warp * 16 + g + 8] = l_rnd[1];
         }
     }
     __syncthreads();
@@ -311,15 +323,16 @@ __global__ void __launch_bounds__(160, 2)
 #pragma unroll
         for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * 16 + r]);
         const float Mu = (M == -INFINITY) ? 0.f : M;
-        float acc = 0.f, l = 0.f;
+        float acc = 0.f, l = 0.f, lr = 0.f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             const float f = ex2_approx(mm[w * 16 + r] - Mu);
             acc += f * mo[(w * 16 + r) * HD + d];
             l += f * ml[w * 16 + r];
+            lr += f * mr[w * 16 + r];
         }
         const int h = h0 + r;
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
         const float L = (l > 0.f) ? (Mu + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         if (p.n_splits == 1) {
             p.out[(size_t(b) * p.Hq + h) * HD + d] = __float2bfloat16_rn(acc * inv_l);

@@ -278,7 +278,9 @@ int fwd_common(const void* q, const void* k, const void* v, void* out, float* ls
     int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, num_splits, pack_gqa, varlen, is_f32);
     if (rc != GQA_OK) return rc;
     if (B == 0 || Sq == 0 || (varlen && Sk == 0)) return GQA_OK;  // nothing to compute
-    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
+    // k and v are never read when there are no keys (dense Sk == 0)
+    const bool reads_kv = varlen || Sk > 0;
+    if (!q || !out || !lse || (reads_kv && (!k || !v))) return GQA_ERR_NULL;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
         !aligned(lse, 4) || (cu && !aligned(cu, 4)))
         return GQA_ERR_ALIGN;

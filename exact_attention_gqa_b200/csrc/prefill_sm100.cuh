@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(320, 1)
                 raise_device_error(kDevBadTile);
             int key_lim = p.causal ? pos + ti.sk - ti.sq + 1 : ti.sk;
             key_lim = min(key_lim, ti.sk);
-            float m_run = -INFINITY, l_run = 0.f;
+            float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
             for (int j = 0; j < nb; ++j) {
                 if (!mbar_wait_warp(bar_s_full + i, s_phase, abort_flag)) goto softmax_done;
                 s_phase ^= 1;
@@ -396,7 +396,7 @@ __global__ void __launch_bounds__(320, 1)
                     m_run = mb;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                float lsum = 0.f;
+                float lsum = 0.f, lrnd = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
@@ -405,8 +405,11 @@ __global__ void __launch_bounds__(320, 1)
                         const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_use));
                         const float p1 =
                             ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_use));
-                        lsum += p0 + p1;
                         pk[e] = pack_bf16x2(p0, p1);
+                        // two row sums: of the exact p (for L) and of the bf16 values
+                        // the P.V MMA consumes (for O / l, an exact convex combination)
+                        lsum += p0 + p1;
+                        lrnd += bf16_lo(pk[e]) + bf16_hi(pk[e]);
                     }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sr[c >> 1][(c & 1) * 16 + e] = pk[e];
@@ -415,6 +418,7 @@ __global__ void __launch_bounds__(320, 1)
                 tmem_st32(tS, sr[0]);
                 tmem_st32(tS + 32, sr[1]);
                 l_run = l_run * alpha + lsum;
+                l_rnd = l_rnd * alpha + lrnd;
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
                     for (int c = 0; c < HD / 32; ++c) {
@@ -440,7 +444,7 @@ __global__ void __launch_bounds__(320, 1)
                     o_phase ^= 1;
                     tc_fence_after();
                 }
-                const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+                const float inv_l = (l_rnd > 0.f) ? 1.f / l_rnd : 0.f;
 #pragma unroll 1
                 for (int c = 0; c < HD / 32; ++c) {
                     uint32_t o[32];

@@ -57,6 +57,8 @@ def call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=8, Hkv=2, S
 @pytest.mark.parametrize("kw,code", [
     (dict(q=None), "GQA_ERR_NULL"),
     (dict(lse=None), "GQA_ERR_NULL"),
+    (dict(k=None), "GQA_ERR_NULL"),
+    (dict(v=None, cu=FAKE), "GQA_ERR_NULL"),          # packed rows are always read
     (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
     (dict(B=-1), "GQA_ERR_SHAPE"),
     (dict(Sk=-3), "GQA_ERR_SHAPE"),
