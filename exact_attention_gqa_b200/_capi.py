@@ -19,6 +19,7 @@ EXPORTS = (
     "gqa_attn_plan",
     "gqa_attn_get_device_error",
     "gqa_attn_strerror",
+    "gqa_attn_decode_noalloc",
 )
 
 STATUS = {

@@ -341,6 +341,82 @@ int fwd_common(const void* q, const void* k, const void* v, void* out, float* ls
     }
 }
 
+// ---------------------------------------------------------------------------- no-alloc decode
+// Scratch for the allocation-free split-KV decode entry point below.  It lives in
+// the library image itself, so every GPU that loads the library holds these bytes
+// until the process exits; the entry point never asks anyone for memory.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GQA_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocScratch {
+    void* ptr = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoallocScratch g_noalloc[64];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array for the current device.  Host code cannot
+// use the array's name as an address (on the host it names a stand-in object), so
+// the address is asked from the runtime once per device, with that device current.
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc[dev].ptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GQA_ERR_CUDA;
+        g_noalloc[dev].ptr = p;
+    }
+    *out = g_noalloc[dev].ptr;
+    return GQA_OK;
+}
+
+template <int HD>
+int launch_decode_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                          int B, int Hq, int Hkv, int Sk, float scale, const Plan& pl,
+                          void* scratch, cudaStream_t stream) {
+    using C = DecodeCfg<HD>;
+    if (cudaFuncSetAttribute(gqa::decode_split_sm100<HD>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    DecodeParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sk = Sk;
+    p.G = Hq / Hkv;
+    p.rows = pl.decode_rows;
+    p.units_per_kv = pl.decode_units;
+    p.n_splits = pl.splits;
+    p.blocks_per_split = pl.blocks_per_split;
+    p.scale_log2 = scale * kLog2e;
+    p.part_o = nullptr;
+    p.part_l = nullptr;
+    if (pl.splits > 1) {
+        // same partial layout as the registered-workspace path: O parts, then L parts
+        const size_t o_bytes = size_t(B) * Hq * pl.splits * HD * 4;
+        p.part_o = static_cast<float*>(scratch);
+        p.part_l = reinterpret_cast<float*>(static_cast<char*>(scratch) +
+                                            ((o_bytes + 255) / 256) * 256);
+    }
+    CUtensorMap tk, tv;
+    const long long rows = (long long)B * Sk;
+    if (!make_map(&tk, k, rows, Hkv, HD, 1, C::BN) || !make_map(&tv, v, rows, Hkv, HD, 1, C::BN))
+        return GQA_ERR_CUDA;
+    dim3 grid(pl.splits, Hkv * pl.decode_units, B);
+    gqa::decode_split_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+    if (pl.splits > 1) {
+        const int rows_bh = B * Hq;
+        gqa::splitkv_combine<HD><<<(rows_bh + 3) / 4, 128, 0, stream>>>(
+            p.part_o, p.part_l, p.out, lse, rows_bh, pl.splits);
+        if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+    }
+    return GQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -418,6 +494,49 @@ const char* gqa_attn_strerror(int code) {
         case GQA_ERR_UNSUPPORTED: return "unsupported device or pack_gqa value";
         default: return "unknown status";
     }
+}
+
+
+// Split-KV decode that allocates nothing: its partial results go to the library's
+// static scratch array instead of a registered workspace.  See gqa_attn.h.
+int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* out,
+                            float* lse, int B, int Hq, int Hkv, int Sk, int D, float scale,
+                            int num_splits, int pack_gqa, cudaStream_t stream) {
+    int rc = check_shape(B, Hq, Hkv, 1, Sk, D, scale, num_splits, pack_gqa, false, false);
+    if (rc != GQA_OK) return rc;
+    if (B == 0) return GQA_OK;
+    const bool reads_kv = Sk > 0;
+    if (!q || !out || !lse || (reads_kv && (!k || !v))) return GQA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    if (Sk == 0) {
+        gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(out), (long long)B * Hq * D, lse, (long long)B * Hq);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
+    Plan pl;
+    make_plan(&pl, B, Hq, Hkv, 1, Sk, num_splits, pack_gqa, false, dev->sms);
+    if (num_splits == 0) {
+        // automatic choice: the largest split count, up to the planned one, whose
+        // partials fit the static scratch (one split needs none)
+        while (pl.splits > 1 && ws_bytes(B, Hq, 1, D, pl.splits) > GQA_NOALLOC_SCRATCH_BYTES) {
+            Plan smaller;
+            make_plan(&smaller, B, Hq, Hkv, 1, Sk, pl.splits - 1, pack_gqa, false, dev->sms);
+            pl = smaller;
+        }
+    }
+    if (ws_bytes(B, Hq, 1, D, pl.splits) > GQA_NOALLOC_SCRATCH_BYTES) return GQA_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc != GQA_OK) return rc;
+    return D == 128 ? launch_decode_noalloc<128>(q, k, v, out, lse, B, Hq, Hkv, Sk, scale, pl,
+                                                 scratch, stream)
+                    : launch_decode_noalloc<64>(q, k, v, out, lse, B, Hq, Hkv, Sk, scale, pl,
+                                                scratch, stream);
 }
 
 }  // extern "C"

@@ -138,6 +138,45 @@ int gqa_attn_plan(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, in
  */
 int gqa_attn_get_device_error(int* host_code, cudaStream_t stream);
 
+/*
+ * Split-KV decode that allocates nothing (no counterpart on the pages; it is an
+ * addition for callers that cannot obtain device memory at call time).
+ *
+ * Who needs it: code that runs where allocation is unavailable or forbidden --
+ * a plugin or custom op handed only its input and output buffers by a host
+ * engine that owns all memory, a real-time loop whose latency budget cannot absorb
+ * cudaMalloc (which may synchronise the device), or a caller with no allocator of
+ * its own.  gqa_attn_fwd's split-KV path needs a workspace registered beforehand;
+ * this entry point needs none: its partial results go to a scratch array of
+ * GQA_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads
+ * the library keeps for the life of the process.
+ *
+ * Computes exactly what gqa_attn_fwd computes for a dense decode step (Sq = 1,
+ * causal or not: one query sees every key) with the same q [B,1,Hq,D], k/v
+ * [B,Sk,Hkv,D], out and lse [B,Hq,1] layouts, bf16 in/out, D 64 or 128, and the
+ * same num_splits (0 = automatic, reduced until the partials fit the scratch) and
+ * pack_gqa meanings.  Nothing is allocated, freed or synchronised: no cudaMalloc,
+ * no cudaFree, no allocating library call.
+ *
+ * Limits and sharing:
+ *   - B * Hq * num_splits * (D + 1) * 4 bytes (plus alignment) must fit in
+ *     GQA_NOALLOC_SCRATCH_BYTES; an explicit num_splits that does not fit returns
+ *     GQA_ERR_WORKSPACE and launches nothing;
+ *   - every call in the process shares the one array per device and leaves its
+ *     partials there; the next call overwrites them (each partial is written
+ *     before it is read within a call, so nothing needs clearing), but calls that
+ *     overlap on the GPU (different streams, or concurrent host threads) race on
+ *     it and must be serialised by the caller;
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ * Returns the same status codes as gqa_attn_fwd.
+ */
+#define GQA_NOALLOC_SCRATCH_BYTES (4u << 20)
+int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* out,
+                            float* lse, int B, int Hq, int Hkv, int Sk, int D, float scale,
+                            int num_splits, int pack_gqa, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char* gqa_attn_strerror(int code);
 
