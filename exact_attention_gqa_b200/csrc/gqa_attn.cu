@@ -202,6 +202,9 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     if (units > INT32_MAX) return GQA_ERR_SHAPE;
     p.n_units = int(units);
     p.causal = causal ? 1 : 0;
+    // dense non-causal: a (batch, head unit)'s position tiles back to back so its K/V
+    // stay in L2; causal and packed batches: longest tiles first
+    p.kv_major = (!causal && !cu) ? 1 : 0;
     p.scale_log2 = scale * kLog2e;
     // Row extents of the 3-D views: exactly the rows the caller allocated
     // (packed variable length: Sk carries the packed row count).

@@ -13,15 +13,19 @@
 //                 heads of one KV head per sub-tile, so K/V are streamed once
 //                 for the whole group (GQA batch-size guide, PackGQA items 1-3);
 //   pack_gqa = 0: rows are 128 consecutive positions of one query head.
-// Work units are spread over a persistent grid, longest first for causal and
-// variable-length batches (sequence-dimension parallelism, FlashAttention-2
-// summary page; attention balancing, Raptor-T abstract).
+// Work units are spread over a persistent grid (sequence-dimension parallelism,
+// FlashAttention-2 summary page).  Causal and variable-length batches run the
+// longest units first (attention balancing, Raptor-T abstract); dense
+// non-causal batches run the position tiles of one (batch, KV head) back to back
+// so that its K and V are re-read from L2 rather than HBM.
 //
 // Roles inside the CTA (320 threads):
 //   warps 0-3  softmax for sub-tile 0 (one thread = one row = one TMEM lane)
 //   warps 4-7  softmax for sub-tile 1
 //   warp 8     tcgen05.mma issuer (one thread), owns the TMEM allocation
-//   warp 9     TMA producer (one thread): Q once per tile, K/V blocks in a ring
+//   warp 9     TMA producer (one thread): Q once per tile (double-buffered when it
+//              fits, so the next tile's Q lands while this one computes), K/V
+//              blocks in a ring
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D)
 // O1 [256+D, 256+2D); P_i (bf16, 64 columns) overwrites the first half of S_i
 // after the softmax has read S_i into registers.
@@ -29,7 +33,9 @@
 // Online softmax in the log2 domain: s2 = s * scale * log2(e).  The running
 // max used for the exponentials is only raised when a block's max exceeds it by
 // more than 8 (a factor 256), so O is rescaled rarely; since O and l always
-// share the same reference max, O / l and L = m + log l are unchanged.
+// share the same reference max, O / l and L = m + log l are unchanged.  The
+// per-element work uses sm_100's paired fp32 instructions (fma/add .f32x2) and
+// three-input max to halve its issue slots.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -48,6 +54,7 @@ struct PrefillParams {
     int n_hu;                // head units: Hkv (pack) or Hq
     int n_units;             // n_mblk * B * n_hu
     int causal;
+    int kv_major;            // 1: tiles of one (batch, head unit) consecutive (L2 reuse)
     float scale_log2;        // scale * log2(e)
 };
 
@@ -59,19 +66,26 @@ struct PrefillCfg {
     static constexpr int ATOM_Q = BM * 128;       // bytes of one Q atom
     static constexpr int ATOM_KV = BN * 128;      // bytes of one K or V atom
     static constexpr int Q_SUB = BM * HD * 2;     // bytes of one Q sub-tile
+    static constexpr int Q_TILE = 2 * Q_SUB;      // both sub-tiles
     static constexpr int KV_TILE = BN * HD * 2;   // bytes of one K or V block
     static constexpr int STAGES = (HD == 128) ? 2 : 4;
+    static constexpr int Q_STAGES = (HD == 128) ? 1 : 2;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + 2 * Q_SUB;
+    static constexpr int OFF_K = OFF_Q + Q_STAGES * Q_TILE;
     static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
     static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
-    static constexpr int NUM_BARS = 2 + 4 * STAGES + 6 + 1;
+    static constexpr int NUM_BARS = 2 * Q_STAGES + 4 * STAGES + 6 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
     static constexpr int TMEM_COLS = 512;
     static constexpr int THREADS = 320;
     __device__ static constexpr uint32_t s_col(int i) { return uint32_t(i) * 128u; }
     __device__ static constexpr uint32_t o_col(int i) { return 256u + uint32_t(i) * HD; }
+    // P (bf16, 64 columns): its own columns when they fit (D = 64), else over S
+    static constexpr bool P_OWN = (HD == 64);
+    __device__ static constexpr uint32_t p_col(int i) {
+        return P_OWN ? 384u + uint32_t(i) * 64u : s_col(i);
+    }
     static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 };
 
@@ -88,11 +102,18 @@ struct TileInfo {
 template <int BN>
 __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
     TileInfo ti;
-    const int per_m = p.B * p.n_hu;
-    ti.m = p.n_mblk - 1 - t / per_m;
-    const int r = t - (t / per_m) * per_m;
-    ti.b = r / p.n_hu;
-    ti.hu = r - ti.b * p.n_hu;
+    if (p.kv_major) {
+        const int bh = t / p.n_mblk;
+        ti.m = t - bh * p.n_mblk;
+        ti.b = bh / p.n_hu;
+        ti.hu = bh - ti.b * p.n_hu;
+    } else {
+        const int per_m = p.B * p.n_hu;
+        ti.m = p.n_mblk - 1 - t / per_m;
+        const int r = t - (t / per_m) * per_m;
+        ti.b = r / p.n_hu;
+        ti.hu = r - ti.b * p.n_hu;
+    }
     if (p.cu_seqlens) {
         const int a = __ldg(p.cu_seqlens + ti.b), e = __ldg(p.cu_seqlens + ti.b + 1);
         ti.q_row0 = ti.k_row0 = a;
@@ -136,13 +157,14 @@ __global__ void __launch_bounds__(320, 1)
     using C = PrefillCfg<HD>;
     constexpr int BN = C::BN;
     constexpr int ST = C::STAGES;
+    constexpr int QS = C::Q_STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-    uint64_t* bar_q_full = bars + 0;
-    uint64_t* bar_q_empty = bars + 1;
-    uint64_t* bar_k_full = bars + 2;
+    uint64_t* bar_q_full = bars;                   // [QS]
+    uint64_t* bar_q_empty = bar_q_full + QS;       // [QS]
+    uint64_t* bar_k_full = bar_q_empty + QS;       // [ST]
     uint64_t* bar_k_empty = bar_k_full + ST;
     uint64_t* bar_v_full = bar_k_empty + ST;
     uint64_t* bar_v_empty = bar_v_full + ST;
@@ -150,6 +172,7 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* bar_p_full = bar_s_full + 2;    // [2]
     uint64_t* bar_o_full = bar_p_full + 2;    // [2]
     uint64_t* bar_drain = bar_o_full + 2;     // MMA completion before exit
+    uint64_t* bar_tok = bar_drain + 1;        // [2] exp-phase turn of each softmax group
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -157,8 +180,10 @@ __global__ void __launch_bounds__(320, 1)
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_q_full, 1);
-        mbar_init(bar_q_empty, 1);
+        for (int s = 0; s < QS; ++s) {
+            mbar_init(bar_q_full + s, 1);
+            mbar_init(bar_q_empty + s, 1);
+        }
         for (int s = 0; s < ST; ++s) {
             mbar_init(bar_k_full + s, 1);
             mbar_init(bar_k_empty + s, 1);
@@ -171,6 +196,8 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(bar_o_full + i, 1);
         }
         mbar_init(bar_drain, 1);
+        mbar_init(bar_tok + 0, 128);
+        mbar_init(bar_tok + 1, 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -197,8 +224,10 @@ __global__ void __launch_bounds__(320, 1)
                 const TileInfo ti = decode_tile<BN>(p, t);
                 const int n = max(ti.nblk[0], ti.nblk[1]);
                 if (n == 0) continue;
-                if (!mbar_wait(bar_q_empty, (qc & 1) ^ 1, abort_flag)) goto producer_done;
-                mbar_arrive_expect_tx(bar_q_full,
+                const int qs = qc % QS;
+                if (!mbar_wait(bar_q_empty + qs, ((qc / QS) & 1) ^ 1, abort_flag))
+                    goto producer_done;
+                mbar_arrive_expect_tx(bar_q_full + qs,
                                       uint32_t(((ti.nblk[0] > 0) + (ti.nblk[1] > 0)) * C::Q_SUB));
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
@@ -207,8 +236,8 @@ __global__ void __launch_bounds__(320, 1)
                     const int z = ti.q_row0 + ti.p0[i];
 #pragma unroll
                     for (int a = 0; a < C::ATOMS; ++a)
-                        tma_load_3d(sQ + i * C::Q_SUB + a * C::ATOM_Q, &tm_q, bar_q_full, a * 64,
-                                    y, z);
+                        tma_load_3d(sQ + qs * C::Q_TILE + i * C::Q_SUB + a * C::ATOM_Q, &tm_q,
+                                    bar_q_full + qs, a * 64, y, z);
                 }
                 ++qc;
                 const int kvh = p.pack ? ti.hu : ti.hu / p.G;
@@ -240,7 +269,10 @@ __global__ void __launch_bounds__(320, 1)
             }
         producer_done:
             // Every copy this thread issued has landed before the CTA may exit.
-            if (qc > 0) drain_wait(bar_q_full, (qc - 1) & 1);
+            for (int s = 0; s < QS; ++s) {
+                const int uq = qc / QS + (s < qc % QS ? 1 : 0);
+                if (uq > 0) drain_wait(bar_q_full + s, (uq - 1) & 1);
+            }
             for (int s = 0; s < ST; ++s) {
                 const int uk = kc / ST + (s < kc % ST ? 1 : 0);  // loads issued into stage s
                 if (uk > 0) drain_wait(bar_k_full + s, (uk - 1) & 1);
@@ -253,44 +285,47 @@ __global__ void __launch_bounds__(320, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, 0, 0);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, 0, 1);
-            const uint32_t sQ = smem_u32(smem + C::OFF_Q);
+            const uint32_t sQ0 = smem_u32(smem + C::OFF_Q);
             const uint32_t sK = smem_u32(smem + C::OFF_K);
             const uint32_t sV = smem_u32(smem + C::OFF_V);
             int qc = 0, kc = 0, vc = 0;
             uint32_t p_phase[2] = {0, 0};
-            auto issue_s = [&](int i, int stage) {
-                const uint32_t qa = sQ + i * C::Q_SUB;
-                const uint32_t ka = sK + stage * C::KV_TILE;
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::ATOM_Q + (kk & 3) * 32;
-                    const uint32_t offk = (kk >> 2) * C::ATOM_KV + (kk & 3) * 32;
-                    umma_ss(tmem + C::s_col(i), sw128_desc(qa + off, 16, 1024),
-                            sw128_desc(ka + offk, 16, 1024), idesc_s, kk > 0);
-                }
+            // Descriptors are built once and advanced by adding (byte offset >> 4) to
+            // the start-address field (no carry: shared addresses stay below 256 KB).
+            const uint64_t dq0 = sw128_desc(sQ0, 16, 1024);
+            const uint64_t dk0 = sw128_desc(sK, 16, 1024);
+            const uint64_t dv0 = sw128_desc(sV, C::ATOM_KV, 1024);
+            constexpr int NS = HD / 16;   // k-steps of S = Q K^T
+            constexpr int NPV = BN / 16;  // k-steps of O += P V
+            auto s_step = [&](uint64_t dq, uint64_t dk, int i, int kk) {
+                const uint32_t oq = ((kk >> 2) * C::ATOM_Q + (kk & 3) * 32) >> 4;
+                const uint32_t ok = ((kk >> 2) * C::ATOM_KV + (kk & 3) * 32) >> 4;
+                umma_ss(tmem + C::s_col(i), dq + oq, dk + ok, idesc_s, kk > 0 ? 1u : 0u);
             };
-            auto issue_pv = [&](int i, int stage, bool accumulate) {
-                const uint32_t va = sV + stage * C::KV_TILE;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_ts(tmem + C::o_col(i), tmem + C::s_col(i) + kk * 8,
-                            sw128_desc(va + kk * 16 * 128, C::ATOM_KV, 1024), idesc_o,
-                            (accumulate || kk > 0) ? 1u : 0u);
+            auto pv_step = [&](uint64_t dv, int i, int kk, bool accumulate) {
+                umma_ts(tmem + C::o_col(i), tmem + C::p_col(i) + kk * 8,
+                        dv + uint64_t((kk * 16 * 128) >> 4), idesc_o,
+                        (accumulate || kk > 0) ? 1u : 0u);
             };
             for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
                 const TileInfo ti = decode_tile<BN>(p, t);
                 const int n = max(ti.nblk[0], ti.nblk[1]);
                 if (n == 0) continue;
-                if (!mbar_wait(bar_q_full, qc & 1, abort_flag)) goto mma_done;
+                const int qs = qc % QS;
+                if (!mbar_wait(bar_q_full + qs, (qc / QS) & 1, abort_flag)) goto mma_done;
                 ++qc;
+                const uint64_t dq = dq0 + uint64_t((qs * C::Q_TILE) >> 4);
                 {
                     const int s = kc % ST;
                     if (!mbar_wait(bar_k_full + s, (kc / ST) & 1, abort_flag)) goto mma_done;
                     tc_fence_after();
+                    const uint64_t dk = dk0 + uint64_t((s * C::KV_TILE) >> 4);
 #pragma unroll
                     for (int i = 0; i < 2; ++i)
                         if (ti.nblk[i] > 0) {
-                            issue_s(i, s);
+                            const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
+#pragma unroll
+                            for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
                             umma_commit(bar_s_full + i);
                         }
                     umma_commit(bar_k_empty + s);
@@ -300,25 +335,44 @@ __global__ void __launch_bounds__(320, 1)
                     const int sv = vc % ST;
                     if (!mbar_wait(bar_v_full + sv, (vc / ST) & 1, abort_flag)) goto mma_done;
                     tc_fence_after();
+                    const uint64_t dv = dv0 + uint64_t((sv * C::KV_TILE) >> 4);
                     int sk_next = -1;
+                    uint64_t dk = 0;
 #pragma unroll
                     for (int i = 0; i < 2; ++i) {
                         if (j >= ti.nblk[i]) continue;
+                        const bool more = j + 1 < ti.nblk[i];
+                        if (more && sk_next < 0) {
+                            sk_next = kc % ST;
+                            if (!mbar_wait(bar_k_full + sk_next, (kc / ST) & 1, abort_flag))
+                                goto mma_done;
+                            dk = dk0 + uint64_t((sk_next * C::KV_TILE) >> 4);
+                        }
                         if (!mbar_wait(bar_p_full + i, p_phase[i], abort_flag)) goto mma_done;
                         p_phase[i] ^= 1;
                         tc_fence_after();
-                        issue_pv(i, sv, j > 0);
-                        if (j + 1 == ti.nblk[i]) umma_commit(bar_o_full + i);
-                        if (j + 1 < ti.nblk[i]) {
-                            if (sk_next < 0) {
-                                sk_next = kc % ST;
-                                if (!mbar_wait(bar_k_full + sk_next, (kc / ST) & 1, abort_flag))
-                                    goto mma_done;
-                                tc_fence_after();
+                        // O_i += P_i(j) V_j and S_i(j+1) = Q_i K_{j+1}^T accumulate into
+                        // different TMEM tiles.  When P has its own columns their k-steps
+                        // are interleaved, so neither chain of dependent accumulations
+                        // stalls the tensor pipe; when P overlays S, every P.V step must
+                        // be issued before S(j+1) overwrites those columns.
+                        const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
+                        if constexpr (C::P_OWN) {
+#pragma unroll
+                            for (int kk = 0; kk < (NPV > NS ? NPV : NS); ++kk) {
+                                if (kk < NPV) pv_step(dv, i, kk, j > 0);
+                                if (more && kk < NS) s_step(dqi, dk, i, kk);
                             }
-                            issue_s(i, sk_next);
-                            umma_commit(bar_s_full + i);
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
+                            if (more) {
+#pragma unroll
+                                for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                            }
                         }
+                        if (!more) umma_commit(bar_o_full + i);
+                        else umma_commit(bar_s_full + i);
                     }
                     umma_commit(bar_v_empty + sv);
                     ++vc;
@@ -327,7 +381,7 @@ __global__ void __launch_bounds__(320, 1)
                         ++kc;
                     }
                 }
-                umma_commit(bar_q_empty);
+                umma_commit(bar_q_empty + qs);
             }
         mma_done:
             // Wait until every MMA issued by this thread has completed.
@@ -341,8 +395,17 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t lane_base = uint32_t((warp & 3) << 5) << 16;
         const uint32_t tS = tmem + lane_base + C::s_col(i);
         const uint32_t tO = tmem + lane_base + C::o_col(i);
+        const uint32_t tP = tmem + lane_base + C::p_col(i);
         const float sl2 = p.scale_log2;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
         uint32_t s_phase = 0, o_phase = 0;
+        // The two groups take turns on the exponential phase (group 0 first), so
+        // that one group's exponentials overlap the MMAs of the other group instead
+        // of both sharing the exp unit and then both waiting for the tensor core.
+        // Every tile has max(n0, n1) turns for both groups, worked or passed.
+        uint32_t turns = 0;
+        uint64_t* tok_mine = bar_tok + i;
+        uint64_t* tok_other = bar_tok + (i ^ 1);
         for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN>(p, t);
             // this warp's sub-tile, selected without runtime array indexing
@@ -350,7 +413,15 @@ __global__ void __launch_bounds__(320, 1)
             const int my_p0 = i ? ti.p0[1] : ti.p0[0];
             const int nb = i ? ti.nblk[1] : ti.nblk[0];
             const int my_full = i ? ti.full_blk[1] : ti.full_blk[0];
-            if (!my_valid) continue;
+            const int nturn = max(ti.nblk[0], ti.nblk[1]);
+            if (!my_valid) {
+                for (int j = 0; j < nturn; ++j, ++turns) {
+                    if (!mbar_wait_warp(tok_mine, (turns & 1) ^ (i == 0 ? 1u : 0u), abort_flag))
+                        goto softmax_done;
+                    mbar_arrive(tok_other);
+                }
+                continue;
+            }
             int pos, head;
             if (p.pack) {
                 pos = my_p0 + r / p.G;
@@ -366,7 +437,13 @@ __global__ void __launch_bounds__(320, 1)
             int key_lim = p.causal ? pos + ti.sk - ti.sq + 1 : ti.sk;
             key_lim = min(key_lim, ti.sk);
             float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
-            for (int j = 0; j < nb; ++j) {
+            for (int j = 0; j < nturn; ++j, ++turns) {
+                if (j >= nb) {  // nothing of ours in this turn: pass it on
+                    if (!mbar_wait_warp(tok_mine, (turns & 1) ^ (i == 0 ? 1u : 0u), abort_flag))
+                        goto softmax_done;
+                    mbar_arrive(tok_other);
+                    continue;
+                }
                 if (!mbar_wait_warp(bar_s_full + i, s_phase, abort_flag)) goto softmax_done;
                 s_phase ^= 1;
                 tc_fence_after();
@@ -384,11 +461,21 @@ __global__ void __launch_bounds__(320, 1)
                         for (int e = 0; e < 32; ++e)
                             if (c * 32 + e >= lim) sr[c][e] = __float_as_uint(-INFINITY);
                 }
-                float mx = -INFINITY;
+                // block row max: four independent three-input max chains
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+                    for (int e = 0; e < 32; e += 8) {
+                        mx0 = fmax3(mx0, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
+                        mx1 = fmax3(mx1, __uint_as_float(sr[c][e + 2]),
+                                    __uint_as_float(sr[c][e + 3]));
+                        mx2 = fmax3(mx2, __uint_as_float(sr[c][e + 4]),
+                                    __uint_as_float(sr[c][e + 5]));
+                        mx3 = fmax3(mx3, __uint_as_float(sr[c][e + 6]),
+                                    __uint_as_float(sr[c][e + 7]));
+                    }
+                const float mx = fmax3(fmaxf(mx0, mx1), mx2, mx3);
                 const float mb = mx * sl2;
                 float alpha = 1.f;
                 if (mb > m_run + C::RESCALE_THRESHOLD) {
@@ -396,30 +483,55 @@ __global__ void __launch_bounds__(320, 1)
                     m_run = mb;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                float lsum = 0.f, lrnd = 0.f;
+                const uint64_t negm2 = f2_pack(-m_use, -m_use);
+                // our turn on the exponential unit
+                if (!mbar_wait_warp(tok_mine, (turns & 1) ^ (i == 0 ? 1u : 0u), abort_flag))
+                    goto softmax_done;
+                // p = 2^(s*scale*log2e - m); two row sums in paired fp32: of the exact p
+                // (for L) and of the bf16 p the P.V MMA consumes (for O / l)
+                uint64_t se0 = 0, se1 = 0, sq0 = 0, sq1 = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * e]), sl2, -m_use));
-                        const float p1 =
-                            ex2_approx(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, -m_use));
+                        const uint64_t a = ffma2(f2_pack(__uint_as_float(sr[c][2 * e]),
+                                                         __uint_as_float(sr[c][2 * e + 1])),
+                                                 sl2x2, negm2);
+                        float a0, a1;
+                        f2_unpack(a, a0, a1);
+                        const float p0 = ex2_approx(a0);
+                        const float p1 = ex2_approx(a1);
                         pk[e] = pack_bf16x2(p0, p1);
-                        // two row sums: of the exact p (for L) and of the bf16 values
-                        // the P.V MMA consumes (for O / l, an exact convex combination)
-                        lsum += p0 + p1;
-                        lrnd += bf16_lo(pk[e]) + bf16_hi(pk[e]);
+                        const uint64_t pe = f2_pack(p0, p1);
+                        const uint64_t pr = f2_pack(bf16_lo(pk[e]), bf16_hi(pk[e]));
+                        if (e & 1) {
+                            se1 = fadd2(se1, pe);
+                            sq1 = fadd2(sq1, pr);
+                        } else {
+                            se0 = fadd2(se0, pe);
+                            sq0 = fadd2(sq0, pr);
+                        }
                     }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sr[c >> 1][(c & 1) * 16 + e] = pk[e];
                 }
-                // P (bf16 pairs) into the first 64 columns of S
-                tmem_st32(tS, sr[0]);
-                tmem_st32(tS + 32, sr[1]);
+                mbar_arrive(tok_other);  // the other group's turn
+                // P (bf16 pairs): its own 64 columns, or the first 64 columns of S
+                tmem_st32(tP, sr[0]);
+                tmem_st32(tP + 32, sr[1]);
+                float lsum, lrnd;
+                {
+                    float x0, x1, y0, y1;
+                    f2_unpack(fadd2(se0, se1), x0, x1);
+                    f2_unpack(fadd2(sq0, sq1), y0, y1);
+                    lsum = x0 + x1;
+                    lrnd = y0 + y1;
+                }
                 l_run = l_run * alpha + lsum;
                 l_rnd = l_rnd * alpha + lrnd;
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    const uint64_t al2 = f2_pack(alpha, alpha);
 #pragma unroll 1
                     for (int c = 0; c < HD / 32; ++c) {
                         uint32_t o[32];
@@ -427,8 +539,15 @@ __global__ void __launch_bounds__(320, 1)
                         tmem_ld_wait();
                         reg_fence(o);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        for (int e = 0; e < 32; e += 2) {
+                            float u0, u1;
+                            f2_unpack(fmul2(f2_pack(__uint_as_float(o[e]),
+                                                    __uint_as_float(o[e + 1])),
+                                            al2),
+                                      u0, u1);
+                            o[e] = __float_as_uint(u0);
+                            o[e + 1] = __float_as_uint(u1);
+                        }
                         tmem_st32(tO + c * 32, o);
                     }
                 }
