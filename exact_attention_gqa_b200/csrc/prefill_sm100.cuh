@@ -358,11 +358,14 @@ __global__ void __launch_bounds__(320, 1)
                         // be issued before S(j+1) overwrites those columns.
                         const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
                         if constexpr (C::P_OWN) {
+                            // S(j+1) first: the softmax needs it next, P.V(j) only later
+                            if (more) {
 #pragma unroll
-                            for (int kk = 0; kk < (NPV > NS ? NPV : NS); ++kk) {
-                                if (kk < NPV) pv_step(dv, i, kk, j > 0);
-                                if (more && kk < NS) s_step(dqi, dk, i, kk);
+                                for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                umma_commit(bar_s_full + i);
                             }
+#pragma unroll
+                            for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
                         } else {
 #pragma unroll
                             for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(320, 1)
                             }
                         }
                         if (!more) umma_commit(bar_o_full + i);
-                        else umma_commit(bar_s_full + i);
+                        else if constexpr (!C::P_OWN) umma_commit(bar_s_full + i);
                     }
                     umma_commit(bar_v_empty + sv);
                     ++vc;
