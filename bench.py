@@ -479,6 +479,72 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def run_decode_sweep(args, local):
+    """Every decode cell: B x num_splits (1, 2, 4, 8, auto) x pack_gqa (1, 0); one line each."""
+    import exact_attention_gqa_b200 as G
+    from exact_attention_gqa_b200 import build
+    build.build()
+    device = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(device)
+    peaks, peak_kind = load_peaks()
+    batches = [int(b) for b in args.batches.split(",")] if args.batches else list(W.DECODE_BATCHES)
+    for B in batches:
+        base = W.decode(B)
+        kv_bytes = W.kv_cache_bytes(B, base.Sk, base.Hkv, base.D)
+        copies = 1 if kv_bytes > 2 * L2_BYTES else 3
+        q = W.make_decode_q(base, device=device)
+        kvs = []
+        for _ in range(copies):
+            k = torch.empty(B, base.Sk, base.Hkv, base.D, dtype=torch.bfloat16, device=device)
+            v = torch.empty_like(k)
+            W.fill_decode_kv(base, k, v)
+            kvs.append((k, v))
+        out = torch.empty_like(q)
+        lse = torch.empty(B, base.Hq, 1, dtype=torch.float32, device=device)
+        nbytes = W.decode_bytes(B, base.Hq, base.Hkv, base.Sk, base.D)
+        for splits in (1, 2, 4, 8, 0):
+            for pack in (1, 0):
+                rc, kern, eff_splits, eff_pack = G.gqa_attn_plan(B, base.Hq, base.Hkv, 1, base.Sk,
+                                                                 base.D, num_splits=splits,
+                                                                 pack_gqa=pack)
+                idx = [0]
+
+                def step():
+                    k, v = kvs[idx[0] % copies]
+                    idx[0] += 1
+                    G.gqa_attn(q, k, v, num_splits=splits, pack_gqa=pack, out=out, lse=lse)
+
+                for _ in range(max(args.warmup, 3)):
+                    step()
+                torch.cuda.synchronize()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                step()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                one = max(e0.elapsed_time(e1), 1e-3)
+                steps = int(max(10, min(5000, 150.0 / one)))
+                e0.record(stream)
+                for _ in range(steps):
+                    step()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / steps
+                gbs = nbytes / (ms * 1e-3) / 1e9
+                print(json.dumps({"metric": METRIC, "sweep": "decode", "B": B, "Sk": base.Sk,
+                                  "num_splits": splits, "pack_gqa": pack,
+                                  "effective_splits": eff_splits, "effective_pack": eff_pack,
+                                  "value": gbs, "unit": "GB/s", "ms_per_step": ms,
+                                  "steps": steps, "kv_copies_rotated": copies,
+                                  "frac_of_measured_copy": gbs / peaks["hbm_gbs"],
+                                  "peak_source": peak_kind,
+                                  "gpu_launches_per_step": 2 if eff_splits > 1 else 1}),
+                      flush=True)
+        del kvs, q, out, lse
+        torch.cuda.empty_cache()
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -488,8 +554,14 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sweep", choices=["decode"], default=None,
+                    help="print one line per decode cell instead of the bench line")
+    ap.add_argument("--batches", default="", help="decode sweep batch sizes (comma list)")
     args = ap.parse_args(argv)
     world, rank, local = dist_setup(args)
+    if args.sweep == "decode":
+        run_decode_sweep(args, local)
+        return
     if args.impl == "reference":
         if args.steps <= 0:
             args.steps = 3
