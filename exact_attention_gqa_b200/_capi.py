@@ -20,6 +20,7 @@ EXPORTS = (
     "gqa_attn_get_device_error",
     "gqa_attn_strerror",
     "gqa_attn_decode_noalloc",
+    "gqa_attn_selftest_timeout",
 )
 
 STATUS = {
@@ -62,6 +63,8 @@ def load() -> ctypes.CDLL:
     lib.gqa_attn_plan.restype = I
     lib.gqa_attn_get_device_error.argtypes = [IP, P]
     lib.gqa_attn_get_device_error.restype = I
+    lib.gqa_attn_selftest_timeout.argtypes = [I, P]
+    lib.gqa_attn_selftest_timeout.restype = I
     lib.gqa_attn_strerror.argtypes = [I]
     lib.gqa_attn_strerror.restype = ctypes.c_char_p
     _lib = lib

@@ -420,6 +420,22 @@ int launch_decode_noalloc(const void* q, const void* k, const void* v, void* out
     return GQA_OK;
 }
 
+// ---------------------------------------------------------------------------- self-test
+// One warp waits, with the kernels' own bounded wait, on an mbarrier that nothing
+// will ever complete; the wait gives up after limit_ns, records the timeout in
+// the device error word and the kernel returns normally.
+__global__ void selftest_wait_timeout(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        gqa::mbar_init(&bar, 1);
+        abort_flag = 0;
+        gqa::fence_mbar_init();
+    }
+    __syncthreads();
+    gqa::mbar_wait_limit(&bar, 0, &abort_flag, limit_ns);
+}
+
 }  // namespace
 
 extern "C" {
@@ -540,6 +556,16 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
                                                  scratch, stream)
                     : launch_decode_noalloc<64>(q, k, v, out, lse, B, Hq, Hkv, Sk, scale, pl,
                                                 scratch, stream);
+}
+
+
+int gqa_attn_selftest_timeout(int limit_ms, cudaStream_t stream) {
+    if (limit_ms < 1 || limit_ms > 1000) return GQA_ERR_SHAPE;
+    DeviceInfo* dev = nullptr;
+    const int rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    selftest_wait_timeout<<<1, 32, 0, stream>>>(uint64_t(limit_ms) * 1000000ull);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -177,6 +177,15 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
                             float* lse, int B, int Hq, int Hkv, int Sk, int D, float scale,
                             int num_splits, int pack_gqa, cudaStream_t stream);
 
+/*
+ * Diagnostic: exercises the kernels' bounded-wait path.  Launches one warp that
+ * waits, with the same bounded mbarrier wait the attention kernels use, on a
+ * barrier nothing completes; after limit_ms (1..1000) the wait gives up, records
+ * device error 1 (wait timed out) and the kernel returns, leaving the context
+ * usable.  Read the code with gqa_attn_get_device_error.  Nothing faults or traps.
+ */
+int gqa_attn_selftest_timeout(int limit_ms, cudaStream_t stream);
+
 /* Static description of a status code. */
 const char* gqa_attn_strerror(int code);
 
