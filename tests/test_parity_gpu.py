@@ -71,6 +71,35 @@ def test_prefill_large_logits():
     compare(out, lse, *oracle.attention(q, k, v, scale=1 / math.sqrt(128), causal=True))
 
 
+def rising_qkv(B, Hq, Hkv, Sq, Sk, D, seed, step_log2=10.0):
+    """Scores that rise block by block: every 128-key block's row max exceeds the
+    previous block's by about `step_log2` in log2 units, so the online softmax must
+    rescale its running output at every block (FlashAttention-2 summary page, online
+    softmax: earlier partial results are rescaled when the running max grows)."""
+    q, k, v = rand_qkv(B, Hq, Hkv, Sq, Sk, D, seed)
+    scale = 1.0 / math.sqrt(D)
+    step = step_log2 / (scale * 8.0 * math.log2(math.e))
+    q[..., 0] = 8.0
+    k[..., 0] = (torch.arange(Sk) // 128).to(torch.float32).mul(step).view(1, Sk, 1).to(k.dtype)
+    return q, k, v
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("pack", [1, 0])
+def test_prefill_rescales_at_every_block(D, causal, pack):
+    q, k, v = rising_qkv(2, 8, 2, 520, 1100, D, seed=31 + D)
+    out, lse = run(q, k, v, causal=causal, pack_gqa=pack)
+    compare(out, lse, *oracle.attention(q, k, v, scale=1 / math.sqrt(D), causal=causal))
+
+
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_decode_rescales_at_every_block(splits):
+    q, k, v = rising_qkv(3, 32, 8, 1, 4000, 128, seed=77)
+    out, lse = run(q, k, v, causal=False, num_splits=splits)
+    compare(out, lse, *oracle.attention(q, k, v, scale=1 / math.sqrt(128), causal=False))
+
+
 def test_pack_on_and_off_agree():
     q, k, v = rand_qkv(2, 16, 4, 333, 333, 128, seed=11)
     a, la = run(q, k, v, causal=True, pack_gqa=1)
