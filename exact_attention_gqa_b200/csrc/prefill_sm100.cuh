@@ -27,8 +27,10 @@
 //              fits, so the next tile's Q lands while this one computes), K/V
 //              blocks in a ring
 // Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D)
-// O1 [256+D, 256+2D); P_i (bf16, 64 columns) overwrites the first half of S_i
-// after the softmax has read S_i into registers.
+// O1 [256+D, 256+2D); P_i (bf16 pairs, 64 columns) has its own columns
+// [384+64i, 448+64i) when D = 64 and otherwise overwrites the first half of S_i
+// after the softmax has read S_i into registers.  The two sub-tiles run their
+// softmax independently; the tensor core alternates between them.
 //
 // Online softmax in the log2 domain: s2 = s * scale * log2(e).  The running
 // max used for the exponentials is only raised when a block's max exceeds it by
@@ -74,7 +76,7 @@ struct PrefillCfg {
     static constexpr int OFF_K = OFF_Q + Q_STAGES * Q_TILE;
     static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
     static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
-    static constexpr int NUM_BARS = 2 * Q_STAGES + 4 * STAGES + 6 + 1 + 2;
+    static constexpr int NUM_BARS = 2 * Q_STAGES + 4 * STAGES + 6 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
     static constexpr int TMEM_COLS = 512;
@@ -170,9 +172,8 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* bar_v_empty = bar_v_full + ST;
     uint64_t* bar_s_full = bar_v_empty + ST;  // [2]
     uint64_t* bar_p_full = bar_s_full + 2;    // [2]
-    uint64_t* bar_o_full = bar_p_full + 2;    // [2]
-    uint64_t* bar_drain = bar_o_full + 2;     // MMA completion before exit
-    uint64_t* bar_tok = bar_drain + 1;        // [2] exp-phase turn of each softmax group
+    uint64_t* bar_o_done = bar_p_full + 2;    // [2] O_i += P_i(j) V_j finished (every block)
+    uint64_t* bar_drain = bar_o_done + 2;     // MMA completion before exit
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -193,11 +194,9 @@ __global__ void __launch_bounds__(320, 1)
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_s_full + i, 1);
             mbar_init(bar_p_full + i, 128);
-            mbar_init(bar_o_full + i, 1);
+            mbar_init(bar_o_done + i, 1);
         }
         mbar_init(bar_drain, 1);
-        mbar_init(bar_tok + 0, 128);
-        mbar_init(bar_tok + 1, 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -351,11 +350,11 @@ __global__ void __launch_bounds__(320, 1)
                         if (!mbar_wait(bar_p_full + i, p_phase[i], abort_flag)) goto mma_done;
                         p_phase[i] ^= 1;
                         tc_fence_after();
-                        // O_i += P_i(j) V_j and S_i(j+1) = Q_i K_{j+1}^T accumulate into
-                        // different TMEM tiles.  When P has its own columns their k-steps
-                        // are interleaved, so neither chain of dependent accumulations
-                        // stalls the tensor pipe; when P overlays S, every P.V step must
-                        // be issued before S(j+1) overwrites those columns.
+                        // When P has its own columns (D = 64), S_i(j+1) = Q_i K_{j+1}^T is
+                        // issued before O_i += P_i(j) V_j, since the softmax needs it first;
+                        // when P overlays S, every P.V step must come before S(j+1)
+                        // overwrites those columns.  o_done_i is committed after every P.V:
+                        // the softmax waits for it before it writes P_i(j+1) or rescales O_i.
                         const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
                         if constexpr (C::P_OWN) {
                             // S(j+1) first: the softmax needs it next, P.V(j) only later
@@ -366,16 +365,17 @@ __global__ void __launch_bounds__(320, 1)
                             }
 #pragma unroll
                             for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
+                            umma_commit(bar_o_done + i);
                         } else {
 #pragma unroll
                             for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
+                            umma_commit(bar_o_done + i);
                             if (more) {
 #pragma unroll
                                 for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                umma_commit(bar_s_full + i);
                             }
                         }
-                        if (!more) umma_commit(bar_o_full + i);
-                        else if constexpr (!C::P_OWN) umma_commit(bar_s_full + i);
                     }
                     umma_commit(bar_v_empty + sv);
                     ++vc;
@@ -402,13 +402,6 @@ __global__ void __launch_bounds__(320, 1)
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
         uint32_t s_phase = 0, o_phase = 0;
-        // The two groups take turns on the exponential phase (group 0 first), so
-        // that one group's exponentials overlap the MMAs of the other group instead
-        // of both sharing the exp unit and then both waiting for the tensor core.
-        // Every tile has max(n0, n1) turns for both groups, worked or passed.
-        uint32_t turns = 0;
-        uint64_t* tok_mine = bar_tok + i;
-        uint64_t* tok_other = bar_tok + (i ^ 1);
         for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN>(p, t);
             // this warp's sub-tile, selected without runtime array indexing
@@ -416,15 +409,7 @@ __global__ void __launch_bounds__(320, 1)
             const int my_p0 = i ? ti.p0[1] : ti.p0[0];
             const int nb = i ? ti.nblk[1] : ti.nblk[0];
             const int my_full = i ? ti.full_blk[1] : ti.full_blk[0];
-            const int nturn = max(ti.nblk[0], ti.nblk[1]);
-            if (!my_valid) {
-                for (int j = 0; j < nturn; ++j, ++turns) {
-                    if (!mbar_wait_warp(tok_mine, (turns & 1) ^ (i == 0 ? 1u : 0u), abort_flag))
-                        goto softmax_done;
-                    mbar_arrive(tok_other);
-                }
-                continue;
-            }
+            if (!my_valid) continue;
             int pos, head;
             if (p.pack) {
                 pos = my_p0 + r / p.G;
@@ -440,13 +425,7 @@ __global__ void __launch_bounds__(320, 1)
             int key_lim = p.causal ? pos + ti.sk - ti.sq + 1 : ti.sk;
             key_lim = min(key_lim, ti.sk);
             float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
-            for (int j = 0; j < nturn; ++j, ++turns) {
-                if (j >= nb) {  // nothing of ours in this turn: pass it on
-                    if (!mbar_wait_warp(tok_mine, (turns & 1) ^ (i == 0 ? 1u : 0u), abort_flag))
-                        goto softmax_done;
-                    mbar_arrive(tok_other);
-                    continue;
-                }
+            for (int j = 0; j < nb; ++j) {
                 if (!mbar_wait_warp(bar_s_full + i, s_phase, abort_flag)) goto softmax_done;
                 s_phase ^= 1;
                 tc_fence_after();
@@ -487,12 +466,12 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
                 const uint64_t negm2 = f2_pack(-m_use, -m_use);
-                // our turn on the exponential unit
-                if (!mbar_wait_warp(tok_mine, (turns & 1) ^ (i == 0 ? 1u : 0u), abort_flag))
-                    goto softmax_done;
-                // p = 2^(s*scale*log2e - m); two row sums in paired fp32: of the exact p
-                // (for L) and of the bf16 p the P.V MMA consumes (for O / l)
+                // p = 2^(s*scale*log2e - m); two row sums in fp32: of the exact p (for L)
+                // and of the bf16 p the P.V MMA consumes (for O / l).  The second sum
+                // takes the bf16 halves either unpacked into paired adds (D = 64) or
+                // through the mixed bf16 + f32 add (D = 128), whichever measured faster.
                 uint64_t se0 = 0, se1 = 0, sq0 = 0, sq1 = 0;
+                float rq0 = 0.f, rq1 = 0.f, rq2 = 0.f, rq3 = 0.f;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
@@ -507,19 +486,34 @@ __global__ void __launch_bounds__(320, 1)
                         const float p1 = ex2_approx(a1);
                         pk[e] = pack_bf16x2(p0, p1);
                         const uint64_t pe = f2_pack(p0, p1);
-                        const uint64_t pr = f2_pack(bf16_lo(pk[e]), bf16_hi(pk[e]));
-                        if (e & 1) {
+                        if (e & 1)
                             se1 = fadd2(se1, pe);
-                            sq1 = fadd2(sq1, pr);
-                        } else {
+                        else
                             se0 = fadd2(se0, pe);
-                            sq0 = fadd2(sq0, pr);
+                        if constexpr (HD == 128) {
+                            if (e & 1)
+                                add_bf16x2_to_f32(pk[e], rq2, rq3);
+                            else
+                                add_bf16x2_to_f32(pk[e], rq0, rq1);
+                        } else {
+                            const uint64_t pr = f2_pack(bf16_lo(pk[e]), bf16_hi(pk[e]));
+                            if (e & 1)
+                                sq1 = fadd2(sq1, pr);
+                            else
+                                sq0 = fadd2(sq0, pr);
                         }
                     }
 #pragma unroll
                     for (int e = 0; e < 16; ++e) sr[c >> 1][(c & 1) * 16 + e] = pk[e];
                 }
-                mbar_arrive(tok_other);  // the other group's turn
+                if constexpr (HD == 128) sq0 = f2_pack(rq0 + rq2, rq1 + rq3);
+                // P.V(j-1) has finished: it no longer reads P's columns and O holds
+                // every block before j (needed before P is overwritten or O rescaled)
+                if (j > 0) {
+                    if (!mbar_wait_warp(bar_o_done + i, o_phase, abort_flag)) goto softmax_done;
+                    o_phase ^= 1;
+                    tc_fence_after();
+                }
                 // P (bf16 pairs): its own 64 columns, or the first 64 columns of S
                 tmem_st32(tP, sr[0]);
                 tmem_st32(tP + 32, sr[1]);
@@ -562,7 +556,7 @@ __global__ void __launch_bounds__(320, 1)
             {
                 const size_t row = size_t(ti.q_row0 + pos) * p.Hq + head;
                 if (nb > 0) {
-                    if (!mbar_wait_warp(bar_o_full + i, o_phase, abort_flag)) goto softmax_done;
+                    if (!mbar_wait_warp(bar_o_done + i, o_phase, abort_flag)) goto softmax_done;
                     o_phase ^= 1;
                     tc_fence_after();
                 }

@@ -58,6 +58,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Same test, but a thread whose phase is still open may sleep in hardware for up to
+// kSuspendHintNs (it wakes as soon as the phase completes) rather than coming back
+// at once, so waiting warps leave the issue slots to the warps that compute.
+constexpr uint32_t kSuspendHintNs = 20000;
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
 
 // Wait for the phase of `bar` with parity `parity` to complete.  Gives up after
 // `limit_ns` (or as soon as *abort is set by another role of the CTA), records
@@ -69,8 +84,8 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
     const uint64_t t0 = globaltimer_ns();
     while (true) {
 #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 4; ++i)
+            if (mbar_try_wait_sleep(bar, parity)) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
             raise_device_error(kDevWaitTimeout);
@@ -272,6 +287,14 @@ __device__ __forceinline__ float bf16_lo(uint32_t packed) {
 }
 __device__ __forceinline__ float bf16_hi(uint32_t packed) {
     return __uint_as_float(packed & 0xffff0000u);
+}
+// lo += float(low bf16 of packed), hi += float(high bf16): sm_100's mixed-precision
+// add (the bf16 operand is widened exactly, then added in f32 round-to-nearest)
+__device__ __forceinline__ void add_bf16x2_to_f32(uint32_t packed, float& lo, float& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(packed));
 }
 
 }  // namespace gqa
