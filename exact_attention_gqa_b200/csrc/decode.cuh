@@ -111,6 +111,9 @@ __global__ void __launch_bounds__(160, 2)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    // the combine kernel (launched as a programmatic dependent) may be scheduled
+    // now; it waits for this grid's completion before it reads any partial
+    griddep_launch_dependents();
     if (threadIdx.x == 0) {
         for (int s = 0; s < ST; ++s) {
             mbar_init(bar_full + s, 1);
@@ -345,43 +348,77 @@ __global__ void __launch_bounds__(160, 2)
     }
 }
 
-// One warp per (batch, query head): O = sum_s exp(L_s - L) O_s, L = logsumexp(L_s).
+// One CTA per (batch, query head), one thread per output dimension:
+// L = M + ln sum_s exp(L_s - M) with M = max_s L_s, then O = sum_s exp(L_s - L) O_s.
+// The split weights are computed once into shared memory, and the weighted sum
+// over splits keeps many independent loads in flight (the partials were just
+// written and sit in L2, so the sum is bound by load latency, not bandwidth).
+constexpr int kCombineMaxSplits = 256;
 template <int HD>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(HD)
     splitkv_combine(const float* __restrict__ part_o, const float* __restrict__ part_l,
                     __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int rows_bh,
                     int n) {
-    const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
+    constexpr int WARPS = HD / 32;
+    __shared__ float wts[kCombineMaxSplits];
+    __shared__ float red[WARPS];
+    __shared__ float s_stat[2];
+    const int w = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_wait();  // the split kernel has finished and its partials are visible
     if (w >= rows_bh) return;
     const float* Ls = part_l + size_t(w) * n;
     float M = -INFINITY;
-    for (int s = lane; s < n; s += 32) M = fmaxf(M, Ls[s]);
+    for (int s = tid; s < n; s += HD) M = fmaxf(M, Ls[s]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    constexpr int PER = HD / 32;
-    float acc[PER];
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    if (tid == 0) {
+        float m = red[0];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-    float L = -INFINITY;
-    if (M != -INFINITY) {
-        float sum = 0.f;
-        for (int s = lane; s < n; s += 32) sum += (Ls[s] == -INFINITY) ? 0.f : expf(Ls[s] - M);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-        L = M + logf(sum);
-        for (int s = 0; s < n; ++s) {
-            const float ls = Ls[s];
-            if (ls == -INFINITY) continue;
-            const float wgt = expf(ls - L);
-            const float* os = part_o + (size_t(w) * n + s) * HD;
-#pragma unroll
-            for (int e = 0; e < PER; ++e) acc[e] += wgt * os[lane + 32 * e];
-        }
+        for (int i = 1; i < WARPS; ++i) m = fmaxf(m, red[i]);
+        s_stat[0] = m;
     }
+    __syncthreads();
+    M = s_stat[0];
+    float sum = 0.f;
+    if (M != -INFINITY)
+        for (int s = tid; s < n; s += HD) sum += (Ls[s] == -INFINITY) ? 0.f : expf(Ls[s] - M);
 #pragma unroll
-    for (int e = 0; e < PER; ++e) out[size_t(w) * HD + lane + 32 * e] = __float2bfloat16_rn(acc[e]);
-    if (lane == 0) lse[w] = L;
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    __syncthreads();
+    if (lane == 0) red[warp] = sum;
+    __syncthreads();
+    if (tid == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int i = 0; i < WARPS; ++i) t += red[i];
+        s_stat[1] = (M == -INFINITY) ? -INFINITY : M + logf(t);
+    }
+    __syncthreads();
+    const float L = s_stat[1];
+    for (int s = tid; s < n; s += HD)
+        wts[s] = (L == -INFINITY || Ls[s] == -INFINITY) ? 0.f : expf(Ls[s] - L);
+    __syncthreads();
+    const float* os = part_o + size_t(w) * n * HD + tid;
+    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    int s = 0;
+#pragma unroll 4
+    for (; s + 4 <= n; s += 4) {
+        const float x0 = os[size_t(s) * HD], x1 = os[size_t(s + 1) * HD];
+        const float x2 = os[size_t(s + 2) * HD], x3 = os[size_t(s + 3) * HD];
+        acc0 += (wts[s] != 0.f) ? wts[s] * x0 : 0.f;
+        acc1 += (wts[s + 1] != 0.f) ? wts[s + 1] * x1 : 0.f;
+        acc2 += (wts[s + 2] != 0.f) ? wts[s + 2] * x2 : 0.f;
+        acc3 += (wts[s + 3] != 0.f) ? wts[s + 3] * x3 : 0.f;
+    }
+    for (; s < n; ++s) {
+        const float x = os[size_t(s) * HD];
+        acc0 += (wts[s] != 0.f) ? wts[s] * x : 0.f;
+    }
+    out[size_t(w) * HD + tid] = __float2bfloat16_rn((acc0 + acc1) + (acc2 + acc3));
+    if (tid == 0) lse[w] = L;
 }
 
 }  // namespace gqa

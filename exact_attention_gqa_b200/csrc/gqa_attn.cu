@@ -24,6 +24,7 @@ using gqa::PrefillParams;
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxSplits = 256;
+static_assert(kMaxSplits <= gqa::kCombineMaxSplits, "combine weights table too small");
 
 enum Kernel { kNone = 0, kPrefill = 1, kDecode = 2, kZeroFill = 3 };
 
@@ -141,9 +142,11 @@ void make_plan(Plan* pl, int B, int Hq, int Hkv, int Sq, int Sk, int num_splits,
         const int nblk = (Sk + DecodeCfg<128>::BN - 1) / DecodeCfg<128>::BN;
         int n = num_splits;
         if (n == 0) {
-            // enough CTAs for two per SM, splits of at least four 64-key blocks
+            // As many splits as keep every CTA on an SM of its own (one CTA per SM
+            // already streams at the HBM rate; a partial second wave only adds a
+            // tail), with splits of at least four 64-key blocks.
             const long long ctas = (long long)B * Hkv * pl->decode_units;
-            const long long want = (2LL * sms + ctas - 1) / ctas;
+            const long long want = sms / ctas;
             n = int(want < 1 ? 1 : (want > 64 ? 64 : want));
             const int max_by_len = nblk / 4 > 0 ? nblk / 4 : 1;
             if (n > max_by_len) n = max_by_len;
@@ -221,6 +224,28 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// The combine runs as a programmatic dependent launch of the split kernel: its CTAs
+// are scheduled while the split kernel drains and wait in griddep_wait() for its
+// completion, which removes the launch gap between the two kernels.
+template <int HD>
+int launch_combine(const float* part_o, const float* part_l, __nv_bfloat16* out, float* lse,
+                   int rows_bh, int n, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows_bh);
+    cfg.blockDim = dim3(HD);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, gqa::splitkv_combine<HD>, part_o, part_l, out, lse, rows_bh, n) !=
+        cudaSuccess)
+        return GQA_ERR_CUDA;
+    return GQA_OK;
+}
+
 template <int HD>
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                   int Hq, int Hkv, int Sk, float scale, const Plan& pl, cudaStream_t stream) {
@@ -266,10 +291,8 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
     if (pl.splits > 1) {
         const int rows_bh = B * Hq;
-        const int blocks = (rows_bh + 3) / 4;
-        gqa::splitkv_combine<HD><<<blocks, 128, 0, stream>>>(
-            p.part_o, p.part_l, p.out, lse, rows_bh, pl.splits);
-        if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+        const int rc = launch_combine<HD>(p.part_o, p.part_l, p.out, lse, rows_bh, pl.splits, stream);
+        if (rc != GQA_OK) return rc;
     }
     return GQA_OK;
 }
@@ -413,9 +436,8 @@ int launch_decode_noalloc(const void* q, const void* k, const void* v, void* out
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
     if (pl.splits > 1) {
         const int rows_bh = B * Hq;
-        gqa::splitkv_combine<HD><<<(rows_bh + 3) / 4, 128, 0, stream>>>(
-            p.part_o, p.part_l, p.out, lse, rows_bh, pl.splits);
-        if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
+        const int rc = launch_combine<HD>(p.part_o, p.part_l, p.out, lse, rows_bh, pl.splits, stream);
+        if (rc != GQA_OK) return rc;
     }
     return GQA_OK;
 }
