@@ -464,11 +464,19 @@ def run_ours(args, world, rank, local):
         achieved = case.bytes / (kernel_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     else:
+        # A timed region of a second or more runs under the power cap, like the
+        # sustained GEMM loop; a short one like the burst figure.
+        sustained = ms_total >= 1000.0 and "bf16_tflops_sustained" in peaks
+        key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
         achieved = case.flops / (kernel_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks[key],
+                "unit": "TFLOP/s", "frac_of_burst": achieved / peaks["bf16_tflops"]}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["peak_source"] = f"{peak_kind} ({'hbm_gbs' if case.decode else 'bf16_tflops'}, burst)"
+    if case.decode:
+        roof["peak_source"] = f"{peak_kind} (hbm_gbs, copy)"
+    else:
+        roof["peak_source"] = (f"{peak_kind} ({key}: timed region {ms_total / 1e3:.1f} s, "
+                               f"{'sustained' if sustained else 'burst'})")
     roof["kernel"] = case.kernel
     tr = load_traffic(w.name, case.kernel)
     roof["traffic"] = tr

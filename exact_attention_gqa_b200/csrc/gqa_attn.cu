@@ -208,6 +208,17 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     // dense non-causal: a (batch, head unit)'s position tiles back to back so its K/V
     // stay in L2; causal and packed batches: longest tiles first
     p.kv_major = (!causal && !cu) ? 1 : 0;
+    {
+        // about 32 MB of K and V per group of (batch, head unit) pairs (an L2 share);
+        // without packing, G consecutive head units read the same KV head
+        const long long kv_per_head = (long long)(cu ? Sq : Sk) * HD * 2 * 2;
+        long long hg = (32LL << 20) / (kv_per_head > 0 ? kv_per_head : 1);
+        if (!pack) hg *= G;
+        const long long per_m = (long long)B * p.n_hu;
+        if (hg < 1) hg = 1;
+        if (hg > per_m) hg = per_m;
+        p.hu_group = int(hg);
+    }
     p.scale_log2 = scale * kLog2e;
     // Row extents of the 3-D views: exactly the rows the caller allocated
     // (packed variable length: Sk carries the packed row count).

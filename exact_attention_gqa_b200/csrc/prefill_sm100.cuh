@@ -57,6 +57,7 @@ struct PrefillParams {
     int n_units;             // n_mblk * B * n_hu
     int causal;
     int kv_major;            // 1: tiles of one (batch, head unit) consecutive (L2 reuse)
+    int hu_group;            // kv_major = 0: (batch, head unit) pairs per longest-first pass
     float scale_log2;        // scale * log2(e)
 };
 
@@ -110,9 +111,26 @@ __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
         ti.b = bh / p.n_hu;
         ti.hu = bh - ti.b * p.n_hu;
     } else {
+        // Longest-first within groups of hu_group (batch, head unit) pairs: a group's
+        // position tiles run from the last (longest under the causal mask) to the
+        // first, then the next group follows.  A group's K and V stay in L2 while
+        // its tiles run, and the tiles still end in short ones.
         const int per_m = p.B * p.n_hu;
-        ti.m = p.n_mblk - 1 - t / per_m;
-        const int r = t - (t / per_m) * per_m;
+        const int hg_full = p.hu_group;
+        const int n_full = per_m / hg_full;
+        const int t_full = n_full * hg_full * p.n_mblk;
+        int c, hg, rem;
+        if (t < t_full) {
+            c = t / (hg_full * p.n_mblk);
+            hg = hg_full;
+            rem = t - c * hg_full * p.n_mblk;
+        } else {
+            c = n_full;
+            hg = per_m - n_full * hg_full;
+            rem = t - t_full;
+        }
+        ti.m = p.n_mblk - 1 - rem / hg;
+        const int r = c * hg_full + (rem - (rem / hg) * hg);
         ti.b = r / p.n_hu;
         ti.hu = r - ti.b * p.n_hu;
     }
