@@ -480,10 +480,10 @@ def run_ours(args, world, rank, local):
     roof["kernel"] = case.kernel
     tr = load_traffic(w.name, case.kernel)
     roof["traffic"] = tr
+    # algorithmic bytes of one launch: q, k, v read once, O and L written once
+    roof["algorithmic_bytes"] = case.in_bytes() + case.out_bytes()
     if tr is not None:
-        roof["traffic_per_algorithmic"] = tr / (case.bytes if case.decode else
-                                                W.prefill_min_bytes(w.B, w.Hq, w.Hkv, w.Sq,
-                                                                    w.Sk, w.D))
+        roof["traffic_per_algorithmic"] = tr / roof["algorithmic_bytes"]
     # ---- CPU baseline (oracle on a bounded sample, rank 0, N=1 only)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
