@@ -225,13 +225,15 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     const long long rows_q = cu ? (long long)Sk : (long long)B * Sq;
     const long long rows_k = cu ? (long long)Sk : (long long)B * Sk;
     p.total_rows = cu ? Sk : 0;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
+    // the output leaves through the same box shape as Q arrives in (one sub-tile)
     if (!make_map(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) ||
         !make_map(&tk, k, rows_k, Hkv, HD, 1, C::BN) ||
-        !make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN))
+        !make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN) ||
+        !make_map(&to, out, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128))
         return GQA_ERR_CUDA;
     const int grid = p.n_units < sms ? p.n_units : sms;
-    gqa::prefill_fwd_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    gqa::prefill_fwd_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 

@@ -76,8 +76,13 @@ struct PrefillCfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_STAGES * Q_TILE;
     static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
-    static constexpr int OFF_BAR = OFF_V + STAGES * KV_TILE;
-    static constexpr int NUM_BARS = 2 * Q_STAGES + 4 * STAGES + 6 + 1;
+    // D = 64: full sub-tiles of O leave through a shared-memory box and one TMA store
+    // (128B-swizzled rows, the same box as Q's); D = 128 has no room and stores rows.
+    static constexpr bool EPI_TMA = (HD == 64);
+    static constexpr int OFF_O = OFF_V + STAGES * KV_TILE;
+    static constexpr int O_SUB = BM * HD * 2;
+    static constexpr int OFF_BAR = OFF_O + (EPI_TMA ? 2 * O_SUB : 0);
+    static constexpr int NUM_BARS = 2 * Q_STAGES + 4 * STAGES + 6 + 1 + 4;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
     static constexpr int TMEM_COLS = 512;
@@ -173,7 +178,8 @@ template <int HD>
 __global__ void __launch_bounds__(320, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
     using C = PrefillCfg<HD>;
     constexpr int BN = C::BN;
     constexpr int ST = C::STAGES;
@@ -192,6 +198,8 @@ __global__ void __launch_bounds__(320, 1)
     uint64_t* bar_p_full = bar_s_full + 2;    // [2]
     uint64_t* bar_o_done = bar_p_full + 2;    // [2] O_i += P_i(j) V_j finished (every block)
     uint64_t* bar_drain = bar_o_done + 2;     // MMA completion before exit
+    uint64_t* bar_epi = bar_drain + 1;        // [2] a sub-tile's O rows are in shared memory
+    uint64_t* bar_ofree = bar_epi + 2;        // [2] the previous O store has read them
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -215,6 +223,10 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(bar_o_done + i, 1);
         }
         mbar_init(bar_drain, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_epi + i, 4);
+            mbar_init(bar_ofree + i, 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -420,6 +432,7 @@ __global__ void __launch_bounds__(320, 1)
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
         uint32_t s_phase = 0, o_phase = 0;
+        uint32_t ec = 0;  // O stores issued through the shared-memory box
         for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
             const TileInfo ti = decode_tile<BN>(p, t);
             // this warp's sub-tile, selected without runtime array indexing
@@ -579,8 +592,60 @@ __global__ void __launch_bounds__(320, 1)
                     tc_fence_after();
                 }
                 const float inv_l = (l_rnd > 0.f) ? 1.f / l_rnd : 0.f;
+                // a sub-tile whose 128 rows are all real leaves through one TMA store
+                const bool tma_out = C::EPI_TMA && (my_p0 + p.sub_pos <= ti.sq);
+                if constexpr (C::EPI_TMA) {
+                    if (tma_out) {
+                        uint8_t* stage = smem + C::OFF_O + i * C::O_SUB;
+                        const uint32_t st_row = smem_u32(stage) + uint32_t(r) * 128u;
+                        if (ec > 0) {  // the previous store has finished reading the box
+                            if (r == 0) {
+                                bulk_wait_read();
+                                mbar_arrive(bar_ofree + i);
+                            }
+                            if (!mbar_wait_warp(bar_ofree + i, (ec - 1) & 1, abort_flag))
+                                goto softmax_done;
+                        }
 #pragma unroll 1
-                for (int c = 0; c < HD / 32; ++c) {
+                        for (int c = 0; c < HD / 32; ++c) {
+                            uint32_t o[32];
+                            if (nb > 0) {
+                                tmem_ld32(tO + c * 32, o);
+                                tmem_ld_wait();
+                                reg_fence(o);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) o[e] = 0u;
+                            }
+                            uint32_t w[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                                   __uint_as_float(o[2 * e + 1]) * inv_l);
+                            // 16-byte chunk q of the row sits at q ^ (row % 8) (128B swizzle)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t q = uint32_t(c * 4 + e);
+                                st_shared_v4(st_row + ((q ^ uint32_t(r & 7)) << 4), w[4 * e],
+                                             w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                            }
+                        }
+                        fence_proxy_async();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar_epi + i);
+                        bool ok = true;
+                        if (r == 0) ok = mbar_wait(bar_epi + i, ec & 1, abort_flag);
+                        if (!__all_sync(0xffffffffu, ok)) goto softmax_done;
+                        if (r == 0) {
+                            tma_store_3d(&tm_o, stage, 0, p.pack ? ti.hu * p.G : ti.hu,
+                                         ti.q_row0 + my_p0);
+                            bulk_commit();
+                        }
+                        ++ec;
+                    }
+                }
+#pragma unroll 1
+                for (int c = 0; c < HD / 32 && !tma_out; ++c) {
                     uint32_t o[32];
                     if (nb > 0) {
                         tmem_ld32(tO + c * 32, o);
@@ -614,7 +679,11 @@ __global__ void __launch_bounds__(320, 1)
                 }
             }
         }
-    softmax_done:;
+    softmax_done:
+        // the thread that issued O stores waits for them before the CTA may exit
+        if constexpr (C::EPI_TMA) {
+            if (r == 0) bulk_wait_all();
+        }
     }
 
     tc_fence_before();
