@@ -83,7 +83,10 @@ typedef enum {
  *   causal       : nonzero for the causal mask
  *   num_splits   : split-KV factor for decode (dense, Sq == 1): 1 = none,
  *                  n > 1 = n contiguous key ranges combined by log-sum-exp
- *                  (needs a workspace, see below), 0 = chosen by the library.
+ *                  (needs a workspace, see below), 0 = chosen by the library
+ *                  (as many splits as give every CTA an SM of its own).  With
+ *                  n > 1 two kernels are enqueued: the split kernel and the
+ *                  combine, the latter as a programmatic dependent launch.
  *                  Must be 0 or 1 for every other shape.
  *   pack_gqa     : 1 = the G query heads of a KV head share one tile (K/V read
  *                  once per group), 0 = one query head per tile, -1 = chosen by

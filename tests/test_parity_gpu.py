@@ -100,6 +100,24 @@ def test_decode_rescales_at_every_block(splits):
     compare(out, lse, *oracle.attention(q, k, v, scale=1 / math.sqrt(128), causal=False))
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_at_the_split_limit(D):
+    """256 splits of one 64-key block each: the most partials the combine takes."""
+    q, k, v = rand_qkv(1, 8, 2, 1, 256 * 64, D, seed=91 + D)
+    rc, kern, splits, pack = gqa_attn_plan(1, 8, 2, 1, 256 * 64, D, num_splits=256)
+    assert kern == "decode_splitkv" and splits == 256
+    out, lse = run(q, k, v, causal=False, num_splits=256)
+    compare(out, lse, *oracle.attention(q, k, v, scale=1 / math.sqrt(D), causal=False))
+
+
+@pytest.mark.parametrize("splits", [2, 0])
+def test_decode_sixteen_heads_per_kv_head(splits):
+    """G = 16 packed in one CTA, D = 64, with and without splits."""
+    q, k, v = rand_qkv(2, 32, 2, 1, 3000, 64, seed=93)
+    out, lse = run(q, k, v, causal=False, num_splits=splits, pack_gqa=1)
+    compare(out, lse, *oracle.attention(q, k, v, scale=1 / math.sqrt(64), causal=False))
+
+
 def test_pack_on_and_off_agree():
     q, k, v = rand_qkv(2, 16, 4, 333, 333, 128, seed=11)
     a, la = run(q, k, v, causal=True, pack_gqa=1)
