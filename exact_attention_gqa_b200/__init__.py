@@ -96,7 +96,8 @@ def _workspace(torch, device, nbytes):
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
         _ws[idx] = buf
-    rc = gqa_attn_set_workspace(ctypes.c_void_p(buf.data_ptr()), buf.numel())
+    with torch.cuda.device(device):  # the registration belongs to this device
+        rc = gqa_attn_set_workspace(ctypes.c_void_p(buf.data_ptr()), buf.numel())
     if rc != 0:
         raise GqaError("gqa_attn_set_workspace", rc)
 
@@ -146,6 +147,14 @@ def gqa_attn(q, k, v, *, causal: bool = False, scale: float | None = None,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):  # the library works on the current device
+        _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
+              pack_gqa, varlen, cu)
+    return out, lse
+
+
+def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits, pack_gqa,
+          varlen, cu):
     stream = _stream_handle(torch, q.device)
     if q.dtype == torch.bfloat16:
         rc, _, splits, _ = gqa_attn_plan(B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
@@ -162,4 +171,3 @@ def gqa_attn(q, k, v, *, causal: bool = False, scale: float | None = None,
                               stream)
         if rc != 0:
             raise GqaError("gqa_attn_fwd_f32", rc)
-    return out, lse

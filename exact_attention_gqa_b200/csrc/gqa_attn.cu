@@ -32,14 +32,14 @@ struct Workspace {
     void* ptr = nullptr;
     size_t bytes = 0;
 };
-Workspace g_ws;
+Workspace g_ws[64];  // one registered split-KV workspace per device
 std::mutex g_mu;
 
 // ---------------------------------------------------------------------------- device
 struct DeviceInfo {
     int ok = 0;       // 1 when the device is sm_100
     int sms = 0;
-    int attrs_set = 0;
+    int attrs_set = 0;  // bit mask of kernels whose shared-memory limit is raised here
 };
 DeviceInfo g_dev[64];
 
@@ -58,6 +58,21 @@ int device_info(DeviceInfo** out) {
     }
     *out = &d;
     return d.ok ? GQA_OK : GQA_ERR_UNSUPPORTED;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (the setting belongs to
+// the device's context, so a process that drives several GPUs needs it on each).
+template <typename Kernel>
+int ensure_smem_limit(Kernel kernel, int bit, int bytes) {
+    DeviceInfo* d = nullptr;
+    const int rc = device_info(&d);
+    if (rc != GQA_OK) return rc;
+    if (d->attrs_set & bit) return GQA_OK;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return GQA_ERR_CUDA;
+    d->attrs_set |= bit;
+    return GQA_OK;
 }
 
 // ---------------------------------------------------------------------------- TMA
@@ -178,13 +193,10 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
                    int Hq, int Hkv, int Sq, int Sk, float scale, int causal, int pack,
                    const int* cu, int sms, cudaStream_t stream) {
     using C = PrefillCfg<HD>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(gqa::prefill_fwd_sm100<HD>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess)
-            return GQA_ERR_CUDA;
-        attr_done = true;
+    {
+        const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD>, HD == 64 ? 1 : 2,
+                                         C::SMEM_BYTES);
+        if (rc != GQA_OK) return rc;
     }
     const int G = Hq / Hkv;
     PrefillParams p;
@@ -263,13 +275,10 @@ template <int HD>
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                   int Hq, int Hkv, int Sk, float scale, const Plan& pl, cudaStream_t stream) {
     using C = DecodeCfg<HD>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(gqa::decode_split_sm100<HD>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES) != cudaSuccess)
-            return GQA_ERR_CUDA;
-        attr_done = true;
+    {
+        const int rc = ensure_smem_limit(gqa::decode_split_sm100<HD>, HD == 64 ? 4 : 8,
+                                         C::SMEM_BYTES);
+        if (rc != GQA_OK) return rc;
     }
     DecodeParams p;
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -289,10 +298,17 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     p.part_l = nullptr;
     if (pl.splits > 1) {
         const size_t need = ws_bytes(B, Hq, 1, HD, pl.splits);
-        if (!g_ws.ptr || g_ws.bytes < need) return GQA_ERR_WORKSPACE;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQA_ERR_CUDA;
+        Workspace ws;
+        {
+            std::lock_guard<std::mutex> lk(g_mu);
+            ws = g_ws[dev];
+        }
+        if (!ws.ptr || ws.bytes < need) return GQA_ERR_WORKSPACE;
         const size_t o_bytes = size_t(B) * Hq * pl.splits * HD * 4;
-        p.part_o = static_cast<float*>(g_ws.ptr);
-        p.part_l = reinterpret_cast<float*>(static_cast<char*>(g_ws.ptr) +
+        p.part_o = static_cast<float*>(ws.ptr);
+        p.part_l = reinterpret_cast<float*>(static_cast<char*>(ws.ptr) +
                                             ((o_bytes + 255) / 256) * 256);
     }
     CUtensorMap tk, tv;
@@ -496,9 +512,12 @@ size_t gqa_attn_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits) {
 
 int gqa_attn_set_workspace(void* dev_ptr, size_t bytes) {
     if (dev_ptr && !aligned(dev_ptr, 16)) return GQA_ERR_ALIGN;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return dev_ptr ? GQA_ERR_CUDA : GQA_OK;  // no device: nothing is registered
     std::lock_guard<std::mutex> lk(g_mu);
-    g_ws.ptr = bytes ? dev_ptr : nullptr;
-    g_ws.bytes = dev_ptr ? bytes : 0;
+    g_ws[dev].ptr = bytes ? dev_ptr : nullptr;
+    g_ws[dev].bytes = dev_ptr ? bytes : 0;
     return GQA_OK;
 }
 

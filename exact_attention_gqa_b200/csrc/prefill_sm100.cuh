@@ -15,9 +15,10 @@
 //   pack_gqa = 0: rows are 128 consecutive positions of one query head.
 // Work units are spread over a persistent grid (sequence-dimension parallelism,
 // FlashAttention-2 summary page).  Causal and variable-length batches run the
-// longest units first (attention balancing, Raptor-T abstract); dense
-// non-causal batches run the position tiles of one (batch, KV head) back to back
-// so that its K and V are re-read from L2 rather than HBM.
+// longest units first (attention balancing, Raptor-T abstract) within groups of
+// (batch, head unit) pairs whose K and V fit a share of L2; dense non-causal
+// batches run the position tiles of one (batch, KV head) back to back so that
+// its K and V are re-read from L2 rather than HBM.
 //
 // Roles inside the CTA (320 threads):
 //   warps 0-3  softmax for sub-tile 0 (one thread = one row = one TMEM lane)
@@ -30,7 +31,9 @@
 // O1 [256+D, 256+2D); P_i (bf16 pairs, 64 columns) has its own columns
 // [384+64i, 448+64i) when D = 64 and otherwise overwrites the first half of S_i
 // after the softmax has read S_i into registers.  The two sub-tiles run their
-// softmax independently; the tensor core alternates between them.
+// softmax independently; the tensor core alternates between them.  At the end of
+// a sub-tile the softmax threads normalise O; with D = 64 a sub-tile whose rows
+// are all real is staged in shared memory and written by one TMA store.
 //
 // Online softmax in the log2 domain: s2 = s * scale * log2(e).  The running
 // max used for the exponentials is only raised when a block's max exceeds it by

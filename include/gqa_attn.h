@@ -115,10 +115,11 @@ int gqa_attn_fwd_f32(const void* q, const void* k, const void* v, void* out, flo
 size_t gqa_attn_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits);
 
 /*
- * Register a caller-owned device buffer as the split-KV workspace of this
- * process (borrowed, never freed by the library; NULL/0 unregisters).  Calls
- * that run concurrently on different streams must not share one workspace.
- * Returns GQA_ERR_ALIGN if dev_ptr is not 16-byte aligned.
+ * Register a caller-owned device buffer as the split-KV workspace of the calling
+ * thread's current device (one registration per device and process; borrowed,
+ * never freed by the library; NULL/0 unregisters).  Calls that run concurrently
+ * on different streams must not share one workspace.  Returns GQA_ERR_ALIGN if
+ * dev_ptr is not 16-byte aligned, GQA_ERR_CUDA if no device can be queried.
  */
 int gqa_attn_set_workspace(void* dev_ptr, size_t bytes);
 
