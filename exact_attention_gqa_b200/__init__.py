@@ -22,7 +22,7 @@ import math
 from . import _capi
 from ._capi import GqaError, STATUS, STATUS_CODE, strerror
 
-__all__ = ["gqa_attn", "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
+__all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
            "gqa_attn_workspace_bytes", "gqa_attn_set_workspace", "gqa_attn_get_device_error",
            "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path"]
 
@@ -171,3 +171,44 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
                               stream)
         if rc != 0:
             raise GqaError("gqa_attn_fwd_f32", rc)
+
+
+def gqa_attn_host(q_h, k_h, v_h, out_h, lse_h, q_d, k_d, v_d, out_d, lse_d, *,
+                  causal: bool = False, scale: float | None = None, num_splits: int = 1,
+                  pack_gqa: int = -1, chunks: int = 0):
+    """Attention on host-resident tensors with the transfers overlapped (gqa_attn_fwd_host).
+
+    q_h, k_h, v_h, out_h, lse_h: CPU tensors (pinned for overlap) in the dense layouts of
+    ``gqa_attn``; q_d ... lse_d: CUDA tensors of the same shapes used as the staging area.
+    Enqueued on the current stream of q_d's device; out_h and lse_h are complete once
+    that stream has been synchronised.
+    """
+    import torch
+
+    B, Sq, Hq, D = q_d.shape
+    _, Sk, Hkv, _ = k_d.shape
+    for h, d in ((q_h, q_d), (k_h, k_d), (v_h, v_d), (out_h, out_d), (lse_h, lse_d)):
+        if h.device.type != "cpu" or d.device != q_d.device or h.shape != d.shape or \
+                h.dtype != d.dtype or not h.is_contiguous() or not d.is_contiguous():
+            raise ValueError("host tensors on the CPU and device tensors on one GPU, "
+                             "same shapes and dtypes, contiguous")
+    if q_d.dtype != torch.bfloat16:
+        raise ValueError("gqa_attn_host takes bf16 q, k, v")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    with torch.cuda.device(q_d.device):
+        n = chunks if chunks > 0 else 8
+        per = -(-B // max(1, min(n, B))) if B else 0
+        need = 0
+        for b in {per, B - (-(-B // per) - 1) * per} if per else ():
+            rc, _, splits, _ = gqa_attn_plan(b, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
+                                             pack_gqa, False)
+            if rc == 0 and splits > 1:
+                need = max(need, gqa_attn_workspace_bytes(b, Hq, Sq, D, splits))
+        _workspace(torch, q_d.device, need)
+        stream = _stream_handle(torch, q_d.device)
+        rc = _capi.load().gqa_attn_fwd_host(
+            _ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(out_h), _ptr(lse_h), _ptr(q_d), _ptr(k_d),
+            _ptr(v_d), _ptr(out_d), _ptr(lse_d), B, Hq, Hkv, Sq, Sk, D, scale,
+            int(bool(causal)), num_splits, pack_gqa, chunks, stream)
+    if rc != 0:
+        raise GqaError("gqa_attn_fwd_host", rc)

@@ -14,6 +14,7 @@ LIB_PATH = pathlib.Path(__file__).resolve().parent / "libgqa_attn.so"
 EXPORTS = (
     "gqa_attn_fwd",
     "gqa_attn_fwd_f32",
+    "gqa_attn_fwd_host",
     "gqa_attn_workspace_bytes",
     "gqa_attn_set_workspace",
     "gqa_attn_plan",
@@ -54,6 +55,9 @@ def load() -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.argtypes = fwd_args
         fn.restype = I
+    lib.gqa_attn_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, I,
+                                      I, P]
+    lib.gqa_attn_fwd_host.restype = I
     lib.gqa_attn_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.gqa_attn_workspace_bytes.restype = Z
     lib.gqa_attn_set_workspace.argtypes = [P, Z]

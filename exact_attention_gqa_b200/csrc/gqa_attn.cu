@@ -489,6 +489,42 @@ __global__ void selftest_wait_timeout(uint64_t limit_ns) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------- host pipeline
+// gqa_attn_fwd_host: three library-owned streams per device (copy in, compute, copy
+// out) and events that chain them chunk by chunk, created on first use and kept.
+constexpr int kMaxChunks = 64;
+struct Pipe {
+    cudaStream_t s_in = nullptr, s_c = nullptr, s_out = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t in_done[kMaxChunks] = {};
+    cudaEvent_t c_done[kMaxChunks] = {};
+    bool ready = false;
+};
+Pipe g_pipe[64];
+std::mutex g_pipe_mu;  // held while a call enqueues, so that its waits see its own records
+
+int pipe_for_device(Pipe** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQA_ERR_CUDA;
+    Pipe& pp = g_pipe[dev];
+    if (!pp.ready) {
+        const unsigned ef = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&pp.s_in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&pp.s_c, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&pp.s_out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&pp.start, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&pp.done, ef) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        for (int c = 0; c < kMaxChunks; ++c)
+            if (cudaEventCreateWithFlags(&pp.in_done[c], ef) != cudaSuccess ||
+                cudaEventCreateWithFlags(&pp.c_done[c], ef) != cudaSuccess)
+                return GQA_ERR_CUDA;
+        pp.ready = true;
+    }
+    *out = &pp;
+    return GQA_OK;
+}
+
 extern "C" {
 
 int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B,
@@ -496,6 +532,81 @@ int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
                  int num_splits, int pack_gqa, const int* cu_seqlens, cudaStream_t stream) {
     return fwd_common(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
                       pack_gqa, cu_seqlens, stream, false);
+}
+
+int gqa_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* out_h,
+                      float* lse_h, void* q_d, void* k_d, void* v_d, void* out_d, float* lse_d,
+                      int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                      int num_splits, int pack_gqa, int chunks, cudaStream_t stream) {
+    int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, num_splits, pack_gqa, false, false);
+    if (rc != GQA_OK) return rc;
+    if (chunks < 0 || chunks > kMaxChunks) return GQA_ERR_SHAPE;
+    if (B == 0 || Sq == 0) return GQA_OK;
+    const bool reads_kv = Sk > 0;
+    if (!q_h || !out_h || !lse_h || !q_d || !out_d || !lse_d ||
+        (reads_kv && (!k_h || !v_h || !k_d || !v_d)))
+        return GQA_ERR_NULL;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    Pipe* pp = nullptr;
+    rc = pipe_for_device(&pp);
+    if (rc != GQA_OK) return rc;
+    // chunks of whole batch elements: [B, S, H, D] and [B, H, S] are batch-major
+    int n = chunks == 0 ? 8 : chunks;
+    if (n > B) n = B;
+    const int per = (B + n - 1) / n;
+    n = (B + per - 1) / per;
+    const size_t qb = size_t(Sq) * Hq * D * 2, kb = size_t(Sk) * Hkv * D * 2;
+    const size_t lb = size_t(Hq) * Sq * 4;
+    auto at = [](const void* base, size_t off) {
+        return static_cast<void*>(static_cast<char*>(const_cast<void*>(base)) + off);
+    };
+    if (cudaEventRecord(pp->start, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_in, pp->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_c, pp->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_out, pp->start, 0) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    int status = GQA_OK;
+    for (int c = 0; c < n && status == GQA_OK; ++c) {
+        const int b0 = c * per, nb = (B - b0 < per) ? B - b0 : per;
+        const size_t oq = size_t(b0) * qb, ok = size_t(b0) * kb, ol = size_t(b0) * lb;
+        if (cudaMemcpyAsync(at(q_d, oq), at(q_h, oq), nb * qb, cudaMemcpyHostToDevice,
+                            pp->s_in) != cudaSuccess ||
+            (reads_kv && (cudaMemcpyAsync(at(k_d, ok), at(k_h, ok), nb * kb,
+                                          cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess ||
+                          cudaMemcpyAsync(at(v_d, ok), at(v_h, ok), nb * kb,
+                                          cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess)) ||
+            cudaEventRecord(pp->in_done[c], pp->s_in) != cudaSuccess ||
+            cudaStreamWaitEvent(pp->s_c, pp->in_done[c], 0) != cudaSuccess) {
+            status = GQA_ERR_CUDA;
+            break;
+        }
+        status = fwd_common(at(q_d, oq), reads_kv ? at(k_d, ok) : nullptr,
+                            reads_kv ? at(v_d, ok) : nullptr, at(out_d, oq),
+                            static_cast<float*>(at(lse_d, ol)), nb, Hq, Hkv, Sq, Sk, D, scale,
+                            causal, num_splits, pack_gqa, nullptr, pp->s_c, false);
+        if (status != GQA_OK) break;
+        if (cudaEventRecord(pp->c_done[c], pp->s_c) != cudaSuccess ||
+            cudaStreamWaitEvent(pp->s_out, pp->c_done[c], 0) != cudaSuccess ||
+            cudaMemcpyAsync(at(out_h, oq), at(out_d, oq), nb * qb, cudaMemcpyDeviceToHost,
+                            pp->s_out) != cudaSuccess ||
+            cudaMemcpyAsync(at(lse_h, ol), at(lse_d, ol), nb * lb, cudaMemcpyDeviceToHost,
+                            pp->s_out) != cudaSuccess)
+            status = GQA_ERR_CUDA;
+    }
+    // whatever was enqueued (all of it, also after an error) finishes before later
+    // work on the caller's stream: join the copy-in and compute streams into copy-out
+    cudaEvent_t tail_c = pp->c_done[0];
+    if (cudaEventRecord(tail_c, pp->s_c) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_out, tail_c, 0) != cudaSuccess ||
+        cudaEventRecord(pp->in_done[0], pp->s_in) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_out, pp->in_done[0], 0) != cudaSuccess ||
+        cudaEventRecord(pp->done, pp->s_out) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, pp->done, 0) != cudaSuccess)
+        status = status == GQA_OK ? GQA_ERR_CUDA : status;
+    return status;
 }
 
 int gqa_attn_fwd_f32(const void* q, const void* k, const void* v, void* out, float* lse, int B,

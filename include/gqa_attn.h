@@ -108,6 +108,30 @@ int gqa_attn_fwd_f32(const void* q, const void* k, const void* v, void* out, flo
                      int num_splits, int pack_gqa, const int* cu_seqlens, cudaStream_t stream);
 
 /*
+ * gqa_attn_fwd on inputs and outputs in host memory, with the transfers overlapped:
+ * the batch is cut into `chunks` groups of whole batch elements (0 = 8; at most 64,
+ * at most B) and, on three streams the library creates once per device, the copy of
+ * chunk c+1 to the device, the attention of chunk c and the copy of chunk c-1's
+ * results back run at the same time.  Dense only (no cu_seqlens), bf16.
+ *   q_h, k_h, v_h, out_h, lse_h : host buffers in gqa_attn_fwd's layouts; page-locked
+ *                  (cudaHostAlloc / cudaHostRegister) for the copies to overlap
+ *   q_d ... lse_d : caller-owned device buffers of the same sizes (the staging area;
+ *                  they hold the inputs and results afterwards)
+ *   other arguments as gqa_attn_fwd; a split-KV decode chunk uses the workspace
+ *                  registered for the current device, sized for its own batch
+ * Ordered after earlier work on `stream`; later work on `stream` waits for all of it.
+ * One call at a time per device from the library's side (calls from several host
+ * threads are serialised while they enqueue).  Returns gqa_attn_fwd's status codes;
+ * GQA_ERR_SHAPE also for chunks < 0 or > 64.  This entry point has no counterpart
+ * on the pages: it exists so that host-resident inputs reach the kernels with the
+ * transfers hidden behind the computation.
+ */
+int gqa_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* out_h,
+                      float* lse_h, void* q_d, void* k_d, void* v_d, void* out_d, float* lse_d,
+                      int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+                      int num_splits, int pack_gqa, int chunks, cudaStream_t stream);
+
+/*
  * Bytes of device workspace gqa_attn_fwd needs for a split-KV decode with the
  * given sizes and num_splits (0 when num_splits <= 1): fp32 partial outputs
  * [B, Hq, Sq, n, D] and partial log-sum-exps [B, Hq, Sq, n].

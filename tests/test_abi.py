@@ -121,3 +121,19 @@ def test_python_front_end_refuses_cpu_tensors():
     q = torch.zeros(1, 4, 2, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):
         G.gqa_attn(q, q[:, :, :1].contiguous(), q[:, :, :1].contiguous())
+
+
+def test_host_pipeline_argument_errors(lib):
+    """gqa_attn_fwd_host validates before it touches a device."""
+    fn = lib.gqa_attn_fwd_host
+    P = ctypes.c_void_p
+    h = P(0x1000)
+    args = [h] * 10 + [2, 8, 2, 16, 16, 64, 0.125, 0, 1, -1]
+    assert fn(*args, 65, None) == G.STATUS_CODE["GQA_ERR_SHAPE"]     # chunks > 64
+    assert fn(*args, -1, None) == G.STATUS_CODE["GQA_ERR_SHAPE"]     # chunks < 0
+    bad = [None] + [h] * 9 + [2, 8, 2, 16, 16, 64, 0.125, 0, 1, -1]
+    assert fn(*bad, 2, None) == G.STATUS_CODE["GQA_ERR_NULL"]
+    wrong_d = [h] * 10 + [2, 8, 2, 16, 16, 96, 0.125, 0, 1, -1]
+    assert fn(*wrong_d, 2, None) == G.STATUS_CODE["GQA_ERR_HEADDIM"]
+    empty = [None] * 10 + [0, 8, 2, 16, 16, 64, 0.125, 0, 1, -1]
+    assert fn(*empty, 2, None) == 0                                  # nothing to do

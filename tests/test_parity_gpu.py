@@ -9,7 +9,8 @@ import torch
 
 import oracle
 import workloads as W
-from exact_attention_gqa_b200 import build, gqa_attn, gqa_attn_get_device_error, gqa_attn_plan
+from exact_attention_gqa_b200 import (build, gqa_attn, gqa_attn_get_device_error, gqa_attn_host,
+                                    gqa_attn_plan)
 from parity import compare
 
 pytestmark = pytest.mark.gpu
@@ -116,6 +117,31 @@ def test_decode_sixteen_heads_per_kv_head(splits):
     q, k, v = rand_qkv(2, 32, 2, 1, 3000, 64, seed=93)
     out, lse = run(q, k, v, causal=False, num_splits=splits, pack_gqa=1)
     compare(out, lse, *oracle.attention(q, k, v, scale=1 / math.sqrt(64), causal=False))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal,splits,chunks", [
+    (5, 8, 2, 300, 300, 64, False, 1, 3),     # ragged chunks (2, 2, 1 batch elements)
+    (4, 16, 4, 257, 513, 128, True, 1, 0),    # default chunking, Sq < Sk
+    (6, 32, 8, 1, 3000, 128, False, 4, 4),    # decode, explicit splits per chunk
+    (3, 8, 2, 64, 0, 64, True, 1, 2),         # no keys: zeros and -inf come back
+])
+def test_host_pipeline_equals_device_path(B, Hq, Hkv, Sq, Sk, D, causal, splits, chunks):
+    """gqa_attn_fwd_host (inputs and outputs in pinned host memory, chunked and
+    overlapped) gives exactly the device path's results."""
+    q, k, v = rand_qkv(B, Hq, Hkv, Sq, Sk, D, seed=B * 7 + Sk + D)
+    ref_o, ref_l = run(q, k, v, causal=causal, num_splits=splits)
+    pin = lambda t: t.contiguous().pin_memory()
+    qh, kh, vh = pin(q), pin(k), pin(v)
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(B, Hq, Sq, dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(q, device=DEV), torch.empty_like(k, device=DEV), \
+        torch.empty_like(v, device=DEV)
+    od, ld = torch.empty_like(qd), torch.empty(B, Hq, Sq, dtype=torch.float32, device=DEV)
+    gqa_attn_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal=causal, num_splits=splits,
+                  chunks=chunks)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, ref_o.cpu()) and torch.equal(lh, ref_l.cpu())
+    compare(oh, lh, *oracle.attention(q, k, v, scale=1 / math.sqrt(D), causal=causal))
 
 
 def test_pack_on_and_off_agree():
