@@ -144,6 +144,24 @@ def test_host_pipeline_equals_device_path(B, Hq, Hkv, Sq, Sk, D, causal, splits,
     compare(oh, lh, *oracle.attention(q, k, v, scale=1 / math.sqrt(D), causal=causal))
 
 
+def test_host_pipeline_decode_auto_splits_per_chunk():
+    """Chunks of 3, 3 and 1 batch elements pick different automatic split counts; the
+    workspace covers the largest and every chunk meets the bar."""
+    B, Hq, Hkv, Sk, D = 7, 32, 8, 5000, 128
+    q, k, v = rand_qkv(B, Hq, Hkv, 1, Sk, D, seed=501)
+    pin = lambda t: t.contiguous().pin_memory()
+    qh, kh, vh = pin(q), pin(k), pin(v)
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(B, Hq, 1, dtype=torch.float32).pin_memory()
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    od, ld = torch.empty_like(qd), torch.empty(B, Hq, 1, dtype=torch.float32, device=DEV)
+    splits = {gqa_attn_plan(b, Hq, Hkv, 1, Sk, D, num_splits=0)[2] for b in (3, 1)}
+    assert len(splits) == 2
+    gqa_attn_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, num_splits=0, chunks=3)
+    torch.cuda.synchronize()
+    compare(oh, lh, *oracle.attention(q, k, v, scale=1 / math.sqrt(D), causal=False))
+
+
 def test_pack_on_and_off_agree():
     q, k, v = rand_qkv(2, 16, 4, 333, 333, 128, seed=11)
     a, la = run(q, k, v, causal=True, pack_gqa=1)
