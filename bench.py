@@ -430,15 +430,9 @@ def run_ours(args, world, rank, local):
                             causal=w.causal, num_splits=w.num_splits if case.decode else 1,
                             pack_gqa=w.pack_gqa)
             return
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        kw = dict(causal=w.causal, out=case.out, lse=case.lse, pack_gqa=w.pack_gqa)
         dcu.copy_(cu_h, non_blocking=True)
-        kw.update(cu_seqlens=dcu, max_seqlen=case.max_len)
-        G.gqa_attn(dq, dk, dv, **kw)
-        ho.copy_(case.out, non_blocking=True)
-        hl.copy_(case.lse, non_blocking=True)
+        G.gqa_attn_host(hq, hk, hv, ho, hl, dq, dk, dv, case.out, case.lse, causal=w.causal,
+                        pack_gqa=w.pack_gqa, cu_seqlens=(cu_h, dcu), max_seqlen=case.max_len)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -512,9 +506,10 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms,
-                    "path": ("gqa_attn_fwd_host: pinned host buffers, 8 batch chunks, copy in / "
-                             "attention / copy out overlapped" if not case.varlen else
-                             "pinned host copies + gqa_attn_fwd on one stream")},
+                    "path": ("gqa_attn_fwd_host" + ("_varlen: 8 chunks of whole sequences"
+                                                      if case.varlen else ": 8 batch chunks")
+                             + ", pinned host buffers, copy in / attention / copy out "
+                               "overlapped")},
             "gpu_launches": steps * case.launches_per_step,
             "clocks": clocks.summary(), "device_error": err,
             "kernel_source": kernel_source_hash(), "library": G.library_path()}

@@ -175,7 +175,7 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
 
 def gqa_attn_host(q_h, k_h, v_h, out_h, lse_h, q_d, k_d, v_d, out_d, lse_d, *,
                   causal: bool = False, scale: float | None = None, num_splits: int = 1,
-                  pack_gqa: int = -1, chunks: int = 0):
+                  pack_gqa: int = -1, chunks: int = 0, cu_seqlens=None, max_seqlen=None):
     """Attention on host-resident tensors with the transfers overlapped (gqa_attn_fwd_host).
 
     q_h, k_h, v_h, out_h, lse_h: CPU tensors (pinned for overlap) in the dense layouts of
@@ -185,6 +185,10 @@ def gqa_attn_host(q_h, k_h, v_h, out_h, lse_h, q_d, k_d, v_d, out_d, lse_d, *,
     """
     import torch
 
+    if cu_seqlens is not None:
+        return _gqa_attn_host_varlen(torch, q_h, k_h, v_h, out_h, lse_h, q_d, k_d, v_d, out_d,
+                                     lse_d, causal, scale, pack_gqa, chunks, cu_seqlens,
+                                     max_seqlen)
     B, Sq, Hq, D = q_d.shape
     _, Sk, Hkv, _ = k_d.shape
     for h, d in ((q_h, q_d), (k_h, k_d), (v_h, v_d), (out_h, out_d), (lse_h, lse_d)):
@@ -212,3 +216,32 @@ def gqa_attn_host(q_h, k_h, v_h, out_h, lse_h, q_d, k_d, v_d, out_d, lse_d, *,
             int(bool(causal)), num_splits, pack_gqa, chunks, stream)
     if rc != 0:
         raise GqaError("gqa_attn_fwd_host", rc)
+
+
+def _gqa_attn_host_varlen(torch, q_h, k_h, v_h, out_h, lse_h, q_d, k_d, v_d, out_d, lse_d, causal,
+                          scale, pack_gqa, chunks, cu_seqlens, max_seqlen):
+    """Packed variable-length form; cu_seqlens = (host int32 [B+1], device int32 [B+1])."""
+    cu_h, cu_d = cu_seqlens
+    total, Hq, D = q_d.shape
+    Hkv = k_d.shape[1]
+    B = cu_h.numel() - 1
+    for h, d in ((q_h, q_d), (k_h, k_d), (v_h, v_d), (out_h, out_d), (lse_h, lse_d)):
+        if h.device.type != "cpu" or d.device != q_d.device or h.shape != d.shape or \
+                h.dtype != d.dtype or not h.is_contiguous() or not d.is_contiguous():
+            raise ValueError("host tensors on the CPU and device tensors on one GPU, "
+                             "same shapes and dtypes, contiguous")
+    if cu_h.device.type != "cpu" or cu_h.dtype != torch.int32 or cu_d.dtype != torch.int32 or \
+            cu_d.device != q_d.device or cu_d.numel() != B + 1:
+        raise ValueError("cu_seqlens = (host int32 [B+1], device int32 [B+1])")
+    cu_h = cu_h.contiguous()
+    if max_seqlen is None:
+        max_seqlen = int((cu_h[1:] - cu_h[:-1]).max()) if B > 0 else 0
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    with torch.cuda.device(q_d.device):
+        stream = _stream_handle(torch, q_d.device)
+        rc = _capi.load().gqa_attn_fwd_host_varlen(
+            _ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(out_h), _ptr(lse_h), _ptr(q_d), _ptr(k_d),
+            _ptr(v_d), _ptr(out_d), _ptr(lse_d), _ptr(cu_h), _ptr(cu_d), B, Hq, Hkv,
+            int(max_seqlen), total, D, scale, int(bool(causal)), pack_gqa, chunks, stream)
+    if rc != 0:
+        raise GqaError("gqa_attn_fwd_host_varlen", rc)

@@ -15,6 +15,7 @@ EXPORTS = (
     "gqa_attn_fwd",
     "gqa_attn_fwd_f32",
     "gqa_attn_fwd_host",
+    "gqa_attn_fwd_host_varlen",
     "gqa_attn_workspace_bytes",
     "gqa_attn_set_workspace",
     "gqa_attn_plan",
@@ -58,6 +59,9 @@ def load() -> ctypes.CDLL:
     lib.gqa_attn_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, I,
                                       I, P]
     lib.gqa_attn_fwd_host.restype = I
+    lib.gqa_attn_fwd_host_varlen.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I,
+                                             I, F, I, I, I, P]
+    lib.gqa_attn_fwd_host_varlen.restype = I
     lib.gqa_attn_workspace_bytes.argtypes = [I, I, I, I, I]
     lib.gqa_attn_workspace_bytes.restype = Z
     lib.gqa_attn_set_workspace.argtypes = [P, Z]

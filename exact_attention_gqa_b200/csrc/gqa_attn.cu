@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "gqa_attn.h"
@@ -619,6 +620,102 @@ int gqa_attn_fwd_f32(const void* q, const void* k, const void* v, void* out, flo
 size_t gqa_attn_workspace_bytes(int B, int Hq, int Sq, int D, int num_splits) {
     if (B <= 0 || Hq <= 0 || Sq <= 0 || D <= 0 || num_splits <= 1) return 0;
     return ws_bytes(B, Hq, Sq, D, num_splits);
+}
+
+int gqa_attn_fwd_host_varlen(const void* q_h, const void* k_h, const void* v_h, void* out_h,
+                             float* lse_h, void* q_d, void* k_d, void* v_d, void* out_d,
+                             float* lse_d, const int* cu_seqlens_h, const int* cu_seqlens_d,
+                             int B, int Hq, int Hkv, int max_seqlen, int total, int D,
+                             float scale, int causal, int pack_gqa, int chunks,
+                             cudaStream_t stream) {
+    int rc = check_shape(B, Hq, Hkv, max_seqlen, total, D, scale, 1, pack_gqa, true, false);
+    if (rc != GQA_OK) return rc;
+    if (chunks < 0 || chunks > kMaxChunks) return GQA_ERR_SHAPE;
+    if (B == 0 || max_seqlen == 0 || total == 0) return GQA_OK;
+    if (!cu_seqlens_h || !cu_seqlens_d || !q_h || !k_h || !v_h || !out_h || !lse_h || !q_d ||
+        !k_d || !v_d || !out_d || !lse_d)
+        return GQA_ERR_NULL;
+    // the host offsets must describe the packed rows: 0 = cu[0] <= ... <= cu[B] = total,
+    // no sequence longer than max_seqlen
+    if (cu_seqlens_h[0] != 0 || cu_seqlens_h[B] != total) return GQA_ERR_SHAPE;
+    for (int b = 0; b < B; ++b) {
+        const int len = cu_seqlens_h[b + 1] - cu_seqlens_h[b];
+        if (len < 0 || len > max_seqlen) return GQA_ERR_SHAPE;
+    }
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    Pipe* pp = nullptr;
+    rc = pipe_for_device(&pp);
+    if (rc != GQA_OK) return rc;
+    const int n_target = chunks == 0 ? 8 : chunks;
+    const long long target = ((long long)total + n_target - 1) / n_target;
+    const size_t qrow = size_t(Hq) * D * 2, krow = size_t(Hkv) * D * 2;
+    auto at = [](const void* base, size_t off) {
+        return static_cast<void*>(static_cast<char*>(const_cast<void*>(base)) + off);
+    };
+    if (cudaEventRecord(pp->start, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_in, pp->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_c, pp->start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_out, pp->start, 0) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    int status = GQA_OK;
+    int s0 = 0, c = 0;
+    while (s0 < B && status == GQA_OK) {
+        // whole sequences until the chunk holds about total / chunks rows
+        int s1 = s0 + 1;
+        while (s1 < B && (long long)cu_seqlens_h[s1] - cu_seqlens_h[s0] < target &&
+               B - s1 > 0 && c + 1 < kMaxChunks)
+            ++s1;
+        if (c + 1 == kMaxChunks) s1 = B;  // the last event pair takes the rest
+        const int r0 = cu_seqlens_h[s0], r1 = cu_seqlens_h[s1];
+        int len_max = 0;
+        for (int b = s0; b < s1; ++b)
+            len_max = std::max(len_max, cu_seqlens_h[b + 1] - cu_seqlens_h[b]);
+        const size_t rows = size_t(r1 - r0);
+        if (rows > 0 &&
+            (cudaMemcpyAsync(at(q_d, r0 * qrow), at(q_h, r0 * qrow), rows * qrow,
+                             cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess ||
+             cudaMemcpyAsync(at(k_d, r0 * krow), at(k_h, r0 * krow), rows * krow,
+                             cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess ||
+             cudaMemcpyAsync(at(v_d, r0 * krow), at(v_h, r0 * krow), rows * krow,
+                             cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess)) {
+            status = GQA_ERR_CUDA;
+            break;
+        }
+        if (cudaEventRecord(pp->in_done[c], pp->s_in) != cudaSuccess ||
+            cudaStreamWaitEvent(pp->s_c, pp->in_done[c], 0) != cudaSuccess) {
+            status = GQA_ERR_CUDA;
+            break;
+        }
+        // the chunk's sequences, addressed through the full buffers and the offsets
+        if (len_max > 0) {
+            status = fwd_common(q_d, k_d, v_d, out_d, lse_d, s1 - s0, Hq, Hkv, len_max, total, D,
+                                scale, causal, 1, pack_gqa, cu_seqlens_d + s0, pp->s_c, false);
+            if (status != GQA_OK) break;
+        }
+        if (cudaEventRecord(pp->c_done[c], pp->s_c) != cudaSuccess ||
+            cudaStreamWaitEvent(pp->s_out, pp->c_done[c], 0) != cudaSuccess ||
+            (rows > 0 &&
+             (cudaMemcpyAsync(at(out_h, r0 * qrow), at(out_d, r0 * qrow), rows * qrow,
+                              cudaMemcpyDeviceToHost, pp->s_out) != cudaSuccess ||
+              cudaMemcpy2DAsync(lse_h + r0, size_t(total) * 4, lse_d + r0, size_t(total) * 4,
+                                rows * 4, size_t(Hq), cudaMemcpyDeviceToHost,
+                                pp->s_out) != cudaSuccess)))
+            status = GQA_ERR_CUDA;
+        s0 = s1;
+        ++c;
+    }
+    cudaEvent_t tail_c = pp->c_done[0];
+    if (cudaEventRecord(tail_c, pp->s_c) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_out, tail_c, 0) != cudaSuccess ||
+        cudaEventRecord(pp->in_done[0], pp->s_in) != cudaSuccess ||
+        cudaStreamWaitEvent(pp->s_out, pp->in_done[0], 0) != cudaSuccess ||
+        cudaEventRecord(pp->done, pp->s_out) != cudaSuccess ||
+        cudaStreamWaitEvent(stream, pp->done, 0) != cudaSuccess)
+        status = status == GQA_OK ? GQA_ERR_CUDA : status;
+    return status;
 }
 
 int gqa_attn_set_workspace(void* dev_ptr, size_t bytes) {

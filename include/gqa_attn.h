@@ -132,6 +132,28 @@ int gqa_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o
                       int num_splits, int pack_gqa, int chunks, cudaStream_t stream);
 
 /*
+ * The packed variable-length form of gqa_attn_fwd_host: chunks of whole sequences
+ * (about total / chunks rows each; 0 = 8 chunks) are copied in, computed and copied
+ * back with the same overlap.
+ *   q_h .. lse_h : host buffers, packed layouts of gqa_attn_fwd (q/out [total, Hq, D],
+ *                  k/v [total, Hkv, D], lse [Hq, total]); page-locked for overlap
+ *   q_d .. lse_d : device buffers of the same sizes
+ *   cu_seqlens_h : host int32[B + 1] (0 = cu[0] <= ... <= cu[B] = total), used to cut
+ *                  the chunks; cu_seqlens_d: the same offsets in device memory, read by
+ *                  the kernels
+ *   max_seqlen   : the longest sequence; total: packed rows
+ * Returns gqa_attn_fwd's status codes; GQA_ERR_SHAPE also when cu_seqlens_h does not
+ * describe `total` rows with no sequence longer than max_seqlen, or for chunks < 0 or
+ * > 64.  No counterpart on the pages (see gqa_attn_fwd_host).
+ */
+int gqa_attn_fwd_host_varlen(const void* q_h, const void* k_h, const void* v_h, void* out_h,
+                             float* lse_h, void* q_d, void* k_d, void* v_d, void* out_d,
+                             float* lse_d, const int* cu_seqlens_h, const int* cu_seqlens_d,
+                             int B, int Hq, int Hkv, int max_seqlen, int total, int D,
+                             float scale, int causal, int pack_gqa, int chunks,
+                             cudaStream_t stream);
+
+/*
  * Bytes of device workspace gqa_attn_fwd needs for a split-KV decode with the
  * given sizes and num_splits (0 when num_splits <= 1): fp32 partial outputs
  * [B, Hq, Sq, n, D] and partial log-sum-exps [B, Hq, Sq, n].

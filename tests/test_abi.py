@@ -137,3 +137,21 @@ def test_host_pipeline_argument_errors(lib):
     assert fn(*wrong_d, 2, None) == G.STATUS_CODE["GQA_ERR_HEADDIM"]
     empty = [None] * 10 + [0, 8, 2, 16, 16, 64, 0.125, 0, 1, -1]
     assert fn(*empty, 2, None) == 0                                  # nothing to do
+
+
+def test_host_pipeline_varlen_checks_offsets(lib):
+    """gqa_attn_fwd_host_varlen rejects host offsets that do not describe the rows."""
+    fn = lib.gqa_attn_fwd_host_varlen
+    P = ctypes.c_void_p
+    h = P(0x1000)
+
+    def call(cu, B, max_len, total, chunks=2):
+        arr = (ctypes.c_int * len(cu))(*cu)
+        return fn(*([h] * 10), ctypes.cast(arr, P), h, B, 8, 2, max_len, total, 64, 0.125, 1,
+                  -1, chunks, None)
+
+    assert call([1, 5, 9], 2, 8, 9) == G.STATUS_CODE["GQA_ERR_SHAPE"]      # cu[0] != 0
+    assert call([0, 5, 8], 2, 8, 9) == G.STATUS_CODE["GQA_ERR_SHAPE"]      # cu[B] != total
+    assert call([0, 6, 5], 2, 8, 5) == G.STATUS_CODE["GQA_ERR_SHAPE"]      # decreasing
+    assert call([0, 6, 9], 2, 5, 9) == G.STATUS_CODE["GQA_ERR_SHAPE"]      # longer than max
+    assert call([0, 5, 9], 2, 8, 9, chunks=65) == G.STATUS_CODE["GQA_ERR_SHAPE"]

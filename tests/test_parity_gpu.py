@@ -162,6 +162,34 @@ def test_host_pipeline_decode_auto_splits_per_chunk():
     compare(oh, lh, *oracle.attention(q, k, v, scale=1 / math.sqrt(D), causal=False))
 
 
+@pytest.mark.parametrize("chunks", [0, 3, 64])
+def test_host_pipeline_varlen_equals_device_path(chunks):
+    """gqa_attn_fwd_host_varlen: chunks of whole sequences, exactly the device path."""
+    lengths = [300, 1, 0, 129, 700, 64, 513, 2]
+    Hq, Hkv, D = 16, 4, 128
+    cu = torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32)
+    total = int(cu[-1])
+    g = torch.Generator().manual_seed(606 + chunks)
+    q = torch.randn(total, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(total, Hkv, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(total, Hkv, D, generator=g).to(torch.bfloat16)
+    cu_d = cu.to(DEV)
+    ref_o, ref_l = gqa_attn(q.to(DEV), k.to(DEV), v.to(DEV), causal=True, cu_seqlens=cu_d,
+                            max_seqlen=max(lengths))
+    torch.cuda.synchronize()
+    pin = lambda t: t.contiguous().pin_memory()
+    qh, kh, vh = pin(q), pin(k), pin(v)
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty(Hq, total, dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(q, device=DEV), torch.empty_like(k, device=DEV), \
+        torch.empty_like(v, device=DEV)
+    od, ld = torch.empty_like(qd), torch.empty(Hq, total, dtype=torch.float32, device=DEV)
+    gqa_attn_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal=True, chunks=chunks,
+                  cu_seqlens=(cu, cu_d), max_seqlen=max(lengths))
+    torch.cuda.synchronize()
+    assert torch.equal(oh, ref_o.cpu()) and torch.equal(lh, ref_l.cpu())
+
+
 def test_pack_on_and_off_agree():
     q, k, v = rand_qkv(2, 16, 4, 333, 333, 128, seed=11)
     a, la = run(q, k, v, causal=True, pack_gqa=1)
