@@ -54,6 +54,10 @@ PREFILL = [
     (1, 32, 8, 129, 129, 128, False, 1),
     (2, 16, 1, 64, 1000, 64, True, 1),    # G = 16, long keys, short queries
     (1, 8, 2, 2, 777, 128, True, 1),      # two query rows
+    (1, 32, 1, 200, 200, 128, True, 1),   # MQA, G = 32: 4 positions per packed sub-tile
+    (2, 8, 2, 3, 20000, 64, True, 1),     # 3 queries against 20000 keys (bottom-right)
+    (1, 64, 8, 257, 257, 64, False, 1),   # G = 8 at D = 64, ragged tail
+    (3, 12, 4, 190, 190, 64, True, 0),    # G = 3 without packing, causal, D = 64
 ]
 
 
