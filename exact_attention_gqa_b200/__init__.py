@@ -22,7 +22,7 @@ import math
 from . import _capi
 from ._capi import GqaError, STATUS, STATUS_CODE, strerror
 
-__all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
+__all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_kvcache", "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
            "gqa_attn_workspace_bytes", "gqa_attn_set_workspace", "gqa_attn_get_device_error",
            "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path"]
 
@@ -171,6 +171,87 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
                               stream)
         if rc != 0:
             raise GqaError("gqa_attn_fwd_f32", rc)
+
+
+def gqa_attn_kvcache(q, k_cache, v_cache, *, seqlens_k=None, max_seqlen_k=None,
+                     block_table=None, window: int = 0, scale: float | None = None,
+                     num_splits: int = 0, pack_gqa: int = -1, out=None, lse=None):
+    """One decode step against a KV cache (gqa_attn_decode_kvcache / _paged).
+
+    q [B, 1, Hq, D] bf16.  Dense cache: k_cache/v_cache [B, Sk, Hkv, D].  Paged
+    cache (block_table given, int32 [B, max_pages]): k_cache/v_cache [num_pages,
+    page_size, Hkv, D].  seqlens_k: int32 [B] keys per sequence (required when
+    paged); max_seqlen_k: a host upper bound of it (read from the tensor when not
+    given, which synchronises).  window > 0 keeps the last `window` keys.
+    Returns (out [B, 1, Hq, D], lse [B, Hq, 1]).
+    """
+    import torch
+
+    paged = block_table is not None
+    tensors = [("q", q), ("k_cache", k_cache), ("v_cache", v_cache)]
+    if seqlens_k is not None:
+        tensors.append(("seqlens_k", seqlens_k))
+    if paged:
+        tensors.append(("block_table", block_table))
+    for name, t in tensors:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k_cache.dtype == v_cache.dtype == torch.bfloat16):
+        raise ValueError("q, k_cache, v_cache must be bf16")
+    if q.dim() != 4 or q.shape[1] != 1 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q is [B, 1, Hq, D]; k_cache/v_cache are 4-D and alike")
+    B, _, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    for name, t in (("seqlens_k", seqlens_k), ("block_table", block_table)):
+        if t is not None and t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    if seqlens_k is not None and seqlens_k.shape != (B,):
+        raise ValueError("seqlens_k must be [B]")
+    if paged:
+        if seqlens_k is None:
+            raise ValueError("a paged cache needs seqlens_k")
+        if block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError("block_table must be [B, max_pages]")
+        num_pages, page_size = k_cache.shape[0], k_cache.shape[1]
+        max_pages = block_table.shape[1]
+        cap = max_pages * page_size
+    else:
+        cap = k_cache.shape[1]
+        if k_cache.shape[0] != B:
+            raise ValueError("a dense cache is [B, Sk, Hkv, D]")
+    if seqlens_k is not None and max_seqlen_k is None:
+        max_seqlen_k = int(seqlens_k.max().item()) if B > 0 else 0
+    keys = int(max_seqlen_k) if seqlens_k is not None else cap
+    if window > 0:
+        keys = min(keys, int(window) + 64)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        stream = _stream_handle(torch, q.device)
+        rc, _, splits, _ = gqa_attn_plan(B, Hq, Hkv, 1, keys, D, scale, False, num_splits,
+                                         pack_gqa, False)
+        if rc == 0 and splits > 1:
+            _workspace(torch, q.device, gqa_attn_workspace_bytes(B, Hq, 1, D, splits))
+        msl = int(max_seqlen_k) if seqlens_k is not None else 0
+        if paged:
+            rc = _capi.load().gqa_attn_decode_paged(
+                _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seqlens_k),
+                _ptr(out), _ptr(lse), B, Hq, Hkv, D, num_pages, page_size, max_pages, msl,
+                scale, int(window), num_splits, pack_gqa, stream)
+            name = "gqa_attn_decode_paged"
+        else:
+            rc = _capi.load().gqa_attn_decode_kvcache(
+                _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens_k), _ptr(out), _ptr(lse), B,
+                Hq, Hkv, cap, D, msl, scale, int(window), num_splits, pack_gqa, stream)
+            name = "gqa_attn_decode_kvcache"
+    if rc != 0:
+        raise GqaError(name, rc)
+    return out, lse
 
 
 def gqa_attn_host(q_h, k_h, v_h, out_h, lse_h, q_d, k_d, v_d, out_d, lse_d, *,

@@ -19,6 +19,16 @@
 // pack_gqa = 1 puts the query heads of one KV head (up to 16) in the rows of
 // one CTA so that K/V are read once per group; pack_gqa = 0 gives every query
 // head its own CTA (the group's CTAs then share K/V through L2).
+//
+// KV-cache forms (Ultralytics GQA glossary, "GQA and related techniques"):
+//   - per-sequence cache lengths: sequence b attends to its first seqlens_k[b] keys;
+//   - PagedAttention: the cache is a pool of fixed-size pages [num_pages, page_size,
+//     Hkv, D] and block_table[b][p] names the page that holds keys
+//     [p * page_size, (p + 1) * page_size) of sequence b; a 64-key block is one TMA
+//     copy per page it touches (page_size a power of two >= 16);
+//   - sliding window: the query, the newest position, sees only the last `window`
+//     keys of its sequence (keys j >= L - window of L cached keys).
+// With any of these, each sequence splits its own key range into num_splits parts.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -34,8 +44,15 @@ struct DecodeParams {
     int rows;                // query heads per CTA (1..16)
     int units_per_kv;        // ceil(G / rows)
     int n_splits;
-    int blocks_per_split;    // 64-key blocks per split
+    int blocks_per_split;    // 64-key blocks per split (whole-cache ranges)
     float scale_log2;
+    // KV-cache forms; the defaults give the dense [B, Sk, Hkv, D] cache of Sk keys
+    const int* seqlens_k = nullptr;    // [B] keys per sequence (<= its capacity)
+    const int* block_table = nullptr;  // [B, max_pages] page of each logical page
+    int max_pages = 0;                 // block_table row length
+    int page_shift = 0;                // log2(page_size)
+    int num_pages = 0;                 // pages in the pool
+    int window = 0;                    // > 0: only the last `window` keys
 };
 
 template <int HD>
@@ -103,11 +120,27 @@ __global__ void __launch_bounds__(160, 2)
     const int kvh = unit / p.units_per_kv;
     const int h0 = kvh * p.G + (unit - kvh * p.units_per_kv) * p.rows;
     const int rows = min(p.rows, kvh * p.G + p.G - h0);
-    const int nblk_total = (p.Sk + C::BN - 1) / C::BN;
-    const int blk0 = split * p.blocks_per_split;
-    const int blk1 = min(blk0 + p.blocks_per_split, nblk_total);
+    // this sequence's keys [key_start, len) and this split's 64-key blocks of them
+    const bool paged = p.block_table != nullptr;
+    int len = p.Sk;
+    if (p.seqlens_k) {
+        const int cap = paged ? (p.max_pages << p.page_shift) : p.Sk;
+        len = __ldg(p.seqlens_k + b);
+        if (len < 0 || len > cap) {
+            if (threadIdx.x == 0) raise_device_error(kDevBadKvIndex);
+            len = min(max(len, 0), cap);
+        }
+    }
+    const int key_start = p.window > 0 ? max(len - p.window, 0) : 0;
+    const int kb_first = key_start / C::BN;
+    const int kb_end = (len + C::BN - 1) / C::BN;
+    const bool per_seq = p.seqlens_k != nullptr || p.window > 0;
+    const int bps = per_seq ? (kb_end - kb_first + p.n_splits - 1) / p.n_splits
+                            : p.blocks_per_split;
+    const int blk0 = kb_first + split * bps;
+    const int blk1 = min(blk0 + bps, kb_end);
     const int nblk = max(blk1 - blk0, 0);
-    const int key_end = min(blk1 * C::BN, p.Sk);
+    const int key_end = min(blk1 * C::BN, len);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -144,13 +177,41 @@ __global__ void __launch_bounds__(160, 2)
                 const int s = c % ST;
                 if (!mbar_wait(bar_empty + s, ((c / ST) & 1) ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar_full + s, 2 * C::TILE);
-                const int z = b * p.Sk + (blk0 + c) * C::BN;
+                const int key0 = (blk0 + c) * C::BN;
+                if (!paged) {
+                    const int z = b * p.Sk + key0;
 #pragma unroll
-                for (int a = 0; a < C::ATOMS; ++a) {
-                    tma_load_3d(smem + C::OFF_K + s * C::TILE + a * C::ATOM, &tm_k, bar_full + s,
-                                a * 64, kvh, z);
-                    tma_load_3d(smem + C::OFF_V + s * C::TILE + a * C::ATOM, &tm_v, bar_full + s,
-                                a * 64, kvh, z);
+                    for (int a = 0; a < C::ATOMS; ++a) {
+                        tma_load_3d(smem + C::OFF_K + s * C::TILE + a * C::ATOM, &tm_k,
+                                    bar_full + s, a * 64, kvh, z);
+                        tma_load_3d(smem + C::OFF_V + s * C::TILE + a * C::ATOM, &tm_v,
+                                    bar_full + s, a * 64, kvh, z);
+                    }
+                } else {
+                    // one copy of min(page_size, 64) rows per page the block touches;
+                    // rows land at their key offset, so the 128B swizzle (a function
+                    // of the shared-memory address) matches a single 64-row copy
+                    const int rows = min(1 << p.page_shift, C::BN);
+                    for (int r0 = 0; r0 < C::BN; r0 += rows) {
+                        // rows past the sequence's end are masked: they are read from
+                        // the block's first page (key0 < len) rather than from table
+                        // entries the sequence may not have filled
+                        const int key = (key0 + r0 < len) ? key0 + r0 : key0;
+                        int page = __ldg(p.block_table + size_t(b) * p.max_pages +
+                                         (key >> p.page_shift));
+                        if (page < 0 || page >= p.num_pages) {
+                            raise_device_error(kDevBadKvIndex);
+                            page = 0;
+                        }
+                        const int z = (page << p.page_shift) + (key & ((1 << p.page_shift) - 1));
+#pragma unroll
+                        for (int a = 0; a < C::ATOMS; ++a) {
+                            tma_load_3d(smem + C::OFF_K + s * C::TILE + a * C::ATOM + r0 * 128,
+                                        &tm_k, bar_full + s, a * 64, kvh, z);
+                            tma_load_3d(smem + C::OFF_V + s * C::TILE + a * C::ATOM + r0 * 128,
+                                        &tm_v, bar_full + s, a * 64, kvh, z);
+                        }
+                    }
                 }
             }
             // every issued copy lands before the CTA may reuse or release the memory
@@ -215,13 +276,16 @@ __global__ void __launch_bounds__(160, 2)
                 mma_bf16_16816(sc[0], qa[kk], b0, b1);
                 mma_bf16_16816(sc[1], qa[kk], b2, b3);
             }
-            // mask keys past the end of this split / of the cache
+            // mask keys past the end of this split / of the sequence, and keys
+            // before the window
             const int kbase = (blk0 + c) * C::BN + warp * 16 + qd;
 #pragma unroll
             for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (kbase + t * 8 + (e & 1) >= key_end) sc[t][e] = -INFINITY;
+                for (int e = 0; e < 4; ++e) {
+                    const int key = kbase + t * 8 + (e & 1);
+                    if (key >= key_end || key < key_start) sc[t][e] = -INFINITY;
+                }
             // online softmax (rows g and g + 8), quad reduction of the block max
             float alpha[2];
 #pragma unroll

@@ -272,9 +272,26 @@ int launch_combine(const float* part_o, const float* part_l, __nv_bfloat16* out,
     return GQA_OK;
 }
 
+// KV-cache forms of a decode launch (decode.cuh); the defaults give the dense cache
+struct KvCacheArgs {
+    const int* seqlens_k = nullptr;    // [B] keys per sequence, or null: Sk each
+    const int* block_table = nullptr;  // [B, max_pages], or null: dense [B, Sk, Hkv, D]
+    int max_pages = 0;
+    int page_size = 0;
+    int num_pages = 0;
+    int window = 0;                    // > 0: last `window` keys only
+};
+
+int log2_exact(int x) {
+    int l = 0;
+    while ((1 << l) < x) ++l;
+    return l;
+}
+
 template <int HD>
 int launch_decode(const void* q, const void* k, const void* v, void* out, float* lse, int B,
-                  int Hq, int Hkv, int Sk, float scale, const Plan& pl, cudaStream_t stream) {
+                  int Hq, int Hkv, int Sk, float scale, const Plan& pl, cudaStream_t stream,
+                  const KvCacheArgs& kv = KvCacheArgs()) {
     using C = DecodeCfg<HD>;
     {
         const int rc = ensure_smem_limit(gqa::decode_split_sm100<HD>, HD == 64 ? 4 : 8,
@@ -297,6 +314,12 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     p.scale_log2 = scale * kLog2e;
     p.part_o = nullptr;
     p.part_l = nullptr;
+    p.seqlens_k = kv.seqlens_k;
+    p.block_table = kv.block_table;
+    p.max_pages = kv.max_pages;
+    p.page_shift = kv.block_table ? log2_exact(kv.page_size) : 0;
+    p.num_pages = kv.num_pages;
+    p.window = kv.window;
     if (pl.splits > 1) {
         const size_t need = ws_bytes(B, Hq, 1, HD, pl.splits);
         int dev = 0;
@@ -313,8 +336,12 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
                                             ((o_bytes + 255) / 256) * 256);
     }
     CUtensorMap tk, tv;
-    const long long rows = (long long)B * Sk;
-    if (!make_map(&tk, k, rows, Hkv, HD, 1, C::BN) || !make_map(&tv, v, rows, Hkv, HD, 1, C::BN))
+    // dense: B * Sk rows in 64-row boxes; paged: the pool's rows in boxes of one page
+    // (at most 64 rows)
+    const long long rows = kv.block_table ? (long long)kv.num_pages * kv.page_size
+                                          : (long long)B * Sk;
+    const int box = kv.block_table ? (kv.page_size < C::BN ? kv.page_size : C::BN) : C::BN;
+    if (!make_map(&tk, k, rows, Hkv, HD, 1, box) || !make_map(&tv, v, rows, Hkv, HD, 1, box))
         return GQA_ERR_CUDA;
     dim3 grid(pl.splits, Hkv * pl.decode_units, B);
     gqa::decode_split_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
@@ -325,6 +352,50 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
         if (rc != GQA_OK) return rc;
     }
     return GQA_OK;
+}
+
+// Decode against a KV cache (dense with per-sequence lengths, or paged), with an
+// optional sliding window.  Sk is the dense cache's keys per sequence (its
+// capacity); for the paged form the capacity is max_pages * page_size.
+int kvcache_common(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                   int Hq, int Hkv, int Sk, int D, int max_seqlen_k, float scale,
+                   const KvCacheArgs& kv, int num_splits, int pack_gqa, cudaStream_t stream) {
+    const bool paged = kv.block_table != nullptr;
+    if (B < 0 || Sk < 0 || max_seqlen_k < 0 || kv.window < 0) return GQA_ERR_SHAPE;
+    if (paged) {
+        if (kv.page_size < 16 || (kv.page_size & (kv.page_size - 1)) != 0 ||
+            kv.num_pages < 1 || kv.max_pages < 1 || !kv.seqlens_k)
+            return kv.seqlens_k ? GQA_ERR_SHAPE : GQA_ERR_NULL;
+        if ((long long)kv.num_pages * kv.page_size > INT32_MAX ||
+            (long long)kv.max_pages * kv.page_size > INT32_MAX)
+            return GQA_ERR_SHAPE;
+        Sk = kv.max_pages * kv.page_size;  // per-sequence capacity
+    }
+    if (max_seqlen_k > Sk) return GQA_ERR_SHAPE;
+    if (!paged && (long long)B * Sk > INT32_MAX) return GQA_ERR_SHAPE;  // 32-bit TMA rows
+    // keys one sequence can touch: its length, or the window plus a partial block
+    int keys = kv.seqlens_k ? max_seqlen_k : Sk;
+    if (kv.window > 0 && keys > kv.window + 64) keys = kv.window + 64;
+    int rc = check_shape(B, Hq, Hkv, 1, keys, D, scale, num_splits, pack_gqa, false, false);
+    if (rc != GQA_OK) return rc;
+    if (B == 0) return GQA_OK;
+    if (!q || !out || !lse || (keys > 0 && (!k || !v))) return GQA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || !aligned(kv.seqlens_k, 4) || !aligned(kv.block_table, 4))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    Plan pl;
+    make_plan(&pl, B, Hq, Hkv, 1, keys, num_splits, pack_gqa, false, dev->sms);
+    if (pl.kernel == kZeroFill) {
+        gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(out), (long long)B * Hq * D, lse, (long long)B * Hq);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
+    if (pl.kernel != kDecode) return GQA_OK;
+    return D == 128 ? launch_decode<128>(q, k, v, out, lse, B, Hq, Hkv, Sk, scale, pl, stream, kv)
+                    : launch_decode<64>(q, k, v, out, lse, B, Hq, Hkv, Sk, scale, pl, stream, kv);
 }
 
 int fwd_common(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
@@ -820,6 +891,34 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
                                                 scratch, stream);
 }
 
+
+int gqa_attn_decode_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                            const int* seqlens_k, void* out, float* lse, int B, int Hq, int Hkv,
+                            int Sk, int D, int max_seqlen_k, float scale, int window,
+                            int num_splits, int pack_gqa, cudaStream_t stream) {
+    KvCacheArgs kv;
+    kv.seqlens_k = seqlens_k;
+    kv.window = window;
+    return kvcache_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Sk, D,
+                          seqlens_k ? max_seqlen_k : Sk, scale, kv, num_splits, pack_gqa, stream);
+}
+
+int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                          const int* block_table, const int* seqlens_k, void* out, float* lse,
+                          int B, int Hq, int Hkv, int D, int num_pages, int page_size,
+                          int max_pages, int max_seqlen_k, float scale, int window,
+                          int num_splits, int pack_gqa, cudaStream_t stream) {
+    if (!block_table) return GQA_ERR_NULL;
+    KvCacheArgs kv;
+    kv.seqlens_k = seqlens_k;
+    kv.block_table = block_table;
+    kv.max_pages = max_pages;
+    kv.page_size = page_size;
+    kv.num_pages = num_pages;
+    kv.window = window;
+    return kvcache_common(q, k_pages, v_pages, out, lse, B, Hq, Hkv, 0, D, max_seqlen_k, scale,
+                          kv, num_splits, pack_gqa, stream);
+}
 
 int gqa_attn_selftest_timeout(int limit_ms, cudaStream_t stream) {
     if (limit_ms < 1 || limit_ms > 1000) return GQA_ERR_SHAPE;

@@ -14,6 +14,7 @@ enum DeviceError : int {
     kDevOk = 0,
     kDevWaitTimeout = 1,   // an mbarrier wait exceeded its time limit
     kDevBadTile = 2,       // a work tile decoded outside the problem
+    kDevBadKvIndex = 3,    // a cache length or page index outside the cache
 };
 __device__ int g_device_error = 0;
 

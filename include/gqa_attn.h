@@ -184,7 +184,7 @@ int gqa_attn_plan(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, in
 /*
  * Read and clear the device error word on `stream` (synchronises that stream).
  * *host_code: 0 none, 1 a pipeline wait timed out, 2 a packed sequence is longer
- * than the Sq that was passed.
+ * than the Sq that was passed, 3 a KV-cache length or page index outside the cache.
  */
 int gqa_attn_get_device_error(int* host_code, cudaStream_t stream);
 
@@ -226,6 +226,62 @@ int gqa_attn_get_device_error(int* host_code, cudaStream_t stream);
 int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* out,
                             float* lse, int B, int Hq, int Hkv, int Sk, int D, float scale,
                             int num_splits, int pack_gqa, cudaStream_t stream);
+
+/*
+ * Decode (one new query position per sequence) against a KV cache, with per-
+ * sequence cache lengths and an optional sliding window.  Ultralytics glossary
+ * "Grouped Query Attention (GQA)": during generation the model keeps the keys and
+ * values of every earlier token in the KV cache and reads all of it for each new
+ * token ("How GQA shrinks the KV cache"); sliding-window attention caps the tokens
+ * each layer attends to ("GQA and related techniques").
+ *
+ * For sequence b with L = seqlens_k[b] cached keys (seqlens_k NULL: L = Sk for
+ * every sequence) and query head h, with c = h / (Hq / Hkv):
+ *   keys j in [j0, L), j0 = max(0, L - window) if window > 0, else 0;
+ *   out[b, h, :] = sum_j softmax_j(scale * q[b,h,:] . k[b,j,c,:]) v[b,j,c,:]
+ *   lse[b, h]    = ln sum_j exp(scale * q[b,h,:] . k[b,j,c,:])
+ * A sequence with no key (L = 0) gets out = 0 and lse = -inf.
+ *
+ * Layouts (device pointers, caller-owned, bf16 unless noted):
+ *   q, out [B, 1, Hq, D]; lse [B, Hq, 1] fp32;
+ *   k_cache, v_cache [B, Sk, Hkv, D]: Sk keys of capacity per sequence, the first
+ *     L of them valid;
+ *   seqlens_k: NULL or device int32 [B] with 0 <= seqlens_k[b] <= Sk; a value
+ *     outside that range raises device error 3 and is clamped.
+ * max_seqlen_k (host): an upper bound of seqlens_k (<= Sk), used to choose
+ *   num_splits; ignored when seqlens_k is NULL.  window >= 0 (0: every key).
+ * num_splits (0 = automatic, from min(max_seqlen_k, window + 64) keys) and
+ *   pack_gqa as for gqa_attn_fwd's decode; each sequence divides its own key range
+ *   into the splits.  D 64 or 128.  Nothing is allocated or synchronised; with
+ *   num_splits > 1 the registered workspace must hold
+ *   gqa_attn_workspace_bytes(B, Hq, 1, D, num_splits).
+ * Returns gqa_attn_fwd's status codes (GQA_ERR_SHAPE also for window < 0,
+ *   max_seqlen_k > Sk).
+ */
+int gqa_attn_decode_kvcache(const void* q, const void* k_cache, const void* v_cache,
+                            const int* seqlens_k, void* out, float* lse, int B, int Hq, int Hkv,
+                            int Sk, int D, int max_seqlen_k, float scale, int window,
+                            int num_splits, int pack_gqa, cudaStream_t stream);
+
+/*
+ * The same decode against a paged KV cache (PagedAttention, Ultralytics glossary
+ * "GQA and related techniques": the cache is allocated in fixed-size blocks).
+ *   k_pages, v_pages [num_pages, page_size, Hkv, D]: a pool of pages;
+ *   block_table: device int32 [B, max_pages]; key j of sequence b is row
+ *     j % page_size of page block_table[b * max_pages + j / page_size];
+ *   seqlens_k: device int32 [B] (required), 0 <= seqlens_k[b] <= max_pages *
+ *     page_size.  Only the table entries of pages holding keys j < seqlens_k[b]
+ *     are read; an entry outside [0, num_pages) raises device error 3 and page 0
+ *     is read in its place.
+ *   page_size: a power of two >= 16; num_pages * page_size < 2^31.
+ * Everything else (window, max_seqlen_k <= max_pages * page_size, num_splits,
+ * pack_gqa, q/out/lse layouts, workspace, errors) as gqa_attn_decode_kvcache.
+ */
+int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                          const int* block_table, const int* seqlens_k, void* out, float* lse,
+                          int B, int Hq, int Hkv, int D, int num_pages, int page_size,
+                          int max_pages, int max_seqlen_k, float scale, int window,
+                          int num_splits, int pack_gqa, cudaStream_t stream);
 
 /*
  * Diagnostic: exercises the kernels' bounded-wait path.  Launches one warp that

@@ -18,6 +18,10 @@ states the passage of the pages it follows in the C source:
                           log-sum-exp weighted combine.
 * ``attention_tiled``  -- the per-step normalised (form 1) and deferred
                           normalisation (form 2) online-softmax forms.
+* ``decode_kvcache``   -- one decode query per sequence against a dense or paged
+                          KV cache with per-sequence lengths and a sliding window
+                          (Ultralytics GQA glossary, KV-cache and related-techniques
+                          sections).
 
 Every function takes float32 numpy arrays (bf16 and fp32 values widen exactly)
 and returns float64 arrays.
@@ -45,6 +49,8 @@ FLAWS = {
     "lse_no_max": 5,
     "fa1_no_rescale": 6,
     "swap_kv": 7,
+    "pages_contiguous": 8,
+    "window_short": 9,
 }
 
 
@@ -76,6 +82,9 @@ def _load():
         lib.oracle_combine.restype = None
         lib.oracle_attention_tiled.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, I, I,
                                                I]
+        lib.oracle_decode_kvcache.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I,
+                                              Dbl, I]
+        lib.oracle_decode_kvcache.restype = I
         lib.oracle_set_flaw.argtypes = [I]
         lib.oracle_set_flaw.restype = None
         lib.oracle_get_flaw.restype = I
@@ -195,3 +204,36 @@ def attention_tiled(q, k, v, *, scale: float, causal: bool, Bm: int, Bn: int, fo
     if rc != 0:
         raise ValueError("oracle_attention_tiled: bad arguments")
     return o, lse
+
+
+def decode_kvcache(q, k_cache, v_cache, *, scale: float, seqlens_k=None, block_table=None,
+                   window: int = 0, threads: int = 0):
+    """Decode against a KV cache.  q [B, 1, Hq, D] or [B, Hq, D]; dense k/v_cache
+    [B, Sk, Hkv, D] or paged [num_pages, page_size, Hkv, D] with block_table
+    [B, max_pages].  Returns (O float64 [B, Hq, D], L float64 [B, Hq])."""
+    q, k, v = _f32(q), _f32(k_cache), _f32(v_cache)
+    B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
+    Hkv = k.shape[2]
+    sl = None if seqlens_k is None else np.ascontiguousarray(_np_int(seqlens_k), dtype=np.int32)
+    bt = None if block_table is None else np.ascontiguousarray(_np_int(block_table),
+                                                                dtype=np.int32)
+    if bt is None:
+        Sk, page_size, max_pages, num_pages = k.shape[1], 0, 0, 0
+    else:
+        Sk, page_size, max_pages, num_pages = 0, k.shape[1], bt.shape[1], k.shape[0]
+    o = np.zeros((B, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq), dtype=np.float64)
+    rc = _load().oracle_decode_kvcache(_ptr(q), _ptr(k), _ptr(v),
+                                       None if bt is None else _ptr(bt),
+                                       None if sl is None else _ptr(sl), _ptr(o), _ptr(lse), B,
+                                       Hq, Hkv, D, Sk, page_size, max_pages, num_pages,
+                                       int(window), float(scale), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_decode_kvcache: bad arguments")
+    return o, lse
+
+
+def _np_int(a):
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").numpy()
+    return a

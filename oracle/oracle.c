@@ -36,6 +36,15 @@
  * Inputs are float32 (bf16 and fp32 values widen to float64 exactly); every
  * arithmetic step is float64.
  *
+ * KV-cache decode (oracle_decode_kvcache): Ultralytics glossary "Grouped Query
+ * Attention (GQA)" -- the KV cache holds the keys and values of every earlier
+ * token and each new token reads all of it ("How GQA shrinks the KV cache");
+ * PagedAttention stores that cache in fixed-size blocks and sliding-window
+ * attention caps the tokens attended to ("GQA and related techniques").  Readings:
+ * key j of sequence b lives in row j % page_size of page block_table[b][j /
+ * page_size]; with a window W > 0 the query (the newest position) attends to the
+ * last W of the L cached keys, j >= L - W.
+ *
  * Return value of every entry point: 0 on success, -1 on bad arguments.
  */
 #include <math.h>
@@ -59,6 +68,8 @@ enum {
     FLAW_LSE_NO_MAX = 5,      /* L = log(l) without adding the max back        */
     FLAW_FA1_NO_RESCALE = 6,  /* tiled FA-1 form drops exp(m_old - m_new)      */
     FLAW_SWAP_KV = 7,         /* uses K where V belongs in O = P V             */
+    FLAW_PAGES_CONTIGUOUS = 8,/* paged cache read as if pages were in order     */
+    FLAW_WINDOW_SHORT = 9,    /* sliding window keeps one key too few           */
 };
 static int g_flaw = FLAW_NONE;
 void oracle_set_flaw(int flaw) { g_flaw = flaw; }
@@ -362,6 +373,109 @@ void oracle_combine(int n, int D, const double* Os, const double* Ls, double* O,
         for (int d = 0; d < D; ++d) O[d] += w * Os[(size_t)s * D + d];
     }
     *L = Lall;
+}
+
+/*
+ * One decode query per sequence against a KV cache, by the plain definition.
+ *   q [B, Hq, D]; o [B, Hq, D]; lse [B, Hq].
+ *   dense (block_table NULL): k_cache, v_cache [B, Sk, Hkv, D];
+ *   paged: k_cache, v_cache [num_pages, page_size, Hkv, D], block_table
+ *     [B, max_pages];
+ *   seqlens_k [B] keys per sequence, or NULL: Sk each (dense only);
+ *   window > 0: keys j in [max(0, L - window), L), else [0, L).
+ * For each (b, h): s_j = scale * q . k_j over those keys, m = max s_j,
+ * p_j = exp(s_j - m), l = sum p_j, O = sum p_j v_j / l, L = m + ln l; no key:
+ * O = 0, L = -inf.
+ */
+int oracle_decode_kvcache(const float* q, const float* k_cache, const float* v_cache,
+                          const int32_t* block_table, const int32_t* seqlens_k, double* o,
+                          double* lse, int B, int Hq, int Hkv, int D, int Sk, int page_size,
+                          int max_pages, int num_pages, int window, double scale, int nthreads)
+{
+    if (!q || !k_cache || !v_cache || !o || !lse) return -1;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0 || window < 0) return -1;
+    const int paged = block_table != NULL;
+    int cap = Sk;
+    if (paged) {
+        if (!seqlens_k || page_size <= 0 || max_pages <= 0 || num_pages <= 0) return -1;
+        cap = max_pages * page_size;
+    } else if (Sk < 0) {
+        return -1;
+    }
+    for (int b = 0; b < B; ++b) {
+        const int L = seqlens_k ? seqlens_k[b] : Sk;
+        if (L < 0 || L > cap) return -1;
+        if (paged)
+            for (int pg = 0; pg < (L + page_size - 1) / page_size; ++pg) {
+                const int32_t e = block_table[(size_t)b * max_pages + pg];
+                if (e < 0 || e >= num_pages) return -1;
+            }
+    }
+    set_threads(nthreads);
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            const int L = seqlens_k ? seqlens_k[b] : Sk;
+            int j0 = 0;
+            if (window > 0) {
+                j0 = L - window;
+                if (g_flaw == FLAW_WINDOW_SHORT) j0 += 1;
+                if (j0 < 0) j0 = 0;
+            }
+            const int c = kv_head_of(h, Hq, Hkv);
+            const float* qv = q + ((size_t)b * Hq + h) * D;
+            double* ob = o + ((size_t)b * Hq + h) * D;
+            double* row = (L > j0) ? malloc(sizeof(double) * (size_t)(L - j0)) : NULL;
+            if (L > j0 && !row) {
+                bad = 1;
+                continue;
+            }
+            /* row index of key j in the cache arrays */
+            size_t* kr = (L > j0) ? malloc(sizeof(size_t) * (size_t)(L - j0)) : NULL;
+            if (L > j0 && !kr) {
+                free(row);
+                bad = 1;
+                continue;
+            }
+            for (int j = j0; j < L; ++j) {
+                size_t r;
+                if (!paged)
+                    r = (size_t)b * Sk + j;
+                else if (g_flaw == FLAW_PAGES_CONTIGUOUS)
+                    r = (size_t)b * max_pages * page_size + j;
+                else
+                    r = (size_t)block_table[(size_t)b * max_pages + j / page_size] * page_size +
+                        (size_t)(j % page_size);
+                kr[j - j0] = r;
+            }
+            double m = -INFINITY;
+            for (int j = j0; j < L; ++j) {
+                const float* kj = k_cache + (kr[j - j0] * Hkv + c) * (size_t)D;
+                row[j - j0] = scale * dot(qv, kj, D);
+                if (row[j - j0] > m) m = row[j - j0];
+            }
+            if (L <= j0) {
+                for (int d = 0; d < D; ++d) ob[d] = 0.0;
+                lse[(size_t)b * Hq + h] = -INFINITY;
+                continue;
+            }
+            double l = 0.0;
+            for (int j = j0; j < L; ++j) {
+                row[j - j0] = exp(row[j - j0] - m);
+                l += row[j - j0];
+            }
+            for (int d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int j = j0; j < L; ++j)
+                    acc += row[j - j0] * (double)v_cache[(kr[j - j0] * Hkv + c) * (size_t)D + d];
+                ob[d] = acc / l;
+            }
+            lse[(size_t)b * Hq + h] = m + log(l);
+            free(row);
+            free(kr);
+        }
+    return bad ? -1 : 0;
 }
 
 /*

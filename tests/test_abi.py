@@ -155,3 +155,56 @@ def test_host_pipeline_varlen_checks_offsets(lib):
     assert call([0, 6, 5], 2, 8, 5) == G.STATUS_CODE["GQA_ERR_SHAPE"]      # decreasing
     assert call([0, 6, 9], 2, 5, 9) == G.STATUS_CODE["GQA_ERR_SHAPE"]      # longer than max
     assert call([0, 5, 9], 2, 8, 9, chunks=65) == G.STATUS_CODE["GQA_ERR_SHAPE"]
+
+
+def kv_call(lib, *, q=FAKE, k=FAKE, v=FAKE, sl=None, out=FAKE, lse=FAKE, B=2, Hq=8, Hkv=2,
+            Sk=100, D=64, msl=0, scale=0.125, window=0, splits=0, pack=-1):
+    return lib.gqa_attn_decode_kvcache(q, k, v, sl, out, lse, B, Hq, Hkv, Sk, D, msl, scale,
+                                       window, splits, pack, None)
+
+
+def paged_call(lib, *, q=FAKE, k=FAKE, v=FAKE, bt=FAKE, sl=FAKE, out=FAKE, lse=FAKE, B=2, Hq=8,
+               Hkv=2, D=64, num_pages=10, page_size=64, max_pages=4, msl=100, scale=0.125,
+               window=0, splits=0, pack=-1):
+    return lib.gqa_attn_decode_paged(q, k, v, bt, sl, out, lse, B, Hq, Hkv, D, num_pages,
+                                     page_size, max_pages, msl, scale, window, splits, pack, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), "GQA_ERR_NULL"),
+    (dict(k=None), "GQA_ERR_NULL"),
+    (dict(window=-1), "GQA_ERR_SHAPE"),
+    (dict(sl=FAKE, msl=101), "GQA_ERR_SHAPE"),        # bound above the capacity
+    (dict(B=70000, Sk=40000), "GQA_ERR_SHAPE"),       # rows past 32-bit TMA coordinates
+    (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
+    (dict(D=96), "GQA_ERR_HEADDIM"),
+    (dict(scale=0.0), "GQA_ERR_SCALE"),
+    (dict(splits=257), "GQA_ERR_SPLITS"),
+    (dict(pack=2), "GQA_ERR_UNSUPPORTED"),
+    (dict(q=ctypes.c_void_p(0x1008)), "GQA_ERR_ALIGN"),
+    (dict(sl=ctypes.c_void_p(0x1002), msl=10), "GQA_ERR_ALIGN"),
+])
+def test_kvcache_argument_errors(lib, kw, code):
+    assert G.STATUS[kv_call(lib, **kw)] == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bt=None), "GQA_ERR_NULL"),
+    (dict(sl=None), "GQA_ERR_NULL"),
+    (dict(page_size=48), "GQA_ERR_SHAPE"),            # not a power of two
+    (dict(page_size=8), "GQA_ERR_SHAPE"),             # below 16
+    (dict(num_pages=0), "GQA_ERR_SHAPE"),
+    (dict(max_pages=0), "GQA_ERR_SHAPE"),
+    (dict(msl=257), "GQA_ERR_SHAPE"),                 # past max_pages * page_size
+    (dict(num_pages=1 << 22, page_size=1024), "GQA_ERR_SHAPE"),
+    (dict(window=-5), "GQA_ERR_SHAPE"),
+    (dict(D=32), "GQA_ERR_HEADDIM"),
+    (dict(bt=ctypes.c_void_p(0x1002)), "GQA_ERR_ALIGN"),
+])
+def test_paged_argument_errors(lib, kw, code):
+    assert G.STATUS[paged_call(lib, **kw)] == code
+
+
+def test_kvcache_empty_batch_is_a_noop(lib):
+    assert kv_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert paged_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0

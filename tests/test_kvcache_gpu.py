@@ -1,0 +1,145 @@
+"""GPU parity of the KV-cache decode entry points against the float64 oracle.
+
+gqa_attn_decode_kvcache (dense cache, per-sequence lengths) and
+gqa_attn_decode_paged (a pool of fixed-size pages and a block table), both with an
+optional sliding window (Ultralytics GQA glossary, "How GQA shrinks the KV cache"
+and "GQA and related techniques").  Inputs are seeded; ragged lengths include 0,
+block and page multiples; unused block-table entries hold -1 so that reading one
+would show as a device error."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_gqa_b200 import build, gqa_attn_get_device_error, gqa_attn_kvcache
+from parity import compare
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    yield
+    torch.cuda.synchronize()
+    assert gqa_attn_get_device_error() == 0
+
+
+def make_cache(B, Hq, Hkv, Sk, D, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, 1, Hq, D, generator=g).bfloat16()
+    k = torch.randn(B, Sk, Hkv, D, generator=g).bfloat16()
+    v = torch.randn(B, Sk, Hkv, D, generator=g).bfloat16()
+    return q, k, v
+
+
+def to_pages(k, v, lens, page_size, seed, spare=5):
+    """Scatter each sequence's first lens[b] keys into a shuffled pool of pages.
+    Table entries past a sequence's last page are -1; unused rows hold noise."""
+    B, Sk, Hkv, D = k.shape
+    max_pages = -(-Sk // page_size)
+    used = [-(-int(n) // page_size) for n in lens]
+    num_pages = sum(used) + spare
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(num_pages, generator=g)
+    kp = (torch.randn(num_pages, page_size, Hkv, D, generator=g) * 3).bfloat16()
+    vp = (torch.randn(num_pages, page_size, Hkv, D, generator=g) * 3).bfloat16()
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b in range(B):
+        for pg in range(used[b]):
+            phys = int(perm[nxt])
+            nxt += 1
+            table[b, pg] = phys
+            j0, j1 = pg * page_size, min((pg + 1) * page_size, int(lens[b]))
+            kp[phys, : j1 - j0] = k[b, j0:j1]
+            vp[phys, : j1 - j0] = v[b, j0:j1]
+    return kp, vp, table
+
+
+def check(out, lse, o_ref, l_ref):
+    compare(out[:, 0], lse[:, :, 0], o_ref, l_ref)
+
+
+LENS = [0, 1, 63, 64, 65, 1500, 2999, 3000]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("window", [0, 1, 100, 2000])
+@pytest.mark.parametrize("splits,pack", [(1, 1), (3, 1), (0, 1), (0, 0)])
+def test_dense_cache_with_lengths(D, window, splits, pack):
+    B, Hq, Hkv, Sk = len(LENS), 32, 8, 3000
+    q, k, v = make_cache(B, Hq, Hkv, Sk, D, seed=D + window + splits)
+    lens = torch.tensor(LENS, dtype=torch.int32)
+    out, lse = gqa_attn_kvcache(q.to(DEV), k.to(DEV), v.to(DEV), seqlens_k=lens.to(DEV),
+                                max_seqlen_k=Sk, window=window, num_splits=splits,
+                                pack_gqa=pack)
+    torch.cuda.synchronize()
+    check(out, lse, *oracle.decode_kvcache(q, k, v, scale=1 / math.sqrt(D), seqlens_k=lens,
+                                           window=window))
+
+
+def test_dense_cache_without_lengths_equals_the_dense_decode():
+    from exact_attention_gqa_b200 import gqa_attn
+    q, k, v = make_cache(3, 16, 4, 1234, 128, seed=5)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    out, lse = gqa_attn_kvcache(qd, kd, vd, num_splits=4)
+    ref_o, ref_l = gqa_attn(qd, kd, vd, num_splits=4)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_o) and torch.equal(lse, ref_l)
+
+
+@pytest.mark.parametrize("page_size", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("window,splits", [(0, 1), (0, 0), (300, 4), (17, 0)])
+def test_paged_cache(page_size, D, window, splits):
+    B, Hq, Hkv, Sk = len(LENS), 16, 4, 3000
+    q, k, v = make_cache(B, Hq, Hkv, Sk, D, seed=page_size + D + window)
+    kp, vp, table = to_pages(k, v, LENS, page_size, seed=page_size * 3 + D)
+    lens = torch.tensor(LENS, dtype=torch.int32)
+    out, lse = gqa_attn_kvcache(q.to(DEV), kp.to(DEV), vp.to(DEV), seqlens_k=lens.to(DEV),
+                                block_table=table.to(DEV), window=window, num_splits=splits)
+    torch.cuda.synchronize()
+    ref = oracle.decode_kvcache(q, kp, vp, scale=1 / math.sqrt(D), seqlens_k=lens,
+                                block_table=table.clamp(min=0), window=window)
+    check(out, lse, *ref)
+    # the same logical cache through the dense entry point
+    dense = oracle.decode_kvcache(q, k, v, scale=1 / math.sqrt(D), seqlens_k=lens, window=window)
+    np.testing.assert_allclose(ref[0], dense[0], rtol=0, atol=1e-12)
+
+
+def test_paged_sixteen_heads_per_kv_head_many_splits():
+    B, Hq, Hkv, Sk, D = 3, 32, 2, 5000, 128
+    lens = [5000, 4097, 1]
+    q, k, v = make_cache(B, Hq, Hkv, Sk, D, seed=11)
+    kp, vp, table = to_pages(k, v, lens, 64, seed=12)
+    tl = torch.tensor(lens, dtype=torch.int32)
+    out, lse = gqa_attn_kvcache(q.to(DEV), kp.to(DEV), vp.to(DEV), seqlens_k=tl.to(DEV),
+                                block_table=table.to(DEV), num_splits=40)
+    torch.cuda.synchronize()
+    check(out, lse, *oracle.decode_kvcache(q, kp, vp, scale=1 / math.sqrt(D), seqlens_k=tl,
+                                           block_table=table.clamp(min=0)))
+
+
+def test_bad_page_and_length_raise_device_error_without_faulting():
+    B, Hq, Hkv, Sk, D = 2, 8, 2, 200, 64
+    q, k, v = make_cache(B, Hq, Hkv, Sk, D, seed=21)
+    lens = [200, 100]
+    kp, vp, table = to_pages(k, v, lens, 64, seed=22)
+    table[1, 0] = kp.shape[0] + 3  # a page that is not in the pool
+    tl = torch.tensor(lens, dtype=torch.int32)
+    out, _ = gqa_attn_kvcache(q.to(DEV), kp.to(DEV), vp.to(DEV), seqlens_k=tl.to(DEV),
+                              block_table=table.to(DEV))
+    torch.cuda.synchronize()
+    assert gqa_attn_get_device_error() == 3
+    assert torch.isfinite(out.float()).all()
+    # a length past the dense cache's capacity is clamped and reported the same way
+    tl2 = torch.tensor([Sk + 5, 3], dtype=torch.int32)
+    gqa_attn_kvcache(q.to(DEV), k.to(DEV), v.to(DEV), seqlens_k=tl2.to(DEV), max_seqlen_k=Sk)
+    torch.cuda.synchronize()
+    assert gqa_attn_get_device_error() == 3
+    assert gqa_attn_get_device_error() == 0

@@ -382,6 +382,104 @@ def test_combine_of_empty_partials():
 
 
 # ---------------------------------------------------------------------------------
+# KV-cache decode: per-sequence lengths, paged storage, sliding window (Ultralytics
+# GQA glossary, "How GQA shrinks the KV cache" and "GQA and related techniques")
+
+def scatter_to_pages(k, v, page_size, seed, spare=3):
+    """Dense caches [B, Sk, Hkv, D] -> a shuffled pool of pages and its block table.
+    Rows no sequence owns hold unrelated values, so a wrong row shows."""
+    B, Sk, Hkv, D = k.shape
+    max_pages = -(-Sk // page_size)
+    num_pages = B * max_pages + spare
+    rng = np.random.default_rng(seed)
+    table = rng.permutation(num_pages)[: B * max_pages].reshape(B, max_pages).astype(np.int32)
+    kp = rnd((num_pages, page_size, Hkv, D), seed + 1, 3.0)
+    vp = rnd((num_pages, page_size, Hkv, D), seed + 2, 3.0)
+    for b in range(B):
+        for pg in range(max_pages):
+            j0, j1 = pg * page_size, min((pg + 1) * page_size, Sk)
+            kp[table[b, pg], : j1 - j0] = k[b, j0:j1]
+            vp[table[b, pg], : j1 - j0] = v[b, j0:j1]
+    return kp, vp, table
+
+
+def kv_sdpa(q, k, v, lens, window, scale):
+    """torch float64 SDPA over each sequence's visible keys, cut from the dense cache."""
+    B, _, Hq, D = q.shape
+    O = np.zeros((B, Hq, D))
+    L = np.zeros((B, Hq))
+    for b in range(B):
+        j1 = int(lens[b])
+        j0 = max(0, j1 - window) if window > 0 else 0
+        if j1 <= j0:
+            L[b] = -np.inf
+            continue
+        o, l = sdpa_ref(q[b:b + 1], k[b:b + 1, j0:j1], v[b:b + 1, j0:j1], scale, False)
+        O[b] = o[0, 0]
+        L[b] = l[0, :, 0]
+    return O, L
+
+
+def assert_kv_close(O, L, Or, Lr):
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isneginf(L), np.isneginf(Lr))
+    fin = np.isfinite(Lr)
+    np.testing.assert_allclose(L[fin], Lr[fin], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", [0, 1, 7, 64, 1000])
+def test_kvcache_lengths_and_window_match_sdpa_on_slices(window):
+    B, Hq, Hkv, Sk, D = 5, 8, 2, 90, 32
+    q, k, v = rnd((B, 1, Hq, D), 40), rnd((B, Sk, Hkv, D), 41), rnd((B, Sk, Hkv, D), 42)
+    lens = np.array([0, 1, 37, 89, 90], dtype=np.int32)
+    O, L = oracle.decode_kvcache(q, k, v, scale=0.2, seqlens_k=lens, window=window)
+    assert_kv_close(O, L, *kv_sdpa(q, k, v, lens, window, 0.2))
+
+
+def test_kvcache_without_lengths_reads_the_whole_cache():
+    B, Hq, Hkv, Sk, D = 2, 6, 3, 21, 8
+    q, k, v = rnd((B, 1, Hq, D), 50), rnd((B, Sk, Hkv, D), 51), rnd((B, Sk, Hkv, D), 52)
+    O, L = oracle.decode_kvcache(q, k, v, scale=0.3)
+    assert_kv_close(O, L, *kv_sdpa(q, k, v, np.full(B, Sk), 0, 0.3))
+
+
+@pytest.mark.parametrize("page_size,window", [(1, 0), (3, 5), (16, 0), (16, 20), (64, 0)])
+def test_kvcache_paged_matches_sdpa(page_size, window):
+    B, Hq, Hkv, Sk, D = 4, 8, 4, 75, 16
+    q, k, v = rnd((B, 1, Hq, D), 60), rnd((B, Sk, Hkv, D), 61), rnd((B, Sk, Hkv, D), 62)
+    lens = np.array([75, 0, 17, 64], dtype=np.int32)
+    kp, vp, table = scatter_to_pages(k, v, page_size, 63)
+    O, L = oracle.decode_kvcache(q, kp, vp, scale=0.25, seqlens_k=lens, block_table=table,
+                                 window=window)
+    assert_kv_close(O, L, *kv_sdpa(q, k, v, lens, window, 0.25))
+
+
+def test_kvcache_window_of_one_returns_the_newest_value():
+    # a single visible key: its value comes out unchanged and L is its logit
+    B, Hq, Hkv, Sk, D = 3, 4, 2, 12, 8
+    q, k, v = rnd((B, 1, Hq, D), 70), rnd((B, Sk, Hkv, D), 71), rnd((B, Sk, Hkv, D), 72)
+    lens = np.array([12, 5, 1], dtype=np.int32)
+    O, L = oracle.decode_kvcache(q, k, v, scale=0.5, seqlens_k=lens, window=1)
+    for b in range(B):
+        for h in range(Hq):
+            c = h // (Hq // Hkv)
+            j = lens[b] - 1
+            np.testing.assert_array_equal(O[b, h], v[b, j, c].astype(np.float64))
+            expect = 0.5 * float(np.dot(q[b, 0, h].astype(np.float64), k[b, j, c].astype(np.float64)))
+            assert abs(L[b, h] - expect) < 1e-12
+
+
+def test_kvcache_rejects_bad_lengths_and_pages():
+    q, k, v = rnd((1, 1, 2, 4), 80), rnd((1, 8, 1, 4), 81), rnd((1, 8, 1, 4), 82)
+    with pytest.raises(ValueError):
+        oracle.decode_kvcache(q, k, v, scale=1.0, seqlens_k=np.array([9], np.int32))
+    with pytest.raises(ValueError):
+        # 12 keys in pages of 8 use both table entries; page 5 is not in the pool of 1
+        oracle.decode_kvcache(q, k, v, scale=1.0, seqlens_k=np.array([12], np.int32),
+                              block_table=np.array([[0, 5]], np.int32))
+
+
+# ---------------------------------------------------------------------------------
 # Pin strength: every planted mistake is caught by at least one pin above
 
 PIN_BATTERY = [
@@ -392,6 +490,8 @@ PIN_BATTERY = [
     lambda: test_brute_force_50_digits(True, 4, 4),
     lambda: test_tiled_forms_equal_full_matrix(7, 5, 1, True, 37, 37),
     lambda: test_equal_keys_average_the_visible_values(),
+    lambda: test_kvcache_lengths_and_window_match_sdpa_on_slices(7),
+    lambda: test_kvcache_paged_matches_sdpa(16, 0),
 ]
 
 
