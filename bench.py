@@ -6,7 +6,8 @@ One step is one forward pass (gqa_attn_fwd through the C ABI) over one batch of 
 workload, with the inputs already resident in HBM.  The default workload is the
 encoder-shaped GQA batch (B=64, Hq=48, Hkv=12, S=512, D=64, bf16, non-causal);
 others: llama (B=4, Hq=32, Hkv=8, S=8192, D=128, causal), llama_stress (q x 4),
-decode_b{1,16,64,128,256} (Sq=1, Sk=32768, split-KV), varlen (32 packed causal
+decode_b{1,16,64,128,256} (Sq=1, Sk=32768, split-KV), decode_paged_bN (the same
+cache in shuffled pages of 256 keys, gqa_attn_kvcache), varlen (32 packed causal
 sequences of 128..8192 tokens).  Prefill workloads report TFLOP/s, decode GB/s.
 
 Under torchrun every rank runs its own copy of the workload (independent batches,
@@ -175,6 +176,8 @@ def workload_by_name(name: str):
         return W.VARLEN
     if name.startswith("decode_b"):
         return W.decode(int(name[len("decode_b"):]), num_splits=0)
+    if name.startswith("decode_paged_b"):
+        return W.decode_paged(int(name[len("decode_paged_b"):]))
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -188,13 +191,20 @@ class Case:
         self.device = device
         self.decode = w.Sq == 1
         self.varlen = bool(w.varlen)
+        self.paged = w.page_size > 0
         if self.decode:
             q = W.make_decode_q(w, device=device)
             # rotate several KV copies when one is not larger than L2
             kv_bytes = W.kv_cache_bytes(w.B, w.Sk, w.Hkv, w.D)
             n_copies = 1 if kv_bytes > 2 * L2_BYTES else 3
             self.kv = []
+            if self.paged:
+                self.table = W.page_table(w).to(device)
+                self.lens = torch.full((w.B,), w.Sk, dtype=torch.int32, device=device)
             for c in range(n_copies):
+                if self.paged:
+                    self.kv.append(W.make_paged_kv(w, self.table, device=device))
+                    continue
                 k = torch.empty(w.B, w.Sk, w.Hkv, w.D, dtype=torch.bfloat16, device=device)
                 v = torch.empty_like(k)
                 W.fill_decode_kv(w, k, v)
@@ -249,6 +259,11 @@ class Case:
         k, v = self.kv[self.i % len(self.kv)]
         self.i += 1
         w = self.w
+        if self.paged:
+            self.G.gqa_attn_kvcache(self.q, k, v, seqlens_k=self.lens, max_seqlen_k=w.Sk,
+                                    block_table=self.table, num_splits=w.num_splits,
+                                    pack_gqa=w.pack_gqa, out=self.out, lse=self.lse)
+            return
         kw = dict(causal=w.causal, out=self.out, lse=self.lse, pack_gqa=w.pack_gqa)
         if self.decode:
             kw["num_splits"] = w.num_splits
@@ -289,6 +304,22 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
     import oracle
     rng = np.random.default_rng(seed)
     cores = oracle.max_threads()
+    if w.Sq == 1 and w.page_size > 0:
+        import dataclasses
+        w1 = dataclasses.replace(w, B=1)
+        table = W.page_table(w1)
+        kp, vp = W.make_paged_kv(w1, table)
+        q = W.make_decode_q(w1)
+        lens = np.full(1, w.Sk, dtype=np.int32)
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.decode_kvcache(q, kp, vp, scale=w.scale, seqlens_k=lens, block_table=table)
+            el += time.perf_counter() - t0
+            n += 1
+        gb = n * W.decode_bytes(1, w.Hq, w.Hkv, w.Sk, w.D) / 1e9
+        return gb / el, (f"{n} x one sequence through its block table (all {w.Hq} heads, "
+                         f"Sk={w.Sk}, pages of {w.page_size})"), cores, el
     if w.Sq == 1:
         k, v = W.make_decode_kv_one(w, 0)
         q = W.make_decode_q(W.decode(1))
@@ -422,7 +453,22 @@ def run_ours(args, world, rank, local):
     cu_h = case.cu.cpu().pin_memory() if case.varlen else None
     dcu = torch.empty_like(case.cu) if case.varlen else None
 
+    if case.paged:
+        ht = case.table.cpu().pin_memory()
+        hs = case.lens.cpu().pin_memory()
+        dt, ds = torch.empty_like(case.table), torch.empty_like(case.lens)
+
     def e2e_step():
+        if case.paged:
+            # the public KV-cache call on inputs copied in from pinned host memory
+            for d, h in ((dq, hq), (dk, hk), (dv, hv), (dt, ht), (ds, hs)):
+                d.copy_(h, non_blocking=True)
+            G.gqa_attn_kvcache(dq, dk, dv, seqlens_k=ds, max_seqlen_k=w.Sk, block_table=dt,
+                               num_splits=w.num_splits, pack_gqa=w.pack_gqa, out=case.out,
+                               lse=case.lse)
+            ho.copy_(case.out, non_blocking=True)
+            hl.copy_(case.lse, non_blocking=True)
+            return
         if not case.varlen:
             # the public host-buffer entry point: batch chunks with copy in, attention and
             # copy out overlapped on the library's streams
@@ -447,7 +493,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     h2d = hq.numel() * hq.element_size() + hk.numel() * 2 + hv.numel() * 2 + \
-        (cu_h.numel() * 4 if cu_h is not None else 0)
+        (cu_h.numel() * 4 if cu_h is not None else 0) + \
+        ((ht.numel() + hs.numel()) * 4 if case.paged else 0)
     d2h = ho.numel() * 2 + hl.numel() * 4
     err = G.gqa_attn_get_device_error()
     if world > 1:
@@ -498,6 +545,9 @@ def run_ours(args, world, rank, local):
                       else "K back-to-back calls")}
     if case.varlen:
         cfg["total_tokens"] = int(case.q.shape[0])
+    if case.paged:
+        cfg["page_size"] = w.page_size
+        cfg["block_table"] = "seeded shuffle of the page pool"
     line = {"metric": METRIC, "value": value, "unit": case.unit, "n_gpus": world,
             "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -506,8 +556,11 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms,
-                    "path": ("gqa_attn_fwd_host" + ("_varlen: 8 chunks of whole sequences"
-                                                      if case.varlen else ": 8 batch chunks")
+                    "path": ("gqa_attn_kvcache on the paged cache after pinned host "
+                             "copies of q, the page pools, the block table and the lengths; "
+                             "results copied back" if case.paged else
+                             "gqa_attn_fwd_host" + ("_varlen: 8 chunks of whole sequences"
+                                                    if case.varlen else ": 8 batch chunks")
                              + ", pinned host buffers, copy in / attention / copy out "
                                "overlapped")},
             "gpu_launches": steps * case.launches_per_step,

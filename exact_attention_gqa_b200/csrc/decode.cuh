@@ -100,7 +100,9 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
     return uint32_t(row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
-template <int HD>
+// PAGED = true reads K and V through p.block_table; the dense instantiation carries
+// none of that code.
+template <int HD, bool PAGED = false>
 __global__ void __launch_bounds__(160, 2)
     decode_split_sm100(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(160, 2)
     const int h0 = kvh * p.G + (unit - kvh * p.units_per_kv) * p.rows;
     const int rows = min(p.rows, kvh * p.G + p.G - h0);
     // this sequence's keys [key_start, len) and this split's 64-key blocks of them
-    const bool paged = p.block_table != nullptr;
+    constexpr bool paged = PAGED;
     int len = p.Sk;
     if (p.seqlens_k) {
         const int cap = paged ? (p.max_pages << p.page_shift) : p.Sk;
@@ -172,8 +174,27 @@ __global__ void __launch_bounds__(160, 2)
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
+            // paged: the pages of block c + 1 are looked up while block c is issued,
+            // so the table read never sits between a free stage and its copies
+            const int rows = paged ? min(1 << p.page_shift, C::BN) : C::BN;
+            const int* trow = paged ? p.block_table + size_t(b) * p.max_pages : nullptr;
+            int pg_cur[4] = {0, 0, 0, 0}, pg_nxt[4] = {0, 0, 0, 0};
+            auto lookup = [&](int blk, int (&pg)[4]) {
+                const int key0 = blk * C::BN;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if (i * rows >= C::BN) break;
+                    // rows past the sequence's end are masked: they are read from the
+                    // block's first page (key0 < len) rather than from table entries the
+                    // sequence may not have filled
+                    const int key = (key0 + i * rows < len) ? key0 + i * rows : key0;
+                    pg[i] = __ldg(trow + (key >> p.page_shift));
+                }
+            };
+            if (paged && nblk > 0) lookup(blk0, pg_cur);
             int c = 0;
             for (; c < nblk; ++c) {
+                if (paged && c + 1 < nblk) lookup(blk0 + c + 1, pg_nxt);
                 const int s = c % ST;
                 if (!mbar_wait(bar_empty + s, ((c / ST) & 1) ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(bar_full + s, 2 * C::TILE);
@@ -191,14 +212,12 @@ __global__ void __launch_bounds__(160, 2)
                     // one copy of min(page_size, 64) rows per page the block touches;
                     // rows land at their key offset, so the 128B swizzle (a function
                     // of the shared-memory address) matches a single 64-row copy
-                    const int rows = min(1 << p.page_shift, C::BN);
-                    for (int r0 = 0; r0 < C::BN; r0 += rows) {
-                        // rows past the sequence's end are masked: they are read from
-                        // the block's first page (key0 < len) rather than from table
-                        // entries the sequence may not have filled
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        if (i * rows >= C::BN) break;
+                        const int r0 = i * rows;
                         const int key = (key0 + r0 < len) ? key0 + r0 : key0;
-                        int page = __ldg(p.block_table + size_t(b) * p.max_pages +
-                                         (key >> p.page_shift));
+                        int page = pg_cur[i];
                         if (page < 0 || page >= p.num_pages) {
                             raise_device_error(kDevBadKvIndex);
                             page = 0;
@@ -212,6 +231,8 @@ __global__ void __launch_bounds__(160, 2)
                                         &tm_v, bar_full + s, a * 64, kvh, z);
                         }
                     }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) pg_cur[i] = pg_nxt[i];
                 }
             }
             // every issued copy lands before the CTA may reuse or release the memory
@@ -277,15 +298,18 @@ __global__ void __launch_bounds__(160, 2)
                 mma_bf16_16816(sc[1], qa[kk], b2, b3);
             }
             // mask keys past the end of this split / of the sequence, and keys
-            // before the window
-            const int kbase = (blk0 + c) * C::BN + warp * 16 + qd;
+            // before the window (only blocks that straddle one of those edges)
+            const int kblk = (blk0 + c) * C::BN;
+            if (kblk + C::BN > key_end || kblk < key_start) {
+                const int kbase = kblk + warp * 16 + qd;
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+                for (int t = 0; t < 2; ++t)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = kbase + t * 8 + (e & 1);
-                    if (key >= key_end || key < key_start) sc[t][e] = -INFINITY;
-                }
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = kbase + t * 8 + (e & 1);
+                        if (key >= key_end || key < key_start) sc[t][e] = -INFINITY;
+                    }
+            }
             // online softmax (rows g and g + 8), quad reduction of the block max
             float alpha[2];
 #pragma unroll

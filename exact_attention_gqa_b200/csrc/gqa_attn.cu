@@ -344,7 +344,14 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     if (!make_map(&tk, k, rows, Hkv, HD, 1, box) || !make_map(&tv, v, rows, Hkv, HD, 1, box))
         return GQA_ERR_CUDA;
     dim3 grid(pl.splits, Hkv * pl.decode_units, B);
-    gqa::decode_split_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    if (kv.block_table) {
+        const int rc = ensure_smem_limit(gqa::decode_split_sm100<HD, true>, HD == 64 ? 16 : 32,
+                                         C::SMEM_BYTES);
+        if (rc != GQA_OK) return rc;
+        gqa::decode_split_sm100<HD, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    } else {
+        gqa::decode_split_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    }
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
     if (pl.splits > 1) {
         const int rows_bh = B * Hq;

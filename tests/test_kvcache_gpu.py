@@ -143,3 +143,28 @@ def test_bad_page_and_length_raise_device_error_without_faulting():
     torch.cuda.synchronize()
     assert gqa_attn_get_device_error() == 3
     assert gqa_attn_get_device_error() == 0
+
+
+def test_full_paged_decode_workload():
+    """The benchmark's paged decode (B=16, Sk=32768, shuffled pages of 256 keys, automatic
+    splits), whole, on the GPU; three sequences checked against the oracle, also with a
+    4096-key window."""
+    import workloads as W
+    w = W.decode_paged(16)
+    table = W.page_table(w).to(DEV)
+    kp, vp = W.make_paged_kv(w, table, device=DEV)
+    q = W.make_decode_q(w, device=DEV)
+    lens = torch.full((w.B,), w.Sk, dtype=torch.int32, device=DEV)
+    rng = np.random.default_rng(16)
+    bs = sorted({0, w.B - 1, int(rng.integers(w.B))})
+    for window in (0, 4096):
+        out, lse = gqa_attn_kvcache(q, kp, vp, seqlens_k=lens, max_seqlen_k=w.Sk,
+                                    block_table=table, window=window)
+        torch.cuda.synchronize()
+        assert torch.isfinite(out.float()).all()
+        for b in bs:
+            idx = table[b].long()
+            kb = kp[idx].reshape(1, w.Sk, w.Hkv, w.D).cpu()
+            vb = vp[idx].reshape(1, w.Sk, w.Hkv, w.D).cpu()
+            ref = oracle.decode_kvcache(q[b:b + 1].cpu(), kb, vb, scale=w.scale, window=window)
+            check(out[b:b + 1], lse[b:b + 1], *ref)

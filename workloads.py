@@ -44,6 +44,7 @@ class Workload:
     pack_gqa: int = 1
     num_splits: int = 1
     varlen: dict = field(default_factory=dict)  # {"n": 32, "lo": 128, "hi": 8192}
+    page_size: int = 0  # > 0: decode against a paged KV cache of pages of this many keys
 
     @property
     def scale(self) -> float:
@@ -75,6 +76,14 @@ def decode(B: int, num_splits: int = 1, pack_gqa: int = 1) -> Workload:
     return Workload(f"decode_b{B}_sk32768_n{num_splits}_pack{pack_gqa}", B=B, Hq=32, Hkv=8,
                     Sq=1, Sk=32768, D=128, dtype="bf16", causal=False, seed=4,
                     pack_gqa=pack_gqa, num_splits=num_splits)
+
+
+def decode_paged(B: int, page_size: int = 256) -> Workload:
+    """The decode workload with its cache stored in shuffled pages (PagedAttention,
+    Ultralytics GQA glossary, "GQA and related techniques")."""
+    return Workload(f"decode_paged_b{B}_sk32768_p{page_size}", B=B, Hq=32, Hkv=8, Sq=1,
+                    Sk=32768, D=128, dtype="bf16", causal=False, seed=4, pack_gqa=1,
+                    num_splits=0, page_size=page_size)
 
 
 VARLEN = Workload("varlen32_len128to8192_causal", B=32, Hq=32, Hkv=8, Sq=0, Sk=0, D=128,
@@ -153,6 +162,29 @@ def fill_decode_kv(w: Workload, k_out: torch.Tensor, v_out: torch.Tensor) -> Non
         kb, vb = make_decode_kv_one(w, b, device=k_out.device)
         k_out[b].copy_(kb)
         v_out[b].copy_(vb)
+
+
+def page_table(w: Workload) -> torch.Tensor:
+    """Block table int32 [B, Sk / page_size]: a seeded shuffle of the page pool, so
+    consecutive keys of a sequence sit in scattered pages."""
+    per = w.Sk // w.page_size
+    g = _gen("cpu", w.seed + 7)
+    return torch.randperm(w.B * per, generator=g).to(torch.int32).reshape(w.B, per)
+
+
+def make_paged_kv(w: Workload, table: torch.Tensor, device="cpu"):
+    """Page pools k/v [B * Sk / page_size, page_size, Hkv, D] holding batch element
+    b's cache (the same values as the dense decode workload) in pages table[b]."""
+    per = w.Sk // w.page_size
+    shape = (w.B * per, w.page_size, w.Hkv, w.D)
+    kp = torch.empty(shape, dtype=w.torch_dtype, device=device)
+    vp = torch.empty(shape, dtype=w.torch_dtype, device=device)
+    idx = table.to(device=device, dtype=torch.int64)
+    for b in range(w.B):
+        kb, vb = make_decode_kv_one(w, b, device=device)
+        kp[idx[b]] = kb.view(per, w.page_size, w.Hkv, w.D)
+        vp[idx[b]] = vb.view(per, w.page_size, w.Hkv, w.D)
+    return kp, vp
 
 
 # ----------------------------------------------------------------------------------
