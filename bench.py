@@ -178,6 +178,8 @@ def workload_by_name(name: str):
         return W.decode(int(name[len("decode_b"):]), num_splits=0)
     if name.startswith("decode_paged_b"):
         return W.decode_paged(int(name[len("decode_paged_b"):]))
+    if name.startswith("decode_fp8_b"):
+        return W.decode_fp8(int(name[len("decode_fp8_b"):]))
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -205,7 +207,8 @@ class Case:
                 if self.paged:
                     self.kv.append(W.make_paged_kv(w, self.table, device=device))
                     continue
-                k = torch.empty(w.B, w.Sk, w.Hkv, w.D, dtype=torch.bfloat16, device=device)
+                k = torch.empty(w.B, w.Sk, w.Hkv, w.D, device=device,
+                                dtype=torch.float8_e4m3fn if w.kv_fp8 else torch.bfloat16)
                 v = torch.empty_like(k)
                 W.fill_decode_kv(w, k, v)
                 self.kv.append((k, v))
@@ -213,8 +216,14 @@ class Case:
             rc, kern, splits, pack = G.gqa_attn_plan(w.B, w.Hq, w.Hkv, 1, w.Sk, w.D,
                                                      num_splits=w.num_splits,
                                                      pack_gqa=w.pack_gqa)
+            if w.kv_fp8 and w.num_splits == 0:
+                # the e4m3 path's own automatic count: two CTAs per SM (whole waves)
+                sms = torch.cuda.get_device_properties(device).multi_processor_count
+                ctas = w.B * w.Hkv * (1 if pack else w.G)
+                splits = max(1, min(64, (2 * sms) // ctas, max(1, (w.Sk // 64) // 4)))
             self.splits, self.pack = splits, pack
-            self.bytes = W.decode_bytes(w.B, w.Hq, w.Hkv, w.Sk, w.D)
+            self.bytes = W.decode_bytes(w.B, w.Hq, w.Hkv, w.Sk, w.D,
+                                        kv_elt=1 if w.kv_fp8 else 2)
             self.flops = W.attention_flops(w.B, w.Hq, 1, w.Sk, w.D, False)
             self.units, self.unit = self.bytes / 1e9, "GB/s"
             self.launches_per_step = 2 if splits > 1 else 1
@@ -250,7 +259,7 @@ class Case:
 
     def in_bytes(self):
         k, v = self.kv[0]
-        return self.q.numel() * 2 + k.numel() * 2 + v.numel() * 2
+        return self.q.numel() * 2 + k.numel() * k.element_size() + v.numel() * v.element_size()
 
     def out_bytes(self):
         return self.out.numel() * 2 + self.lse.numel() * 4
@@ -259,6 +268,11 @@ class Case:
         k, v = self.kv[self.i % len(self.kv)]
         self.i += 1
         w = self.w
+        if w.kv_fp8:
+            self.G.gqa_attn_kvcache(self.q, k, v, k_scale=W.FP8_SCALE, v_scale=W.FP8_SCALE,
+                                    num_splits=w.num_splits, pack_gqa=w.pack_gqa, out=self.out,
+                                    lse=self.lse)
+            return
         if self.paged:
             self.G.gqa_attn_kvcache(self.q, k, v, seqlens_k=self.lens, max_seqlen_k=w.Sk,
                                     block_table=self.table, num_splits=w.num_splits,
@@ -320,6 +334,21 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
         gb = n * W.decode_bytes(1, w.Hq, w.Hkv, w.Sk, w.D) / 1e9
         return gb / el, (f"{n} x one sequence through its block table (all {w.Hq} heads, "
                          f"Sk={w.Sk}, pages of {w.page_size})"), cores, el
+    if w.Sq == 1 and w.kv_fp8:
+        kb, vb = W.make_decode_kv_one(w, 0)
+        k8 = (kb.float() / W.FP8_SCALE).to(torch.float8_e4m3fn)[None]
+        v8 = (vb.float() / W.FP8_SCALE).to(torch.float8_e4m3fn)[None]
+        q = W.make_decode_q(W.decode(1))
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.decode_kvcache(q, k8, v8, scale=w.scale, k_scale=W.FP8_SCALE,
+                                  v_scale=W.FP8_SCALE)
+            el += time.perf_counter() - t0
+            n += 1
+        gb = n * W.decode_bytes(1, w.Hq, w.Hkv, w.Sk, w.D, kv_elt=1) / 1e9
+        return gb / el, (f"{n} x one batch element of the e4m3 cache (all {w.Hq} heads, "
+                         f"Sk={w.Sk})"), cores, el
     if w.Sq == 1:
         k, v = W.make_decode_kv_one(w, 0)
         q = W.make_decode_q(W.decode(1))
@@ -459,6 +488,15 @@ def run_ours(args, world, rank, local):
         dt, ds = torch.empty_like(case.table), torch.empty_like(case.lens)
 
     def e2e_step():
+        if w.kv_fp8:
+            for d, h in ((dq, hq), (dk, hk), (dv, hv)):
+                d.copy_(h, non_blocking=True)
+            G.gqa_attn_kvcache(dq, dk, dv, k_scale=W.FP8_SCALE, v_scale=W.FP8_SCALE,
+                               num_splits=w.num_splits, pack_gqa=w.pack_gqa, out=case.out,
+                               lse=case.lse)
+            ho.copy_(case.out, non_blocking=True)
+            hl.copy_(case.lse, non_blocking=True)
+            return
         if case.paged:
             # the public KV-cache call on inputs copied in from pinned host memory
             for d, h in ((dq, hq), (dk, hk), (dv, hv), (dt, ht), (ds, hs)):
@@ -492,7 +530,8 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
-    h2d = hq.numel() * hq.element_size() + hk.numel() * 2 + hv.numel() * 2 + \
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + \
+        hv.numel() * hv.element_size() + \
         (cu_h.numel() * 4 if cu_h is not None else 0) + \
         ((ht.numel() + hs.numel()) * 4 if case.paged else 0)
     d2h = ho.numel() * 2 + hl.numel() * 4
@@ -545,6 +584,8 @@ def run_ours(args, world, rank, local):
                       else "K back-to-back calls")}
     if case.varlen:
         cfg["total_tokens"] = int(case.q.shape[0])
+    if w.kv_fp8:
+        cfg["kv_cache"] = f"e4m3 codes, k_scale = v_scale = {W.FP8_SCALE}"
     if case.paged:
         cfg["page_size"] = w.page_size
         cfg["block_table"] = "seeded shuffle of the page pool"
@@ -556,7 +597,9 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms,
-                    "path": ("gqa_attn_kvcache on the paged cache after pinned host "
+                    "path": ("gqa_attn_kvcache on the e4m3 cache after pinned host copies "
+                             "of q and the caches; results copied back" if w.kv_fp8 else
+                             "gqa_attn_kvcache on the paged cache after pinned host "
                              "copies of q, the page pools, the block table and the lengths; "
                              "results copied back" if case.paged else
                              "gqa_attn_fwd_host" + ("_varlen: 8 chunks of whole sequences"

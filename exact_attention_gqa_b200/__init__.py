@@ -175,15 +175,17 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
 
 def gqa_attn_kvcache(q, k_cache, v_cache, *, seqlens_k=None, max_seqlen_k=None,
                      block_table=None, window: int = 0, scale: float | None = None,
-                     num_splits: int = 0, pack_gqa: int = -1, out=None, lse=None):
-    """One decode step against a KV cache (gqa_attn_decode_kvcache / _paged).
+                     num_splits: int = 0, pack_gqa: int = -1, k_scale: float | None = None,
+                     v_scale: float | None = None, out=None, lse=None):
+    """One decode step against a KV cache (gqa_attn_decode_kvcache / _paged / _fp8).
 
     q [B, 1, Hq, D] bf16.  Dense cache: k_cache/v_cache [B, Sk, Hkv, D].  Paged
     cache (block_table given, int32 [B, max_pages]): k_cache/v_cache [num_pages,
     page_size, Hkv, D].  seqlens_k: int32 [B] keys per sequence (required when
     paged); max_seqlen_k: a host upper bound of it (read from the tensor when not
     given, which synchronises).  window > 0 keeps the last `window` keys.
-    Returns (out [B, 1, Hq, D], lse [B, Hq, 1]).
+    An e4m3 cache (torch.float8_e4m3fn or uint8 codes) needs k_scale and v_scale: the
+    stored value is code * scale.  Returns (out [B, 1, Hq, D], lse [B, Hq, 1]).
     """
     import torch
 
@@ -198,8 +200,17 @@ def gqa_attn_kvcache(q, k_cache, v_cache, *, seqlens_k=None, max_seqlen_k=None,
             raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
-    if not (q.dtype == k_cache.dtype == v_cache.dtype == torch.bfloat16):
-        raise ValueError("q, k_cache, v_cache must be bf16")
+    fp8_types = (torch.uint8, getattr(torch, "float8_e4m3fn", torch.uint8))
+    fp8 = k_cache.dtype in fp8_types
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bf16")
+    if fp8:
+        if v_cache.dtype not in fp8_types:
+            raise ValueError("k_cache and v_cache must both be e4m3 (or both bf16)")
+        if k_scale is None or v_scale is None:
+            raise ValueError("an e4m3 cache needs k_scale and v_scale")
+    elif not (k_cache.dtype == v_cache.dtype == torch.bfloat16):
+        raise ValueError("k_cache, v_cache must be bf16 or e4m3")
     if q.dim() != 4 or q.shape[1] != 1 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
         raise ValueError("q is [B, 1, Hq, D]; k_cache/v_cache are 4-D and alike")
     B, _, Hq, D = q.shape
@@ -235,10 +246,20 @@ def gqa_attn_kvcache(q, k_cache, v_cache, *, seqlens_k=None, max_seqlen_k=None,
         stream = _stream_handle(torch, q.device)
         rc, _, splits, _ = gqa_attn_plan(B, Hq, Hkv, 1, keys, D, scale, False, num_splits,
                                          pack_gqa, False)
+        if fp8 and num_splits == 0:
+            splits = 64  # the e4m3 path picks its own count, at most 64
         if rc == 0 and splits > 1:
             _workspace(torch, q.device, gqa_attn_workspace_bytes(B, Hq, 1, D, splits))
         msl = int(max_seqlen_k) if seqlens_k is not None else 0
-        if paged:
+        if fp8:
+            rc = _capi.load().gqa_attn_decode_fp8(
+                _ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale),
+                _ptr(block_table), _ptr(seqlens_k), _ptr(out), _ptr(lse), B, Hq, Hkv, D,
+                0 if paged else cap, num_pages if paged else 0, page_size if paged else 0,
+                max_pages if paged else 0, msl if (paged or seqlens_k is not None) else cap,
+                scale, int(window), num_splits, pack_gqa, stream)
+            name = "gqa_attn_decode_fp8"
+        elif paged:
             rc = _capi.load().gqa_attn_decode_paged(
                 _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), _ptr(seqlens_k),
                 _ptr(out), _ptr(lse), B, Hq, Hkv, D, num_pages, page_size, max_pages, msl,

@@ -24,6 +24,7 @@ EXPORTS = (
     "gqa_attn_decode_noalloc",
     "gqa_attn_decode_kvcache",
     "gqa_attn_decode_paged",
+    "gqa_attn_decode_fp8",
     "gqa_attn_selftest_timeout",
 )
 
@@ -78,6 +79,9 @@ def load() -> ctypes.CDLL:
     lib.gqa_attn_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,
                                           I, P]
     lib.gqa_attn_decode_paged.restype = I
+    lib.gqa_attn_decode_fp8.argtypes = [P, P, P, F, F, P, P, P, P, I, I, I, I, I, I, I, I, I, F,
+                                        I, I, I, P]
+    lib.gqa_attn_decode_fp8.restype = I
     lib.gqa_attn_selftest_timeout.argtypes = [I, P]
     lib.gqa_attn_selftest_timeout.restype = I
     lib.gqa_attn_strerror.argtypes = [I]

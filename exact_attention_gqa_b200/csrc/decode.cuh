@@ -29,7 +29,18 @@
 //   - sliding window: the query, the newest position, sees only the last `window`
 //     keys of its sequence (keys j >= L - window of L cached keys).
 // With any of these, each sequence splits its own key range into num_splits parts.
+//
+// FP8 cache (KV8): K and V stored as e4m3 with one scale each per tensor.  The 8-bit
+// tiles land by TMA in an unswizzled ring; each consumer warp converts its own 16
+// keys of K and V to f16 in a swizzled buffer of its own, frees the stage, and runs
+// the f16 form of the same MMAs (q is rounded to f16 once, P is packed as f16).  Every
+// e4m3 value is an f16 value, so the conversion is exact; the K scale is folded into
+// the softmax scale, O is multiplied by the V scale.  (An integer form of the
+// conversion, shifting the byte into f16 bit positions, measured no faster: it frees
+// the conversion unit but doubles the instructions per element.)
 #pragma once
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 
 namespace gqa {
@@ -53,6 +64,7 @@ struct DecodeParams {
     int page_shift = 0;                // log2(page_size)
     int num_pages = 0;                 // pages in the pool
     int window = 0;                    // > 0: only the last `window` keys
+    float v_scale = 1.f;               // e4m3 cache: value of one V code unit
 };
 
 template <int HD>
@@ -71,6 +83,62 @@ struct DecodeCfg {
         (OFF_MISC + 16 > MERGE_BYTES ? OFF_MISC + 16 : MERGE_BYTES) + 1024;
     static constexpr int THREADS = 160;
 };
+
+// e4m3 K/V: 8-bit stages (rows of HD bytes, no swizzle) and per-warp f16 copies of the
+// warp's 16 keys in the 128B-swizzled layout the ldmatrix addressing expects
+template <int HD>
+struct DecodeCfg8 {
+    static constexpr int BN = 64;
+    static constexpr int TILE = BN * HD;        // bytes of K (or V) per stage
+    static constexpr int STAGES = 4;
+    static constexpr int WATOM = 16 * 128;      // a warp's 16 keys x 64 dims in f16
+    static constexpr int WTILE = 16 * HD * 2;   // a warp's 16 keys, all dims, f16
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = STAGES * TILE;
+    static constexpr int OFF_W = 2 * STAGES * TILE;  // [4 warps][K, V][WTILE]
+    static constexpr int OFF_BAR = OFF_W + 4 * 2 * WTILE;
+    static constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
+    static constexpr int MERGE_BYTES = 4 * 16 * (HD + 3) * 4;
+    static constexpr int SMEM_BYTES =
+        (OFF_MISC + 16 > MERGE_BYTES ? OFF_MISC + 16 : MERGE_BYTES) + 1024;
+    static constexpr int THREADS = 160;
+};
+
+// four e4m3 values (byte i = element i) -> two f16x2 words (elements 0,1 and 2,3)
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(x));
+}
+// lo += float(low f16 of packed), hi += float(high f16): mixed-precision adds
+__device__ __forceinline__ void add_f16x2_to_f32(uint32_t packed, float& lo, float& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "add.rn.f32.f16 %0, l, %0;\n\tadd.rn.f32.f16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(packed));
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// bf16x2 -> f16x2 (round to nearest; |x| > 65504 becomes inf)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
+    return pack_f16x2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void st_shared_v4u(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d));
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -93,6 +161,23 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// the same with f16 inputs
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+    if constexpr (F16)
+        mma_f16_16816(d, a, b0, b1);
+    else
+        mma_bf16_16816(d, a, b0, b1);
+}
 
 // Byte offset of the 16-byte chunk holding dims [8c, 8c+8) of row `row` in a
 // 128B-swizzled [rows x 64 dims] atom written by TMA.
@@ -101,12 +186,12 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int chunk) {
 }
 
 // PAGED = true reads K and V through p.block_table; the dense instantiation carries
-// none of that code.
-template <int HD, bool PAGED = false>
+// none of that code.  KV8 = true: K and V are e4m3 (see the top of the file).
+template <int HD, bool PAGED = false, bool KV8 = false>
 __global__ void __launch_bounds__(160, 2)
     decode_split_sm100(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-    using C = DecodeCfg<HD>;
+    using C = std::conditional_t<KV8, DecodeCfg8<HD>, DecodeCfg<HD>>;
     constexpr int ST = C::STAGES;
     constexpr int KSTEPS = HD / 16;
     extern __shared__ uint8_t smem_raw[];
@@ -191,6 +276,23 @@ __global__ void __launch_bounds__(160, 2)
                     pg[i] = __ldg(trow + (key >> p.page_shift));
                 }
             };
+            // copies of rows [r0, r0 + box) of stage s from tensor row z
+            auto load_rows = [&](int s, int r0, int z) {
+                if constexpr (KV8) {
+                    tma_load_3d(smem + C::OFF_K + s * C::TILE + r0 * HD, &tm_k, bar_full + s, 0,
+                                kvh, z);
+                    tma_load_3d(smem + C::OFF_V + s * C::TILE + r0 * HD, &tm_v, bar_full + s, 0,
+                                kvh, z);
+                } else {
+#pragma unroll
+                    for (int a = 0; a < C::ATOMS; ++a) {
+                        tma_load_3d(smem + C::OFF_K + s * C::TILE + a * C::ATOM + r0 * 128,
+                                    &tm_k, bar_full + s, a * 64, kvh, z);
+                        tma_load_3d(smem + C::OFF_V + s * C::TILE + a * C::ATOM + r0 * 128,
+                                    &tm_v, bar_full + s, a * 64, kvh, z);
+                    }
+                }
+            };
             if (paged && nblk > 0) lookup(blk0, pg_cur);
             int c = 0;
             for (; c < nblk; ++c) {
@@ -200,14 +302,7 @@ __global__ void __launch_bounds__(160, 2)
                 mbar_arrive_expect_tx(bar_full + s, 2 * C::TILE);
                 const int key0 = (blk0 + c) * C::BN;
                 if (!paged) {
-                    const int z = b * p.Sk + key0;
-#pragma unroll
-                    for (int a = 0; a < C::ATOMS; ++a) {
-                        tma_load_3d(smem + C::OFF_K + s * C::TILE + a * C::ATOM, &tm_k,
-                                    bar_full + s, a * 64, kvh, z);
-                        tma_load_3d(smem + C::OFF_V + s * C::TILE + a * C::ATOM, &tm_v,
-                                    bar_full + s, a * 64, kvh, z);
-                    }
+                    load_rows(s, 0, b * p.Sk + key0);
                 } else {
                     // one copy of min(page_size, 64) rows per page the block touches;
                     // rows land at their key offset, so the 128B swizzle (a function
@@ -222,14 +317,8 @@ __global__ void __launch_bounds__(160, 2)
                             raise_device_error(kDevBadKvIndex);
                             page = 0;
                         }
-                        const int z = (page << p.page_shift) + (key & ((1 << p.page_shift) - 1));
-#pragma unroll
-                        for (int a = 0; a < C::ATOMS; ++a) {
-                            tma_load_3d(smem + C::OFF_K + s * C::TILE + a * C::ATOM + r0 * 128,
-                                        &tm_k, bar_full + s, a * 64, kvh, z);
-                            tma_load_3d(smem + C::OFF_V + s * C::TILE + a * C::ATOM + r0 * 128,
-                                        &tm_v, bar_full + s, a * 64, kvh, z);
-                        }
+                        load_rows(s, r0,
+                                  (page << p.page_shift) + (key & ((1 << p.page_shift) - 1)));
                     }
 #pragma unroll
                     for (int i = 0; i < 4; ++i) pg_cur[i] = pg_nxt[i];
@@ -267,10 +356,23 @@ __global__ void __launch_bounds__(160, 2)
                 qa[kk][1] = v1 ? __ldg(qrow1 + (kk * 16 + qd) / 2) : 0u;
                 qa[kk][2] = v0 ? __ldg(qrow0 + (kk * 16 + 8 + qd) / 2) : 0u;
                 qa[kk][3] = v1 ? __ldg(qrow1 + (kk * 16 + 8 + qd) / 2) : 0u;
+                if constexpr (KV8) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) qa[kk][e] = bf16x2_to_f16x2(qa[kk][e]);
+                }
             }
         }
         const uint32_t sK0 = smem_u32(smem + C::OFF_K);
         const uint32_t sV0 = smem_u32(smem + C::OFF_V);
+        // KV8: this warp's f16 copies of its 16 keys; ldmatrix rows count from the warp's
+        // first key there, and an atom (64 dims) holds 16 rows
+        uint32_t wK = 0, wV = 0;
+        if constexpr (KV8) {
+            wK = smem_u32(smem + C::OFF_W + warp * 2 * C::WTILE);
+            wV = wK + C::WTILE;
+        }
+        constexpr int ATOM_B = KV8 ? 16 * 128 : 64 * 128;
+        const int row0 = KV8 ? warp * 16 : 0;
         // ldmatrix row addresses: lane provides row (lane & 7) of matrix (lane >> 3)
         const int mat = lane >> 3, mrow = lane & 7;
         // QK: matrices (keys +0/+8) x (dim chunk +0/+1): key = 16w + (mat>>1)*8 + mrow
@@ -282,8 +384,66 @@ __global__ void __launch_bounds__(160, 2)
         for (int c = 0; c < nblk; ++c) {
             const int s = c % ST;
             if (!mbar_wait_warp(bar_full + s, (c / ST) & 1, abort_flag)) break;
-            const uint32_t sK = sK0 + s * C::TILE;
-            const uint32_t sV = sV0 + s * C::TILE;
+            uint32_t sK = sK0 + s * C::TILE;
+            uint32_t sV = sV0 + s * C::TILE;
+            // keys past the end may be unwritten cache memory (a page's or the dense
+            // cache's unused rows): their P is 0, but 0 * NaN would still reach O, so this
+            // warp zeroes its own V rows there; the stage is handed back to TMA only after
+            // a proxy fence orders these writes before the next copy into it
+            bool zeroed = false;
+            if constexpr (!KV8) {
+                const int r_end = key_end - (blk0 + c) * C::BN - warp * 16;  // rows kept
+                if (r_end < 16) {
+                    zeroed = true;
+                    constexpr int CH = 16 * C::ATOMS * 8;  // 16-byte chunks of 16 rows
+                    for (int ci = lane; ci < CH; ci += 32) {
+                        const int row = ci / (C::ATOMS * 8);
+                        if (row < r_end) continue;
+                        const int rest = ci - row * (C::ATOMS * 8);
+                        const int a = rest >> 3, q16 = rest & 7;
+                        st_shared_v4u(sV + uint32_t(a * C::ATOM + (warp * 16 + row) * 128 +
+                                                    q16 * 16),
+                                      0u, 0u, 0u, 0u);
+                    }
+                    __syncwarp();
+                }
+            }
+            if constexpr (KV8) {
+                // e4m3 rows of this warp's 16 keys -> f16, 16-byte chunks read in order
+                // (conflict-free) and written to the swizzled atoms; then the stage is free
+                __syncwarp();  // the previous block's ldmatrix reads of wK / wV are done
+                // lane -> one 8-dim chunk: the loads are consecutive 8-byte pieces and
+                // each group of 8 lanes stores one 128-byte row of an atom (every bank
+                // once), so neither side has bank conflicts
+                const int r_keep = key_end - (blk0 + c) * C::BN - warp * 16;  // rows kept
+#pragma unroll
+                for (int kv = 0; kv < 2; ++kv) {
+                    const uint32_t src = (kv ? sV : sK) + uint32_t(warp * 16 * HD);
+                    const uint32_t dst = kv ? wV : wK;
+#pragma unroll
+                    for (int it = 0; it < HD / 16; ++it) {
+                        const int ci = it * 32 + lane;       // 8-dim chunk of the warp's rows
+                        const int row = ci / (HD / 8);       // key within the warp's 16
+                        const int ch = ci - row * (HD / 8);  // f16 chunk index over HD / 8
+                        uint32_t x0, x1;
+                        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                                     : "=r"(x0), "=r"(x1)
+                                     : "r"(src + uint32_t(ci * 8)));
+                        uint32_t h[4];
+                        e4m3x4_to_f16x4(x0, h[0], h[1]);
+                        e4m3x4_to_f16x4(x1, h[2], h[3]);
+                        // keys past the end may be unwritten cache memory: their P is 0,
+                        // and 0 * NaN would still reach O, so they become zeros
+                        if (row >= r_keep) h[0] = h[1] = h[2] = h[3] = 0u;
+                        st_shared_v4u(dst + uint32_t((ch >> 3) * ATOM_B) + sw128_off(row, ch),
+                                      h[0], h[1], h[2], h[3]);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_empty + s);
+                sK = wK;
+                sV = wV;
+            }
             float sc[2][4];
 #pragma unroll
             for (int t = 0; t < 2; ++t)
@@ -293,9 +453,10 @@ __global__ void __launch_bounds__(160, 2)
             for (int kk = 0; kk < KSTEPS; ++kk) {
                 const int chunk = kk * 2 + chunk_qk;
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(sK + (chunk >> 3) * C::ATOM + sw128_off(key_qk, chunk), b0, b1, b2, b3);
-                mma_bf16_16816(sc[0], qa[kk], b0, b1);
-                mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                ldsm_x4(sK + (chunk >> 3) * ATOM_B + sw128_off(key_qk - row0, chunk), b0, b1, b2,
+                        b3);
+                mma_16816<KV8>(sc[0], qa[kk], b0, b1);
+                mma_16816<KV8>(sc[1], qa[kk], b2, b3);
             }
             // mask keys past the end of this split / of the sequence, and keys
             // before the window (only blocks that straddle one of those edges)
@@ -336,20 +497,37 @@ __global__ void __launch_bounds__(160, 2)
                         const float mu = (m_run[hr] == -INFINITY) ? 0.f : m_run[hr];
                         pr[t][e] = ex2_approx(fmaf(sc[t][e], sl2, -mu));
                     }
-                pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-                pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-                pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-                pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+                if constexpr (KV8) {
+                    pa[0] = pack_f16x2(pr[0][0], pr[0][1]);
+                    pa[1] = pack_f16x2(pr[0][2], pr[0][3]);
+                    pa[2] = pack_f16x2(pr[1][0], pr[1][1]);
+                    pa[3] = pack_f16x2(pr[1][2], pr[1][3]);
+                } else {
+                    pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+                    pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+                    pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+                    pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+                }
                 // two row sums: exact p (for L) and the bf16 weights the MMA consumes
                 // (for O / l); rows g: pa[0], pa[2]; rows g + 8: pa[1], pa[3]
 #pragma unroll
                 for (int hr = 0; hr < 2; ++hr)
                     l_part[hr] = l_part[hr] * alpha[hr] + pr[0][2 * hr] + pr[0][2 * hr + 1] +
                                  pr[1][2 * hr] + pr[1][2 * hr + 1];
-                l_rnd[0] = l_rnd[0] * alpha[0] + bf16_lo(pa[0]) + bf16_hi(pa[0]) +
-                           bf16_lo(pa[2]) + bf16_hi(pa[2]);
-                l_rnd[1] = l_rnd[1] * alpha[1] + bf16_lo(pa[1]) + bf16_hi(pa[1]) +
-                           bf16_lo(pa[3]) + bf16_hi(pa[3]);
+                if constexpr (KV8) {
+                    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+                    add_f16x2_to_f32(pa[0], a0, a1);
+                    add_f16x2_to_f32(pa[2], a0, a1);
+                    add_f16x2_to_f32(pa[1], b0, b1);
+                    add_f16x2_to_f32(pa[3], b0, b1);
+                    l_rnd[0] = l_rnd[0] * alpha[0] + (a0 + a1);
+                    l_rnd[1] = l_rnd[1] * alpha[1] + (b0 + b1);
+                } else {
+                    l_rnd[0] = l_rnd[0] * alpha[0] + bf16_lo(pa[0]) + bf16_hi(pa[0]) +
+                               bf16_lo(pa[2]) + bf16_hi(pa[2]);
+                    l_rnd[1] = l_rnd[1] * alpha[1] + bf16_lo(pa[1]) + bf16_hi(pa[1]) +
+                               bf16_lo(pa[3]) + bf16_hi(pa[3]);
+                }
             }
             if (alpha[0] != 1.f || alpha[1] != 1.f) {
 #pragma unroll
@@ -364,12 +542,14 @@ __global__ void __launch_bounds__(160, 2)
             for (int nt = 0; nt < KSTEPS; ++nt) {
                 const int chunk = nt * 2 + chunk_pv;
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(sV + (chunk >> 3) * C::ATOM + sw128_off(key_pv, chunk), b0, b1, b2, b3);
-                mma_bf16_16816(o[2 * nt], pa, b0, b1);
-                mma_bf16_16816(o[2 * nt + 1], pa, b2, b3);
+                ldsm_x4_t(sV + (chunk >> 3) * ATOM_B + sw128_off(key_pv - row0, chunk), b0, b1, b2,
+                          b3);
+                mma_16816<KV8>(o[2 * nt], pa, b0, b1);
+                mma_16816<KV8>(o[2 * nt + 1], pa, b2, b3);
             }
+            if (zeroed) fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_empty + s);
+            if (!KV8 && lane == 0) mbar_arrive(bar_empty + s);
         }
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
@@ -423,7 +603,7 @@ __global__ void __launch_bounds__(160, 2)
             lr += f * mr[w * 16 + r];
         }
         const int h = h0 + r;
-        const float inv_l = (lr > 0.f) ? 1.f / lr : 0.f;
+        const float inv_l = (lr > 0.f) ? (KV8 ? p.v_scale : 1.f) / lr : 0.f;
         const float L = (l > 0.f) ? (Mu + __log2f(l)) * 0.69314718055994531f : -INFINITY;
         if (p.n_splits == 1) {
             p.out[(size_t(b) * p.Hq + h) * HD + d] = __float2bfloat16_rn(acc * inv_l);

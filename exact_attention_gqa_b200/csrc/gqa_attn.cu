@@ -111,6 +111,21 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int heads, int D
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 8-bit [rows, heads, D] view (e4m3 K/V): boxes of {D bytes, 1 head, box_rows}, no swizzle
+bool make_map_u8(CUtensorMap* m, const void* base, long long rows, int heads, int D,
+                 int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(heads), cuuint64_t(rows)};
+    cuuint64_t strides[2] = {cuuint64_t(D), cuuint64_t(heads) * D};
+    cuuint32_t box[3] = {cuuint32_t(D), 1u, cuuint32_t(box_rows)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------- plan
 struct Plan {
     int kernel = kNone;
@@ -280,6 +295,8 @@ struct KvCacheArgs {
     int page_size = 0;
     int num_pages = 0;
     int window = 0;                    // > 0: last `window` keys only
+    bool fp8 = false;                  // K and V are e4m3 codes
+    float k_scale = 1.f, v_scale = 1.f;  // value of one code unit of K and of V
 };
 
 int log2_exact(int x) {
@@ -320,6 +337,10 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     p.page_shift = kv.block_table ? log2_exact(kv.page_size) : 0;
     p.num_pages = kv.num_pages;
     p.window = kv.window;
+    if (kv.fp8) {
+        p.scale_log2 = scale * kv.k_scale * kLog2e;  // logits of the decoded keys
+        p.v_scale = kv.v_scale;
+    }
     if (pl.splits > 1) {
         const size_t need = ws_bytes(B, Hq, 1, HD, pl.splits);
         int dev = 0;
@@ -341,17 +362,30 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     const long long rows = kv.block_table ? (long long)kv.num_pages * kv.page_size
                                           : (long long)B * Sk;
     const int box = kv.block_table ? (kv.page_size < C::BN ? kv.page_size : C::BN) : C::BN;
-    if (!make_map(&tk, k, rows, Hkv, HD, 1, box) || !make_map(&tv, v, rows, Hkv, HD, 1, box))
-        return GQA_ERR_CUDA;
+    const bool maps = kv.fp8 ? (make_map_u8(&tk, k, rows, Hkv, HD, box) &&
+                                make_map_u8(&tv, v, rows, Hkv, HD, box))
+                             : (make_map(&tk, k, rows, Hkv, HD, 1, box) &&
+                                make_map(&tv, v, rows, Hkv, HD, 1, box));
+    if (!maps) return GQA_ERR_CUDA;
     dim3 grid(pl.splits, Hkv * pl.decode_units, B);
-    if (kv.block_table) {
-        const int rc = ensure_smem_limit(gqa::decode_split_sm100<HD, true>, HD == 64 ? 16 : 32,
-                                         C::SMEM_BYTES);
+    // one instantiation per (paged, e4m3) pair; each raises its own shared-memory limit
+    auto launch = [&](auto kernel, int bit, int smem) -> int {
+        const int rc = ensure_smem_limit(kernel, bit, smem);
         if (rc != GQA_OK) return rc;
-        gqa::decode_split_sm100<HD, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
-    } else {
+        kernel<<<grid, C::THREADS, smem, stream>>>(tk, tv, p);
+        return GQA_OK;
+    };
+    constexpr int SM8 = gqa::DecodeCfg8<HD>::SMEM_BYTES;
+    const int sh = HD == 64 ? 0 : 1;
+    int rc = GQA_OK;
+    if (kv.fp8)
+        rc = kv.block_table ? launch(gqa::decode_split_sm100<HD, true, true>, 256 << sh, SM8)
+                            : launch(gqa::decode_split_sm100<HD, false, true>, 64 << sh, SM8);
+    else if (kv.block_table)
+        rc = launch(gqa::decode_split_sm100<HD, true>, 16 << sh, C::SMEM_BYTES);
+    else
         gqa::decode_split_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tk, tv, p);
-    }
+    if (rc != GQA_OK) return rc;
     if (cudaGetLastError() != cudaSuccess) return GQA_ERR_CUDA;
     if (pl.splits > 1) {
         const int rows_bh = B * Hq;
@@ -369,6 +403,9 @@ int kvcache_common(const void* q, const void* k, const void* v, void* out, float
                    const KvCacheArgs& kv, int num_splits, int pack_gqa, cudaStream_t stream) {
     const bool paged = kv.block_table != nullptr;
     if (B < 0 || Sk < 0 || max_seqlen_k < 0 || kv.window < 0) return GQA_ERR_SHAPE;
+    if (kv.fp8 && !(std::isfinite(kv.k_scale) && kv.k_scale > 0.f &&
+                    std::isfinite(kv.v_scale) && kv.v_scale > 0.f))
+        return GQA_ERR_SCALE;
     if (paged) {
         if (kv.page_size < 16 || (kv.page_size & (kv.page_size - 1)) != 0 ||
             kv.num_pages < 1 || kv.max_pages < 1 || !kv.seqlens_k)
@@ -395,6 +432,18 @@ int kvcache_common(const void* q, const void* k, const void* v, void* out, float
     if (rc != GQA_OK) return rc;
     Plan pl;
     make_plan(&pl, B, Hq, Hkv, 1, keys, num_splits, pack_gqa, false, dev->sms);
+    if (kv.fp8 && num_splits == 0 && pl.kernel == kDecode) {
+        // the e4m3 kernel converts every element, so one CTA per SM leaves each SM
+        // sub-partition a single warp; two resident CTAs per SM (they fit) measured
+        // faster at every batch size
+        const long long ctas = (long long)B * Hkv * pl.decode_units;
+        const int nblk = (keys + 63) / 64;
+        long long n = (2LL * dev->sms) / ctas;  // whole waves: at most two CTAs per SM
+        if (n < 1) n = 1;
+        if (n > 64) n = 64;
+        if (n > nblk / 4) n = nblk / 4 > 0 ? nblk / 4 : 1;
+        make_plan(&pl, B, Hq, Hkv, 1, keys, int(n), pack_gqa, false, dev->sms);
+    }
     if (pl.kernel == kZeroFill) {
         gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
             static_cast<__nv_bfloat16*>(out), (long long)B * Hq * D, lse, (long long)B * Hq);
@@ -925,6 +974,29 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
     kv.window = window;
     return kvcache_common(q, k_pages, v_pages, out, lse, B, Hq, Hkv, 0, D, max_seqlen_k, scale,
                           kv, num_splits, pack_gqa, stream);
+}
+
+int gqa_attn_decode_fp8(const void* q, const void* k8, const void* v8, float k_scale,
+                        float v_scale, const int* block_table, const int* seqlens_k, void* out,
+                        float* lse, int B, int Hq, int Hkv, int D, int Sk, int num_pages,
+                        int page_size, int max_pages, int max_seqlen_k, float scale, int window,
+                        int num_splits, int pack_gqa, cudaStream_t stream) {
+    KvCacheArgs kv;
+    kv.seqlens_k = seqlens_k;
+    kv.window = window;
+    kv.fp8 = true;
+    kv.k_scale = k_scale;
+    kv.v_scale = v_scale;
+    if (block_table) {
+        kv.block_table = block_table;
+        kv.max_pages = max_pages;
+        kv.page_size = page_size;
+        kv.num_pages = num_pages;
+        Sk = 0;
+    }
+    return kvcache_common(q, k8, v8, out, lse, B, Hq, Hkv, Sk, D,
+                          (seqlens_k || block_table) ? max_seqlen_k : Sk, scale, kv, num_splits,
+                          pack_gqa, stream);
 }
 
 int gqa_attn_selftest_timeout(int limit_ms, cudaStream_t stream) {

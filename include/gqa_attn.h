@@ -284,6 +284,34 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
                           int num_splits, int pack_gqa, cudaStream_t stream);
 
 /*
+ * The same decode against a KV cache stored in 8 bits: every K and V element is an
+ * e4m3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; subnormals below
+ * 2^-6; largest finite 448; the NaN codes 0x7f and 0xff are not propagated: they are
+ * read as +-480), and the stored value is
+ * code_value * k_scale (keys) or code_value * v_scale (values), one scale per tensor.
+ * The attention is gqa_attn_decode_kvcache's on those decoded values.  The GQA
+ * batch-size guide names FP8 as the way to lower memory-bandwidth pressure (hardware
+ * adaptation section, Hopper item; precision row of its production checklist); the
+ * cache is read once in 8 bits, half the bytes of bf16.
+ *   block_table NULL: k8, v8 [B, Sk, Hkv, D] uint8 codes (num_pages, page_size and
+ *     max_pages ignored);
+ *   block_table given: k8, v8 [num_pages, page_size, Hkv, D] codes with
+ *     gqa_attn_decode_paged's table, lengths and page rules (Sk ignored);
+ *   q bf16 [B, 1, Hq, D] (rounded to f16 for the products: |q| must stay below
+ *     65504), out bf16 [B, 1, Hq, D], lse fp32 [B, Hq, 1]; k_scale, v_scale finite
+ *     and > 0 (GQA_ERR_SCALE otherwise).
+ * num_splits = 0 chooses up to 64 splits so that two CTAs share each SM (the 8-bit
+ * path converts every element and needs the extra warps); a registered workspace of
+ * gqa_attn_workspace_bytes(B, Hq, 1, D, 64) always suffices.  Status codes, window,
+ * explicit splits and pack_gqa as gqa_attn_decode_kvcache.
+ */
+int gqa_attn_decode_fp8(const void* q, const void* k8, const void* v8, float k_scale,
+                        float v_scale, const int* block_table, const int* seqlens_k, void* out,
+                        float* lse, int B, int Hq, int Hkv, int D, int Sk, int num_pages,
+                        int page_size, int max_pages, int max_seqlen_k, float scale, int window,
+                        int num_splits, int pack_gqa, cudaStream_t stream);
+
+/*
  * Diagnostic: exercises the kernels' bounded-wait path.  Launches one warp that
  * waits, with the same bounded mbarrier wait the attention kernels use, on a
  * barrier nothing completes; after limit_ms (1..1000) the wait gives up, records

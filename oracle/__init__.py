@@ -51,6 +51,7 @@ FLAWS = {
     "swap_kv": 7,
     "pages_contiguous": 8,
     "window_short": 9,
+    "e4m3_bias": 10,
 }
 
 
@@ -85,6 +86,11 @@ def _load():
         lib.oracle_decode_kvcache.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I,
                                               Dbl, I]
         lib.oracle_decode_kvcache.restype = I
+        lib.oracle_decode_kvcache_e4m3.argtypes = [P, P, P, Dbl, Dbl, P, P, P, P, I, I, I, I, I,
+                                                   I, I, I, I, Dbl, I]
+        lib.oracle_decode_kvcache_e4m3.restype = I
+        lib.oracle_e4m3_table.argtypes = [P]
+        lib.oracle_e4m3_table.restype = None
         lib.oracle_set_flaw.argtypes = [I]
         lib.oracle_set_flaw.restype = None
         lib.oracle_get_flaw.restype = I
@@ -206,12 +212,36 @@ def attention_tiled(q, k, v, *, scale: float, causal: bool, Bm: int, Bn: int, fo
     return o, lse
 
 
+def e4m3_table() -> np.ndarray:
+    """Values of the 256 e4m3 codes (float64; NaN for 0x7f and 0xff)."""
+    out = np.zeros(256, dtype=np.float64)
+    _load().oracle_e4m3_table(_ptr(out))
+    return out
+
+
+def _codes(a):
+    if hasattr(a, "detach"):  # torch uint8 or float8_e4m3fn: the raw bytes
+        import torch
+        a = a.detach().to("cpu")
+        if a.dtype != torch.uint8:
+            a = a.view(torch.uint8)
+        a = a.numpy()
+    return np.ascontiguousarray(a, dtype=np.uint8)
+
+
 def decode_kvcache(q, k_cache, v_cache, *, scale: float, seqlens_k=None, block_table=None,
-                   window: int = 0, threads: int = 0):
+                   window: int = 0, k_scale=None, v_scale=None, threads: int = 0):
     """Decode against a KV cache.  q [B, 1, Hq, D] or [B, Hq, D]; dense k/v_cache
     [B, Sk, Hkv, D] or paged [num_pages, page_size, Hkv, D] with block_table
-    [B, max_pages].  Returns (O float64 [B, Hq, D], L float64 [B, Hq])."""
-    q, k, v = _f32(q), _f32(k_cache), _f32(v_cache)
+    [B, max_pages].  With k_scale/v_scale the caches are e4m3 codes (uint8 or
+    float8_e4m3fn) whose values are code * scale.  Returns (O float64 [B, Hq, D],
+    L float64 [B, Hq])."""
+    fp8 = k_scale is not None
+    q = _f32(q)
+    if fp8:
+        k, v = _codes(k_cache), _codes(v_cache)
+    else:
+        k, v = _f32(k_cache), _f32(v_cache)
     B, Hq, D = q.shape[0], q.shape[-2], q.shape[-1]
     Hkv = k.shape[2]
     sl = None if seqlens_k is None else np.ascontiguousarray(_np_int(seqlens_k), dtype=np.int32)
@@ -223,11 +253,14 @@ def decode_kvcache(q, k_cache, v_cache, *, scale: float, seqlens_k=None, block_t
         Sk, page_size, max_pages, num_pages = 0, k.shape[1], bt.shape[1], k.shape[0]
     o = np.zeros((B, Hq, D), dtype=np.float64)
     lse = np.zeros((B, Hq), dtype=np.float64)
-    rc = _load().oracle_decode_kvcache(_ptr(q), _ptr(k), _ptr(v),
-                                       None if bt is None else _ptr(bt),
-                                       None if sl is None else _ptr(sl), _ptr(o), _ptr(lse), B,
-                                       Hq, Hkv, D, Sk, page_size, max_pages, num_pages,
-                                       int(window), float(scale), int(threads))
+    args = (None if bt is None else _ptr(bt), None if sl is None else _ptr(sl), _ptr(o),
+            _ptr(lse), B, Hq, Hkv, D, Sk, page_size, max_pages, num_pages, int(window),
+            float(scale), int(threads))
+    if fp8:
+        rc = _load().oracle_decode_kvcache_e4m3(_ptr(q), _ptr(k), _ptr(v), float(k_scale),
+                                                float(v_scale), *args)
+    else:
+        rc = _load().oracle_decode_kvcache(_ptr(q), _ptr(k), _ptr(v), *args)
     if rc != 0:
         raise ValueError("oracle_decode_kvcache: bad arguments")
     return o, lse

@@ -44,6 +44,10 @@
  * key j of sequence b lives in row j % page_size of page block_table[b][j /
  * page_size]; with a window W > 0 the query (the newest position) attends to the
  * last W of the L cached keys, j >= L - W.
+ * FP8 cache: the GQA batch-size guide names FP8 (hardware adaptation section) without
+ * a format; reading: e4m3 codes (sign, 4-bit exponent with bias 7, 3-bit mantissa,
+ * subnormals 2^-6 * m/8, codes 0x7f / 0xff NaN, no infinities), one scale per tensor,
+ * stored value = code value * scale.
  *
  * Return value of every entry point: 0 on success, -1 on bad arguments.
  */
@@ -70,6 +74,7 @@ enum {
     FLAW_SWAP_KV = 7,         /* uses K where V belongs in O = P V             */
     FLAW_PAGES_CONTIGUOUS = 8,/* paged cache read as if pages were in order     */
     FLAW_WINDOW_SHORT = 9,    /* sliding window keeps one key too few           */
+    FLAW_E4M3_BIAS = 10,      /* e4m3 exponent bias 8 instead of 7              */
 };
 static int g_flaw = FLAW_NONE;
 void oracle_set_flaw(int flaw) { g_flaw = flaw; }
@@ -375,6 +380,37 @@ void oracle_combine(int n, int D, const double* Os, const double* Ls, double* O,
     *L = Lall;
 }
 
+/* Value of one e4m3 code. */
+static double e4m3_value(uint8_t c)
+{
+    const int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    const int bias = (g_flaw == FLAW_E4M3_BIAS) ? 8 : 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = (e == 0) ? ldexp((double)m / 8.0, 1 - bias)
+                                : ldexp(1.0 + (double)m / 8.0, e - bias);
+    return sign ? -mag : mag;
+}
+
+/* All 256 code values (out[256]). */
+void oracle_e4m3_table(double* out)
+{
+    for (int c = 0; c < 256; ++c) out[c] = e4m3_value((uint8_t)c);
+}
+
+/* Element of a cache: float value, or e4m3 code times its scale (lut holds the 256
+ * code values, filled by e4m3_value for each call). */
+typedef struct {
+    const float* f;
+    const uint8_t* c;
+    double scale;
+    const double* lut;
+} cache_src;
+
+static double cache_at(const cache_src* src, size_t i)
+{
+    return src->f ? (double)src->f[i] : src->lut[src->c[i]] * src->scale;
+}
+
 /*
  * One decode query per sequence against a KV cache, by the plain definition.
  *   q [B, Hq, D]; o [B, Hq, D]; lse [B, Hq].
@@ -387,12 +423,12 @@ void oracle_combine(int n, int D, const double* Os, const double* Ls, double* O,
  * p_j = exp(s_j - m), l = sum p_j, O = sum p_j v_j / l, L = m + ln l; no key:
  * O = 0, L = -inf.
  */
-int oracle_decode_kvcache(const float* q, const float* k_cache, const float* v_cache,
-                          const int32_t* block_table, const int32_t* seqlens_k, double* o,
-                          double* lse, int B, int Hq, int Hkv, int D, int Sk, int page_size,
-                          int max_pages, int num_pages, int window, double scale, int nthreads)
+static int decode_core(const float* q, const cache_src* ks, const cache_src* vs,
+                       const int32_t* block_table, const int32_t* seqlens_k, double* o,
+                       double* lse, int B, int Hq, int Hkv, int D, int Sk, int page_size,
+                       int max_pages, int num_pages, int window, double scale, int nthreads)
 {
-    if (!q || !k_cache || !v_cache || !o || !lse) return -1;
+    if (!q || !(ks->f || ks->c) || !(vs->f || vs->c) || !o || !lse) return -1;
     if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0 || window < 0) return -1;
     const int paged = block_table != NULL;
     int cap = Sk;
@@ -451,8 +487,10 @@ int oracle_decode_kvcache(const float* q, const float* k_cache, const float* v_c
             }
             double m = -INFINITY;
             for (int j = j0; j < L; ++j) {
-                const float* kj = k_cache + (kr[j - j0] * Hkv + c) * (size_t)D;
-                row[j - j0] = scale * dot(qv, kj, D);
+                const size_t kb = (kr[j - j0] * Hkv + c) * (size_t)D;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += (double)qv[d] * cache_at(ks, kb + d);
+                row[j - j0] = scale * acc;
                 if (row[j - j0] > m) m = row[j - j0];
             }
             if (L <= j0) {
@@ -468,7 +506,7 @@ int oracle_decode_kvcache(const float* q, const float* k_cache, const float* v_c
             for (int d = 0; d < D; ++d) {
                 double acc = 0.0;
                 for (int j = j0; j < L; ++j)
-                    acc += row[j - j0] * (double)v_cache[(kr[j - j0] * Hkv + c) * (size_t)D + d];
+                    acc += row[j - j0] * cache_at(vs, (kr[j - j0] * Hkv + c) * (size_t)D + d);
                 ob[d] = acc / l;
             }
             lse[(size_t)b * Hq + h] = m + log(l);
@@ -476,6 +514,31 @@ int oracle_decode_kvcache(const float* q, const float* k_cache, const float* v_c
             free(kr);
         }
     return bad ? -1 : 0;
+}
+
+int oracle_decode_kvcache(const float* q, const float* k_cache, const float* v_cache,
+                          const int32_t* block_table, const int32_t* seqlens_k, double* o,
+                          double* lse, int B, int Hq, int Hkv, int D, int Sk, int page_size,
+                          int max_pages, int num_pages, int window, double scale, int nthreads)
+{
+    const cache_src ks = {k_cache, NULL, 1.0, NULL}, vs = {v_cache, NULL, 1.0, NULL};
+    return decode_core(q, &ks, &vs, block_table, seqlens_k, o, lse, B, Hq, Hkv, D, Sk,
+                       page_size, max_pages, num_pages, window, scale, nthreads);
+}
+
+/* The same with e4m3 codes: key element = value(code) * k_scale, likewise for V. */
+int oracle_decode_kvcache_e4m3(const float* q, const uint8_t* k8, const uint8_t* v8,
+                               double k_scale, double v_scale, const int32_t* block_table,
+                               const int32_t* seqlens_k, double* o, double* lse, int B, int Hq,
+                               int Hkv, int D, int Sk, int page_size, int max_pages,
+                               int num_pages, int window, double scale, int nthreads)
+{
+    if (!k8 || !v8) return -1;
+    double lut[256];
+    oracle_e4m3_table(lut);
+    const cache_src ks = {NULL, k8, k_scale, lut}, vs = {NULL, v8, v_scale, lut};
+    return decode_core(q, &ks, &vs, block_table, seqlens_k, o, lse, B, Hq, Hkv, D, Sk,
+                       page_size, max_pages, num_pages, window, scale, nthreads);
 }
 
 /*

@@ -208,3 +208,32 @@ def test_paged_argument_errors(lib, kw, code):
 def test_kvcache_empty_batch_is_a_noop(lib):
     assert kv_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
     assert paged_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+
+
+def fp8_call(lib, *, q=FAKE, k=FAKE, v=FAKE, ks=0.5, vs=0.5, bt=None, sl=None, out=FAKE,
+             lse=FAKE, B=2, Hq=8, Hkv=2, D=128, Sk=64, num_pages=0, page_size=0, max_pages=0,
+             msl=0, scale=0.125, window=0, splits=0, pack=-1):
+    return lib.gqa_attn_decode_fp8(q, k, v, ks, vs, bt, sl, out, lse, B, Hq, Hkv, D, Sk,
+                                   num_pages, page_size, max_pages, msl, scale, window, splits,
+                                   pack, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(ks=0.0), "GQA_ERR_SCALE"),
+    (dict(vs=-1.0), "GQA_ERR_SCALE"),
+    (dict(ks=float("nan")), "GQA_ERR_SCALE"),
+    (dict(vs=float("inf")), "GQA_ERR_SCALE"),
+    (dict(k=None), "GQA_ERR_NULL"),
+    (dict(D=96), "GQA_ERR_HEADDIM"),
+    (dict(window=-1), "GQA_ERR_SHAPE"),
+    (dict(sl=FAKE, msl=65), "GQA_ERR_SHAPE"),
+    (dict(bt=FAKE, sl=FAKE, num_pages=4, page_size=24, max_pages=2, msl=10), "GQA_ERR_SHAPE"),
+    (dict(bt=FAKE, sl=None, num_pages=4, page_size=64, max_pages=2, msl=10), "GQA_ERR_NULL"),
+    (dict(v=ctypes.c_void_p(0x1004)), "GQA_ERR_ALIGN"),
+])
+def test_fp8_argument_errors(lib, kw, code):
+    assert G.STATUS[fp8_call(lib, **kw)] == code
+
+
+def test_fp8_empty_batch_is_a_noop(lib):
+    assert fp8_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0

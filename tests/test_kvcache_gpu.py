@@ -168,3 +168,120 @@ def test_full_paged_decode_workload():
             vb = vp[idx].reshape(1, w.Sk, w.Hkv, w.D).cpu()
             ref = oracle.decode_kvcache(q[b:b + 1].cpu(), kb, vb, scale=w.scale, window=window)
             check(out[b:b + 1], lse[b:b + 1], *ref)
+
+
+# ------------------------------------------------------------------ e4m3 (FP8) cache
+def e4m3_cache(B, Sk, Hkv, D, seed, spread=50.0):
+    """Finite e4m3 codes of N(0, spread^2) draws (|x| stays far below 448)."""
+    g = torch.Generator().manual_seed(seed)
+    k = (torch.randn(B, Sk, Hkv, D, generator=g) * spread).to(torch.float8_e4m3fn)
+    v = (torch.randn(B, Sk, Hkv, D, generator=g) * spread).to(torch.float8_e4m3fn)
+    return k, v
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("window,splits,pack", [(0, 1, 1), (0, 0, 1), (100, 3, 0), (2000, 0, 1)])
+def test_fp8_dense_cache(D, window, splits, pack):
+    B, Hq, Hkv, Sk = len(LENS), 32, 8, 3000
+    q, _, _ = make_cache(B, Hq, Hkv, 1, D, seed=D + window)
+    k8, v8 = e4m3_cache(B, Sk, Hkv, D, seed=D + splits)
+    ks, vs = 1 / 50, 1 / 40
+    lens = torch.tensor(LENS, dtype=torch.int32)
+    out, lse = gqa_attn_kvcache(q.to(DEV), k8.to(DEV), v8.to(DEV), seqlens_k=lens.to(DEV),
+                                max_seqlen_k=Sk, window=window, num_splits=splits,
+                                pack_gqa=pack, k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    check(out, lse, *oracle.decode_kvcache(q, k8, v8, scale=1 / math.sqrt(D), seqlens_k=lens,
+                                           window=window, k_scale=ks, v_scale=vs))
+
+
+@pytest.mark.parametrize("page_size", [16, 256])
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp8_paged_cache_as_uint8_codes(page_size, D):
+    B, Hq, Hkv, Sk = len(LENS), 16, 4, 3000
+    q, _, _ = make_cache(B, Hq, Hkv, 1, D, seed=page_size + D)
+    k8, v8 = e4m3_cache(B, Sk, Hkv, D, seed=page_size * 7 + D)
+    ku, vu = k8.view(torch.uint8), v8.view(torch.uint8)
+    # pages of codes through the same shuffled table as the bf16 test
+    kp, vp, table = to_pages(ku.view(torch.int8).float(), vu.view(torch.int8).float(), LENS,
+                             page_size, seed=page_size + 1)
+    kp = kp.float().round().to(torch.int8).view(torch.uint8)
+    vp = vp.float().round().to(torch.int8).view(torch.uint8)
+    lens = torch.tensor(LENS, dtype=torch.int32)
+    out, lse = gqa_attn_kvcache(q.to(DEV), kp.to(DEV), vp.to(DEV), seqlens_k=lens.to(DEV),
+                                block_table=table.to(DEV), window=300, k_scale=0.02,
+                                v_scale=0.03)
+    torch.cuda.synchronize()
+    ref = oracle.decode_kvcache(q, kp, vp, scale=1 / math.sqrt(D), seqlens_k=lens,
+                                block_table=table.clamp(min=0), window=300, k_scale=0.02,
+                                v_scale=0.03)
+    check(out, lse, *ref)
+    dense = oracle.decode_kvcache(q, ku, vu, scale=1 / math.sqrt(D), seqlens_k=lens, window=300,
+                                  k_scale=0.02, v_scale=0.03)
+    np.testing.assert_allclose(ref[0], dense[0], rtol=0, atol=1e-12)
+
+
+def test_full_fp8_decode_workload():
+    """The benchmark's e4m3 decode (B=16, Sk=32768, automatic splits) on the GPU, three
+    sequences checked against the oracle's e4m3 decode."""
+    import workloads as W
+    w = W.decode_fp8(16)
+    q = W.make_decode_q(w, device=DEV)
+    k8 = torch.empty(w.B, w.Sk, w.Hkv, w.D, dtype=torch.float8_e4m3fn, device=DEV)
+    v8 = torch.empty_like(k8)
+    W.fill_decode_kv(w, k8, v8)
+    out, lse = gqa_attn_kvcache(q, k8, v8, k_scale=W.FP8_SCALE, v_scale=W.FP8_SCALE)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(8)
+    for b in sorted({0, w.B - 1, int(rng.integers(w.B))}):
+        ref = oracle.decode_kvcache(q[b:b + 1].cpu(), k8[b:b + 1].cpu(), v8[b:b + 1].cpu(),
+                                    scale=w.scale, k_scale=W.FP8_SCALE, v_scale=W.FP8_SCALE)
+        check(out[b:b + 1], lse[b:b + 1], *ref)
+
+
+def nan_like(shape, fp8):
+    if fp8:
+        return torch.full(shape, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn)
+    return torch.full(shape, float("nan"), dtype=torch.bfloat16)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+@pytest.mark.parametrize("page_size", [0, 16, 64])
+def test_unwritten_cache_rows_holding_nan_never_reach_the_output(fp8, page_size):
+    """Rows a sequence does not own (past its length, in its last page or in the dense
+    cache's spare capacity) hold NaN: their weight is 0, and nothing of them may show."""
+    B, Hq, Hkv, Sk, D = 4, 16, 4, 700, 128
+    lens = [700, 1, 300, 65]
+    q, k, v = make_cache(B, Hq, Hkv, Sk, D, seed=31 + page_size)
+    if fp8:
+        k, v = e4m3_cache(B, Sk, Hkv, D, seed=32 + page_size)
+    for b, n in enumerate(lens):
+        k[b, n:] = nan_like(k[b, n:].shape, fp8)
+        v[b, n:] = nan_like(v[b, n:].shape, fp8)
+    kw = dict(k_scale=0.02, v_scale=0.02) if fp8 else {}
+    tl = torch.tensor(lens, dtype=torch.int32)
+    if page_size == 0:
+        kc, vc, table = k, v, None
+    else:
+        per = -(-Sk // page_size)
+        used = [-(-n // page_size) for n in lens]
+        kc = nan_like((sum(used) + 3, page_size, Hkv, D), fp8)
+        vc = nan_like((sum(used) + 3, page_size, Hkv, D), fp8)
+        table = torch.full((B, per), -1, dtype=torch.int32)
+        perm = torch.randperm(kc.shape[0], generator=torch.Generator().manual_seed(5))
+        nxt = 0
+        for b, n in enumerate(lens):
+            for pg in range(used[b]):
+                phys = int(perm[nxt])
+                nxt += 1
+                table[b, pg] = phys
+                j1 = min((pg + 1) * page_size, n)
+                kc[phys, : j1 - pg * page_size] = k[b, pg * page_size:j1]
+                vc[phys, : j1 - pg * page_size] = v[b, pg * page_size:j1]
+    out, lse = gqa_attn_kvcache(q.to(DEV), kc.to(DEV), vc.to(DEV), seqlens_k=tl.to(DEV),
+                                max_seqlen_k=Sk,
+                                block_table=None if table is None else table.to(DEV), **kw)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    check(out, lse, *oracle.decode_kvcache(q, k, v, scale=1 / math.sqrt(D), seqlens_k=tl, **kw))

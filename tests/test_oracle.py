@@ -479,6 +479,54 @@ def test_kvcache_rejects_bad_lengths_and_pages():
                               block_table=np.array([[0, 5]], np.int32))
 
 
+def test_e4m3_table_matches_torch_float8():
+    # every code: torch's float8_e4m3fn decoding (a library routine) is the reference
+    t = oracle.e4m3_table()
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn)
+    ref = ref.double().numpy()
+    assert np.array_equal(np.isnan(t), np.isnan(ref))
+    np.testing.assert_array_equal(t[~np.isnan(t)], ref[~np.isnan(ref)])
+    assert t[0x7E] == 448.0 and t[0x01] == 2.0 ** -9 and t[0x38] == 1.0
+
+
+def e4m3_codes(shape, seed, spread=1.0):
+    """Random finite e4m3 codes (torch rounds normal draws to the format)."""
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(*shape, generator=g) * spread
+    return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def decoded(codes, scale):
+    return codes.view(torch.float8_e4m3fn).double().numpy() * scale
+
+
+@pytest.mark.parametrize("window", [0, 9])
+def test_kvcache_e4m3_matches_sdpa_on_decoded_values(window):
+    B, Hq, Hkv, Sk, D = 3, 8, 2, 70, 16
+    q = rnd((B, 1, Hq, D), 90)
+    k8, v8 = e4m3_codes((B, Sk, Hkv, D), 91, 40.0), e4m3_codes((B, Sk, Hkv, D), 92, 40.0)
+    ks, vs = 0.03125, 0.0217
+    lens = np.array([70, 33, 0], dtype=np.int32)
+    O, L = oracle.decode_kvcache(q, k8, v8, scale=0.25, seqlens_k=lens, window=window,
+                                 k_scale=ks, v_scale=vs)
+    assert_kv_close(O, L, *kv_sdpa(q, decoded(k8, ks), decoded(v8, vs), lens, window, 0.25))
+
+
+def test_kvcache_e4m3_paged_matches_sdpa():
+    B, Hq, Hkv, Sk, D = 2, 4, 1, 48, 8
+    q = rnd((B, 1, Hq, D), 93)
+    k8, v8 = e4m3_codes((B, Sk, Hkv, D), 94, 8.0), e4m3_codes((B, Sk, Hkv, D), 95, 8.0)
+    lens = np.array([48, 20], dtype=np.int32)
+    kp, vp, table = scatter_to_pages(k8.numpy().astype(np.float32),
+                                     v8.numpy().astype(np.float32), 16, 96)
+    # owned rows hold the codes exactly; the noise in unowned rows becomes small codes
+    kp = np.ascontiguousarray(np.clip(np.abs(kp), 0, 255)).astype(np.uint8)
+    vp = np.ascontiguousarray(np.clip(np.abs(vp), 0, 255)).astype(np.uint8)
+    O, L = oracle.decode_kvcache(q, kp, vp, scale=0.5, seqlens_k=lens, block_table=table,
+                                 k_scale=0.1, v_scale=0.2)
+    assert_kv_close(O, L, *kv_sdpa(q, decoded(k8, 0.1), decoded(v8, 0.2), lens, 0, 0.5))
+
+
 # ---------------------------------------------------------------------------------
 # Pin strength: every planted mistake is caught by at least one pin above
 
@@ -492,6 +540,7 @@ PIN_BATTERY = [
     lambda: test_equal_keys_average_the_visible_values(),
     lambda: test_kvcache_lengths_and_window_match_sdpa_on_slices(7),
     lambda: test_kvcache_paged_matches_sdpa(16, 0),
+    lambda: test_e4m3_table_matches_torch_float8(),
 ]
 
 

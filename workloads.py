@@ -45,6 +45,7 @@ class Workload:
     num_splits: int = 1
     varlen: dict = field(default_factory=dict)  # {"n": 32, "lo": 128, "hi": 8192}
     page_size: int = 0  # > 0: decode against a paged KV cache of pages of this many keys
+    kv_fp8: bool = False  # decode against an e4m3 KV cache (scale FP8_SCALE)
 
     @property
     def scale(self) -> float:
@@ -84,6 +85,16 @@ def decode_paged(B: int, page_size: int = 256) -> Workload:
     return Workload(f"decode_paged_b{B}_sk32768_p{page_size}", B=B, Hq=32, Hkv=8, Sq=1,
                     Sk=32768, D=128, dtype="bf16", causal=False, seed=4, pack_gqa=1,
                     num_splits=0, page_size=page_size)
+
+
+FP8_SCALE = 1.0 / 32.0  # e4m3 cache: the bf16 values times 32, rounded to e4m3
+
+
+def decode_fp8(B: int) -> Workload:
+    """The decode workload with its cache in 8 bits (FP8 for decode bandwidth, GQA
+    batch-size guide, hardware adaptation section)."""
+    return Workload(f"decode_fp8_b{B}_sk32768", B=B, Hq=32, Hkv=8, Sq=1, Sk=32768, D=128,
+                    dtype="bf16", causal=False, seed=4, pack_gqa=1, num_splits=0, kv_fp8=True)
 
 
 VARLEN = Workload("varlen32_len128to8192_causal", B=32, Hq=32, Hkv=8, Sq=0, Sk=0, D=128,
@@ -157,9 +168,12 @@ def make_decode_kv_one(w: Workload, b: int, device="cpu"):
 
 
 def fill_decode_kv(w: Workload, k_out: torch.Tensor, v_out: torch.Tensor) -> None:
-    """Fill preallocated k/v [B,Sk,Hkv,D] element by element (on their device)."""
+    """Fill preallocated k/v [B,Sk,Hkv,D] element by element (on their device).  An
+    e4m3 (float8_e4m3fn) destination gets the values divided by FP8_SCALE, rounded."""
     for b in range(k_out.shape[0]):
         kb, vb = make_decode_kv_one(w, b, device=k_out.device)
+        if k_out.dtype != kb.dtype:
+            kb, vb = (t.float() / FP8_SCALE for t in (kb, vb))
         k_out[b].copy_(kb)
         v_out[b].copy_(vb)
 
@@ -217,9 +231,12 @@ def kv_cache_bytes(batch: int, seq: int, Hkv: int, D: int, bytes_per_elt: int = 
     return 2 * batch * seq * D * Hkv * bytes_per_elt * layers
 
 
-def decode_bytes(B: int, Hq: int, Hkv: int, Sk: int, D: int, elt: int = 2) -> int:
-    """Algorithmic HBM bytes of one decode step: K and V once, q, O (elt) and L (fp32)."""
-    return kv_cache_bytes(B, Sk, Hkv, D, elt) + 2 * B * Hq * D * elt + 4 * B * Hq
+def decode_bytes(B: int, Hq: int, Hkv: int, Sk: int, D: int, elt: int = 2,
+                 kv_elt: int | None = None) -> int:
+    """Algorithmic HBM bytes of one decode step: K and V once (kv_elt bytes each, default
+    elt), q and O (elt), L (fp32)."""
+    kv_elt = elt if kv_elt is None else kv_elt
+    return kv_cache_bytes(B, Sk, Hkv, D, kv_elt) + 2 * B * Hq * D * elt + 4 * B * Hq
 
 
 def prefill_min_bytes(B: int, Hq: int, Hkv: int, Sq: int, Sk: int, D: int, elt: int = 2):
