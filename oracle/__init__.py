@@ -18,6 +18,8 @@ states the passage of the pages it follows in the C source:
                           log-sum-exp weighted combine.
 * ``attention_tiled``  -- the per-step normalised (form 1) and deferred
                           normalisation (form 2) online-softmax forms.
+* ``attention_blocksparse`` -- attention restricted to a (query block, key block)
+                          pattern (Raptor-T abstract: BigBird's block-sparse attention).
 * ``decode_kvcache``   -- one decode query per sequence against a dense or paged
                           KV cache with per-sequence lengths and a sliding window
                           (Ultralytics GQA glossary, KV-cache and related-techniques
@@ -52,6 +54,7 @@ FLAWS = {
     "pages_contiguous": 8,
     "window_short": 9,
     "e4m3_bias": 10,
+    "sparse_row": 11,
 }
 
 
@@ -89,6 +92,9 @@ def _load():
         lib.oracle_decode_kvcache_e4m3.argtypes = [P, P, P, Dbl, Dbl, P, P, P, P, I, I, I, I, I,
                                                    I, I, I, I, Dbl, I]
         lib.oracle_decode_kvcache_e4m3.restype = I
+        lib.oracle_attention_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, P, P,
+                                                     I, I]
+        lib.oracle_attention_blocksparse.restype = I
         lib.oracle_e4m3_table.argtypes = [P]
         lib.oracle_e4m3_table.restype = None
         lib.oracle_set_flaw.argtypes = [I]
@@ -270,3 +276,23 @@ def _np_int(a):
     if hasattr(a, "detach"):
         a = a.detach().to("cpu").numpy()
     return a
+
+
+def attention_blocksparse(q, k, v, row_ptr, col, *, scale: float, blk: int = 128,
+                          threads: int = 0):
+    """Dense-layout attention restricted to a block pattern (CSR rows of key blocks per
+    query block of blk positions).  Returns (O float64 like q, L float64 [B,Hq,Sq])."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    B, Hq, Hkv, Sq, Sk, D = _dims(q, k, None)
+    rp = np.ascontiguousarray(_np_int(row_ptr), dtype=np.int32)
+    cl = np.ascontiguousarray(_np_int(col), dtype=np.int32)
+    if cl.size == 0:
+        cl = np.zeros(1, dtype=np.int32)
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    rc = _load().oracle_attention_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
+                                              Hq, Hkv, Sq, Sk, D, float(scale), _ptr(rp),
+                                              _ptr(cl), int(blk), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_blocksparse: bad arguments")
+    return o, lse

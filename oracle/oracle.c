@@ -49,6 +49,13 @@
  * subnormals 2^-6 * m/8, codes 0x7f / 0xff NaN, no infinities), one scale per tensor,
  * stored value = code value * scale.
  *
+ * Block-sparse attention (oracle_attention_blocksparse): Raptor-T abstract, research
+ * background -- BigBird cuts the input into blocks of a block size and computes
+ * attention between blocks; several attention patterns combine into the final one.
+ * Reading: a pattern of (query block, key block) pairs given as rows of key blocks
+ * (CSR: row_ptr[n_qblk + 1], col[nnz]); key j is visible to query i iff block
+ * j / blk is in row i / blk; otherwise exactly the definition above (non-causal).
+ *
  * Return value of every entry point: 0 on success, -1 on bad arguments.
  */
 #include <math.h>
@@ -75,6 +82,7 @@ enum {
     FLAW_PAGES_CONTIGUOUS = 8,/* paged cache read as if pages were in order     */
     FLAW_WINDOW_SHORT = 9,    /* sliding window keeps one key too few           */
     FLAW_E4M3_BIAS = 10,      /* e4m3 exponent bias 8 instead of 7              */
+    FLAW_SPARSE_ROW = 11,     /* block pattern row of the next query block       */
 };
 static int g_flaw = FLAW_NONE;
 void oracle_set_flaw(int flaw) { g_flaw = flaw; }
@@ -378,6 +386,81 @@ void oracle_combine(int n, int D, const double* Os, const double* Ls, double* O,
         for (int d = 0; d < D; ++d) O[d] += w * Os[(size_t)s * D + d];
     }
     *L = Lall;
+}
+
+/*
+ * Exact attention restricted to a block pattern (dense layout, non-causal).
+ * row_ptr[n_qblk + 1], col[nnz]: key blocks of each query block of `blk` positions;
+ * n_qblk = ceil(Sq / blk).  o like q, lse [B, Hq, Sq].  A row whose blocks hold no
+ * key gets O = 0, L = -inf.
+ */
+int oracle_attention_blocksparse(const float* q, const float* k, const float* v, double* o,
+                                 double* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                                 double scale, const int32_t* row_ptr, const int32_t* col,
+                                 int blk, int nthreads)
+{
+    if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, NULL) || !o || !lse || !row_ptr || !col ||
+        blk <= 0)
+        return -1;
+    const int n_qblk = (Sq + blk - 1) / blk, n_kblk = (Sk + blk - 1) / blk;
+    if (row_ptr[0] != 0) return -1;
+    for (int r = 0; r < n_qblk; ++r) {
+        if (row_ptr[r + 1] < row_ptr[r]) return -1;
+        for (int e = row_ptr[r]; e < row_ptr[r + 1]; ++e)
+            if (col[e] < 0 || col[e] >= n_kblk) return -1;
+    }
+    set_threads(nthreads);
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            size_t q_row0, lse_off, lse_step;
+            head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, 0, NULL, b, h,
+                                     &q_row0, &lse_off, &lse_step);
+            double* row = malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+            unsigned char* vis = malloc((size_t)(Sk > 0 ? Sk : 1));
+            if (!row || !vis) {
+                free(row);
+                free(vis);
+                bad = 1;
+                continue;
+            }
+            for (int i = 0; i < Sq; ++i) {
+                int qb = i / blk;
+                if (g_flaw == FLAW_SPARSE_ROW && qb + 1 < n_qblk) qb += 1;
+                memset(vis, 0, (size_t)Sk);
+                for (int e = row_ptr[qb]; e < row_ptr[qb + 1]; ++e)
+                    for (int j = col[e] * blk; j < (col[e] + 1) * blk && j < Sk; ++j) vis[j] = 1;
+                const float* qi = hv.q + (size_t)i * hv.q_stride;
+                double m = -INFINITY;
+                for (int j = 0; j < Sk; ++j) {
+                    row[j] = vis[j] ? scale * dot(qi, hv.k + (size_t)j * hv.kv_stride, D)
+                                    : -INFINITY;
+                    if (row[j] > m) m = row[j];
+                }
+                double* oi = o + ((q_row0 + i) * Hq + h) * (size_t)D;
+                if (m == -INFINITY) {
+                    for (int d = 0; d < D; ++d) oi[d] = 0.0;
+                    lse[lse_off + (size_t)i * lse_step] = -INFINITY;
+                    continue;
+                }
+                double l = 0.0;
+                for (int j = 0; j < Sk; ++j) {
+                    row[j] = (row[j] == -INFINITY) ? 0.0 : exp(row[j] - m);
+                    l += row[j];
+                }
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j < Sk; ++j)
+                        if (row[j] != 0.0) acc += row[j] * (double)hv.v[(size_t)j * hv.kv_stride + d];
+                    oi[d] = acc / l;
+                }
+                lse[lse_off + (size_t)i * lse_step] = m + log(l);
+            }
+            free(row);
+            free(vis);
+        }
+    return bad ? -1 : 0;
 }
 
 /* Value of one e4m3 code. */

@@ -528,6 +528,87 @@ def test_kvcache_e4m3_paged_matches_sdpa():
 
 
 # ---------------------------------------------------------------------------------
+# Block-sparse attention (Raptor-T abstract: BigBird's block pattern)
+
+def random_pattern(n_q, n_k, seed, density=0.35, empty_rows=()):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for r in range(n_q):
+        cols = [] if r in empty_rows else sorted(set(
+            np.flatnonzero(rng.random(n_k) < density).tolist()) | {min(r, n_k - 1)})
+        rows.append(cols)
+    row_ptr = np.zeros(n_q + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum([len(c) for c in rows])
+    col = np.array([c for cols in rows for c in cols], dtype=np.int32)
+    return row_ptr, col
+
+
+def expand_pattern(row_ptr, col, Sq, Sk, blk):
+    mask = np.zeros((Sq, Sk), dtype=bool)
+    for r in range(len(row_ptr) - 1):
+        for c in col[row_ptr[r]:row_ptr[r + 1]]:
+            mask[r * blk:(r + 1) * blk, c * blk:(c + 1) * blk] = True
+    return mask
+
+
+def masked_sdpa(q, k, v, scale, mask):
+    """torch float64 SDPA with a boolean element mask, and logsumexp; rows without a
+    visible key are O = 0, L = -inf."""
+    qt, kt, vt = bshd_to_bhsd64(q), bshd_to_bhsd64(k), bshd_to_bhsd64(v)
+    G = qt.shape[1] // kt.shape[1]
+    kf, vf = kt.repeat_interleave(G, dim=1), vt.repeat_interleave(G, dim=1)
+    m = torch.from_numpy(mask)
+    s = (scale * qt @ kf.transpose(-1, -2)).masked_fill(~m, float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    dead = ~m.any(dim=-1)
+    live = torch.from_numpy(np.where(mask.any(axis=1))[0])
+    o = torch.zeros_like(qt)
+    if live.numel():
+        o[:, :, live] = F.scaled_dot_product_attention(qt[:, :, live], kf, vf,
+                                                       attn_mask=m[live], scale=scale)
+    lse[..., dead] = float("-inf")
+    return o.transpose(1, 2).numpy(), lse.numpy()
+
+
+@pytest.mark.parametrize("Sq,Sk,blk,seed", [(300, 333, 128, 1), (96, 80, 16, 2), (64, 200, 8, 3)])
+def test_blocksparse_matches_sdpa_with_the_expanded_mask(Sq, Sk, blk, seed):
+    B, Hq, Hkv, D = 2, 8, 2, 16
+    q, k, v = rnd((B, Sq, Hq, D), seed), rnd((B, Sk, Hkv, D), seed + 10), \
+        rnd((B, Sk, Hkv, D), seed + 20)
+    n_q, n_k = -(-Sq // blk), -(-Sk // blk)
+    row_ptr, col = random_pattern(n_q, n_k, seed, empty_rows=(1,))
+    O, L = oracle.attention_blocksparse(q, k, v, row_ptr, col, scale=0.3, blk=blk)
+    Or, Lr = masked_sdpa(q, k, v, 0.3, expand_pattern(row_ptr, col, Sq, Sk, blk))
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isneginf(L), np.isneginf(Lr))
+    fin = np.isfinite(Lr)
+    np.testing.assert_allclose(L[fin], Lr[fin], rtol=0, atol=1e-12)
+    assert np.all(O[:, blk:2 * blk] == 0)  # the empty query block
+
+
+def test_blocksparse_with_every_block_is_dense_attention():
+    B, Hq, Hkv, Sq, Sk, D = 1, 4, 2, 70, 90, 8
+    q, k, v = rnd((B, Sq, Hq, D), 30), rnd((B, Sk, Hkv, D), 31), rnd((B, Sk, Hkv, D), 32)
+    n_q, n_k = -(-Sq // 16), -(-Sk // 16)
+    row_ptr = np.arange(n_q + 1, dtype=np.int32) * n_k
+    col = np.tile(np.arange(n_k, dtype=np.int32), n_q)
+    O, L = oracle.attention_blocksparse(q, k, v, row_ptr, col, scale=0.5, blk=16)
+    Or, Lr = sdpa_ref(q, k, v, 0.5, False)
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, Lr, rtol=0, atol=1e-12)
+
+
+def test_blocksparse_rejects_bad_patterns():
+    q, k, v = rnd((1, 20, 2, 4), 40), rnd((1, 20, 1, 4), 41), rnd((1, 20, 1, 4), 42)
+    with pytest.raises(ValueError):  # key block 3 does not exist for 20 keys in blocks of 8
+        oracle.attention_blocksparse(q, k, v, np.array([0, 1, 1, 1], np.int32),
+                                     np.array([3], np.int32), scale=1.0, blk=8)
+    with pytest.raises(ValueError):  # row pointers must not decrease
+        oracle.attention_blocksparse(q, k, v, np.array([0, 2, 1, 2], np.int32),
+                                     np.array([0, 1], np.int32), scale=1.0, blk=8)
+
+
+# ---------------------------------------------------------------------------------
 # Pin strength: every planted mistake is caught by at least one pin above
 
 PIN_BATTERY = [
@@ -541,6 +622,7 @@ PIN_BATTERY = [
     lambda: test_kvcache_lengths_and_window_match_sdpa_on_slices(7),
     lambda: test_kvcache_paged_matches_sdpa(16, 0),
     lambda: test_e4m3_table_matches_torch_float8(),
+    lambda: test_blocksparse_matches_sdpa_with_the_expanded_mask(96, 80, 16, 2),
 ]
 
 
