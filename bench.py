@@ -7,8 +7,10 @@ workload, with the inputs already resident in HBM.  The default workload is the
 encoder-shaped GQA batch (B=64, Hq=48, Hkv=12, S=512, D=64, bf16, non-causal);
 others: llama (B=4, Hq=32, Hkv=8, S=8192, D=128, causal), llama_stress (q x 4),
 decode_b{1,16,64,128,256} (Sq=1, Sk=32768, split-KV), decode_paged_bN (the same
-cache in shuffled pages of 256 keys, gqa_attn_kvcache), varlen (32 packed causal
-sequences of 128..8192 tokens).  Prefill workloads report TFLOP/s, decode GB/s.
+cache in shuffled pages of 256 keys, gqa_attn_kvcache), decode_fp8_bN (that cache in
+e4m3), varlen (32 packed causal sequences of 128..8192 tokens), bigbird (the Llama
+shape, non-causal, with a BigBird-style block pattern over 128-blocks,
+gqa_attn_blocksparse).  Prefill workloads report TFLOP/s, decode GB/s.
 
 Under torchrun every rank runs its own copy of the workload (independent batches,
 no collective on the data path: weak scaling); the time is the max over ranks.
@@ -174,6 +176,8 @@ def workload_by_name(name: str):
         return W.LLAMA_STRESS
     if name == "varlen":
         return W.VARLEN
+    if name == "bigbird":
+        return W.BIGBIRD
     if name.startswith("decode_b"):
         return W.decode(int(name[len("decode_b"):]), num_splits=0)
     if name.startswith("decode_paged_b"):
@@ -228,6 +232,16 @@ class Case:
             self.units, self.unit = self.bytes / 1e9, "GB/s"
             self.launches_per_step = 2 if splits > 1 else 1
             self.kernel = "decode_split_sm100"
+        elif w.block_sparse:
+            q, k, v = W.make_qkv(w, device=device)
+            self.q, self.kv = q, [(k, v)]
+            rp, col = W.bigbird_pattern(w)
+            self.rp, self.col = rp.to(device), col.to(device)
+            self.flops = W.blocksparse_flops(w, rp, col)
+            self.units, self.unit = self.flops / 1e12, "TFLOP/s"
+            self.launches_per_step = 1
+            self.kernel = "prefill_fwd_sm100"
+            self.splits, self.pack = 1, 1
         elif self.varlen:
             lengths = W.varlen_lengths(w)
             q, k, v, cu = W.make_varlen(w, device=device, lengths=lengths)
@@ -268,6 +282,10 @@ class Case:
         k, v = self.kv[self.i % len(self.kv)]
         self.i += 1
         w = self.w
+        if w.block_sparse:
+            self.G.gqa_attn_blocksparse(self.q, k, v, self.rp, self.col, out=self.out,
+                                        lse=self.lse)
+            return
         if w.kv_fp8:
             self.G.gqa_attn_kvcache(self.q, k, v, k_scale=W.FP8_SCALE, v_scale=W.FP8_SCALE,
                                     num_splits=w.num_splits, pack_gqa=w.pack_gqa, out=self.out,
@@ -334,6 +352,21 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
         gb = n * W.decode_bytes(1, w.Hq, w.Hkv, w.Sk, w.D) / 1e9
         return gb / el, (f"{n} x one sequence through its block table (all {w.Hq} heads, "
                          f"Sk={w.Sk}, pages of {w.page_size})"), cores, el
+    if w.block_sparse:
+        q, k, v = W.make_qkv(w, B=1)
+        q, k, v = q[:, :, : w.G].contiguous(), k[:, :, :1].contiguous(), v[:, :, :1].contiguous()
+        rp, col = W.bigbird_pattern(w)
+        import dataclasses
+        w1 = dataclasses.replace(w, B=1, Hq=w.G, Hkv=1)
+        flops = W.blocksparse_flops(w1, rp, col)
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.attention_blocksparse(q, k, v, rp, col, scale=w.scale, blk=128)
+            el += time.perf_counter() - t0
+            n += 1
+        return (n * flops / 1e12 / el,
+                f"{n} x batch element 0, the {w.G} query heads of KV head 0", cores, el)
     if w.Sq == 1 and w.kv_fp8:
         kb, vb = W.make_decode_kv_one(w, 0)
         k8 = (kb.float() / W.FP8_SCALE).to(torch.float8_e4m3fn)[None]
@@ -487,7 +520,18 @@ def run_ours(args, world, rank, local):
         hs = case.lens.cpu().pin_memory()
         dt, ds = torch.empty_like(case.table), torch.empty_like(case.lens)
 
+    if w.block_sparse:
+        hrp, hcol = case.rp.cpu().pin_memory(), case.col.cpu().pin_memory()
+        drp, dcol = torch.empty_like(case.rp), torch.empty_like(case.col)
+
     def e2e_step():
+        if w.block_sparse:
+            for d, h in ((dq, hq), (dk, hk), (dv, hv), (drp, hrp), (dcol, hcol)):
+                d.copy_(h, non_blocking=True)
+            G.gqa_attn_blocksparse(dq, dk, dv, drp, dcol, out=case.out, lse=case.lse)
+            ho.copy_(case.out, non_blocking=True)
+            hl.copy_(case.lse, non_blocking=True)
+            return
         if w.kv_fp8:
             for d, h in ((dq, hq), (dk, hk), (dv, hv)):
                 d.copy_(h, non_blocking=True)
@@ -533,7 +577,8 @@ def run_ours(args, world, rank, local):
     h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + \
         hv.numel() * hv.element_size() + \
         (cu_h.numel() * 4 if cu_h is not None else 0) + \
-        ((ht.numel() + hs.numel()) * 4 if case.paged else 0)
+        ((ht.numel() + hs.numel()) * 4 if case.paged else 0) + \
+        ((hrp.numel() + hcol.numel()) * 4 if w.block_sparse else 0)
     d2h = ho.numel() * 2 + hl.numel() * 4
     err = G.gqa_attn_get_device_error()
     if world > 1:
@@ -586,6 +631,9 @@ def run_ours(args, world, rank, local):
         cfg["total_tokens"] = int(case.q.shape[0])
     if w.kv_fp8:
         cfg["kv_cache"] = f"e4m3 codes, k_scale = v_scale = {W.FP8_SCALE}"
+    if w.block_sparse:
+        cfg["block_pattern"] = dict(w.block_sparse, block=128, blocks=int(case.col.numel()),
+                                    of=int((case.rp.numel() - 1) * -(-w.Sk // 128)))
     if case.paged:
         cfg["page_size"] = w.page_size
         cfg["block_table"] = "seeded shuffle of the page pool"
@@ -597,7 +645,9 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms,
-                    "path": ("gqa_attn_kvcache on the e4m3 cache after pinned host copies "
+                    "path": ("gqa_attn_blocksparse after pinned host copies of q, k, v and "
+                             "the block pattern; results copied back" if w.block_sparse else
+                             "gqa_attn_kvcache on the e4m3 cache after pinned host copies "
                              "of q and the caches; results copied back" if w.kv_fp8 else
                              "gqa_attn_kvcache on the paged cache after pinned host "
                              "copies of q, the page pools, the block table and the lengths; "

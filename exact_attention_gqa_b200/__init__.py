@@ -22,7 +22,8 @@ import math
 from . import _capi
 from ._capi import GqaError, STATUS, STATUS_CODE, strerror
 
-__all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_kvcache", "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
+__all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_kvcache", "gqa_attn_blocksparse",
+           "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
            "gqa_attn_workspace_bytes", "gqa_attn_set_workspace", "gqa_attn_get_device_error",
            "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path"]
 
@@ -171,6 +172,47 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
                               stream)
         if rc != 0:
             raise GqaError("gqa_attn_fwd_f32", rc)
+
+
+def gqa_attn_blocksparse(q, k, v, blk_row_ptr, blk_col, *, scale: float | None = None,
+                         out=None, lse=None):
+    """Non-causal attention restricted to a block pattern (gqa_attn_fwd_blocksparse).
+
+    q [B, Sq, Hq, D], k/v [B, Sk, Hkv, D] bf16 (Hq / Hkv >= 2 and dividing 128);
+    blk_row_ptr int32 [ceil(Sq / 128) + 1] and blk_col int32 [nnz] on the GPU: the
+    128-key blocks each 128-position query block attends to.  Returns (out, lse).
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v), ("blk_row_ptr", blk_row_ptr),
+                    ("blk_col", blk_col)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype == torch.bfloat16):
+        raise ValueError("q, k, v must be bf16")
+    if blk_row_ptr.dtype != torch.int32 or blk_col.dtype != torch.int32:
+        raise ValueError("the block pattern is int32")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("dense inputs are q [B, Sq, Hq, D], k/v [B, Sk, Hkv, D]")
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    if blk_row_ptr.numel() != -(-Sq // 128) + 1:
+        raise ValueError("blk_row_ptr must have ceil(Sq / 128) + 1 entries")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    col = blk_col if blk_col.numel() else torch.zeros(1, dtype=torch.int32, device=q.device)
+    with torch.cuda.device(q.device):
+        rc = _capi.load().gqa_attn_fwd_blocksparse(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
+            _ptr(blk_row_ptr), _ptr(col), _stream_handle(torch, q.device))
+    if rc != 0:
+        raise GqaError("gqa_attn_fwd_blocksparse", rc)
+    return out, lse
 
 
 def gqa_attn_kvcache(q, k_cache, v_cache, *, seqlens_k=None, max_seqlen_k=None,

@@ -22,6 +22,7 @@ EXPORTS = (
     "gqa_attn_get_device_error",
     "gqa_attn_strerror",
     "gqa_attn_decode_noalloc",
+    "gqa_attn_fwd_blocksparse",
     "gqa_attn_decode_kvcache",
     "gqa_attn_decode_paged",
     "gqa_attn_decode_fp8",
@@ -74,6 +75,8 @@ def load() -> ctypes.CDLL:
     lib.gqa_attn_plan.restype = I
     lib.gqa_attn_get_device_error.argtypes = [IP, P]
     lib.gqa_attn_get_device_error.restype = I
+    lib.gqa_attn_fwd_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P]
+    lib.gqa_attn_fwd_blocksparse.restype = I
     lib.gqa_attn_decode_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, P]
     lib.gqa_attn_decode_kvcache.restype = I
     lib.gqa_attn_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,

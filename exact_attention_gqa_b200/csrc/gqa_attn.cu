@@ -207,7 +207,8 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 template <int HD>
 int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                    int Hq, int Hkv, int Sq, int Sk, float scale, int causal, int pack,
-                   const int* cu, int sms, cudaStream_t stream) {
+                   const int* cu, int sms, cudaStream_t stream,
+                   const int* blk_row_ptr = nullptr, const int* blk_col = nullptr) {
     using C = PrefillCfg<HD>;
     {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD>, HD == 64 ? 1 : 2,
@@ -248,6 +249,9 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
         p.hu_group = int(hg);
     }
     p.scale_log2 = scale * kLog2e;
+    p.blk_row_ptr = blk_row_ptr;
+    p.blk_col = blk_col;
+    p.n_kblk = (Sk + C::BN - 1) / C::BN;
     // Row extents of the 3-D views: exactly the rows the caller allocated
     // (packed variable length: Sk carries the packed row count).
     const long long rows_q = cu ? (long long)Sk : (long long)B * Sq;
@@ -261,7 +265,15 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
         !make_map(&to, out, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128))
         return GQA_ERR_CUDA;
     const int grid = p.n_units < sms ? p.n_units : sms;
-    gqa::prefill_fwd_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+    if (blk_row_ptr) {
+        const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD, true>, HD == 64 ? 1024 : 2048,
+                                         C::SMEM_BYTES);
+        if (rc != GQA_OK) return rc;
+        gqa::prefill_fwd_sm100<HD, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv,
+                                                                                     to, p);
+    } else {
+        gqa::prefill_fwd_sm100<HD><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+    }
     return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
@@ -947,6 +959,35 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
                                                 scratch, stream);
 }
 
+
+int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, float* lse,
+                             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                             const int* blk_row_ptr, const int* blk_col, cudaStream_t stream) {
+    int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, 1, 1, false, false);
+    if (rc != GQA_OK) return rc;
+    const int G = Hq / Hkv;
+    // a CTA tile (2 x 128 / G positions) must lie inside one 128-position query block
+    if (G < 2 || 128 % G != 0) return GQA_ERR_UNSUPPORTED;
+    if (B == 0 || Sq == 0) return GQA_OK;
+    if (!q || !out || !lse || !blk_row_ptr || !blk_col || (Sk > 0 && (!k || !v)))
+        return GQA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || !aligned(blk_row_ptr, 4) || !aligned(blk_col, 4))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    if (Sk == 0) {
+        gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(out), (long long)B * Sq * Hq * D, lse,
+            (long long)B * Hq * Sq);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
+    return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 0, 1,
+                                          nullptr, dev->sms, stream, blk_row_ptr, blk_col)
+                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 0, 1,
+                                         nullptr, dev->sms, stream, blk_row_ptr, blk_col);
+}
 
 int gqa_attn_decode_kvcache(const void* q, const void* k_cache, const void* v_cache,
                             const int* seqlens_k, void* out, float* lse, int B, int Hq, int Hkv,

@@ -35,6 +35,11 @@
 // a sub-tile the softmax threads normalise O; with D = 64 a sub-tile whose rows
 // are all real is staged in shared memory and written by one TMA store.
 //
+// Block-sparse form (Raptor-T abstract: BigBird computes attention between blocks of
+// a fixed size, several patterns combined): blk_row_ptr / blk_col list, per query block
+// of 128 positions, the 128-key blocks it attends to; a CTA tile (at most 128 positions,
+// PackGQA with G >= 2) lies in one query block and walks that list instead of 0..n-1.
+//
 // Online softmax in the log2 domain: s2 = s * scale * log2(e).  The running
 // max used for the exponentials is only raised when a block's max exceeds it by
 // more than 8 (a factor 256), so O is rescaled rarely; since O and l always
@@ -62,6 +67,10 @@ struct PrefillParams {
     int kv_major;            // 1: tiles of one (batch, head unit) consecutive (L2 reuse)
     int hu_group;            // kv_major = 0: (batch, head unit) pairs per longest-first pass
     float scale_log2;        // scale * log2(e)
+    // block-sparse: CSR rows of 128-key blocks per 128-position query block (nullptr: dense)
+    const int* blk_row_ptr = nullptr;  // [ceil(Sq / 128) + 1]
+    const int* blk_col = nullptr;      // [nnz], ascending within a row
+    int n_kblk = 0;                    // ceil(Sk / 128): key blocks that exist
 };
 
 template <int HD>
@@ -108,9 +117,10 @@ struct TileInfo {
     int nblk[2];          // K/V blocks each sub-tile visits (0: nothing to compute)
     int valid[2];         // sub-tile holds at least one real query row
     int full_blk[2];      // blocks [0, full_blk) need no mask for any row
+    int kb0;              // block-sparse: first entry of this tile's row in blk_col
 };
 
-template <int BN>
+template <int BN, bool SPARSE = false>
 __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
     TileInfo ti;
     if (p.kv_major) {
@@ -163,7 +173,29 @@ __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
         int first_lim = p.causal ? min(ti.sk, p0 + ti.sk - ti.sq + 1) : ti.sk;
         ti.full_blk[i] = first_lim > 0 ? first_lim / BN : 0;
     }
+    ti.kb0 = 0;
+    if constexpr (SPARSE) {
+        // both sub-tiles lie in query block qb and share its list of key blocks
+        const int qb = (ti.m * 2 * p.sub_pos) >> 7;
+        const int r0 = __ldg(p.blk_row_ptr + qb), r1 = __ldg(p.blk_row_ptr + qb + 1);
+        ti.kb0 = r0;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) ti.nblk[i] = ti.valid[i] ? max(r1 - r0, 0) : 0;
+    }
     return ti;
+}
+
+// Key block of a tile's j-th step: j itself (dense) or the j-th entry of the tile's
+// row of the block pattern; an index past the keys is reported and clamped.
+template <bool SPARSE>
+__device__ __forceinline__ int sparse_block(const PrefillParams& p, const TileInfo& ti, int j) {
+    if constexpr (!SPARSE) return j;
+    int kb = __ldg(p.blk_col + ti.kb0 + j);
+    if (kb < 0 || kb >= p.n_kblk) {
+        raise_device_error(kDevBadTile);
+        kb = 0;
+    }
+    return kb;
 }
 
 // Wait that ignores the abort flag (used to drain in-flight copies before exit).
@@ -177,7 +209,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
-template <int HD>
+// SPARSE = true walks the block pattern of p.blk_row_ptr / p.blk_col; the dense
+// instantiation carries none of that code.
+template <int HD, bool SPARSE = false>
 __global__ void __launch_bounds__(320, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -253,7 +287,7 @@ __global__ void __launch_bounds__(320, 1)
             uint8_t* sV = smem + C::OFF_V;
             int qc = 0, kc = 0, vc = 0;
             for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
-                const TileInfo ti = decode_tile<BN>(p, t);
+                const TileInfo ti = decode_tile<BN, SPARSE>(p, t);
                 const int n = max(ti.nblk[0], ti.nblk[1]);
                 if (n == 0) continue;
                 const int qs = qc % QS;
@@ -274,7 +308,7 @@ __global__ void __launch_bounds__(320, 1)
                 ++qc;
                 const int kvh = p.pack ? ti.hu : ti.hu / p.G;
                 for (int j = 0; j < n; ++j) {
-                    const int z = ti.k_row0 + j * BN;
+                    const int z = ti.k_row0 + sparse_block<SPARSE>(p, ti, j) * BN;
                     {
                         const int s = kc % ST;
                         if (!mbar_wait(bar_k_empty + s, ((kc / ST) & 1) ^ 1, abort_flag))
@@ -340,7 +374,7 @@ __global__ void __launch_bounds__(320, 1)
                         (accumulate || kk > 0) ? 1u : 0u);
             };
             for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
-                const TileInfo ti = decode_tile<BN>(p, t);
+                const TileInfo ti = decode_tile<BN, SPARSE>(p, t);
                 const int n = max(ti.nblk[0], ti.nblk[1]);
                 if (n == 0) continue;
                 const int qs = qc % QS;
@@ -437,7 +471,7 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t s_phase = 0, o_phase = 0;
         uint32_t ec = 0;  // O stores issued through the shared-memory box
         for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
-            const TileInfo ti = decode_tile<BN>(p, t);
+            const TileInfo ti = decode_tile<BN, SPARSE>(p, t);
             // this warp's sub-tile, selected without runtime array indexing
             const int my_valid = i ? ti.valid[1] : ti.valid[0];
             const int my_p0 = i ? ti.p0[1] : ti.p0[0];
@@ -469,8 +503,15 @@ __global__ void __launch_bounds__(320, 1)
                 tmem_ld_wait();
 #pragma unroll
                 for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-                if (j >= my_full) {
-                    const int lim = key_lim - j * BN;
+                // keys of this block past the row's limit (causal diagonal, sequence end)
+                int kbj = j;
+                bool need_mask = j >= my_full;
+                if constexpr (SPARSE) {
+                    kbj = sparse_block<SPARSE>(p, ti, j);
+                    need_mask = (kbj + 1) * BN > key_lim;
+                }
+                if (need_mask) {
+                    const int lim = key_lim - kbj * BN;
 #pragma unroll
                     for (int c = 0; c < 4; ++c)
 #pragma unroll

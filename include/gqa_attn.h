@@ -228,6 +228,26 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
                             int num_splits, int pack_gqa, cudaStream_t stream);
 
 /*
+ * Block-sparse attention: gqa_attn_fwd's dense, non-causal forward restricted to a
+ * pattern of (query block, key block) pairs with blocks of 128 positions and 128 keys
+ * (Raptor-T abstract: BigBird divides the input into blocks of a block size and
+ * computes attention between blocks, several patterns combined into one).
+ *   key j is visible to query i iff j / 128 is in row i / 128 of the pattern;
+ *   blk_row_ptr: device int32 [ceil(Sq / 128) + 1], blk_row_ptr[0] = 0, non-
+ *     decreasing; blk_col: device int32 [blk_row_ptr[last]], the key blocks of each
+ *     row, in [0, ceil(Sk / 128)) (an entry outside raises device error 2 and block 0
+ *     is read in its place), ascending within a row (any order gives the same result);
+ *   the pattern is the same for every batch element and head;
+ *   a query whose blocks hold no key gets O = 0, L = -inf.
+ * Layouts, dtypes (bf16 only), D (64, 128) and errors as gqa_attn_fwd.  PackGQA is
+ * always on, and the group size G = Hq / Hkv must be >= 2 and divide 128 (one CTA tile
+ * of 256 / G positions then lies in one query block); otherwise GQA_ERR_UNSUPPORTED.
+ */
+int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, float* lse,
+                             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
+                             const int* blk_row_ptr, const int* blk_col, cudaStream_t stream);
+
+/*
  * Decode (one new query position per sequence) against a KV cache, with per-
  * sequence cache lengths and an optional sliding window.  Ultralytics glossary
  * "Grouped Query Attention (GQA)": during generation the model keeps the keys and

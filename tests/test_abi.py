@@ -237,3 +237,28 @@ def test_fp8_argument_errors(lib, kw, code):
 
 def test_fp8_empty_batch_is_a_noop(lib):
     assert fp8_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+
+
+def sparse_call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=8, Hkv=2, Sq=256,
+                Sk=256, D=128, scale=0.125, rp=FAKE, col=FAKE):
+    return lib.gqa_attn_fwd_blocksparse(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, rp,
+                                        col, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=8, Hkv=8), "GQA_ERR_UNSUPPORTED"),     # G = 1: a tile spans two query blocks
+    (dict(Hq=6, Hkv=2), "GQA_ERR_UNSUPPORTED"),     # G = 3 does not divide 128
+    (dict(rp=None), "GQA_ERR_NULL"),
+    (dict(col=None), "GQA_ERR_NULL"),
+    (dict(q=None), "GQA_ERR_NULL"),
+    (dict(D=96), "GQA_ERR_HEADDIM"),
+    (dict(scale=-1.0), "GQA_ERR_SCALE"),
+    (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
+    (dict(col=ctypes.c_void_p(0x1002)), "GQA_ERR_ALIGN"),
+])
+def test_blocksparse_argument_errors(lib, kw, code):
+    assert G.STATUS[sparse_call(lib, **kw)] == code
+
+
+def test_blocksparse_empty_batch_is_a_noop(lib):
+    assert sparse_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0

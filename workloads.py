@@ -46,6 +46,7 @@ class Workload:
     varlen: dict = field(default_factory=dict)  # {"n": 32, "lo": 128, "hi": 8192}
     page_size: int = 0  # > 0: decode against a paged KV cache of pages of this many keys
     kv_fp8: bool = False  # decode against an e4m3 KV cache (scale FP8_SCALE)
+    block_sparse: dict = field(default_factory=dict)  # {"window": 3, "global": 2, "random": 3}
 
     @property
     def scale(self) -> float:
@@ -95,6 +96,50 @@ def decode_fp8(B: int) -> Workload:
     batch-size guide, hardware adaptation section)."""
     return Workload(f"decode_fp8_b{B}_sk32768", B=B, Hq=32, Hkv=8, Sq=1, Sk=32768, D=128,
                     dtype="bf16", causal=False, seed=4, pack_gqa=1, num_splits=0, kv_fp8=True)
+
+
+BIGBIRD = Workload("bigbird_b4_s8192_blk128", B=4, Hq=32, Hkv=8, Sq=8192, Sk=8192, D=128,
+                   dtype="bf16", causal=False, seed=6,
+                   block_sparse={"window": 3, "global": 2, "random": 3})
+
+
+def bigbird_pattern(w: Workload):
+    """BigBird-style block pattern over 128-position blocks (Raptor-T abstract: several
+    patterns combined): a window of `window` blocks around the diagonal, `global` blocks
+    every row attends to and whose rows attend to everything, and `random` more blocks
+    per row drawn from a seeded generator.  Returns CSR (row_ptr, col) int32 tensors."""
+    blk = 128
+    n_q, n_k = -(-w.Sq // blk), -(-w.Sk // blk)
+    bs = w.block_sparse
+    g = _gen("cpu", w.seed + 101)
+    rows = []
+    for r in range(n_q):
+        if r < bs["global"]:
+            rows.append(list(range(n_k)))
+            continue
+        cols = set(range(min(bs["global"], n_k)))
+        half = bs["window"] // 2
+        cols |= {c for c in range(r - half, r + half + 1) if 0 <= c < n_k}
+        rnd = torch.randperm(n_k, generator=g)[: bs["random"]].tolist()
+        cols |= set(rnd)
+        rows.append(sorted(cols))
+    row_ptr = torch.zeros(n_q + 1, dtype=torch.int32)
+    row_ptr[1:] = torch.cumsum(torch.tensor([len(c) for c in rows]), 0)
+    col = torch.tensor([c for cs in rows for c in cs], dtype=torch.int32)
+    return row_ptr, col
+
+
+def blocksparse_flops(w: Workload, row_ptr, col) -> int:
+    """4*D flops per visible (query, key) pair per head under the block pattern."""
+    blk = 128
+    pairs = 0
+    rp = row_ptr.tolist()
+    cl = col.tolist()
+    for r in range(len(rp) - 1):
+        rows_in = min(blk, w.Sq - r * blk)
+        keys = sum(min(blk, w.Sk - c * blk) for c in cl[rp[r]:rp[r + 1]])
+        pairs += rows_in * keys
+    return 4 * w.D * pairs * w.B * w.Hq
 
 
 VARLEN = Workload("varlen32_len128to8192_causal", B=32, Hq=32, Hkv=8, Sq=0, Sk=0, D=128,
