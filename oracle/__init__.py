@@ -18,6 +18,7 @@ states the passage of the pages it follows in the C source:
                           log-sum-exp weighted combine.
 * ``attention_tiled``  -- the per-step normalised (form 1) and deferred
                           normalisation (form 2) online-softmax forms.
+* ``attention_backward`` -- dQ, dK, dV for a given dO (FA-2 page, backward pass).
 * ``attention_blocksparse`` -- attention restricted to a (query block, key block)
                           pattern (Raptor-T abstract: BigBird's block-sparse attention).
 * ``decode_kvcache``   -- one decode query per sequence against a dense or paged
@@ -55,6 +56,7 @@ FLAWS = {
     "window_short": 9,
     "e4m3_bias": 10,
     "sparse_row": 11,
+    "bwd_no_d": 12,
 }
 
 
@@ -95,6 +97,9 @@ def _load():
         lib.oracle_attention_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, P, P,
                                                      I, I]
         lib.oracle_attention_blocksparse.restype = I
+        lib.oracle_attention_backward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, Dbl, I,
+                                                  I]
+        lib.oracle_attention_backward.restype = I
         lib.oracle_e4m3_table.argtypes = [P]
         lib.oracle_e4m3_table.restype = None
         lib.oracle_set_flaw.argtypes = [I]
@@ -296,3 +301,18 @@ def attention_blocksparse(q, k, v, row_ptr, col, *, scale: float, blk: int = 128
     if rc != 0:
         raise ValueError("oracle_attention_blocksparse: bad arguments")
     return o, lse
+
+
+def attention_backward(q, k, v, dout, *, scale: float, causal: bool, threads: int = 0):
+    """Gradients (dQ like q, dK and dV like k; float64) of the forward for a given dO."""
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, Hq, Hkv, Sq, Sk, D = _dims(q, k, None)
+    dq = np.zeros(q.shape, dtype=np.float64)
+    dk = np.zeros(k.shape, dtype=np.float64)
+    dv = np.zeros(k.shape, dtype=np.float64)
+    rc = _load().oracle_attention_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq),
+                                           _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D,
+                                           float(scale), int(bool(causal)), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_backward: bad arguments")
+    return dq, dk, dv

@@ -56,6 +56,14 @@
  * (CSR: row_ptr[n_qblk + 1], col[nnz]); key j is visible to query i iff block
  * j / blk is in row i / blk; otherwise exactly the definition above (non-causal).
  *
+ * Backward (oracle_attention_backward): FA-2 summary page, parallelism paragraph of the
+ * backward pass -- dK and dV accumulate per key/value column block, dQ is shared; GQA
+ * paragraph -- dK and dV are summed over the query heads that share a K/V head.  The
+ * page gives no formulas; these are the derivatives of the definition above (L's
+ * derivative is not needed: only dO is given):
+ *   dV = P^T dO;  dP = dO V^T;  D_i = sum_j P_ij dP_ij;  dS = P * (dP - D);
+ *   dQ = scale * dS K;  dK = scale * dS^T Q.
+ *
  * Return value of every entry point: 0 on success, -1 on bad arguments.
  */
 #include <math.h>
@@ -83,6 +91,7 @@ enum {
     FLAW_WINDOW_SHORT = 9,    /* sliding window keeps one key too few           */
     FLAW_E4M3_BIAS = 10,      /* e4m3 exponent bias 8 instead of 7              */
     FLAW_SPARSE_ROW = 11,     /* block pattern row of the next query block       */
+    FLAW_BWD_NO_D = 12,       /* backward: dS = P * dP, without subtracting D    */
 };
 static int g_flaw = FLAW_NONE;
 void oracle_set_flaw(int flaw) { g_flaw = flaw; }
@@ -386,6 +395,88 @@ void oracle_combine(int n, int D, const double* Os, const double* Ls, double* O,
         for (int d = 0; d < D; ++d) O[d] += w * Os[(size_t)s * D + d];
     }
     *L = Lall;
+}
+
+/*
+ * Gradients of O = attention(Q, K, V) for a given dO (dense layout, optional causal
+ * mask with the forward's bottom-right alignment).  dq like q; dk, dv like k (summed
+ * over the G query heads of each K/V head).  Rows without a visible key contribute
+ * nothing.  P is recomputed in float64 from the definition.
+ */
+int oracle_attention_backward(const float* q, const float* k, const float* v, const float* dout,
+                              double* dq, double* dk, double* dv, int B, int Hq, int Hkv,
+                              int Sq, int Sk, int D, double scale, int causal, int nthreads)
+{
+    if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, NULL) || !dout || !dq || !dk || !dv)
+        return -1;
+    const int G = Hq / Hkv;
+    memset(dq, 0, sizeof(double) * (size_t)B * Sq * Hq * D);
+    memset(dk, 0, sizeof(double) * (size_t)B * Sk * Hkv * D);
+    memset(dv, 0, sizeof(double) * (size_t)B * Sk * Hkv * D);
+    set_threads(nthreads);
+    int bad = 0;
+    /* one (sequence, K/V head) per task: its dk, dv rows are written by it alone */
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < Hkv; ++c) {
+            double* P = malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+            double* dP = malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+            if (!P || !dP) {
+                free(P);
+                free(dP);
+                bad = 1;
+                continue;
+            }
+            for (int h = c * G; h < (c + 1) * G; ++h) {
+                size_t q_row0, lse_off, lse_step;
+                head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, NULL, b,
+                                         h, &q_row0, &lse_off, &lse_step);
+                const size_t k_row0 = (size_t)b * Sk;
+                for (int i = 0; i < Sq; ++i) {
+                    const float* qi = hv.q + (size_t)i * hv.q_stride;
+                    const float* doi = dout + ((q_row0 + i) * Hq + h) * (size_t)D;
+                    double m = -INFINITY;
+                    for (int j = 0; j < Sk; ++j) {
+                        P[j] = key_visible(i, j, Sq, Sk, causal)
+                                   ? scale * dot(qi, hv.k + (size_t)j * hv.kv_stride, D)
+                                   : -INFINITY;
+                        if (P[j] > m) m = P[j];
+                    }
+                    if (m == -INFINITY) continue; /* no visible key: no gradient */
+                    double l = 0.0;
+                    for (int j = 0; j < Sk; ++j) {
+                        P[j] = (P[j] == -INFINITY) ? 0.0 : exp(P[j] - m);
+                        l += P[j];
+                    }
+                    double Di = 0.0;
+                    for (int j = 0; j < Sk; ++j) {
+                        P[j] /= l;
+                        dP[j] = 0.0;
+                        if (P[j] == 0.0) continue;
+                        for (int d = 0; d < D; ++d)
+                            dP[j] += (double)doi[d] * (double)hv.v[(size_t)j * hv.kv_stride + d];
+                        Di += P[j] * dP[j];
+                    }
+                    if (g_flaw == FLAW_BWD_NO_D) Di = 0.0;
+                    double* dqi = dq + ((q_row0 + i) * Hq + h) * (size_t)D;
+                    for (int j = 0; j < Sk; ++j) {
+                        if (P[j] == 0.0) continue;
+                        const double dS = P[j] * (dP[j] - Di);
+                        const float* kj = hv.k + (size_t)j * hv.kv_stride;
+                        double* dkj = dk + ((k_row0 + j) * Hkv + c) * (size_t)D;
+                        double* dvj = dv + ((k_row0 + j) * Hkv + c) * (size_t)D;
+                        for (int d = 0; d < D; ++d) {
+                            dqi[d] += scale * dS * (double)kj[d];
+                            dkj[d] += scale * dS * (double)qi[d];
+                            dvj[d] += P[j] * (double)doi[d];
+                        }
+                    }
+                }
+            }
+            free(P);
+            free(dP);
+        }
+    return bad ? -1 : 0;
 }
 
 /*

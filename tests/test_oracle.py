@@ -609,6 +609,63 @@ def test_blocksparse_rejects_bad_patterns():
 
 
 # ---------------------------------------------------------------------------------
+# Backward (FA-2 page: dK, dV per K/V block, dQ shared; GQA: dK, dV summed over heads)
+
+def autograd_ref(q, k, v, do, scale, causal):
+    """torch float64 autograd through scaled_dot_product_attention (enable_gqa), with
+    the forward's bottom-right causal mask; returns dq, dk, dv in [B, S, H, D]."""
+    qt, kt, vt = (bshd_to_bhsd64(a).clone().requires_grad_(True) for a in (q, k, v))
+    mask = None
+    if causal:
+        Sq, Sk = qt.shape[2], kt.shape[2]
+        mask = torch.ones(Sq, Sk, dtype=torch.bool).tril(diagonal=Sk - Sq)
+    o = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale,
+                                       enable_gqa=True)
+    o.backward(bshd_to_bhsd64(do))
+    return tuple(t.grad.transpose(1, 2).numpy() for t in (qt, kt, vt))
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal", [
+    (2, 8, 2, 33, 33, 16, True),     # GQA, causal, Sq = Sk
+    (1, 6, 2, 20, 45, 8, True),      # Sq < Sk, bottom-right
+    (2, 4, 1, 17, 29, 16, False),    # MQA
+    (1, 3, 3, 12, 12, 32, False),    # MHA
+])
+def test_backward_matches_torch_autograd_float64(B, Hq, Hkv, Sq, Sk, D, causal):
+    seed = B * 100 + Sq + Sk
+    q, k, v = rnd((B, Sq, Hq, D), seed), rnd((B, Sk, Hkv, D), seed + 1), \
+        rnd((B, Sk, Hkv, D), seed + 2)
+    do = rnd((B, Sq, Hq, D), seed + 3)
+    got = oracle.attention_backward(q, k, v, do, scale=0.4, causal=causal)
+    for g, r in zip(got, autograd_ref(q, k, v, do, 0.4, causal)):
+        np.testing.assert_allclose(g, r, rtol=0, atol=1e-11)
+
+
+def test_backward_matches_finite_differences_of_the_forward():
+    # d/dx of sum(O * dO) by central differences of the (separately pinned) forward
+    B, Hq, Hkv, Sq, Sk, D = 1, 2, 1, 4, 5, 3
+    q, k, v = rnd((B, Sq, Hq, D), 60), rnd((B, Sk, Hkv, D), 61), rnd((B, Sk, Hkv, D), 62)
+    do = rnd((B, Sq, Hq, D), 63)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, scale=0.7, causal=True)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.attention(q_, k_, v_, scale=0.7, causal=True)
+        return float(np.sum(o * do.astype(np.float64)))
+
+    h = 2.0 ** -8  # exact in float32 next to values of order 1
+    for arr, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        for idx in np.ndindex(arr.shape):
+            plus, minus = arr.copy(), arr.copy()
+            plus[idx] += h
+            minus[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = plus, minus
+            num = (loss(*args_p) - loss(*args_m)) / (float(plus[idx]) - float(minus[idx]))
+            assert abs(num - grad[idx]) < 2e-4, (which, idx, num, grad[idx])
+
+
+# ---------------------------------------------------------------------------------
 # Pin strength: every planted mistake is caught by at least one pin above
 
 PIN_BATTERY = [
@@ -623,6 +680,7 @@ PIN_BATTERY = [
     lambda: test_kvcache_paged_matches_sdpa(16, 0),
     lambda: test_e4m3_table_matches_torch_float8(),
     lambda: test_blocksparse_matches_sdpa_with_the_expanded_mask(96, 80, 16, 2),
+    lambda: test_backward_matches_torch_autograd_float64(2, 8, 2, 33, 33, 16, True),
 ]
 
 
