@@ -10,7 +10,8 @@ decode_b{1,16,64,128,256} (Sq=1, Sk=32768, split-KV), decode_paged_bN (the same
 cache in shuffled pages of 256 keys, gqa_attn_kvcache), decode_fp8_bN (that cache in
 e4m3), varlen (32 packed causal sequences of 128..8192 tokens), bigbird (the Llama
 shape, non-causal, with a BigBird-style block pattern over 128-blocks,
-gqa_attn_blocksparse).  Prefill workloads report TFLOP/s, decode GB/s.
+gqa_attn_blocksparse), llama_bwd (the backward pass of the Llama shape: dQ, dK, dV,
+gqa_attn_backward).  Prefill workloads report TFLOP/s, decode GB/s.
 
 Under torchrun every rank runs its own copy of the workload (independent batches,
 no collective on the data path: weak scaling); the time is the max over ranks.
@@ -178,6 +179,8 @@ def workload_by_name(name: str):
         return W.VARLEN
     if name == "bigbird":
         return W.BIGBIRD
+    if name == "llama_bwd":
+        return W.LLAMA_BWD
     if name.startswith("decode_b"):
         return W.decode(int(name[len("decode_b"):]), num_splits=0)
     if name.startswith("decode_paged_b"):
@@ -232,6 +235,18 @@ class Case:
             self.units, self.unit = self.bytes / 1e9, "GB/s"
             self.launches_per_step = 2 if splits > 1 else 1
             self.kernel = "decode_split_sm100"
+        elif w.backward:
+            q, k, v = W.make_qkv(w, device=device)
+            self.q, self.kv = q, [(k, v)]
+            self.do = W.make_dout(w, device=device)
+            self.fwd_out, self.fwd_lse = G.gqa_attn(q, k, v, causal=w.causal)
+            self.grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+            # the backward's five products against the forward's two
+            self.flops = int(2.5 * W.attention_flops(w.B, w.Hq, w.Sq, w.Sk, w.D, w.causal))
+            self.units, self.unit = self.flops / 1e12, "TFLOP/s"
+            self.launches_per_step = 3
+            self.kernel = "bwd_dkdv + bwd_dq"
+            self.splits, self.pack = 1, 0
         elif w.block_sparse:
             q, k, v = W.make_qkv(w, device=device)
             self.q, self.kv = q, [(k, v)]
@@ -282,6 +297,11 @@ class Case:
         k, v = self.kv[self.i % len(self.kv)]
         self.i += 1
         w = self.w
+        if w.backward:
+            dq, dk, dv = self.grads
+            self.G.gqa_attn_backward(self.q, k, v, self.fwd_out, self.fwd_lse, self.do,
+                                     causal=w.causal, dq=dq, dk=dk, dv=dv)
+            return
         if w.block_sparse:
             self.G.gqa_attn_blocksparse(self.q, k, v, self.rp, self.col, out=self.out,
                                         lse=self.lse)
@@ -352,6 +372,22 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
         gb = n * W.decode_bytes(1, w.Hq, w.Hkv, w.Sk, w.D) / 1e9
         return gb / el, (f"{n} x one sequence through its block table (all {w.Hq} heads, "
                          f"Sk={w.Sk}, pages of {w.page_size})"), cores, el
+    if w.backward:
+        # batch element 0, the query heads of K/V head 0, the first 2048 positions (with
+        # the causal mask those queries see only those keys: a problem of its own)
+        S = 2048
+        q, k, v = W.make_qkv(w, B=1, Sq=S, Sk=S)
+        q, k, v = q[:, :, : w.G].contiguous(), k[:, :, :1].contiguous(), v[:, :, :1].contiguous()
+        do = torch.randn(1, S, w.G, w.D, generator=torch.Generator().manual_seed(7)).bfloat16()
+        flops = int(2.5 * W.attention_flops(1, w.G, S, S, w.D, w.causal))
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.attention_backward(q, k, v, do, scale=w.scale, causal=w.causal)
+            el += time.perf_counter() - t0
+            n += 1
+        return (n * flops / 1e12 / el, f"{n} x the backward of batch element 0, the {w.G} "
+                f"query heads of K/V head 0, positions 0..{S - 1}", cores, el)
     if w.block_sparse:
         q, k, v = W.make_qkv(w, B=1)
         q, k, v = q[:, :, : w.G].contiguous(), k[:, :, :1].contiguous(), v[:, :, :1].contiguous()
@@ -520,11 +556,26 @@ def run_ours(args, world, rank, local):
         hs = case.lens.cpu().pin_memory()
         dt, ds = torch.empty_like(case.table), torch.empty_like(case.lens)
 
+    if w.backward:
+        hout, hlse = case.fwd_out.cpu().pin_memory(), case.fwd_lse.cpu().pin_memory()
+        hdo = case.do.cpu().pin_memory()
+        dout_d, dlse_d, ddo_d = (torch.empty_like(t) for t in (case.fwd_out, case.fwd_lse,
+                                                               case.do))
+        hgrads = tuple(torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in case.grads)
     if w.block_sparse:
         hrp, hcol = case.rp.cpu().pin_memory(), case.col.cpu().pin_memory()
         drp, dcol = torch.empty_like(case.rp), torch.empty_like(case.col)
 
     def e2e_step():
+        if w.backward:
+            for d, h in ((dq, hq), (dk, hk), (dv, hv), (dout_d, hout), (dlse_d, hlse),
+                         (ddo_d, hdo)):
+                d.copy_(h, non_blocking=True)
+            gd = G.gqa_attn_backward(dq, dk, dv, dout_d, dlse_d, ddo_d, causal=w.causal,
+                                     dq=case.grads[0], dk=case.grads[1], dv=case.grads[2])
+            for h, d in zip(hgrads, gd):
+                h.copy_(d, non_blocking=True)
+            return
         if w.block_sparse:
             for d, h in ((dq, hq), (dk, hk), (dv, hv), (drp, hrp), (dcol, hcol)):
                 d.copy_(h, non_blocking=True)
@@ -580,6 +631,9 @@ def run_ours(args, world, rank, local):
         ((ht.numel() + hs.numel()) * 4 if case.paged else 0) + \
         ((hrp.numel() + hcol.numel()) * 4 if w.block_sparse else 0)
     d2h = ho.numel() * 2 + hl.numel() * 4
+    if w.backward:
+        h2d += hout.numel() * 2 + hlse.numel() * 4 + hdo.numel() * 2
+        d2h = sum(t.numel() * 2 for t in hgrads)
     err = G.gqa_attn_get_device_error()
     if world > 1:
         import torch.distributed as dist
@@ -631,6 +685,9 @@ def run_ours(args, world, rank, local):
         cfg["total_tokens"] = int(case.q.shape[0])
     if w.kv_fp8:
         cfg["kv_cache"] = f"e4m3 codes, k_scale = v_scale = {W.FP8_SCALE}"
+    if w.backward:
+        cfg["pass"] = "backward: dQ, dK, dV for a seeded dO (O and L from the forward)"
+        cfg["flops"] = "2.5 x the forward's (five products against two)"
     if w.block_sparse:
         cfg["block_pattern"] = dict(w.block_sparse, block=128, blocks=int(case.col.numel()),
                                     of=int((case.rp.numel() - 1) * -(-w.Sk // 128)))
@@ -645,7 +702,9 @@ def run_ours(args, world, rank, local):
             "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms,
-                    "path": ("gqa_attn_blocksparse after pinned host copies of q, k, v and "
+                    "path": ("gqa_attn_backward after pinned host copies of q, k, v, O, L "
+                             "and dO; dQ, dK, dV copied back" if w.backward else
+                             "gqa_attn_blocksparse after pinned host copies of q, k, v and "
                              "the block pattern; results copied back" if w.block_sparse else
                              "gqa_attn_kvcache on the e4m3 cache after pinned host copies "
                              "of q and the caches; results copied back" if w.kv_fp8 else

@@ -23,6 +23,7 @@ from . import _capi
 from ._capi import GqaError, STATUS, STATUS_CODE, strerror
 
 __all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_kvcache", "gqa_attn_blocksparse",
+           "gqa_attn_backward",
            "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
            "gqa_attn_workspace_bytes", "gqa_attn_set_workspace", "gqa_attn_get_device_error",
            "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path"]
@@ -172,6 +173,44 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
                               stream)
         if rc != 0:
             raise GqaError("gqa_attn_fwd_f32", rc)
+
+
+def gqa_attn_backward(q, k, v, out, lse, dout, *, causal: bool = False,
+                      scale: float | None = None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV of gqa_attn's dense forward for the gradient dout (gqa_attn_bwd).
+
+    q, out, dout [B, Sq, Hq, D], k/v [B, Sk, Hkv, D] bf16 on the GPU; lse [B, Hq, Sq] as
+    gqa_attn returned it for the same inputs, causal and scale.  Returns (dq, dk, dv).
+    """
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype == dout.dtype == torch.bfloat16):
+        raise ValueError("q, k, v, out, dout must be bf16")
+    if lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape or out.shape != q.shape \
+            or dout.shape != q.shape:
+        raise ValueError("q/out/dout [B, Sq, Hq, D], k/v [B, Sk, Hkv, D]")
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    lib = _capi.load()
+    with torch.cuda.device(q.device):
+        _workspace(torch, q.device, lib.gqa_attn_bwd_workspace_bytes(B, Hq, Sq))
+        rc = lib.gqa_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Sk, D, scale,
+                              int(bool(causal)), _stream_handle(torch, q.device))
+    if rc != 0:
+        raise GqaError("gqa_attn_bwd", rc)
+    return dq, dk, dv
 
 
 def gqa_attn_blocksparse(q, k, v, blk_row_ptr, blk_col, *, scale: float | None = None,

@@ -23,6 +23,8 @@ EXPORTS = (
     "gqa_attn_strerror",
     "gqa_attn_decode_noalloc",
     "gqa_attn_fwd_blocksparse",
+    "gqa_attn_bwd_workspace_bytes",
+    "gqa_attn_bwd",
     "gqa_attn_decode_kvcache",
     "gqa_attn_decode_paged",
     "gqa_attn_decode_fp8",
@@ -75,6 +77,10 @@ def load() -> ctypes.CDLL:
     lib.gqa_attn_plan.restype = I
     lib.gqa_attn_get_device_error.argtypes = [IP, P]
     lib.gqa_attn_get_device_error.restype = I
+    lib.gqa_attn_bwd_workspace_bytes.argtypes = [I, I, I]
+    lib.gqa_attn_bwd_workspace_bytes.restype = Z
+    lib.gqa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
+    lib.gqa_attn_bwd.restype = I
     lib.gqa_attn_fwd_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P]
     lib.gqa_attn_fwd_blocksparse.restype = I
     lib.gqa_attn_decode_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, P]

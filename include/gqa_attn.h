@@ -228,6 +228,25 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
                             int num_splits, int pack_gqa, cudaStream_t stream);
 
 /*
+ * Backward pass of the dense forward: dQ, dK, dV for a given dO (FA-2 summary page,
+ * backward paragraph: dK and dV accumulate per K/V column block, dQ is shared between
+ * them; GQA paragraph: dK and dV are summed over the query heads sharing a K/V head).
+ * With P recomputed from lse and D_i = rowsum(dO_i * O_i):
+ *   dV = P^T dO;  dS = P * (dO V^T - D);  dK = scale dS^T Q;  dQ = scale dS K.
+ * q, out, dout, dq [B, Sq, Hq, D]; k, v, dk, dv [B, Sk, Hkv, D] (bf16, contiguous);
+ * lse [B, Hq, Sq] fp32 as gqa_attn_fwd wrote it with the same q, k, v, scale and
+ * causal; D 64 or 128; causal as gqa_attn_fwd (bottom-right).  Every output element is
+ * written (no accumulation into the caller's buffers, no atomics: run to run the
+ * results are bit-identical).  The registered workspace (gqa_attn_set_workspace) must
+ * hold gqa_attn_bwd_workspace_bytes(B, Hq, Sq) bytes (GQA_ERR_WORKSPACE otherwise);
+ * nothing is allocated or synchronised.  Status codes as gqa_attn_fwd.
+ */
+size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Sq);
+int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq,
+                 int Sk, int D, float scale, int causal, cudaStream_t stream);
+
+/*
  * Block-sparse attention: gqa_attn_fwd's dense, non-causal forward restricted to a
  * pattern of (query block, key block) pairs with blocks of 128 positions and 128 keys
  * (Raptor-T abstract: BigBird divides the input into blocks of a block size and

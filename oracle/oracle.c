@@ -401,7 +401,8 @@ void oracle_combine(int n, int D, const double* Os, const double* Ls, double* O,
  * Gradients of O = attention(Q, K, V) for a given dO (dense layout, optional causal
  * mask with the forward's bottom-right alignment).  dq like q; dk, dv like k (summed
  * over the G query heads of each K/V head).  Rows without a visible key contribute
- * nothing.  P is recomputed in float64 from the definition.
+ * nothing.  P is recomputed in float64 from the definition.  Needs B*Hq*Sk*D*16 bytes
+ * of host memory for the per-head partial dk, dv.
  */
 int oracle_attention_backward(const float* q, const float* k, const float* v, const float* dout,
                               double* dq, double* dk, double* dv, int B, int Hq, int Hkv,
@@ -410,15 +411,20 @@ int oracle_attention_backward(const float* q, const float* k, const float* v, co
     if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, NULL) || !dout || !dq || !dk || !dv)
         return -1;
     const int G = Hq / Hkv;
+    const size_t kv_elems = (size_t)Sk * D;  /* one head's dk (or dv) */
     memset(dq, 0, sizeof(double) * (size_t)B * Sq * Hq * D);
     memset(dk, 0, sizeof(double) * (size_t)B * Sk * Hkv * D);
     memset(dv, 0, sizeof(double) * (size_t)B * Sk * Hkv * D);
+    /* each (sequence, query head) accumulates its dk, dv into a buffer of its own; the
+     * G heads of a K/V head are summed afterwards, in head order */
+    double* part = malloc(sizeof(double) * 2 * kv_elems * (size_t)B * Hq + 1);
+    if (!part) return -1;
+    memset(part, 0, sizeof(double) * 2 * kv_elems * (size_t)B * Hq);
     set_threads(nthreads);
     int bad = 0;
-    /* one (sequence, K/V head) per task: its dk, dv rows are written by it alone */
 #pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
     for (int b = 0; b < B; ++b)
-        for (int c = 0; c < Hkv; ++c) {
+        for (int h = 0; h < Hq; ++h) {
             double* P = malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
             double* dP = malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
             if (!P || !dP) {
@@ -427,55 +433,66 @@ int oracle_attention_backward(const float* q, const float* k, const float* v, co
                 bad = 1;
                 continue;
             }
-            for (int h = c * G; h < (c + 1) * G; ++h) {
-                size_t q_row0, lse_off, lse_step;
-                head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, NULL, b,
-                                         h, &q_row0, &lse_off, &lse_step);
-                const size_t k_row0 = (size_t)b * Sk;
-                for (int i = 0; i < Sq; ++i) {
-                    const float* qi = hv.q + (size_t)i * hv.q_stride;
-                    const float* doi = dout + ((q_row0 + i) * Hq + h) * (size_t)D;
-                    double m = -INFINITY;
-                    for (int j = 0; j < Sk; ++j) {
-                        P[j] = key_visible(i, j, Sq, Sk, causal)
-                                   ? scale * dot(qi, hv.k + (size_t)j * hv.kv_stride, D)
-                                   : -INFINITY;
-                        if (P[j] > m) m = P[j];
-                    }
-                    if (m == -INFINITY) continue; /* no visible key: no gradient */
-                    double l = 0.0;
-                    for (int j = 0; j < Sk; ++j) {
-                        P[j] = (P[j] == -INFINITY) ? 0.0 : exp(P[j] - m);
-                        l += P[j];
-                    }
-                    double Di = 0.0;
-                    for (int j = 0; j < Sk; ++j) {
-                        P[j] /= l;
-                        dP[j] = 0.0;
-                        if (P[j] == 0.0) continue;
-                        for (int d = 0; d < D; ++d)
-                            dP[j] += (double)doi[d] * (double)hv.v[(size_t)j * hv.kv_stride + d];
-                        Di += P[j] * dP[j];
-                    }
-                    if (g_flaw == FLAW_BWD_NO_D) Di = 0.0;
-                    double* dqi = dq + ((q_row0 + i) * Hq + h) * (size_t)D;
-                    for (int j = 0; j < Sk; ++j) {
-                        if (P[j] == 0.0) continue;
-                        const double dS = P[j] * (dP[j] - Di);
-                        const float* kj = hv.k + (size_t)j * hv.kv_stride;
-                        double* dkj = dk + ((k_row0 + j) * Hkv + c) * (size_t)D;
-                        double* dvj = dv + ((k_row0 + j) * Hkv + c) * (size_t)D;
-                        for (int d = 0; d < D; ++d) {
-                            dqi[d] += scale * dS * (double)kj[d];
-                            dkj[d] += scale * dS * (double)qi[d];
-                            dvj[d] += P[j] * (double)doi[d];
-                        }
+            double* pdk = part + 2 * kv_elems * ((size_t)b * Hq + h);
+            double* pdv = pdk + kv_elems;
+            size_t q_row0, lse_off, lse_step;
+            head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, NULL, b, h,
+                                     &q_row0, &lse_off, &lse_step);
+            for (int i = 0; i < Sq; ++i) {
+                const float* qi = hv.q + (size_t)i * hv.q_stride;
+                const float* doi = dout + ((q_row0 + i) * Hq + h) * (size_t)D;
+                double m = -INFINITY;
+                for (int j = 0; j < Sk; ++j) {
+                    P[j] = key_visible(i, j, Sq, Sk, causal)
+                               ? scale * dot(qi, hv.k + (size_t)j * hv.kv_stride, D)
+                               : -INFINITY;
+                    if (P[j] > m) m = P[j];
+                }
+                if (m == -INFINITY) continue; /* no visible key: no gradient */
+                double l = 0.0;
+                for (int j = 0; j < Sk; ++j) {
+                    P[j] = (P[j] == -INFINITY) ? 0.0 : exp(P[j] - m);
+                    l += P[j];
+                }
+                double Di = 0.0;
+                for (int j = 0; j < Sk; ++j) {
+                    P[j] /= l;
+                    dP[j] = 0.0;
+                    if (P[j] == 0.0) continue;
+                    for (int d = 0; d < D; ++d)
+                        dP[j] += (double)doi[d] * (double)hv.v[(size_t)j * hv.kv_stride + d];
+                    Di += P[j] * dP[j];
+                }
+                if (g_flaw == FLAW_BWD_NO_D) Di = 0.0;
+                double* dqi = dq + ((q_row0 + i) * Hq + h) * (size_t)D;
+                for (int j = 0; j < Sk; ++j) {
+                    if (P[j] == 0.0) continue;
+                    const double dS = P[j] * (dP[j] - Di);
+                    const float* kj = hv.k + (size_t)j * hv.kv_stride;
+                    for (int d = 0; d < D; ++d) {
+                        dqi[d] += scale * dS * (double)kj[d];
+                        pdk[(size_t)j * D + d] += scale * dS * (double)qi[d];
+                        pdv[(size_t)j * D + d] += P[j] * (double)doi[d];
                     }
                 }
             }
             free(P);
             free(dP);
         }
+    if (!bad)
+        for (int b = 0; b < B; ++b)
+            for (int c = 0; c < Hkv; ++c)
+                for (int h = c * G; h < (c + 1) * G; ++h) {
+                    const double* pdk = part + 2 * kv_elems * ((size_t)b * Hq + h);
+                    const double* pdv = pdk + kv_elems;
+                    for (int j = 0; j < Sk; ++j)
+                        for (int d = 0; d < D; ++d) {
+                            const size_t o = (((size_t)b * Sk + j) * Hkv + c) * D + d;
+                            dk[o] += pdk[(size_t)j * D + d];
+                            dv[o] += pdv[(size_t)j * D + d];
+                        }
+                }
+    free(part);
     return bad ? -1 : 0;
 }
 

@@ -6,6 +6,11 @@ output element whose reference magnitude is so large that one bf16 ulp exceeds
 1e-2 (|O| >= 2) may differ by up to that ulp instead: rounding to bf16 alone
 can use half of it.  fp32 path: max |dO| <= 1e-4, max |dL| <= 1e-4.
 Rows with no visible key must give exactly O = 0 and L = -inf.
+
+Backward (bf16 gradients, P and dS rounded to bf16 before their products, outputs
+rounded to bf16: each about 2^-9 relative): the forward's bar scaled by the
+gradient's magnitude, max |d| <= 1e-2 * max(1, max |ref|) and
+mean |d| <= 1e-3 * max(1, mean |ref|).
 """
 import numpy as np
 
@@ -49,4 +54,24 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, *, f32=False):
     assert np.all(err <= allowed), stats
     assert stats["mean_abs"] <= BF16_MEAN_ABS, stats
     assert stats["max_lse"] <= BF16_MAX_LSE, stats
+    return stats
+
+
+GRAD_MAX_REL = 1e-2
+GRAD_MEAN_REL = 1e-3
+
+
+def compare_grad(g_gpu, ref):
+    """Assert the backward bar for one gradient tensor; returns the observed errors."""
+    g = to_np(g_gpu) if not isinstance(g_gpu, np.ndarray) else g_gpu.astype(np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert g.shape == ref.shape, (g.shape, ref.shape)
+    assert np.all(np.isfinite(g)), "non-finite gradient"
+    err = np.abs(g - ref)
+    big = max(1.0, float(np.abs(ref).max(initial=0.0)))
+    typ = max(1.0, float(np.abs(ref).mean())) if ref.size else 1.0
+    stats = {"max_abs": float(err.max(initial=0.0)), "mean_abs": float(err.mean()) if err.size else 0.0,
+             "max_ref": big, "mean_ref": typ}
+    assert stats["max_abs"] <= GRAD_MAX_REL * big, stats
+    assert stats["mean_abs"] <= GRAD_MEAN_REL * typ, stats
     return stats

@@ -47,6 +47,7 @@ class Workload:
     page_size: int = 0  # > 0: decode against a paged KV cache of pages of this many keys
     kv_fp8: bool = False  # decode against an e4m3 KV cache (scale FP8_SCALE)
     block_sparse: dict = field(default_factory=dict)  # {"window": 3, "global": 2, "random": 3}
+    backward: bool = False  # time the backward pass (dQ, dK, dV) of this forward
 
     @property
     def scale(self) -> float:
@@ -68,6 +69,8 @@ ENCODER = Workload("encoder_b64_h48kv12_s512_d64", B=64, Hq=48, Hkv=12, Sq=512, 
                    D=64, dtype="bf16", causal=False, seed=1)
 LLAMA = Workload("llama8b_prefill_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8192, Sk=8192,
                  D=128, dtype="bf16", causal=True, seed=2)
+LLAMA_BWD = Workload("llama8b_backward_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8192, Sk=8192,
+                     D=128, dtype="bf16", causal=True, seed=2, backward=True)
 LLAMA_STRESS = Workload("llama8b_prefill_b4_s8192_causal_qx4", B=4, Hq=32, Hkv=8, Sq=8192,
                         Sk=8192, D=128, dtype="bf16", causal=True, seed=3, q_mult=4.0)
 DECODE_BATCHES = (1, 16, 64, 128, 256)
@@ -166,6 +169,13 @@ def make_qkv(w: Workload, device="cpu", *, B=None, Sq=None, Sk=None):
     if w.q_mult != 1.0:
         q = q * w.q_mult
     return tuple(t.transpose(1, 2).contiguous() for t in (q, k, v))
+
+
+def make_dout(w: Workload, device="cpu"):
+    """The output gradient dO [B, Sq, Hq, D] for the backward pass (seeded N(0, 1))."""
+    g = _gen(device, w.seed + 500)
+    d = torch.randn(w.B, w.Hq, w.Sq, w.D, generator=g, device=device).to(w.torch_dtype)
+    return d.transpose(1, 2).contiguous()
 
 
 def varlen_lengths(w: Workload, n=None, lo=None, hi=None) -> torch.Tensor:
