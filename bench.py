@@ -43,15 +43,17 @@ import workloads as W  # noqa: E402
 METRIC = "GQA attn fwd TFLOP/s (prefill) & KV-read GB/s (decode), % roofline, 1×B200"
 L2_BYTES = 126 * 2**20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["exact_attention_gqa_b200/csrc/" + f for f in
-                  ("sm100_ptx.cuh", "prefill_sm100.cuh", "decode.cuh", "gqa_attn.cu")]
+_FWD_SOURCES = ("sm100_ptx.cuh", "prefill_sm100.cuh", "decode.cuh", "gqa_attn.cu")
+# the sources each timed kernel is built from (its traffic line is keyed by their hash)
+KERNEL_SOURCES = {"forward": _FWD_SOURCES,
+                  "backward": _FWD_SOURCES + ("backward.cuh", "backward_host.cuh")}
 
 
 # ----------------------------------------------------------------------------- helpers
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str = "") -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        h.update((ROOT / f).read_bytes())
+    for f in KERNEL_SOURCES["backward" if kernel.startswith("bwd") else "forward"]:
+        h.update((ROOT / "exact_attention_gqa_b200" / "csrc" / f).read_bytes())
     return h.hexdigest()[:12]
 
 
@@ -68,7 +70,7 @@ def load_traffic(workload: str, kernel: str):
     f = ROOT / "profiles" / "dram_traffic.txt"
     if not f.exists():
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel)
     for line in f.read_text().splitlines():
         parts = line.split()
         if len(parts) >= 4 and not line.startswith("#") and parts[0] == workload \
@@ -717,7 +719,7 @@ def run_ours(args, world, rank, local):
                                "overlapped")},
             "gpu_launches": steps * case.launches_per_step,
             "clocks": clocks.summary(), "device_error": err,
-            "kernel_source": kernel_source_hash(), "library": G.library_path()}
+            "kernel_source": kernel_source_hash(case.kernel), "library": G.library_path()}
     print(json.dumps(line), flush=True)
 
 
