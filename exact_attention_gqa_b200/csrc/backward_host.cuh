@@ -4,7 +4,7 @@
 // helpers it uses; kept apart so the forward's translation unit text does not change
 // with the backward.
 #pragma once
-#include "backward.cuh"
+#include "backward_tc.cuh"
 
 extern "C" {
 
@@ -46,38 +46,52 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
         ws = g_ws[dev];
     }
     if (!ws.ptr || ws.bytes < gqa_attn_bwd_workspace_bytes(B, Hq, Sq)) return GQA_ERR_WORKSPACE;
-    gqa::BwdParams p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.k = static_cast<const __nv_bfloat16*>(k);
-    p.v = static_cast<const __nv_bfloat16*>(v);
+    gqa::BwdParams p;  // D = rowsum(dO * O)
     p.o = static_cast<const __nv_bfloat16*>(out);
     p.dout = static_cast<const __nv_bfloat16*>(dout);
-    p.lse = lse;
     p.dvec = static_cast<float*>(ws.ptr);
-    p.dq = static_cast<__nv_bfloat16*>(dq);
-    p.dk = static_cast<__nv_bfloat16*>(dk);
-    p.dv = static_cast<__nv_bfloat16*>(dv);
     p.B = B;
     p.Hq = Hq;
-    p.Hkv = Hkv;
     p.Sq = Sq;
-    p.Sk = Sk;
-    p.G = Hq / Hkv;
-    p.causal = causal ? 1 : 0;
-    p.scale = scale;
-    p.scale_log2 = scale * kLog2e;
+    gqa::BwdTcParams tp;
+    tp.lse = lse;
+    tp.dvec = static_cast<const float*>(ws.ptr);
+    tp.B = B;
+    tp.Hq = Hq;
+    tp.Hkv = Hkv;
+    tp.Sq = Sq;
+    tp.Sk = Sk;
+    tp.G = Hq / Hkv;
+    tp.causal = causal ? 1 : 0;
+    tp.scale = scale;
+    tp.scale_log2 = scale * kLog2e;
+    // [rows, heads, D] views: 128-row boxes for the resident tiles, 64-row for the stream
+    CUtensorMap mq128, mo128, mk128, mv128, mq64, mo64, mk64, mv64;
+    const long long rq = (long long)B * Sq, rk = (long long)B * Sk;
+    if (!make_map(&mq128, q, rq, Hq, D, 1, 128) || !make_map(&mo128, dout, rq, Hq, D, 1, 128) ||
+        !make_map(&mk128, k, rk, Hkv, D, 1, 128) || !make_map(&mv128, v, rk, Hkv, D, 1, 128) ||
+        !make_map(&mq64, q, rq, Hq, D, 1, 64) || !make_map(&mo64, dout, rq, Hq, D, 1, 64) ||
+        !make_map(&mk64, k, rk, Hkv, D, 1, 64) || !make_map(&mv64, v, rk, Hkv, D, 1, 64))
+        return GQA_ERR_CUDA;
     auto launch = [&](auto tag) -> int {
         constexpr int HD = decltype(tag)::value;
-        constexpr int S1 = gqa::bwd_dkdv_smem<HD>(), S2 = gqa::bwd_dq_smem<HD>();
+        constexpr int S1 = gqa::BwdTcCfg<HD, false>::SMEM, S2 = gqa::BwdTcCfg<HD, true>::SMEM;
         const int sh = HD == 64 ? 0 : 1;
-        int r = ensure_smem_limit(gqa::bwd_dkdv<HD>, 4096 << sh, S1);
-        if (r == GQA_OK) r = ensure_smem_limit(gqa::bwd_dq<HD>, 16384 << sh, S2);
+        int r = ensure_smem_limit(gqa::bwd_tc<HD, false>, 4096 << sh, S1);
+        if (r == GQA_OK) r = ensure_smem_limit(gqa::bwd_tc<HD, true>, 16384 << sh, S2);
         if (r != GQA_OK) return r;
         const long long rows = (long long)B * Sq * Hq;
         gqa::bwd_dot_do_o<HD><<<unsigned((rows + 7) / 8), 256, 0, stream>>>(p);
-        gqa::bwd_dkdv<HD><<<dim3((Sk + gqa::kBwdKeys - 1) / gqa::kBwdKeys, Hkv, B), 128, S1,
-                            stream>>>(p);
-        gqa::bwd_dq<HD><<<dim3((Sq + gqa::kBwdQ - 1) / gqa::kBwdQ, Hq, B), 128, S2, stream>>>(p);
+        gqa::BwdTcParams t1 = tp;
+        t1.out0 = static_cast<__nv_bfloat16*>(dk);
+        t1.out1 = static_cast<__nv_bfloat16*>(dv);
+        gqa::bwd_tc<HD, false><<<dim3((Sk + 127) / 128, Hkv, B), 320, S1, stream>>>(
+            mk128, mv128, mq64, mo64, t1);
+        gqa::BwdTcParams t2 = tp;
+        t2.out0 = static_cast<__nv_bfloat16*>(dq);
+        t2.out1 = nullptr;
+        gqa::bwd_tc<HD, true><<<dim3((Sq + 127) / 128, Hq, B), 320, S2, stream>>>(
+            mq128, mo128, mk64, mv64, t2);
         return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
     };
     return D == 128 ? launch(std::integral_constant<int, 128>())
