@@ -11,7 +11,7 @@ cache in shuffled pages of 256 keys, gqa_attn_kvcache), decode_fp8_bN (that cach
 e4m3), varlen (32 packed causal sequences of 128..8192 tokens), bigbird (the Llama
 shape, non-causal, with a BigBird-style block pattern over 128-blocks,
 gqa_attn_blocksparse), llama_bwd (the backward pass of the Llama shape: dQ, dK, dV,
-gqa_attn_backward).  Prefill workloads report TFLOP/s, decode GB/s.
+gqa_attn_backward; llama_bwd_b1: one batch element of it).  Prefill workloads report TFLOP/s, decode GB/s.
 
 Under torchrun every rank runs its own copy of the workload (independent batches,
 no collective on the data path: weak scaling); the time is the max over ranks.
@@ -183,6 +183,8 @@ def workload_by_name(name: str):
         return W.BIGBIRD
     if name == "llama_bwd":
         return W.LLAMA_BWD
+    if name == "llama_bwd_b1":
+        return W.LLAMA_BWD_B1
     if name.startswith("decode_b"):
         return W.decode(int(name[len("decode_b"):]), num_splits=0)
     if name.startswith("decode_paged_b"):
@@ -247,7 +249,7 @@ class Case:
             self.flops = int(2.5 * W.attention_flops(w.B, w.Hq, w.Sq, w.Sk, w.D, w.causal))
             self.units, self.unit = self.flops / 1e12, "TFLOP/s"
             self.launches_per_step = 3
-            self.kernel = "bwd_dkdv + bwd_dq"
+            self.kernel = "bwd_tc"
             self.splits, self.pack = 1, 0
         elif w.block_sparse:
             q, k, v = W.make_qkv(w, device=device)

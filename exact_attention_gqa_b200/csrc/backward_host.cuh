@@ -6,6 +6,10 @@
 #pragma once
 #include "backward_tc.cuh"
 
+#ifndef GQA_BWD_EW
+#define GQA_BWD_EW 8
+#endif
+
 extern "C" {
 
 size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Sq) {
@@ -75,22 +79,25 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
         return GQA_ERR_CUDA;
     auto launch = [&](auto tag) -> int {
         constexpr int HD = decltype(tag)::value;
-        constexpr int S1 = gqa::BwdTcCfg<HD, false>::SMEM, S2 = gqa::BwdTcCfg<HD, true>::SMEM;
+        constexpr int EW = GQA_BWD_EW;
+        using C1 = gqa::BwdTcCfg<HD, false, EW>;
+        using C2 = gqa::BwdTcCfg<HD, true, EW>;
+        constexpr int S1 = C1::SMEM, S2 = C2::SMEM;
         const int sh = HD == 64 ? 0 : 1;
-        int r = ensure_smem_limit(gqa::bwd_tc<HD, false>, 4096 << sh, S1);
-        if (r == GQA_OK) r = ensure_smem_limit(gqa::bwd_tc<HD, true>, 16384 << sh, S2);
+        int r = ensure_smem_limit(gqa::bwd_tc<HD, false, EW>, 4096 << sh, S1);
+        if (r == GQA_OK) r = ensure_smem_limit(gqa::bwd_tc<HD, true, EW>, 16384 << sh, S2);
         if (r != GQA_OK) return r;
         const long long rows = (long long)B * Sq * Hq;
         gqa::bwd_dot_do_o<HD><<<unsigned((rows + 7) / 8), 256, 0, stream>>>(p);
         gqa::BwdTcParams t1 = tp;
         t1.out0 = static_cast<__nv_bfloat16*>(dk);
         t1.out1 = static_cast<__nv_bfloat16*>(dv);
-        gqa::bwd_tc<HD, false><<<dim3((Sk + 127) / 128, Hkv, B), 320, S1, stream>>>(
+        gqa::bwd_tc<HD, false, EW><<<dim3((Sk + 127) / 128, Hkv, B), C1::THREADS, S1, stream>>>(
             mk128, mv128, mq64, mo64, t1);
         gqa::BwdTcParams t2 = tp;
         t2.out0 = static_cast<__nv_bfloat16*>(dq);
         t2.out1 = nullptr;
-        gqa::bwd_tc<HD, true><<<dim3((Sq + 127) / 128, Hq, B), 320, S2, stream>>>(
+        gqa::bwd_tc<HD, true, EW><<<dim3((Sq + 127) / 128, Hq, B), C2::THREADS, S2, stream>>>(
             mq128, mo128, mk64, mv64, t2);
         return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
     };

@@ -42,10 +42,13 @@ struct BwdTcParams {
     float scale_log2;  // scale * log2(e)
 };
 
-template <int HD, bool DQ>
+template <int HD, bool DQ, int EW>
 struct BwdTcCfg {
     static constexpr int M = 128;       // resident rows
     static constexpr int N = 64;        // streamed rows per block
+    static constexpr int NG = EW / 4;   // column groups: warps per TMEM lane quarter
+    static constexpr int CW = N / NG;   // columns of S (and dP) per elementwise warp
+    static constexpr int THREADS = 32 * (EW + 2);
     static constexpr int CH = HD / 64;  // 64-dimension chunks (one 128-byte swizzle atom wide)
     static constexpr int STAGES = HD == 128 ? 4 : 6;
     static constexpr int RES_ATOM = M * 128;  // one chunk of a resident tile
@@ -56,7 +59,7 @@ struct BwdTcCfg {
     static constexpr int OFF_X = 0;
     static constexpr int OFF_Y = RES_TILE;
     static constexpr int OFF_ST = 2 * RES_TILE;
-    static constexpr int OFF_LD = OFF_ST + STAGES * STAGE;  // [STAGES][2][N] fp32: L log2, D
+    static constexpr int OFF_LD = OFF_ST + STAGES * STAGE;  // [STAGES][2][N] fp32: -L log2e, -D
     static constexpr int LD_BYTES = DQ ? 0 : STAGES * 2 * N * 4;
     static constexpr int OFF_BAR = OFF_LD + LD_BYTES;
     static constexpr int NBAR = 1 + 2 * STAGES + 2 + 2 + 1 + 1;
@@ -71,6 +74,29 @@ struct BwdTcCfg {
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[16]) {
+    tmem_ld16(taddr, r);
+}
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[32]) {
+    tmem_ld32(taddr, r);
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -80,15 +106,24 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[15])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[8]) {
+    tmem_st8(taddr, r);
+}
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[16]) {
+    tmem_st16(taddr, r);
+}
 
-template <int HD, bool DQ>
-__global__ void __launch_bounds__(320, 1)
+template <int HD, bool DQ, int EW>
+__global__ void __launch_bounds__(BwdTcCfg<HD, DQ, EW>::THREADS, 1)
     bwd_tc(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_y,
            const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
            const BwdTcParams p) {
-    using C = BwdTcCfg<HD, DQ>;
+    using C = BwdTcCfg<HD, DQ, EW>;
     constexpr int N = C::N;
     constexpr int ST = C::STAGES;
+    constexpr int CW = C::CW;
+    constexpr int WP = EW;      // producer warp
+    constexpr int WM = EW + 1;  // MMA warp
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -147,14 +182,14 @@ __global__ void __launch_bounds__(320, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_sp + i, 1);
-            mbar_init(bar_p + i, 8);
+            mbar_init(bar_p + i, EW);
         }
         mbar_init(bar_acc, 1);
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 9) {
+    if (warp == WM) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
         tmem_relinquish();
     }
@@ -163,7 +198,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 8) {
+    if (warp == WP) {
         // ------------------------------------------------------------ TMA producer
         const int zx = DQ ? b * p.Sq + r0 : b * p.Sk + r0;
         if (lane == 0 && n > 0) {
@@ -185,15 +220,15 @@ __global__ void __launch_bounds__(320, 1)
             int s0, hs;
             block(t, s0, hs);
             if constexpr (!DQ) {
-                // L (log2 units) and D of the block's 64 queries; 0 past the end
+                // -L (log2 units) and -D of the block's 64 queries; 0 past the end
                 const size_t row = (size_t(b) * p.Hq + hs) * p.Sq;
                 float* dst = sLD + s * 2 * N;
 #pragma unroll
                 for (int k = 0; k < N / 32; ++k) {
                     const int i = s0 + k * 32 + lane;
                     const bool ok = i < p.Sq;
-                    dst[k * 32 + lane] = ok ? p.lse[row + i] * 1.4426950408889634f : 0.f;
-                    dst[N + k * 32 + lane] = ok ? p.dvec[row + i] : 0.f;
+                    dst[k * 32 + lane] = ok ? p.lse[row + i] * -1.4426950408889634f : 0.f;
+                    dst[N + k * 32 + lane] = ok ? -p.dvec[row + i] : 0.f;
                 }
                 __syncwarp();
             }
@@ -217,7 +252,7 @@ __global__ void __launch_bounds__(320, 1)
                 if (u > 0) drain_wait(bar_full + s, (u - 1) & 1);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == WM) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && n > 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, N, 0, 0);
@@ -233,8 +268,11 @@ __global__ void __launch_bounds__(320, 1)
             auto str_off = [](int kk) {
                 return uint64_t(((kk >> 2) * C::STR_ATOM + (kk & 3) * 32) >> 4);
             };
-            // P / dS of stream rows 16 kk .. +15: packed columns written by half kk >> 1
-            auto p_col = [](int kk) { return uint32_t((kk >> 1) * 32 + (kk & 1) * 8); };
+            // P / dS of stream rows 16 kk .. +15: the packed columns that the warp holding
+            // S columns [16 kk / CW * CW, + CW) wrote at the start of its slice
+            auto p_col = [](int kk) {
+                return uint32_t((16 * kk / CW) * CW + (16 * kk % CW) / 2);
+            };
             if (!mbar_wait(bar_x, 0, abort_flag)) goto mma_done;
             for (int t = 0; t <= n; ++t) {
                 if (t < n) {
@@ -284,15 +322,16 @@ __global__ void __launch_bounds__(320, 1)
         const int lq = warp & 3, hf = warp >> 2;
         const int row = lq * 32 + lane;  // resident row of this thread
         const uint32_t lane_base = uint32_t(lq * 32) << 16;
-        const float sl2 = p.scale_log2;
-        // dQ: L and D belong to this thread's query row
-        float l2_row = 0.f, d_row = 0.f;
+        const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
+        // dQ: -L (log2 units) and -D belong to this thread's query row
+        uint64_t nl_row = 0, nd_row = 0;
         if constexpr (DQ) {
             const int i = r0 + row;
             if (i < p.Sq) {
                 const size_t li = (size_t(b) * p.Hq + hx) * p.Sq + i;
-                l2_row = p.lse[li] * 1.4426950408889634f;
-                d_row = p.dvec[li];
+                const float nl = p.lse[li] * -1.4426950408889634f, nd = -p.dvec[li];
+                nl_row = f2_pack(nl, nl);
+                nd_row = f2_pack(nd, nd);
             }
         }
         bool ok = true;
@@ -303,25 +342,23 @@ __global__ void __launch_bounds__(320, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t tS = tmem + lane_base + C::BUF0 + bf * C::BUF + hf * 32;
-            uint32_t sr[32], dr[32];
-            tmem_ld32(tS, sr);
-            tmem_ld32(tS + N, dr);
+            const uint32_t tS = tmem + lane_base + C::BUF0 + bf * C::BUF + hf * CW;
+            uint32_t sr[CW], dr[CW];
+            tmem_ld_cols(tS, sr);
+            tmem_ld_cols(tS + N, dr);
             int s0, hs;
             block(t, s0, hs);
-            const int col0 = s0 + hf * 32;  // first streamed row (column) of this half
+            const int col0 = s0 + hf * CW;  // first streamed row (column) of this slice
             const float* lcol = nullptr;
-            const float* dcol = nullptr;
             if constexpr (!DQ) {
                 const int s = t % ST;
-                // L, D were written before the block's full barrier completed
+                // -L, -D were written before the block's full barrier completed
                 if (!mbar_wait_warp(bar_full + s, (t / ST) & 1, abort_flag)) {
                     tmem_ld_wait();
                     ok = false;
                     break;
                 }
-                lcol = sLD + s * 2 * N + hf * 32;
-                dcol = lcol + N;
+                lcol = sLD + s * 2 * N + hf * CW;
             }
             tmem_ld_wait();
             reg_fence(sr);
@@ -329,58 +366,69 @@ __global__ void __launch_bounds__(320, 1)
             // causal / ragged masking, decided per warp
             bool need_mask;
             if constexpr (DQ) {
-                need_mask = col0 + 32 > p.Sk ||
-                            (p.causal && col0 + 31 > r0 + lq * 32 + shift);
+                need_mask = col0 + CW > p.Sk ||
+                            (p.causal && col0 + CW - 1 > r0 + lq * 32 + shift);
             } else {
-                need_mask = col0 + 32 > p.Sq ||
+                need_mask = col0 + CW > p.Sq ||
                             (p.causal && r0 + lq * 32 + 31 > col0 + shift);
             }
-            uint32_t pp[16], dd[16];
+            uint32_t pp[CW / 2], dd[CW / 2];
 #pragma unroll
-            for (int e8 = 0; e8 < 32; e8 += 8) {
-                float lv[8], dv8[8];
+            for (int e8 = 0; e8 < CW; e8 += 8) {
+                uint64_t nl[4], nd[4];
                 if constexpr (DQ) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        lv[q] = l2_row;
-                        dv8[q] = d_row;
+                    for (int q = 0; q < 4; ++q) {
+                        nl[q] = nl_row;
+                        nd[q] = nd_row;
                     }
                 } else {
                     const float4 l0 = *reinterpret_cast<const float4*>(lcol + e8);
                     const float4 l1 = *reinterpret_cast<const float4*>(lcol + e8 + 4);
-                    const float4 d0 = *reinterpret_cast<const float4*>(dcol + e8);
-                    const float4 d1 = *reinterpret_cast<const float4*>(dcol + e8 + 4);
-                    lv[0] = l0.x; lv[1] = l0.y; lv[2] = l0.z; lv[3] = l0.w;
-                    lv[4] = l1.x; lv[5] = l1.y; lv[6] = l1.z; lv[7] = l1.w;
-                    dv8[0] = d0.x; dv8[1] = d0.y; dv8[2] = d0.z; dv8[3] = d0.w;
-                    dv8[4] = d1.x; dv8[5] = d1.y; dv8[6] = d1.z; dv8[7] = d1.w;
+                    const float4 d0 = *reinterpret_cast<const float4*>(lcol + N + e8);
+                    const float4 d1 = *reinterpret_cast<const float4*>(lcol + N + e8 + 4);
+                    nl[0] = f2_pack(l0.x, l0.y);
+                    nl[1] = f2_pack(l0.z, l0.w);
+                    nl[2] = f2_pack(l1.x, l1.y);
+                    nl[3] = f2_pack(l1.z, l1.w);
+                    nd[0] = f2_pack(d0.x, d0.y);
+                    nd[1] = f2_pack(d0.z, d0.w);
+                    nd[2] = f2_pack(d1.x, d1.y);
+                    nd[3] = f2_pack(d1.z, d1.w);
                 }
 #pragma unroll
                 for (int e2 = 0; e2 < 8; e2 += 2) {
                     const int e = e8 + e2;
-                    float pv[2], dsv[2];
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        float pr = ex2_approx(fmaf(__uint_as_float(sr[e + q]), sl2, -lv[e2 + q]));
-                        if (need_mask) {
-                            const int cidx = col0 + e + q;
-                            bool vis;
-                            if constexpr (DQ) {
-                                vis = cidx < p.Sk && (!p.causal || cidx <= r0 + row + shift);
-                            } else {
-                                vis = cidx < p.Sq && (!p.causal || r0 + row <= cidx + shift);
-                            }
-                            if (!vis) pr = 0.f;
+                    float a0, a1;
+                    f2_unpack(ffma2(f2_pack(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])),
+                                    sl2x2, nl[e2 >> 1]),
+                              a0, a1);
+                    float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+                    if (need_mask) {
+                        const int c0 = col0 + e;
+                        bool v0, v1;
+                        if constexpr (DQ) {
+                            v0 = c0 < p.Sk && (!p.causal || c0 <= r0 + row + shift);
+                            v1 = c0 + 1 < p.Sk && (!p.causal || c0 + 1 <= r0 + row + shift);
+                        } else {
+                            v0 = c0 < p.Sq && (!p.causal || r0 + row <= c0 + shift);
+                            v1 = c0 + 1 < p.Sq && (!p.causal || r0 + row <= c0 + 1 + shift);
                         }
-                        pv[q] = pr;
-                        dsv[q] = pr * (__uint_as_float(dr[e + q]) - dv8[e2 + q]);
+                        if (!v0) p0 = 0.f;
+                        if (!v1) p1 = 0.f;
                     }
-                    pp[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-                    dd[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+                    float s0v, s1v;
+                    f2_unpack(fmul2(f2_pack(p0, p1),
+                                    fadd2(f2_pack(__uint_as_float(dr[e]),
+                                                  __uint_as_float(dr[e + 1])),
+                                          nd[e2 >> 1])),
+                              s0v, s1v);
+                    pp[e >> 1] = pack_bf16x2(p0, p1);
+                    dd[e >> 1] = pack_bf16x2(s0v, s1v);
                 }
             }
-            tmem_st16(tS, pp);
-            tmem_st16(tS + N, dd);
+            tmem_st_cols(tS, pp);
+            tmem_st_cols(tS + N, dd);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -393,6 +441,7 @@ __global__ void __launch_bounds__(320, 1)
             const int rg = r0 + row;
             const bool live = DQ ? rg < p.Sq : rg < p.Sk;
             constexpr int NACC = DQ ? 1 : 2;
+            constexpr int AW = HD / C::NG;  // accumulator columns per warp
 #pragma unroll
             for (int a = 0; a < NACC; ++a) {
                 const uint32_t acol = a == 0 ? C::ACC2 : C::ACC1;
@@ -401,21 +450,21 @@ __global__ void __launch_bounds__(320, 1)
                     DQ ? p.out0 + ((size_t(b) * p.Sq + rg) * p.Hq + hx) * HD
                        : (a == 0 ? p.out0 : p.out1) + ((size_t(b) * p.Sk + rg) * p.Hkv + c) * HD;
 #pragma unroll
-                for (int k = 0; k < HD / 64; ++k) {
-                    const int col = hf * (HD / 2) + k * 32;
-                    uint32_t r[32];
+                for (int k = 0; k < AW / 16; ++k) {
+                    const int col = hf * AW + k * 16;
+                    uint32_t r[16];
                     if (n > 0) {
-                        tmem_ld32(tmem + lane_base + acol + col, r);
+                        tmem_ld16(tmem + lane_base + acol + col, r);
                         tmem_ld_wait();
                         reg_fence(r);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) r[e] = 0u;
+                        for (int e = 0; e < 16; ++e) r[e] = 0u;
                     }
                     if (live) {
                         uint4* o4 = reinterpret_cast<uint4*>(dst + col);
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
+                        for (int v = 0; v < 2; ++v)
                             o4[v] = make_uint4(
                                 pack_bf16x2(__uint_as_float(r[8 * v]) * mul,
                                             __uint_as_float(r[8 * v + 1]) * mul),
@@ -434,7 +483,7 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 9) tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == WM) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace gqa

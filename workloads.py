@@ -69,7 +69,10 @@ ENCODER = Workload("encoder_b64_h48kv12_s512_d64", B=64, Hq=48, Hkv=12, Sq=512, 
                    D=64, dtype="bf16", causal=False, seed=1)
 LLAMA = Workload("llama8b_prefill_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8192, Sk=8192,
                  D=128, dtype="bf16", causal=True, seed=2)
+# the backward of the Llama prefill shape (and one batch element of it, for profiles)
 LLAMA_BWD = Workload("llama8b_backward_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8192, Sk=8192,
+                     D=128, dtype="bf16", causal=True, seed=2, backward=True)
+LLAMA_BWD_B1 = Workload("llama8b_backward_b1_s8192_causal", B=1, Hq=32, Hkv=8, Sq=8192, Sk=8192,
                      D=128, dtype="bf16", causal=True, seed=2, backward=True)
 LLAMA_STRESS = Workload("llama8b_prefill_b4_s8192_causal_qx4", B=4, Hq=32, Hkv=8, Sq=8192,
                         Sk=8192, D=128, dtype="bf16", causal=True, seed=3, q_mult=4.0)
