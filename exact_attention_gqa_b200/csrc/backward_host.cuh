@@ -69,13 +69,19 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
     tp.causal = causal ? 1 : 0;
     tp.scale = scale;
     tp.scale_log2 = scale * kLog2e;
-    // [rows, heads, D] views: 128-row boxes for the resident tiles, 64-row for the stream
-    CUtensorMap mq128, mo128, mk128, mv128, mq64, mo64, mk64, mv64;
+    // [rows, heads, D] views: 128-row boxes for the resident tiles; the streamed blocks
+    // are 64 query rows (dK/dV launch) and 96 key rows (dQ launch)
+    constexpr int NQB = gqa::BwdTcCfg<128, false, GQA_BWD_EW>::N;
+    constexpr int NKB = gqa::BwdTcCfg<128, true, GQA_BWD_EW>::N;
+    static_assert(NQB == gqa::BwdTcCfg<64, false, GQA_BWD_EW>::N &&
+                      NKB == gqa::BwdTcCfg<64, true, GQA_BWD_EW>::N,
+                  "block rows do not depend on D");
+    CUtensorMap mq128, mo128, mk128, mv128, mqs, mos, mks, mvs;
     const long long rq = (long long)B * Sq, rk = (long long)B * Sk;
     if (!make_map(&mq128, q, rq, Hq, D, 1, 128) || !make_map(&mo128, dout, rq, Hq, D, 1, 128) ||
         !make_map(&mk128, k, rk, Hkv, D, 1, 128) || !make_map(&mv128, v, rk, Hkv, D, 1, 128) ||
-        !make_map(&mq64, q, rq, Hq, D, 1, 64) || !make_map(&mo64, dout, rq, Hq, D, 1, 64) ||
-        !make_map(&mk64, k, rk, Hkv, D, 1, 64) || !make_map(&mv64, v, rk, Hkv, D, 1, 64))
+        !make_map(&mqs, q, rq, Hq, D, 1, NQB) || !make_map(&mos, dout, rq, Hq, D, 1, NQB) ||
+        !make_map(&mks, k, rk, Hkv, D, 1, NKB) || !make_map(&mvs, v, rk, Hkv, D, 1, NKB))
         return GQA_ERR_CUDA;
     auto launch = [&](auto tag) -> int {
         constexpr int HD = decltype(tag)::value;
@@ -93,12 +99,12 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
         t1.out0 = static_cast<__nv_bfloat16*>(dk);
         t1.out1 = static_cast<__nv_bfloat16*>(dv);
         gqa::bwd_tc<HD, false, EW><<<dim3((Sk + 127) / 128, Hkv, B), C1::THREADS, S1, stream>>>(
-            mk128, mv128, mq64, mo64, t1);
+            mk128, mv128, mqs, mos, t1);
         gqa::BwdTcParams t2 = tp;
         t2.out0 = static_cast<__nv_bfloat16*>(dq);
         t2.out1 = nullptr;
         gqa::bwd_tc<HD, true, EW><<<dim3((Sq + 127) / 128, Hq, B), C2::THREADS, S2, stream>>>(
-            mq128, mo128, mk64, mv64, t2);
+            mq128, mo128, mks, mvs, t2);
         return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
     };
     return D == 128 ? launch(std::integral_constant<int, 128>())

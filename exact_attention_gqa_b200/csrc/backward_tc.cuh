@@ -45,12 +45,13 @@ struct BwdTcParams {
 template <int HD, bool DQ, int EW>
 struct BwdTcCfg {
     static constexpr int M = 128;       // resident rows
-    static constexpr int N = 64;        // streamed rows per block
+    // streamed rows per block: the dQ role has TMEM room for two 96-column S/dP pairs
+    static constexpr int N = DQ ? 96 : 64;
     static constexpr int NG = EW / 4;   // column groups: warps per TMEM lane quarter
     static constexpr int CW = N / NG;   // columns of S (and dP) per elementwise warp
     static constexpr int THREADS = 32 * (EW + 2);
     static constexpr int CH = HD / 64;  // 64-dimension chunks (one 128-byte swizzle atom wide)
-    static constexpr int STAGES = HD == 128 ? 4 : 6;
+    static constexpr int STAGES = HD == 128 ? (DQ ? 3 : 4) : 6;
     static constexpr int RES_ATOM = M * 128;  // one chunk of a resident tile
     static constexpr int RES_TILE = CH * RES_ATOM;
     static constexpr int STR_ATOM = N * 128;  // one chunk of a streamed block
@@ -84,11 +85,19 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr)
         : "memory");
 }
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[16]) {
-    tmem_ld16(taddr, r);
-}
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[32]) {
-    tmem_ld32(taddr, r);
+// NC consecutive columns: x32 loads when NC is a multiple of 32, else x16 loads
+// (each load starts at a column aligned to its width)
+template <int NC>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NC]) {
+    if constexpr (NC % 32 == 0) {
+#pragma unroll
+        for (int i = 0; i < NC / 32; ++i)
+            tmem_ld32(taddr + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * i));
+    } else {
+#pragma unroll
+        for (int i = 0; i < NC / 16; ++i)
+            tmem_ld16(taddr + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(r + 16 * i));
+    }
 }
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
     asm volatile(
@@ -106,11 +115,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[15])
         : "memory");
 }
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[8]) {
-    tmem_st8(taddr, r);
-}
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[16]) {
-    tmem_st16(taddr, r);
+// NC consecutive columns (8, 16 or 24): x16 stores, then an x8 store for the rest
+template <int NC>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[NC]) {
+#pragma unroll
+    for (int i = 0; i < NC / 16; ++i)
+        tmem_st16(taddr + 16 * i, *reinterpret_cast<const uint32_t(*)[16]>(r + 16 * i));
+    if constexpr (NC % 16 == 8)
+        tmem_st8(taddr + NC - 8, *reinterpret_cast<const uint32_t(*)[8]>(r + NC - 8));
 }
 
 template <int HD, bool DQ, int EW>

@@ -59,10 +59,53 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, *, f32=False):
 
 GRAD_MAX_REL = 1e-2
 GRAD_MEAN_REL = 1e-3
+GRAD_MODEL_FACTOR = 1.5
 
 
-def compare_grad(g_gpu, ref):
-    """Assert the backward bar for one gradient tensor; returns the observed errors."""
+def bf16_backward_model(q, k, v, do, scale, causal):
+    """Rounding model of the backward's stated arithmetic, for the tolerance only: the
+    products of bf16 inputs accumulated in fp32, P and dS rounded to bf16 before the
+    accumulating products, O and the gradients rounded to bf16.  Its distance from the
+    float64 oracle is the error that arithmetic makes on these inputs; it shares nothing
+    with the CUDA path.  Returns dq, dk, dv as float64 arrays in the input layouts."""
+    import torch
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    out = [np.zeros(q.shape), np.zeros(k.shape), np.zeros(v.shape)]
+    l2e = 1.4426950408889634
+    for b in range(B):
+        for c in range(Hkv):
+            hs = slice(c * G, (c + 1) * G)
+            qf = q[b, :, hs].float().transpose(0, 1)           # [G, Sq, D]
+            dof = do[b, :, hs].float().transpose(0, 1)
+            kf = k[b, :, c].float()                             # [Sk, D]
+            vf = v[b, :, c].float()
+            s = qf @ kf.T                                       # [G, Sq, Sk]
+            if causal:
+                vis = torch.ones(Sq, Sk, dtype=torch.bool).tril(diagonal=Sk - Sq)
+                s = s.masked_fill(~vis, float("-inf"))
+            lse = torch.logsumexp(s.double() * scale, -1)
+            o = torch.softmax(s.double() * scale, -1).nan_to_num(0.0) @ vf.double()
+            o = o.float().bfloat16().float()
+            p = torch.exp2(s * (scale * l2e) - (lse * l2e).float()[..., None]).nan_to_num(0.0)
+            dsv = p * (dof @ vf.T - (dof * o).sum(-1, keepdim=True))
+            pb, dsb = p.bfloat16().float(), dsv.bfloat16().float()
+            dq = (scale * dsb @ kf).bfloat16().double()
+            dk = (scale * (dsb.transpose(1, 2) @ qf).sum(0)).bfloat16().double()
+            dv = (pb.transpose(1, 2) @ dof).sum(0).bfloat16().double()
+            out[0][b, :, hs] = dq.transpose(0, 1).numpy()
+            out[1][b, :, c] = dk.numpy()
+            out[2][b, :, c] = dv.numpy()
+    return out
+
+
+def compare_grad(g_gpu, ref, model=None):
+    """Assert the backward bar for one gradient tensor; returns the observed errors.
+    Fixed bar: max |err| <= 1e-2 max(1, max|ref|), mean |err| <= 1e-3 max(1, mean|ref|).
+    With `model` (bf16_backward_model's tensor), each bound is at least 1.5 x the
+    model's own max / mean distance from the oracle: long reductions (dK, dV summed
+    over G Sq rows) carry more bf16 rounding than the fixed bar allows."""
     g = to_np(g_gpu) if not isinstance(g_gpu, np.ndarray) else g_gpu.astype(np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert g.shape == ref.shape, (g.shape, ref.shape)
@@ -70,8 +113,13 @@ def compare_grad(g_gpu, ref):
     err = np.abs(g - ref)
     big = max(1.0, float(np.abs(ref).max(initial=0.0)))
     typ = max(1.0, float(np.abs(ref).mean())) if ref.size else 1.0
+    max_bar, mean_bar = GRAD_MAX_REL * big, GRAD_MEAN_REL * typ
+    if model is not None and ref.size:
+        merr = np.abs(np.asarray(model, dtype=np.float64) - ref)
+        max_bar = max(max_bar, GRAD_MODEL_FACTOR * float(merr.max()))
+        mean_bar = max(mean_bar, GRAD_MODEL_FACTOR * float(merr.mean()))
     stats = {"max_abs": float(err.max(initial=0.0)), "mean_abs": float(err.mean()) if err.size else 0.0,
-             "max_ref": big, "mean_ref": typ}
-    assert stats["max_abs"] <= GRAD_MAX_REL * big, stats
-    assert stats["mean_abs"] <= GRAD_MEAN_REL * typ, stats
+             "max_bar": max_bar, "mean_bar": mean_bar}
+    assert stats["max_abs"] <= max_bar, stats
+    assert stats["mean_abs"] <= mean_bar, stats
     return stats

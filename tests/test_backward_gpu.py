@@ -9,7 +9,7 @@ import torch
 import oracle
 from exact_attention_gqa_b200 import build, gqa_attn, gqa_attn_backward, \
     gqa_attn_get_device_error
-from parity import compare_grad
+from parity import bf16_backward_model, compare_grad
 
 pytestmark = pytest.mark.gpu
 
@@ -54,8 +54,9 @@ def test_backward_matches_oracle(B, Hq, Hkv, Sq, Sk, D, causal):
     q, k, v, do = inputs(B, Hq, Hkv, Sq, Sk, D, seed=B + Sq + Sk + D)
     grads = run_bwd(q, k, v, do, causal)
     ref = oracle.attention_backward(q, k, v, do, scale=1 / math.sqrt(D), causal=causal)
-    for g, r in zip(grads, ref):
-        compare_grad(g, r)
+    model = bf16_backward_model(q, k, v, do, 1 / math.sqrt(D), causal)
+    for g, r, m in zip(grads, ref, model):
+        compare_grad(g, r, m)
 
 
 def test_backward_is_bitwise_reproducible():
@@ -74,6 +75,33 @@ def test_queries_without_keys_get_zero_gradient():
     ref = oracle.attention_backward(q, k, v, do, scale=0.125, causal=True)
     for g, r in zip((dq, dk, dv), ref):
         compare_grad(g, r)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_query_blocks_without_any_key(D):
+    # causal with Sq - Sk >= 128: whole 128-query blocks see no key (their dQ launch
+    # streams nothing and writes zeros); the later rows are checked against the oracle
+    q, k, v, do = inputs(1, 4, 2, 400, 100, D, seed=13 + D)
+    dq, dk, dv = run_bwd(q, k, v, do, True)
+    assert torch.all(dq[:, :300] == 0)
+    ref = oracle.attention_backward(q, k, v, do, scale=1 / math.sqrt(D), causal=True)
+    model = bf16_backward_model(q, k, v, do, 1 / math.sqrt(D), True)
+    for g, r, m in zip((dq, dk, dv), ref, model):
+        compare_grad(g, r, m)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal", [
+    (1, 16, 2, 520, 390, 64, True),    # G = 8, several key and query blocks, Sq > Sk
+    (2, 2, 2, 129, 1100, 128, True),   # MHA, one row past a block, long keys
+    (1, 4, 1, 700, 65, 128, False),    # one key past a 64-key block
+])
+def test_backward_multiblock_shapes(B, Hq, Hkv, Sq, Sk, D, causal):
+    q, k, v, do = inputs(B, Hq, Hkv, Sq, Sk, D, seed=B * 7 + Sq + Sk)
+    grads = run_bwd(q, k, v, do, causal)
+    ref = oracle.attention_backward(q, k, v, do, scale=1 / math.sqrt(D), causal=causal)
+    model = bf16_backward_model(q, k, v, do, 1 / math.sqrt(D), causal)
+    for g, r, m in zip(grads, ref, model):
+        compare_grad(g, r, m)
 
 
 def test_no_keys_gives_zero_dq():

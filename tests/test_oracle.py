@@ -665,6 +665,21 @@ def test_backward_matches_finite_differences_of_the_forward():
             assert abs(num - grad[idx]) < 2e-4, (which, idx, num, grad[idx])
 
 
+def test_bf16_backward_model_tracks_the_oracle():
+    # the tolerance model of the backward's bf16 arithmetic: close to the exact
+    # gradients (its error is rounding, a fraction of a percent), but not equal to them
+    from parity import bf16_backward_model
+    q, k, v = rnd((1, 40, 4, 16), 70), rnd((1, 50, 2, 16), 71), rnd((1, 50, 2, 16), 72)
+    do = rnd((1, 40, 4, 16), 73)
+    tq, tk, tv, tdo = (torch.from_numpy(a).bfloat16() for a in (q, k, v, do))
+    exact = oracle.attention_backward(tq, tk, tv, tdo, scale=0.25, causal=True)
+    model = bf16_backward_model(tq, tk, tv, tdo, 0.25, True)
+    for m, r in zip(model, exact):
+        err = np.abs(m - r)
+        assert 0 < err.max() <= 1e-2 * max(1.0, np.abs(r).max())
+        assert err.mean() <= 2e-3 * max(1.0, np.abs(r).mean())
+
+
 # ---------------------------------------------------------------------------------
 # Pin strength: every planted mistake is caught by at least one pin above
 
