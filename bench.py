@@ -471,6 +471,21 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
 
 
 # ----------------------------------------------------------------------------- arms
+def workload_config(w) -> dict:
+    """The workload's own keys of the JSON line's config (both arms)."""
+    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Sk": w.Sk,
+           "D": w.D, "causal": w.causal}
+    if w.kv_fp8:
+        cfg["kv_cache"] = f"e4m3 codes, k_scale = v_scale = {W.FP8_SCALE}"
+    if w.backward:
+        cfg["pass"] = "backward: dQ, dK, dV for a seeded dO (O and L from the forward)"
+        cfg["flops"] = "2.5 x the forward's (five products against two)"
+    if w.page_size:
+        cfg["page_size"] = w.page_size
+        cfg["block_table"] = "seeded shuffle of the page pool"
+    return cfg
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -487,7 +502,7 @@ def run_reference(args, world, rank):
             "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(e for _, e in per_step),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name},
+            "config": workload_config(w),
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                              "sample": f"each step: {desc}"},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
@@ -677,27 +692,19 @@ def run_ours(args, world, rank, local):
         v_cpu, desc, cores, el = oracle_sample(w, target_s=args.cpu_seconds, max_s=30.0)
         cpu = {"value": v_cpu, "unit": case.unit, "cores": cores, "kind": "oracle",
                "sample": f"{desc}; {el:.1f} s of float64 CPU work"}
-    cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Sq": w.Sq, "Sk": w.Sk,
-           "D": w.D, "causal": w.causal, "pack_gqa": case.pack, "num_splits": case.splits,
+    cfg = workload_config(w)
+    cfg.update({"pack_gqa": case.pack, "num_splits": case.splits,
            "per_rank": "independent copy of the workload on every rank",
            "l2": ("inputs larger than L2 (%.0f MB per step)" % (case.in_bytes() / 1e6)
                   if case.in_bytes() > L2_BYTES or len(case.kv) > 1 else "inputs fit in L2"),
            "kv_copies_rotated": len(case.kv),
            "timing": ("CUDA graph of the K steps, replayed once" if case.decode
-                      else "K back-to-back calls")}
+                      else "K back-to-back calls")})
     if case.varlen:
         cfg["total_tokens"] = int(case.q.shape[0])
-    if w.kv_fp8:
-        cfg["kv_cache"] = f"e4m3 codes, k_scale = v_scale = {W.FP8_SCALE}"
-    if w.backward:
-        cfg["pass"] = "backward: dQ, dK, dV for a seeded dO (O and L from the forward)"
-        cfg["flops"] = "2.5 x the forward's (five products against two)"
     if w.block_sparse:
         cfg["block_pattern"] = dict(w.block_sparse, block=128, blocks=int(case.col.numel()),
                                     of=int((case.rp.numel() - 1) * -(-w.Sk // 128)))
-    if case.paged:
-        cfg["page_size"] = w.page_size
-        cfg["block_table"] = "seeded shuffle of the page pool"
     line = {"metric": METRIC, "value": value, "unit": case.unit, "n_gpus": world,
             "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
