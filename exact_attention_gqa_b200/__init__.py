@@ -184,20 +184,31 @@ def gqa_attn_backward(q, k, v, out, lse, dout, *, causal: bool = False,
     """
     import torch
 
-    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout)):
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
-        if not t.is_contiguous():
-            raise ValueError(f"{name} must be contiguous")
-    if not (q.dtype == k.dtype == v.dtype == out.dtype == dout.dtype == torch.bfloat16):
-        raise ValueError("q, k, v, out, dout must be bf16")
-    if lse.dtype != torch.float32:
-        raise ValueError("lse must be fp32")
     if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape or out.shape != q.shape \
             or dout.shape != q.shape:
         raise ValueError("q/out/dout [B, Sq, Hq, D], k/v [B, Sk, Hkv, D]")
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
+    if k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("k/v must match q in batch and head dimension")
+    if tuple(lse.shape) != (B, Hq, Sq):
+        raise ValueError(f"lse must be [B, Hq, Sq] = {(B, Hq, Sq)}, got {tuple(lse.shape)}")
+    if not (q.dtype == k.dtype == v.dtype == out.dtype == dout.dtype == torch.bfloat16):
+        raise ValueError("q, k, v, out, dout must be bf16")
+    if lse.dtype != torch.float32:
+        raise ValueError("lse must be fp32")
+    for name, g, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if g is not None and (g.shape != like.shape or g.dtype != like.dtype
+                              or g.device != like.device or not g.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like its input, "
+                             "on the same device")
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse), ("dout", dout)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if t.device != q.device:
+            raise ValueError(f"{name} must be on q's device")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk

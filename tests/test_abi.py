@@ -262,3 +262,55 @@ def test_blocksparse_argument_errors(lib, kw, code):
 
 def test_blocksparse_empty_batch_is_a_noop(lib):
     assert sparse_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+
+
+# ---------------------------------------------------------------------------- backward
+def bwd_call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE,
+             dv=FAKE, B=1, Hq=8, Hkv=2, Sq=256, Sk=256, D=128, scale=0.125, causal=1):
+    return lib.gqa_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, scale,
+                            causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=96), "GQA_ERR_HEADDIM"),
+    (dict(scale=-1.0), "GQA_ERR_SCALE"),
+    (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
+    (dict(Sq=-1), "GQA_ERR_SHAPE"),
+    (dict(q=None), "GQA_ERR_NULL"),
+    (dict(lse=None), "GQA_ERR_NULL"),
+    (dict(dout=None), "GQA_ERR_NULL"),
+    (dict(dk=None), "GQA_ERR_NULL"),
+    (dict(dv=ctypes.c_void_p(0x1008)), "GQA_ERR_ALIGN"),
+    (dict(lse=ctypes.c_void_p(0x1002)), "GQA_ERR_ALIGN"),
+])
+def test_backward_argument_errors(lib, kw, code):
+    assert G.STATUS[bwd_call(lib, **kw)] == code
+
+
+def test_backward_empty_problems_are_noops(lib):
+    assert bwd_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None, dout=None, dq=None,
+                    dk=None, dv=None) == 0
+    assert bwd_call(lib, Sq=0, Sk=0, q=None, k=None, v=None, out=None, lse=None, dout=None,
+                    dq=None, dk=None, dv=None) == 0
+
+
+def test_backward_workspace_bytes(lib):
+    # one fp32 D_i per (batch, query head, row), rounded up to 256 bytes
+    assert lib.gqa_attn_bwd_workspace_bytes(2, 3, 5) == 256
+    assert lib.gqa_attn_bwd_workspace_bytes(4, 32, 8192) == 4 * 32 * 8192 * 4
+    assert lib.gqa_attn_bwd_workspace_bytes(0, 32, 8192) == 0
+
+
+def test_backward_front_end_checks_shapes_first():
+    import torch
+    q = torch.zeros(1, 16, 4, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 20, 2, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 4, 16)
+    with pytest.raises(ValueError, match="lse must be"):
+        G.gqa_attn_backward(q, k, k, q, lse[:, :, :8], q)
+    with pytest.raises(ValueError, match="dk must be"):
+        G.gqa_attn_backward(q, k, k, q, lse, q, dk=torch.zeros(1, 20, 2, 32, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="k/v must match"):
+        G.gqa_attn_backward(q, k[..., :32], k[..., :32], q, lse, q)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        G.gqa_attn_backward(q, k, k, q, lse, q)
