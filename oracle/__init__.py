@@ -21,6 +21,8 @@ states the passage of the pages it follows in the C source:
 * ``attention_backward`` -- dQ, dK, dV for a given dO (FA-2 page, backward pass).
 * ``attention_blocksparse`` -- attention restricted to a (query block, key block)
                           pattern (Raptor-T abstract: BigBird's block-sparse attention).
+* ``attention_e4m3``   -- the forward on e4m3 Q, K, V codes with one scale per tensor
+                          (the batch-size guide's FP8 precision lever).
 * ``decode_kvcache``   -- one decode query per sequence against a dense or paged
                           KV cache with per-sequence lengths and a sliding window
                           (Ultralytics GQA glossary, KV-cache and related-techniques
@@ -57,6 +59,7 @@ FLAWS = {
     "e4m3_bias": 10,
     "sparse_row": 11,
     "bwd_no_d": 12,
+    "e4m3_no_vscale": 13,
 }
 
 
@@ -94,6 +97,9 @@ def _load():
         lib.oracle_decode_kvcache_e4m3.argtypes = [P, P, P, Dbl, Dbl, P, P, P, P, I, I, I, I, I,
                                                    I, I, I, I, Dbl, I]
         lib.oracle_decode_kvcache_e4m3.restype = I
+        lib.oracle_attention_e4m3.argtypes = [P, P, P, Dbl, Dbl, Dbl, P, P, I, I, I, I, I, I,
+                                              Dbl, I, P, I]
+        lib.oracle_attention_e4m3.restype = I
         lib.oracle_attention_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, P, P,
                                                      I, I]
         lib.oracle_attention_blocksparse.restype = I
@@ -238,6 +244,26 @@ def _codes(a):
             a = a.view(torch.uint8)
         a = a.numpy()
     return np.ascontiguousarray(a, dtype=np.uint8)
+
+
+def attention_e4m3(q8, k8, v8, *, q_scale: float, k_scale: float, v_scale: float,
+                   scale: float, causal: bool, cu_seqlens=None, threads: int = 0):
+    """Forward on e4m3 codes (uint8 or float8_e4m3fn; element = value(code) * scale of
+    its tensor), layouts as ``attention``.  Returns (O float64 like q, L float64)."""
+    q, k, v = _codes(q8), _codes(k8), _codes(v8)
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    B, Hq, Hkv, Sq, Sk, D = _dims(q, k, cu)
+    if v.shape != k.shape:
+        raise ValueError("v must have the shape of k")
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((Hq, q.shape[0]) if cu is not None else (B, Hq, Sq), dtype=np.float64)
+    rc = _load().oracle_attention_e4m3(_ptr(q), _ptr(k), _ptr(v), float(q_scale),
+                                       float(k_scale), float(v_scale), _ptr(o), _ptr(lse), B,
+                                       Hq, Hkv, Sq, Sk, D, float(scale), int(bool(causal)),
+                                       None if cu is None else _ptr(cu), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_e4m3: bad arguments or a NaN code")
+    return o, lse
 
 
 def decode_kvcache(q, k_cache, v_cache, *, scale: float, seqlens_k=None, block_table=None,

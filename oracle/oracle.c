@@ -92,6 +92,7 @@ enum {
     FLAW_E4M3_BIAS = 10,      /* e4m3 exponent bias 8 instead of 7              */
     FLAW_SPARSE_ROW = 11,     /* block pattern row of the next query block       */
     FLAW_BWD_NO_D = 12,       /* backward: dS = P * dP, without subtracting D    */
+    FLAW_E4M3_NO_VSCALE = 13, /* e4m3 prefill: O left without the V scale        */
 };
 static int g_flaw = FLAW_NONE;
 void oracle_set_flaw(int flaw) { g_flaw = flaw; }
@@ -730,6 +731,50 @@ int oracle_decode_kvcache_e4m3(const float* q, const uint8_t* k8, const uint8_t*
     const cache_src ks = {NULL, k8, k_scale, lut}, vs = {NULL, v8, v_scale, lut};
     return decode_core(q, &ks, &vs, block_table, seqlens_k, o, lse, B, Hq, Hkv, D, Sk,
                        page_size, max_pages, num_pages, window, scale, nthreads);
+}
+
+/*
+ * Prefill with e4m3 Q, K and V (the batch-size guide names FP8 as the precision that
+ * lowers memory-bandwidth pressure: hardware adaptation section, Hopper item, and the
+ * precision row of its production checklist).  Each tensor holds codes with one scale:
+ * element = value(code) * scale of that tensor.  The result is the plain definition
+ * on those elements: S = scale * (q_scale Q)(k_scale K)^T, P = softmax(S),
+ * O = P (v_scale V), L = m + ln l.  The code values are exact in float, so the codes
+ * are decoded once and the per-tensor scales enter in double: q_scale * k_scale with
+ * the logit scale, v_scale on O.  A NaN code (0x7f, 0xff) is rejected.
+ */
+int oracle_attention_e4m3(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                          double q_scale, double k_scale, double v_scale, double* o,
+                          double* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                          double scale, int causal, const int32_t* cu_seqlens, int nthreads)
+{
+    if (check_args(q8, k8, v8, B, Hq, Hkv, Sq, Sk, D, cu_seqlens) || !o || !lse) return -1;
+    const size_t nq = (size_t)(cu_seqlens ? cu_seqlens[B] : B * Sq) * Hq * D;
+    const size_t nk = (size_t)(cu_seqlens ? cu_seqlens[B] : B * Sk) * Hkv * D;
+    float* q = (float*)malloc(sizeof(float) * (nq ? nq : 1));
+    float* k = (float*)malloc(sizeof(float) * (nk ? nk : 1));
+    float* v = (float*)malloc(sizeof(float) * (nk ? nk : 1));
+    int rc = (q && k && v) ? 0 : -1;
+    double lut[256];
+    oracle_e4m3_table(lut);
+    for (size_t i = 0; rc == 0 && i < nq; ++i) {
+        if (isnan(lut[q8[i]])) rc = -1;
+        q[i] = (float)lut[q8[i]];
+    }
+    for (size_t i = 0; rc == 0 && i < nk; ++i) {
+        if (isnan(lut[k8[i]]) || isnan(lut[v8[i]])) rc = -1;
+        k[i] = (float)lut[k8[i]];
+        v[i] = (float)lut[v8[i]];
+    }
+    if (rc == 0)
+        rc = oracle_attention(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, scale * q_scale * k_scale,
+                              causal, cu_seqlens, nthreads);
+    if (rc == 0 && g_flaw != FLAW_E4M3_NO_VSCALE)
+        for (size_t i = 0; i < nq; ++i) o[i] *= v_scale;
+    free(q);
+    free(k);
+    free(v);
+    return rc;
 }
 
 /*

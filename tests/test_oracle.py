@@ -665,6 +665,58 @@ def test_backward_matches_finite_differences_of_the_forward():
             assert abs(num - grad[idx]) < 2e-4, (which, idx, num, grad[idx])
 
 
+# ---------------------------------------------------------------------------------
+# e4m3 prefill (the batch-size guide's FP8 lever): element = value(code) * tensor scale
+
+def e4m3_tensors(shape, seed, spread=3.0):
+    """float8_e4m3fn tensors from seeded normal draws (torch rounds to the format)."""
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(*shape, generator=g) * spread).to(torch.float8_e4m3fn)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D,causal", [
+    (2, 8, 2, 33, 33, 16, True),    # GQA, causal
+    (1, 6, 2, 20, 45, 8, True),     # Sq < Sk, bottom-right
+    (2, 4, 1, 17, 29, 16, False),   # MQA
+])
+def test_e4m3_prefill_matches_sdpa_on_torch_decoded_values(B, Hq, Hkv, Sq, Sk, D, causal):
+    q8, k8, v8 = e4m3_tensors((B, Sq, Hq, D), 80), e4m3_tensors((B, Sk, Hkv, D), 81), \
+        e4m3_tensors((B, Sk, Hkv, D), 82)
+    qs, ks, vs, scale = 0.75, 0.125, 3.0, 0.3
+    o, lse = oracle.attention_e4m3(q8, k8, v8, q_scale=qs, k_scale=ks, v_scale=vs,
+                                   scale=scale, causal=causal)
+    dec = [(t.to(torch.float64) * sc).numpy() for t, sc in ((q8, qs), (k8, ks), (v8, vs))]
+    o_ref, lse_ref = sdpa_ref(*dec, scale, causal, bottom_right=causal and Sq != Sk)
+    assert np.max(np.abs(o - o_ref)) < 1e-11 * max(1.0, np.abs(o_ref).max())
+    assert np.max(np.abs(lse - lse_ref)) < 1e-11 * max(1.0, np.abs(lse_ref).max())
+
+
+def test_e4m3_prefill_varlen_is_per_sequence():
+    lens = [5, 0, 17, 9]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    q8, k8, v8 = e4m3_tensors((cu[-1], 4, 16), 83), e4m3_tensors((cu[-1], 2, 16), 84), \
+        e4m3_tensors((cu[-1], 2, 16), 85)
+    o, lse = oracle.attention_e4m3(q8, k8, v8, q_scale=0.5, k_scale=2.0, v_scale=0.25,
+                                   scale=0.2, causal=True, cu_seqlens=cu)
+    for b, n in enumerate(lens):
+        if n == 0:
+            continue
+        sl = slice(cu[b], cu[b + 1])
+        ob, lb = oracle.attention_e4m3(q8[sl][None], k8[sl][None], v8[sl][None], q_scale=0.5,
+                                       k_scale=2.0, v_scale=0.25, scale=0.2, causal=True)
+        assert np.array_equal(o[sl], ob[0]) and np.array_equal(lse[:, sl], lb[0])
+
+
+def test_e4m3_prefill_rejects_nan_codes():
+    q8 = e4m3_tensors((1, 4, 2, 8), 86)
+    k8 = e4m3_tensors((1, 4, 1, 8), 87)
+    bad = k8.view(torch.uint8).clone()
+    bad[0, 2, 0, 3] = 0x7F
+    with pytest.raises(ValueError):
+        oracle.attention_e4m3(q8, bad, k8, q_scale=1, k_scale=1, v_scale=1, scale=0.3,
+                              causal=False)
+
+
 def test_bf16_backward_model_tracks_the_oracle():
     # the tolerance model of the backward's bf16 arithmetic: close to the exact
     # gradients (its error is rounding, a fraction of a percent), but not equal to them
@@ -696,6 +748,7 @@ PIN_BATTERY = [
     lambda: test_e4m3_table_matches_torch_float8(),
     lambda: test_blocksparse_matches_sdpa_with_the_expanded_mask(96, 80, 16, 2),
     lambda: test_backward_matches_torch_autograd_float64(2, 8, 2, 33, 33, 16, True),
+    lambda: test_e4m3_prefill_matches_sdpa_on_torch_decoded_values(2, 8, 2, 33, 33, 16, True),
 ]
 
 
