@@ -19,6 +19,8 @@ states the passage of the pages it follows in the C source:
 * ``attention_tiled``  -- the per-step normalised (form 1) and deferred
                           normalisation (form 2) online-softmax forms.
 * ``attention_backward`` -- dQ, dK, dV for a given dO (FA-2 page, backward pass).
+* ``attention_blocksparse_varlen`` -- the block pattern over packed sequences, each
+                          padded only to whole blocks (Raptor-T's minimum padding).
 * ``attention_blocksparse`` -- attention restricted to a (query block, key block)
                           pattern (Raptor-T abstract: BigBird's block-sparse attention).
 * ``attention_e4m3``   -- the forward on e4m3 Q, K, V codes with one scale per tensor
@@ -60,6 +62,7 @@ FLAWS = {
     "sparse_row": 11,
     "bwd_no_d": 12,
     "e4m3_no_vscale": 13,
+    "sparse_maxpad": 14,
 }
 
 
@@ -100,6 +103,9 @@ def _load():
         lib.oracle_attention_e4m3.argtypes = [P, P, P, Dbl, Dbl, Dbl, P, P, I, I, I, I, I, I,
                                               Dbl, I, P, I]
         lib.oracle_attention_e4m3.restype = I
+        lib.oracle_attention_blocksparse_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, Dbl,
+                                                            P, P, I, I]
+        lib.oracle_attention_blocksparse_varlen.restype = I
         lib.oracle_attention_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, P, P,
                                                      I, I]
         lib.oracle_attention_blocksparse.restype = I
@@ -326,6 +332,33 @@ def attention_blocksparse(q, k, v, row_ptr, col, *, scale: float, blk: int = 128
                                               _ptr(cl), int(blk), int(threads))
     if rc != 0:
         raise ValueError("oracle_attention_blocksparse: bad arguments")
+    return o, lse
+
+
+def attention_blocksparse_varlen(q, k, v, cu_seqlens, row_ptr, col, *, scale: float,
+                                 blk: int = 128, threads: int = 0):
+    """Packed sequences ([total, H, D]), each with its own block pattern: the pattern's
+    rows are the query blocks of sequence 0, then of sequence 1, ... (ceil(n_b / blk)
+    each), col entries are key blocks of the same sequence.  Returns (O float64 like q,
+    L float64 [Hq, total])."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    cu = np.ascontiguousarray(_np_int(cu_seqlens), dtype=np.int32)
+    B, Hq, Hkv, _, _, D = _dims(q, k, cu)
+    rp = np.ascontiguousarray(_np_int(row_ptr), dtype=np.int32)
+    cl = np.ascontiguousarray(_np_int(col), dtype=np.int32)
+    if cl.size == 0:
+        cl = np.zeros(1, dtype=np.int32)
+    n_rows = int(sum(-(-(int(cu[b + 1]) - int(cu[b])) // blk) for b in range(B)))
+    if rp.size != n_rows + 1:
+        raise ValueError(f"row_ptr must hold {n_rows + 1} entries (one row per block)")
+    o = np.zeros(q.shape, dtype=np.float64)
+    lse = np.zeros((Hq, q.shape[0]), dtype=np.float64)
+    rc = _load().oracle_attention_blocksparse_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                                     _ptr(lse), _ptr(cu), B, Hq, Hkv, D,
+                                                     float(scale), _ptr(rp), _ptr(cl),
+                                                     int(blk), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_attention_blocksparse_varlen: bad arguments")
     return o, lse
 
 

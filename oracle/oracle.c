@@ -93,6 +93,8 @@ enum {
     FLAW_SPARSE_ROW = 11,     /* block pattern row of the next query block       */
     FLAW_BWD_NO_D = 12,       /* backward: dS = P * dP, without subtracting D    */
     FLAW_E4M3_NO_VSCALE = 13, /* e4m3 prefill: O left without the V scale        */
+    FLAW_SPARSE_MAXPAD = 14,  /* varlen pattern rows numbered as if every sequence
+                                 were padded to the longest one                 */
 };
 static int g_flaw = FLAW_NONE;
 void oracle_set_flaw(int flaw) { g_flaw = flaw; }
@@ -569,6 +571,105 @@ int oracle_attention_blocksparse(const float* q, const float* k, const float* v,
             free(row);
             free(vis);
         }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Block-sparse attention over packed variable-length sequences with minimum padding
+ * (Raptor-T abstract: BigBird's block-sparse attention; its minimum-padding algorithm
+ * pads each sequence only to whole blocks instead of to the longest sequence).
+ * Sequence b holds n_b = cu[b+1] - cu[b] positions and ceil(n_b / blk) blocks; its
+ * query blocks are rows blk_off[b] .. blk_off[b] + ceil(n_b / blk) - 1 of the pattern,
+ * blk_off[b] = sum over earlier sequences of their block counts, and their col entries
+ * are key blocks of the same sequence, 0 .. ceil(n_b / blk) - 1.  Non-causal, self
+ * attention within each sequence.  q, k, v, o packed [total, H, D], lse [Hq, total].
+ */
+int oracle_attention_blocksparse_varlen(const float* q, const float* k, const float* v,
+                                        double* o, double* lse, const int32_t* cu, int B,
+                                        int Hq, int Hkv, int D, double scale,
+                                        const int32_t* row_ptr, const int32_t* col, int blk,
+                                        int nthreads)
+{
+    if (check_args(q, k, v, B, Hq, Hkv, 0, 0, D, cu) || !o || !lse || !row_ptr || !col ||
+        blk <= 0)
+        return -1;
+    int32_t* off = (int32_t*)malloc(sizeof(int32_t) * (size_t)(B + 1));
+    if (!off) return -1;
+    int maxlen = 0;
+    for (int b = 0; b < B; ++b)
+        if (cu[b + 1] - cu[b] > maxlen) maxlen = cu[b + 1] - cu[b];
+    off[0] = 0;
+    for (int b = 0; b < B; ++b) off[b + 1] = off[b] + (cu[b + 1] - cu[b] + blk - 1) / blk;
+    int bad = row_ptr[0] != 0;
+    for (int b = 0; b < B && !bad; ++b) {
+        const int nkb = (cu[b + 1] - cu[b] + blk - 1) / blk;
+        for (int r = off[b]; r < off[b] + nkb && !bad; ++r) {
+            if (row_ptr[r + 1] < row_ptr[r]) bad = 1;
+            for (int e = row_ptr[r]; e < row_ptr[r + 1] && !bad; ++e)
+                if (col[e] < 0 || col[e] >= nkb) bad = 1;
+        }
+    }
+    if (bad) {
+        free(off);
+        return -1;
+    }
+    set_threads(nthreads);
+#pragma omp parallel for collapse(2) schedule(dynamic) reduction(| : bad)
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hq; ++h) {
+            size_t q_row0, lse_off, lse_step;
+            head_view hv = make_view(q, k, v, B, Hq, Hkv, 0, 0, D, scale, 0, cu, b, h, &q_row0,
+                                     &lse_off, &lse_step);
+            const int n = hv.Sq, nqb = (n + blk - 1) / blk;
+            double* row = malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+            unsigned char* vis = malloc((size_t)(n > 0 ? n : 1));
+            if (!row || !vis) {
+                free(row);
+                free(vis);
+                bad = 1;
+                continue;
+            }
+            for (int i = 0; i < n; ++i) {
+                int qb = i / blk;
+                if (g_flaw == FLAW_SPARSE_ROW && qb + 1 < nqb) qb += 1;
+                int r = off[b] + qb;
+                if (g_flaw == FLAW_SPARSE_MAXPAD) { /* rows of max-padded sequences */
+                    r = b * ((maxlen + blk - 1) / blk) + qb;
+                    if (r >= off[B]) r = off[B] - 1;
+                }
+                memset(vis, 0, (size_t)n);
+                for (int e = row_ptr[r]; e < row_ptr[r + 1]; ++e)
+                    for (int j = col[e] * blk; j < (col[e] + 1) * blk && j < n; ++j) vis[j] = 1;
+                const float* qi = hv.q + (size_t)i * hv.q_stride;
+                double m = -INFINITY;
+                for (int j = 0; j < n; ++j) {
+                    row[j] = vis[j] ? scale * dot(qi, hv.k + (size_t)j * hv.kv_stride, D)
+                                    : -INFINITY;
+                    if (row[j] > m) m = row[j];
+                }
+                double* oi = o + ((q_row0 + i) * Hq + h) * (size_t)D;
+                if (m == -INFINITY) {
+                    for (int d = 0; d < D; ++d) oi[d] = 0.0;
+                    lse[lse_off + (size_t)i * lse_step] = -INFINITY;
+                    continue;
+                }
+                double l = 0.0;
+                for (int j = 0; j < n; ++j) {
+                    row[j] = (row[j] == -INFINITY) ? 0.0 : exp(row[j] - m);
+                    l += row[j];
+                }
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int j = 0; j < n; ++j)
+                        if (row[j] != 0.0) acc += row[j] * (double)hv.v[(size_t)j * hv.kv_stride + d];
+                    oi[d] = acc / l;
+                }
+                lse[lse_off + (size_t)i * lse_step] = m + log(l);
+            }
+            free(row);
+            free(vis);
+        }
+    free(off);
     return bad ? -1 : 0;
 }
 

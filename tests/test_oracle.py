@@ -609,6 +609,72 @@ def test_blocksparse_rejects_bad_patterns():
 
 
 # ---------------------------------------------------------------------------------
+# Block-sparse over packed sequences with minimum padding (Raptor-T abstract)
+
+VARLEN_LENS = [50, 0, 130, 17, 260, 33]
+
+
+def varlen_sparse_case(blk, seed):
+    cu = np.concatenate([[0], np.cumsum(VARLEN_LENS)]).astype(np.int32)
+    total, Hq, Hkv, D = int(cu[-1]), 4, 2, 16
+    q, k, v = rnd((total, Hq, D), seed), rnd((total, Hkv, D), seed + 1), \
+        rnd((total, Hkv, D), seed + 2)
+    rp, cl = W.bigbird_pattern_varlen(VARLEN_LENS, {"window": 3, "global": 1, "random": 2},
+                                      seed=seed + 3, blk=blk)
+    return cu, q, k, v, rp.numpy(), cl.numpy()
+
+
+@pytest.mark.parametrize("blk,seed", [(16, 90), (32, 95)])
+def test_blocksparse_varlen_matches_sdpa_per_sequence(blk, seed):
+    cu, q, k, v, rp, cl = varlen_sparse_case(blk, seed)
+    O, L = oracle.attention_blocksparse_varlen(q, k, v, cu, rp, cl, scale=0.3, blk=blk)
+    row0 = 0  # first pattern row of the sequence: its blocks follow the earlier ones'
+    for b, n in enumerate(VARLEN_LENS):
+        nb = -(-n // blk)
+        sl = slice(cu[b], cu[b + 1])
+        if n:
+            sub_rp = rp[row0:row0 + nb + 1] - rp[row0]
+            sub_cl = cl[rp[row0]:rp[row0 + nb]]
+            mask = expand_pattern(sub_rp, sub_cl, n, n, blk)
+            Or, Lr = masked_sdpa(q[sl][None], k[sl][None], v[sl][None], 0.3, mask)
+            np.testing.assert_allclose(O[sl], Or[0], rtol=0, atol=1e-12)
+            Lb = L[:, sl]
+            assert np.array_equal(np.isneginf(Lb), np.isneginf(Lr[0]))
+            fin = np.isfinite(Lr[0])
+            np.testing.assert_allclose(Lb[fin], Lr[0][fin], rtol=0, atol=1e-12)
+        row0 += nb
+
+
+def test_blocksparse_varlen_equals_the_dense_form_per_sequence():
+    blk = 16
+    cu, q, k, v, rp, cl = varlen_sparse_case(blk, 97)
+    O, L = oracle.attention_blocksparse_varlen(q, k, v, cu, rp, cl, scale=0.25, blk=blk)
+    row0 = 0
+    for b, n in enumerate(VARLEN_LENS):
+        nb = -(-n // blk)
+        if n:
+            sl = slice(cu[b], cu[b + 1])
+            sub_rp = rp[row0:row0 + nb + 1] - rp[row0]
+            Od, Ld = oracle.attention_blocksparse(q[sl][None], k[sl][None], v[sl][None], sub_rp,
+                                                  cl[rp[row0]:rp[row0 + nb]], scale=0.25,
+                                                  blk=blk)
+            np.testing.assert_allclose(O[sl], Od[0], rtol=0, atol=1e-13)
+            np.testing.assert_allclose(L[:, sl], Ld[0], rtol=0, atol=1e-13)
+        row0 += nb
+
+
+def test_blocksparse_varlen_rejects_blocks_of_other_sequences():
+    blk = 16
+    cu, q, k, v, rp, cl = varlen_sparse_case(blk, 99)
+    bad = cl.copy()
+    bad[0] = 4  # sequence 0 (50 positions) has key blocks 0..3 only
+    with pytest.raises(ValueError):
+        oracle.attention_blocksparse_varlen(q, k, v, cu, rp, bad, scale=0.3, blk=blk)
+    with pytest.raises(ValueError):  # one row per block of every sequence
+        oracle.attention_blocksparse_varlen(q, k, v, cu, rp[:-1], cl, scale=0.3, blk=blk)
+
+
+# ---------------------------------------------------------------------------------
 # Backward (FA-2 page: dK, dV per K/V block, dQ shared; GQA: dK, dV summed over heads)
 
 def autograd_ref(q, k, v, do, scale, causal):
@@ -749,6 +815,7 @@ PIN_BATTERY = [
     lambda: test_blocksparse_matches_sdpa_with_the_expanded_mask(96, 80, 16, 2),
     lambda: test_backward_matches_torch_autograd_float64(2, 8, 2, 33, 33, 16, True),
     lambda: test_e4m3_prefill_matches_sdpa_on_torch_decoded_values(2, 8, 2, 33, 33, 16, True),
+    lambda: test_blocksparse_varlen_matches_sdpa_per_sequence(16, 90),
 ]
 
 

@@ -135,6 +135,31 @@ def bigbird_pattern(w: Workload):
     return row_ptr, col
 
 
+def bigbird_pattern_varlen(lengths, block_sparse: dict, seed: int, blk: int = 128):
+    """Per-sequence BigBird-style patterns for packed sequences with minimum padding:
+    sequence b has ceil(n_b / blk) query and key blocks, its rows follow those of the
+    earlier sequences, its col entries count its own key blocks.  The pattern of each
+    sequence is built as in bigbird_pattern (window, global, seeded random blocks)."""
+    g = _gen("cpu", seed)
+    rows = []
+    for n in [int(x) for x in lengths]:
+        nb = -(-n // blk)
+        for r in range(nb):
+            if r < block_sparse["global"]:
+                rows.append(list(range(nb)))
+                continue
+            cols = set(range(min(block_sparse["global"], nb)))
+            half = block_sparse["window"] // 2
+            cols |= {c for c in range(r - half, r + half + 1) if 0 <= c < nb}
+            cols |= set(torch.randperm(nb, generator=g)[: block_sparse["random"]].tolist())
+            rows.append(sorted(cols))
+    row_ptr = torch.zeros(len(rows) + 1, dtype=torch.int32)
+    if rows:
+        row_ptr[1:] = torch.cumsum(torch.tensor([len(c) for c in rows]), 0)
+    col = torch.tensor([c for cs in rows for c in cs], dtype=torch.int32)
+    return row_ptr, col
+
+
 def blocksparse_flops(w: Workload, row_ptr, col) -> int:
     """4*D flops per visible (query, key) pair per head under the block pattern."""
     blk = 128
