@@ -29,6 +29,7 @@ import os
 import pathlib
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -90,11 +91,21 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.tmp = False
 
     def __enter__(self):
-        out_dir = ROOT / "gpurun_out"
-        out_dir.mkdir(exist_ok=True)
-        self.path = out_dir / f"clocks_rank{os.environ.get('RANK', '0')}.csv"
+        # the raw samples go to GQA_CLOCKS_DIR when set (kept for inspection), else to a
+        # temporary file; the JSON line carries their summary either way
+        out_dir = os.environ.get("GQA_CLOCKS_DIR")
+        name = f"clocks_rank{os.environ.get('RANK', '0')}.csv"
+        if out_dir:
+            pathlib.Path(out_dir).mkdir(parents=True, exist_ok=True)
+            self.path = pathlib.Path(out_dir) / name
+        else:
+            fd, tmp = tempfile.mkstemp(prefix="gqa_", suffix="_" + name)
+            os.close(fd)
+            self.path = pathlib.Path(tmp)
+            self.tmp = True
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -117,7 +128,10 @@ class ClockSampler:
         if self.proc is None or not self.path or not self.path.exists():
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         rows = []
-        for line in self.path.read_text().splitlines():
+        text = self.path.read_text()
+        if self.tmp:
+            self.path.unlink(missing_ok=True)
+        for line in text.splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
