@@ -125,12 +125,12 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if self.proc is None or not self.path or not self.path.exists():
+        text = self.path.read_text() if self.path and self.path.exists() else ""
+        if self.tmp and self.path:
+            self.path.unlink(missing_ok=True)
+        if self.proc is None or not text:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         rows = []
-        text = self.path.read_text()
-        if self.tmp:
-            self.path.unlink(missing_ok=True)
         for line in text.splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
