@@ -88,6 +88,7 @@ def gqa_attn_get_device_error(stream=None) -> int:
 
 # ------------------------------------------------------------------ torch front end
 _ws = {}  # device index -> torch buffer registered as the split-KV workspace
+_ws_retired = []  # buffers replaced by a larger one, kept alive for in-flight kernels
 
 
 def _workspace(torch, device, nbytes):
@@ -96,7 +97,12 @@ def _workspace(torch, device, nbytes):
     idx = device.index if device.index is not None else torch.cuda.current_device()
     buf = _ws.get(idx)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        # grow geometrically; a replaced buffer stays alive (a kernel on another stream
+        # may still read it), which keeps at most about twice the largest size
+        old = 0 if buf is None else buf.numel()
+        if buf is not None:
+            _ws_retired.append(buf)
+        buf = torch.empty(max(nbytes, 2 * old, 1 << 20), dtype=torch.uint8, device=device)
         _ws[idx] = buf
     with torch.cuda.device(device):  # the registration belongs to this device
         rc = gqa_attn_set_workspace(ctypes.c_void_p(buf.data_ptr()), buf.numel())
