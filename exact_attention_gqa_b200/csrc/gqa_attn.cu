@@ -8,6 +8,8 @@
 #include <cstring>
 #include <algorithm>
 #include <mutex>
+#include <queue>
+#include <vector>
 
 #include "gqa_attn.h"
 #include "sm100_ptx.cuh"
@@ -208,7 +210,9 @@ template <int HD>
 int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                    int Hq, int Hkv, int Sq, int Sk, float scale, int causal, int pack,
                    const int* cu, int sms, cudaStream_t stream,
-                   const int* blk_row_ptr = nullptr, const int* blk_col = nullptr) {
+                   const int* blk_row_ptr = nullptr, const int* blk_col = nullptr,
+                   const int* blk_off = nullptr, const int* tile_order = nullptr,
+                   int n_order = 0, int order_grid = 0) {
     using C = PrefillCfg<HD>;
     {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD>, HD == 64 ? 1 : 2,
@@ -252,6 +256,9 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     p.blk_row_ptr = blk_row_ptr;
     p.blk_col = blk_col;
     p.n_kblk = (Sk + C::BN - 1) / C::BN;
+    p.blk_off = blk_off;
+    p.tile_order = tile_order;
+    if (tile_order) p.n_units = n_order;  // the balanced order lists every step
     // Row extents of the 3-D views: exactly the rows the caller allocated
     // (packed variable length: Sk carries the packed row count).
     const long long rows_q = cu ? (long long)Sk : (long long)B * Sq;
@@ -264,7 +271,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
         !make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN) ||
         !make_map(&to, out, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128))
         return GQA_ERR_CUDA;
-    const int grid = p.n_units < sms ? p.n_units : sms;
+    const int grid = tile_order ? order_grid : (p.n_units < sms ? p.n_units : sms);
     if (blk_row_ptr) {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD, true>, HD == 64 ? 1024 : 2048,
                                          C::SMEM_BYTES);
@@ -987,6 +994,100 @@ int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                                           nullptr, dev->sms, stream, blk_row_ptr, blk_col)
                     : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 0, 1,
                                          nullptr, dev->sms, stream, blk_row_ptr, blk_col);
+}
+
+int gqa_attn_sparse_varlen_schedule(const int* cu_seqlens, const int* blk_row_ptr, int B,
+                                    int Hq, int Hkv, int max_seqlen, int grid, int* blk_off,
+                                    int* order, int order_cap, int* n_order, int* order_grid) {
+    if (!cu_seqlens || !blk_row_ptr || !blk_off || !n_order || !order_grid || B < 0 ||
+        Hq <= 0 || Hkv <= 0 ||
+        Hq % Hkv != 0 || max_seqlen < 0 || grid <= 0 || order_cap < 0 || (order_cap && !order))
+        return GQA_ERR_NULL;
+    const int G = Hq / Hkv;
+    if (G < 2 || 128 % G != 0) return GQA_ERR_UNSUPPORTED;
+    // minimum padding: sequence b owns ceil(n_b / 128) pattern rows, after the earlier ones
+    blk_off[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        const int n = cu_seqlens[b + 1] - cu_seqlens[b];
+        if (n < 0 || n > max_seqlen) return GQA_ERR_SHAPE;
+        blk_off[b + 1] = blk_off[b] + (n + 127) / 128;
+    }
+    // units (b, kv head, m) as the kernel linearises them; cost = key blocks of the row
+    // times the sub-tiles that hold positions, plus one block for the tile's fixed work
+    const int sub = 128 / G, n_mblk = (max_seqlen + 2 * sub - 1) / (2 * sub);
+    struct Unit { long long cost; int u; };
+    std::vector<Unit> units;
+    for (int b = 0; b < B; ++b) {
+        const int n = cu_seqlens[b + 1] - cu_seqlens[b];
+        for (int m = 0; m < n_mblk; ++m) {
+            const int p0 = m * 2 * sub;
+            if (p0 >= n) break;
+            const int qb = blk_off[b] + p0 / 128;
+            const int row = blk_row_ptr[qb + 1] - blk_row_ptr[qb];
+            if (row < 0) return GQA_ERR_SHAPE;
+            const int subs = 1 + (p0 + sub < n ? 1 : 0);
+            for (int h = 0; h < Hkv; ++h)
+                units.push_back({(long long)row * subs + 1, (b * Hkv + h) * n_mblk + m});
+        }
+    }
+    // longest processing time first: each unit goes to the CTA with the least work so far
+    std::stable_sort(units.begin(), units.end(),
+                     [](const Unit& a, const Unit& c) { return a.cost > c.cost; });
+    const int g = (int)std::min<size_t>((size_t)grid, std::max<size_t>(units.size(), 1));
+    std::vector<std::vector<int>> lists(g);
+    using Load = std::pair<long long, int>;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < g; ++c) heap.push({0, c});
+    for (const Unit& x : units) {
+        Load top = heap.top();
+        heap.pop();
+        lists[top.second].push_back(x.u);
+        heap.push({top.first + x.cost, top.second});
+    }
+    size_t depth = 0;
+    for (const auto& l : lists) depth = std::max(depth, l.size());
+    const long long need = (long long)g * (long long)depth;
+    if (need > INT32_MAX) return GQA_ERR_SHAPE;
+    *n_order = (int)need;
+    *order_grid = g;
+    if (need > order_cap) return GQA_ERR_WORKSPACE;  // *n_order says how many entries
+    // CTA c takes steps c, c + g, c + 2 g, ... of the persistent loop
+    for (size_t k = 0; k < depth; ++k)
+        for (int c = 0; c < g; ++c)
+            order[k * g + c] = k < lists[c].size() ? lists[c][k] : -1;
+    return GQA_OK;
+}
+
+int gqa_attn_fwd_blocksparse_varlen(const void* q, const void* k, const void* v, void* out,
+                                    float* lse, const int* cu_seqlens, const int* blk_off,
+                                    int B, int Hq, int Hkv, int max_seqlen, int total, int D,
+                                    float scale, const int* blk_row_ptr, const int* blk_col,
+                                    const int* tile_order, int n_order, int order_grid,
+                                    cudaStream_t stream) {
+    int rc = check_shape(B, Hq, Hkv, max_seqlen, total, D, scale, 1, 1, true, false);
+    if (rc != GQA_OK) return rc;
+    const int G = Hq / Hkv;
+    if (G < 2 || 128 % G != 0) return GQA_ERR_UNSUPPORTED;
+    if (B == 0 || max_seqlen == 0 || total == 0) return GQA_OK;
+    if (!q || !k || !v || !out || !lse || !cu_seqlens || !blk_off || !blk_row_ptr || !blk_col)
+        return GQA_ERR_NULL;
+    if (tile_order && (n_order <= 0 || order_grid <= 0 || n_order % order_grid != 0))
+        return GQA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || !aligned(blk_row_ptr, 4) || !aligned(blk_col, 4) ||
+        !aligned(cu_seqlens, 4) || !aligned(blk_off, 4) || !aligned(tile_order, 4))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, max_seqlen, total,
+                                          scale, 0, 1, cu_seqlens, dev->sms, stream,
+                                          blk_row_ptr, blk_col, blk_off, tile_order, n_order,
+                                          order_grid)
+                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, max_seqlen, total,
+                                         scale, 0, 1, cu_seqlens, dev->sms, stream,
+                                         blk_row_ptr, blk_col, blk_off, tile_order, n_order,
+                                         order_grid);
 }
 
 int gqa_attn_decode_kvcache(const void* q, const void* k_cache, const void* v_cache,

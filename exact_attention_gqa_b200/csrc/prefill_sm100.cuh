@@ -71,6 +71,12 @@ struct PrefillParams {
     const int* blk_row_ptr = nullptr;  // [ceil(Sq / 128) + 1]
     const int* blk_col = nullptr;      // [nnz], ascending within a row
     int n_kblk = 0;                    // ceil(Sk / 128): key blocks that exist
+    // block-sparse over packed sequences (minimum padding): first pattern row of each
+    // sequence, [B + 1] (prefix sum of ceil(n_b / 128)); nullptr: one dense pattern
+    const int* blk_off = nullptr;
+    // optional tile order (attention balancing): entry t is the unit the persistent
+    // loop's t-th step takes, as (b * n_hu + hu) * n_mblk + m, or -1 for no tile
+    const int* tile_order = nullptr;
 };
 
 template <int HD>
@@ -123,7 +129,15 @@ struct TileInfo {
 template <int BN, bool SPARSE = false>
 __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
     TileInfo ti;
-    if (p.kv_major) {
+    bool none = false;
+    if constexpr (SPARSE) {
+        if (p.tile_order) {  // balanced order: unit index in the (b, hu, m) linearisation
+            const int u = __ldg(p.tile_order + t);
+            none = u < 0;
+            t = none ? 0 : u;
+        }
+    }
+    if (p.kv_major || (SPARSE && p.tile_order)) {
         const int bh = t / p.n_mblk;
         ti.m = t - bh * p.n_mblk;
         ti.b = bh / p.n_hu;
@@ -175,12 +189,15 @@ __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
     }
     ti.kb0 = 0;
     if constexpr (SPARSE) {
-        // both sub-tiles lie in query block qb and share its list of key blocks
-        const int qb = (ti.m * 2 * p.sub_pos) >> 7;
-        const int r0 = __ldg(p.blk_row_ptr + qb), r1 = __ldg(p.blk_row_ptr + qb + 1);
+        // both sub-tiles lie in query block qb (of this sequence) and share its list of
+        // key blocks; packed sequences start at their own first pattern row
+        const int qb = ((ti.m * 2 * p.sub_pos) >> 7) + (p.blk_off ? __ldg(p.blk_off + ti.b) : 0);
+        const bool any = !none && (ti.valid[0] || ti.valid[1]);
+        const int r0 = any ? __ldg(p.blk_row_ptr + qb) : 0;
+        const int r1 = any ? __ldg(p.blk_row_ptr + qb + 1) : 0;
         ti.kb0 = r0;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) ti.nblk[i] = ti.valid[i] ? max(r1 - r0, 0) : 0;
+        for (int i = 0; i < 2; ++i) ti.nblk[i] = (ti.valid[i] && !none) ? max(r1 - r0, 0) : 0;
     }
     return ti;
 }
@@ -191,7 +208,7 @@ template <bool SPARSE>
 __device__ __forceinline__ int sparse_block(const PrefillParams& p, const TileInfo& ti, int j) {
     if constexpr (!SPARSE) return j;
     int kb = __ldg(p.blk_col + ti.kb0 + j);
-    if (kb < 0 || kb >= p.n_kblk) {
+    if (kb < 0 || kb >= (ti.sk + 127) >> 7) {  // key blocks of this sequence
         raise_device_error(kDevBadTile);
         kb = 0;
     }

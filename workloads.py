@@ -160,6 +160,18 @@ def bigbird_pattern_varlen(lengths, block_sparse: dict, seed: int, blk: int = 12
     return row_ptr, col
 
 
+def blocksparse_varlen_flops(lengths, row_ptr, col, Hq: int, D: int, blk: int = 128) -> int:
+    """4*D flops per visible (query, key) pair per head over packed sequences."""
+    rp, cl = row_ptr.tolist(), col.tolist()
+    pairs, r = 0, 0
+    for n in [int(x) for x in lengths]:
+        for qb in range(-(-n // blk)):
+            rows_in = min(blk, n - qb * blk)
+            pairs += rows_in * sum(min(blk, n - c * blk) for c in cl[rp[r]:rp[r + 1]])
+            r += 1
+    return 4 * D * pairs * Hq
+
+
 def blocksparse_flops(w: Workload, row_ptr, col) -> int:
     """4*D flops per visible (query, key) pair per head under the block pattern."""
     blk = 128
@@ -176,6 +188,11 @@ def blocksparse_flops(w: Workload, row_ptr, col) -> int:
 VARLEN = Workload("varlen32_len128to8192_causal", B=32, Hq=32, Hkv=8, Sq=0, Sk=0, D=128,
                   dtype="bf16", causal=True, seed=5,
                   varlen={"n": 32, "lo": 128, "hi": 8192})
+# the same 32 lengths (seed 5), non-causal, a BigBird-style pattern per sequence
+BIGBIRD_VARLEN = Workload("bigbird_varlen32_len128to8192_blk128", B=32, Hq=32, Hkv=8, Sq=0,
+                          Sk=0, D=128, dtype="bf16", causal=False, seed=5,
+                          varlen={"n": 32, "lo": 128, "hi": 8192},
+                          block_sparse={"window": 3, "global": 2, "random": 3})
 
 
 def _gen(device, seed: int) -> torch.Generator:
