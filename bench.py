@@ -197,6 +197,8 @@ def workload_by_name(name: str):
         return W.BIGBIRD
     if name == "bigbird_varlen":
         return W.BIGBIRD_VARLEN
+    if name == "llama_fp8":
+        return W.LLAMA_FP8
     if name == "llama_bwd":
         return W.LLAMA_BWD
     if name == "llama_bwd_b1":
@@ -267,6 +269,14 @@ class Case:
             self.launches_per_step = 3
             self.kernel = "bwd_tc"
             self.splits, self.pack = 1, 0
+        elif w.qkv_fp8:
+            q8, k8, v8 = W.make_qkv_e4m3(w, device=device)
+            self.q, self.kv = q8, [(k8, v8)]
+            self.flops = W.attention_flops(w.B, w.Hq, w.Sq, w.Sk, w.D, w.causal)
+            self.units, self.unit = self.flops / 1e12, "TFLOP/s"
+            self.launches_per_step = 1
+            self.kernel = "prefill_fwd_sm100"
+            self.splits, self.pack = 1, 1
         elif w.block_sparse and self.varlen:
             lengths = W.varlen_lengths(w)
             q, k, v, cu = W.make_varlen(w, device=device, lengths=lengths)
@@ -315,7 +325,7 @@ class Case:
             rc, kern, self.splits, self.pack = G.gqa_attn_plan(w.B, w.Hq, w.Hkv, w.Sq, w.Sk,
                                                                w.D, causal=w.causal,
                                                                pack_gqa=w.pack_gqa)
-        self.out = torch.empty_like(self.q)
+        self.out = torch.empty(self.q.shape, dtype=torch.bfloat16, device=device)
         if self.varlen:
             self.lse = torch.empty(w.Hq, self.q.shape[0], dtype=torch.float32, device=device)
         else:
@@ -325,7 +335,8 @@ class Case:
 
     def in_bytes(self):
         k, v = self.kv[0]
-        return self.q.numel() * 2 + k.numel() * k.element_size() + v.numel() * v.element_size()
+        return (self.q.numel() * self.q.element_size() + k.numel() * k.element_size() +
+                v.numel() * v.element_size())
 
     def out_bytes(self):
         return self.out.numel() * 2 + self.lse.numel() * 4
@@ -338,6 +349,11 @@ class Case:
             dq, dk, dv = self.grads
             self.G.gqa_attn_backward(self.q, k, v, self.fwd_out, self.fwd_lse, self.do,
                                      causal=w.causal, dq=dq, dk=dk, dv=dv)
+            return
+        if w.qkv_fp8:
+            sc = W.FP8_PREFILL_SCALE
+            self.G.gqa_attn_fp8(self.q, k, v, q_scale=sc, k_scale=sc, v_scale=sc,
+                                causal=w.causal, out=self.out, lse=self.lse)
             return
         if w.block_sparse and self.varlen:
             self.G.gqa_attn_blocksparse_varlen(self.q, k, v, self.cu, self.rp, self.col,
@@ -430,6 +446,22 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
             n += 1
         return (n * flops / 1e12 / el, f"{n} x the backward of batch element 0, the {w.G} "
                 f"query heads of K/V head 0, positions 0..{S - 1}", cores, el)
+    if w.qkv_fp8:
+        S = 1024
+        q8, k8, v8 = W.make_qkv_e4m3(w, B=1, Sq=S, Sk=S)
+        q8, k8, v8 = q8[:, :, : w.G].contiguous(), k8[:, :, :1].contiguous(), \
+            v8[:, :, :1].contiguous()
+        sc = W.FP8_PREFILL_SCALE
+        flops = W.attention_flops(1, w.G, S, S, w.D, w.causal)
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.attention_e4m3(q8, k8, v8, q_scale=sc, k_scale=sc, v_scale=sc,
+                                  scale=w.scale, causal=w.causal)
+            el += time.perf_counter() - t0
+            n += 1
+        return (n * flops / 1e12 / el, f"{n} x the e4m3 forward of batch element 0, the "
+                f"{w.G} query heads of K/V head 0, positions 0..{S - 1}", cores, el)
     if w.block_sparse and w.varlen:
         lengths = W.varlen_lengths(w).tolist()
         q, k, v, cu = W.make_varlen(w, lengths=lengths)
@@ -532,6 +564,8 @@ def workload_config(w) -> dict:
            "D": w.D, "causal": w.causal}
     if w.kv_fp8:
         cfg["kv_cache"] = f"e4m3 codes, k_scale = v_scale = {W.FP8_SCALE}"
+    if w.qkv_fp8:
+        cfg["inputs"] = f"e4m3 codes, q_scale = k_scale = v_scale = {W.FP8_PREFILL_SCALE}"
     if w.backward:
         cfg["pass"] = "backward: dQ, dK, dV for a seeded dO (O and L from the forward)"
         cfg["flops"] = "2.5 x the forward's (five products against two)"
@@ -650,6 +684,15 @@ def run_ours(args, world, rank, local):
             for h, d in zip(hgrads, gd):
                 h.copy_(d, non_blocking=True)
             return
+        if w.qkv_fp8:
+            sc = W.FP8_PREFILL_SCALE
+            for d, h in ((dq, hq), (dk, hk), (dv, hv)):
+                d.copy_(h, non_blocking=True)
+            G.gqa_attn_fp8(dq, dk, dv, q_scale=sc, k_scale=sc, v_scale=sc, causal=w.causal,
+                           out=case.out, lse=case.lse)
+            ho.copy_(case.out, non_blocking=True)
+            hl.copy_(case.lse, non_blocking=True)
+            return
         if w.block_sparse and case.varlen:
             # the schedule from the host copies of the offsets and the pattern, then the
             # inputs in, the attention, the results out
@@ -740,14 +783,18 @@ def run_ours(args, world, rank, local):
         sustained = ms_total >= 1000.0 and "bf16_tflops_sustained" in peaks
         key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
         achieved = case.flops / (kernel_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks[key],
-                "unit": "TFLOP/s", "frac_of_burst": achieved / peaks["bf16_tflops"]}
+        # an e4m3 contraction: the measured bf16 figure times the nominal 2x of fp8
+        ratio = 2.0 if w.qkv_fp8 else 1.0
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks[key] * ratio,
+                "unit": "TFLOP/s",
+                "frac_of_burst": achieved / (peaks["bf16_tflops"] * ratio)}
     roof["frac"] = roof["achieved"] / roof["peak"]
     if case.decode:
         roof["peak_source"] = f"{peak_kind} (hbm_gbs, copy)"
     else:
         roof["peak_source"] = (f"{peak_kind} ({key}: timed region {ms_total / 1e3:.1f} s, "
-                               f"{'sustained' if sustained else 'burst'})")
+                               f"{'sustained' if sustained else 'burst'})"
+                               + (" x 2, the nominal e4m3 / bf16 ratio" if w.qkv_fp8 else ""))
     roof["kernel"] = case.kernel
     tr = load_traffic(w.name, case.kernel)
     roof["traffic"] = tr
@@ -781,14 +828,18 @@ def run_ours(args, world, rank, local):
             cfg["tile_order"] = "host schedule: longest first onto the least loaded CTA"
     line = {"metric": METRIC, "value": value, "unit": case.unit, "n_gpus": world,
             "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) bf16)", "config": cfg, "roofline": roof,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if w.qkv_fp8 else "bf16",
+            "data": "synthetic (seeded N(0,1) bf16)" + (", as e4m3 codes" if w.qkv_fp8 else ""),
+            "config": cfg, "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms,
                     "path": ("gqa_attn_backward after pinned host copies of q, k, v, O, L "
                              "and dO; dQ, dK, dV copied back" if w.backward else
+                             "gqa_attn_fp8 after pinned host copies of the e4m3 q, k, v; "
+                             "results copied back" if w.qkv_fp8 else
                              "gqa_attn_blocksparse_varlen_plan on the host offsets and "
                              "pattern, pinned host copies of q, k, v, cu_seqlens and the "
                              "pattern, gqa_attn_blocksparse_varlen; results copied back"

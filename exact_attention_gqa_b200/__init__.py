@@ -28,7 +28,7 @@ __all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_kvcache", "gqa_attn_blockspars
            "gqa_attn_workspace_bytes", "gqa_attn_set_workspace", "gqa_attn_get_device_error",
            "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path",
            "gqa_attn_blocksparse_varlen", "gqa_attn_blocksparse_varlen_plan",
-           "SparseVarlenPlan"]
+           "SparseVarlenPlan", "gqa_attn_fp8"]
 
 KERNEL_NAMES = {0: "none", 1: "prefill_sm100", 2: "decode_splitkv", 3: "zero_fill"}
 
@@ -175,6 +175,51 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
                               stream)
         if rc != 0:
             raise GqaError("gqa_attn_fwd_f32", rc)
+
+
+def gqa_attn_fp8(q8, k8, v8, *, q_scale: float, k_scale: float, v_scale: float,
+                 causal: bool = False, scale: float | None = None, cu_seqlens=None,
+                 max_seqlen: int | None = None, out=None, lse=None):
+    """Prefill on e4m3 codes (gqa_attn_fwd_fp8): q8 [B, Sq, Hq, 128], k8/v8 [B, Sk, Hkv,
+    128] as torch.float8_e4m3fn or uint8 on the GPU (or packed [total, H, 128] with
+    cu_seqlens and max_seqlen); element = value(code) * its tensor's scale.  Returns
+    (out bf16 like q8, lse)."""
+    import torch
+
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+            raise ValueError(f"{name} must hold e4m3 codes (uint8 or float8_e4m3fn)")
+    varlen = cu_seqlens is not None
+    if varlen:
+        if q8.dim() != 3 or k8.dim() != 3 or v8.shape != k8.shape or max_seqlen is None:
+            raise ValueError("packed q8 [total, Hq, D], k8/v8 [total, Hkv, D], max_seqlen")
+        total, Hq, D = q8.shape
+        Hkv = k8.shape[1]
+        B, Sq, Sk = cu_seqlens.numel() - 1, int(max_seqlen), total
+        lse_shape = (Hq, total)
+    else:
+        if q8.dim() != 4 or k8.dim() != 4 or v8.shape != k8.shape:
+            raise ValueError("q8 [B, Sq, Hq, D], k8/v8 [B, Sk, Hkv, D]")
+        B, Sq, Hq, D = q8.shape
+        _, Sk, Hkv, _ = k8.shape
+        lse_shape = (B, Hq, Sq)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device) if out is None else out
+    lse = torch.empty(lse_shape, dtype=torch.float32, device=q8.device) if lse is None else lse
+    lib = _capi.load()
+    with torch.cuda.device(q8.device):
+        rc = lib.gqa_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), B, Hq,
+                                  Hkv, Sq, Sk, D, scale, float(q_scale), float(k_scale),
+                                  float(v_scale), int(bool(causal)),
+                                  _ptr(cu_seqlens) if varlen else None,
+                                  _stream_handle(torch, q8.device))
+    if rc != 0:
+        raise GqaError("gqa_attn_fwd_fp8", rc)
+    return out, lse
 
 
 class SparseVarlenPlan:

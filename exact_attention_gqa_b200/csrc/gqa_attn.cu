@@ -128,6 +128,22 @@ bool make_map_u8(CUtensorMap* m, const void* base, long long rows, int heads, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 8-bit [rows, heads, D] view with 128-byte swizzle: boxes of {128 bytes, box_h,
+// box_rows} (e4m3 Q, K, V of the prefill; D = 128 is one swizzle atom)
+bool make_map_u8_sw128(CUtensorMap* m, const void* base, long long rows, int heads, int D,
+                       int box_h, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(heads), cuuint64_t(rows)};
+    cuuint64_t strides[2] = {cuuint64_t(D), cuuint64_t(heads) * D};
+    cuuint32_t box[3] = {128u, cuuint32_t(box_h), cuuint32_t(box_rows)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------- plan
 struct Plan {
     int kernel = kNone;
@@ -206,15 +222,16 @@ size_t ws_bytes(int B, int Hq, int Sq, int D, int n) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-template <int HD>
+template <int HD, bool FP8 = false>
 int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                    int Hq, int Hkv, int Sq, int Sk, float scale, int causal, int pack,
                    const int* cu, int sms, cudaStream_t stream,
                    const int* blk_row_ptr = nullptr, const int* blk_col = nullptr,
                    const int* blk_off = nullptr, const int* tile_order = nullptr,
-                   int n_order = 0, int order_grid = 0) {
-    using C = PrefillCfg<HD>;
-    {
+                   int n_order = 0, int order_grid = 0, float qk_scale = 1.f,
+                   float o_scale = 1.f) {
+    using C = PrefillCfg<HD, FP8>;
+    if constexpr (!FP8) {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD>, HD == 64 ? 1 : 2,
                                          C::SMEM_BYTES);
         if (rc != GQA_OK) return rc;
@@ -252,7 +269,8 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
         if (hg > per_m) hg = per_m;
         p.hu_group = int(hg);
     }
-    p.scale_log2 = scale * kLog2e;
+    p.scale_log2 = scale * qk_scale * kLog2e;  // e4m3: the Q and K code units folded in
+    p.o_scale = o_scale;
     p.blk_row_ptr = blk_row_ptr;
     p.blk_col = blk_col;
     p.n_kblk = (Sk + C::BN - 1) / C::BN;
@@ -266,12 +284,26 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     p.total_rows = cu ? Sk : 0;
     CUtensorMap tq, tk, tv, to;
     // the output leaves through the same box shape as Q arrives in (one sub-tile)
-    if (!make_map(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) ||
-        !make_map(&tk, k, rows_k, Hkv, HD, 1, C::BN) ||
-        !make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN) ||
-        !make_map(&to, out, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128))
+    bool maps_ok;
+    if constexpr (FP8)
+        maps_ok = make_map_u8_sw128(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) &&
+                  make_map_u8_sw128(&tk, k, rows_k, Hkv, HD, 1, C::BN) &&
+                  make_map_u8_sw128(&tv, v, rows_k, Hkv, HD, 1, C::BN);
+    else
+        maps_ok = make_map(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) &&
+                  make_map(&tk, k, rows_k, Hkv, HD, 1, C::BN) &&
+                  make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN);
+    if (!maps_ok || !make_map(&to, out, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128))
         return GQA_ERR_CUDA;
     const int grid = tile_order ? order_grid : (p.n_units < sms ? p.n_units : sms);
+    if constexpr (FP8) {
+        const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD, false, true>, 65536,
+                                         C::SMEM_BYTES);
+        if (rc != GQA_OK) return rc;
+        gqa::prefill_fwd_sm100<HD, false, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
+            tq, tk, tv, to, p);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
     if (blk_row_ptr) {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD, true>, HD == 64 ? 1024 : 2048,
                                          C::SMEM_BYTES);
@@ -994,6 +1026,39 @@ int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                                           nullptr, dev->sms, stream, blk_row_ptr, blk_col)
                     : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 0, 1,
                                          nullptr, dev->sms, stream, blk_row_ptr, blk_col);
+}
+
+int gqa_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* out, float* lse,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, float q_scale,
+                     float k_scale, float v_scale, int causal, const int* cu_seqlens,
+                     cudaStream_t stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, 1, -1, varlen, false);
+    if (rc != GQA_OK) return rc;
+    if (D != 128) return GQA_ERR_HEADDIM;
+    if (!(std::isfinite(q_scale) && q_scale > 0.f && std::isfinite(k_scale) && k_scale > 0.f &&
+          std::isfinite(v_scale) && v_scale > 0.f))
+        return GQA_ERR_SCALE;
+    if (B == 0 || Sq == 0 || (varlen && Sk == 0)) return GQA_OK;
+    const bool reads_kv = varlen || Sk > 0;
+    if (!q8 || !out || !lse || (reads_kv && (!k8 || !v8))) return GQA_ERR_NULL;
+    if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || (varlen && !aligned(cu_seqlens, 4)))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    if (!varlen && Sk == 0) {
+        gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(out), (long long)B * Sq * Hq * D, lse,
+            (long long)B * Hq * Sq);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
+    Plan pl;
+    make_plan(&pl, B, Hq, Hkv, Sq, Sk, 1, -1, varlen, dev->sms);
+    return launch_prefill<128, true>(q8, k8, v8, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal,
+                                     pl.pack, cu_seqlens, dev->sms, stream, nullptr, nullptr,
+                                     nullptr, nullptr, 0, 0, q_scale * k_scale, v_scale);
 }
 
 int gqa_attn_sparse_varlen_schedule(const int* cu_seqlens, const int* blk_row_ptr, int B,

@@ -267,6 +267,24 @@ int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                              const int* blk_row_ptr, const int* blk_col, cudaStream_t stream);
 
 /*
+ * Prefill forward on e4m3 Q, K and V with one scale per tensor (the batch-size guide
+ * names FP8 as the precision that lowers memory-bandwidth pressure: hardware adaptation
+ * section, Hopper item; precision row of its production checklist).
+ *   element = value(code) * scale of its tensor; q8 [B, Sq, Hq, D], k8/v8 [B, Sk, Hkv,
+ *   D] bytes (or packed [total, H, D] with cu_seqlens as gqa_attn_fwd); D = 128;
+ *   out bf16 like q, lse fp32 as gqa_attn_fwd; causal as gqa_attn_fwd.
+ * S = Q K^T and O += P V run as 8-bit tensor-core products (kind::f8f6f4, fp32
+ * accumulation); P is rounded to e4m3 (relative to the running row max, times 2^7),
+ * O is normalised by the sum of the unrounded p.  Codes 0x7f / 0xff (NaN) are not
+ * supported.  Errors as gqa_attn_fwd, plus GQA_ERR_SCALE for a scale that is not
+ * finite and positive.
+ */
+int gqa_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* out, float* lse,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, float q_scale,
+                     float k_scale, float v_scale, int causal, const int* cu_seqlens,
+                     cudaStream_t stream);
+
+/*
  * Block-sparse attention over packed variable-length sequences with minimum padding
  * (Raptor-T abstract: BigBird's block-sparse attention; the minimum-padding algorithm
  * pads each sequence only to whole blocks instead of to the longest sequence; the

@@ -408,3 +408,29 @@ def test_blocksparse_varlen_argument_errors(lib):
     assert call(order=FAKE, n_order=10, grid=3) == "GQA_ERR_SHAPE"
     assert call(cu=ctypes.c_void_p(0x1002)) == "GQA_ERR_ALIGN"
     assert call(B=0) == "GQA_OK"
+
+
+# ---------------------------------------------------------------- e4m3 prefill
+def fp8_prefill_call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=8, Hkv=2, Sq=256,
+             Sk=256, D=128, scale=0.125, qs=1.0, ks=1.0, vs=1.0, causal=1, cu=None):
+    return lib.gqa_attn_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, qs, ks, vs,
+                                causal, cu, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=64), "GQA_ERR_HEADDIM"),
+    (dict(qs=0.0), "GQA_ERR_SCALE"),
+    (dict(vs=float("inf")), "GQA_ERR_SCALE"),
+    (dict(scale=-1.0), "GQA_ERR_SCALE"),
+    (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
+    (dict(q=None), "GQA_ERR_NULL"),
+    (dict(v=None), "GQA_ERR_NULL"),
+    (dict(k=ctypes.c_void_p(0x1004)), "GQA_ERR_ALIGN"),
+])
+def test_fp8_prefill_argument_errors(lib, kw, code):
+    assert G.STATUS[fp8_prefill_call(lib, **kw)] == code
+
+
+def test_fp8_prefill_empty_problems_are_noops(lib):
+    assert fp8_prefill_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert fp8_prefill_call(lib, Sq=0, q=None, k=None, v=None, out=None, lse=None) == 0
