@@ -204,12 +204,15 @@ __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
         // both sub-tiles lie in query block qb (of this sequence) and share its list of
         // key blocks; packed sequences start at their own first pattern row
         const int qb = ((ti.m * 2 * p.sub_pos) >> 7) + (p.blk_off ? __ldg(p.blk_off + ti.b) : 0);
-        const bool any = !none && (ti.valid[0] || ti.valid[1]);
+        // an empty slot of the balanced order is no tile at all: no role may touch the
+        // unit it decoded to (the softmax warps key their epilogue on `valid`)
+        if (none) ti.valid[0] = ti.valid[1] = 0;
+        const bool any = ti.valid[0] || ti.valid[1];
         const int r0 = any ? __ldg(p.blk_row_ptr + qb) : 0;
         const int r1 = any ? __ldg(p.blk_row_ptr + qb + 1) : 0;
         ti.kb0 = r0;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) ti.nblk[i] = (ti.valid[i] && !none) ? max(r1 - r0, 0) : 0;
+        for (int i = 0; i < 2; ++i) ti.nblk[i] = ti.valid[i] ? max(r1 - r0, 0) : 0;
     }
     return ti;
 }
