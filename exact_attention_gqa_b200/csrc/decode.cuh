@@ -421,7 +421,9 @@ __global__ void __launch_bounds__(160, 2)
                 for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(qv[hr][e]));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
                 amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                const float sc_row = amax > 0.f ? exp2f(floorf(log2f(224.f / amax))) : 1.f;
+                // 2^floor(log2(224 / amax)), capped so that it stays finite for tiny rows
+                const float sc_row =
+                    amax > 0.f ? fminf(exp2f(floorf(log2f(224.f / amax))), 0x1p100f) : 1.f;
                 sl2r[hr] = sl2 / sc_row;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
