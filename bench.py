@@ -195,6 +195,10 @@ def workload_by_name(name: str):
         return W.VARLEN
     if name == "bigbird":
         return W.BIGBIRD
+    if name == "bigbird_varlen":
+        return W.BIGBIRD_VARLEN
+    if name == "llama_fp8":
+        return W.LLAMA_FP8
     if name == "llama_bwd":
         return W.LLAMA_BWD
     if name == "llama_bwd_b1":
@@ -265,6 +269,31 @@ class Case:
             self.launches_per_step = 3
             self.kernel = "bwd_tc"
             self.splits, self.pack = 1, 0
+        elif w.qkv_fp8:
+            q8, k8, v8 = W.make_qkv_e4m3(w, device=device)
+            self.q, self.kv = q8, [(k8, v8)]
+            self.flops = W.attention_flops(w.B, w.Hq, w.Sq, w.Sk, w.D, w.causal)
+            self.units, self.unit = self.flops / 1e12, "TFLOP/s"
+            self.launches_per_step = 1
+            self.kernel = "prefill_fwd_sm100"
+            self.splits, self.pack = 1, 1
+        elif w.block_sparse and self.varlen:
+            lengths = W.varlen_lengths(w)
+            q, k, v, cu = W.make_varlen(w, device=device, lengths=lengths)
+            self.q, self.kv, self.cu = q, [(k, v)], cu.to(device)
+            self.max_len = int(lengths.max())
+            self.lengths = lengths
+            rp, col = W.bigbird_pattern_varlen(lengths.tolist(), w.block_sparse,
+                                               seed=w.seed + 101)
+            self.rp, self.col = rp.to(device), col.to(device)
+            self.plan = G.gqa_attn_blocksparse_varlen_plan(cu, rp, Hq=w.Hq, Hkv=w.Hkv,
+                                                           max_seqlen=self.max_len,
+                                                           device=device)
+            self.flops = W.blocksparse_varlen_flops(lengths.tolist(), rp, col, w.Hq, w.D)
+            self.units, self.unit = self.flops / 1e12, "TFLOP/s"
+            self.launches_per_step = 1
+            self.kernel = "prefill_fwd_sm100"
+            self.splits, self.pack = 1, 1
         elif w.block_sparse:
             q, k, v = W.make_qkv(w, device=device)
             self.q, self.kv = q, [(k, v)]
@@ -296,7 +325,7 @@ class Case:
             rc, kern, self.splits, self.pack = G.gqa_attn_plan(w.B, w.Hq, w.Hkv, w.Sq, w.Sk,
                                                                w.D, causal=w.causal,
                                                                pack_gqa=w.pack_gqa)
-        self.out = torch.empty_like(self.q)
+        self.out = torch.empty(self.q.shape, dtype=torch.bfloat16, device=device)
         if self.varlen:
             self.lse = torch.empty(w.Hq, self.q.shape[0], dtype=torch.float32, device=device)
         else:
@@ -306,7 +335,8 @@ class Case:
 
     def in_bytes(self):
         k, v = self.kv[0]
-        return self.q.numel() * 2 + k.numel() * k.element_size() + v.numel() * v.element_size()
+        return (self.q.numel() * self.q.element_size() + k.numel() * k.element_size() +
+                v.numel() * v.element_size())
 
     def out_bytes(self):
         return self.out.numel() * 2 + self.lse.numel() * 4
@@ -319,6 +349,16 @@ class Case:
             dq, dk, dv = self.grads
             self.G.gqa_attn_backward(self.q, k, v, self.fwd_out, self.fwd_lse, self.do,
                                      causal=w.causal, dq=dq, dk=dk, dv=dv)
+            return
+        if w.qkv_fp8:
+            sc = W.FP8_PREFILL_SCALE
+            self.G.gqa_attn_fp8(self.q, k, v, q_scale=sc, k_scale=sc, v_scale=sc,
+                                causal=w.causal, out=self.out, lse=self.lse)
+            return
+        if w.block_sparse and self.varlen:
+            self.G.gqa_attn_blocksparse_varlen(self.q, k, v, self.cu, self.rp, self.col,
+                                               max_seqlen=self.max_len, plan=self.plan,
+                                               out=self.out, lse=self.lse)
             return
         if w.block_sparse:
             self.G.gqa_attn_blocksparse(self.q, k, v, self.rp, self.col, out=self.out,
@@ -406,6 +446,39 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
             n += 1
         return (n * flops / 1e12 / el, f"{n} x the backward of batch element 0, the {w.G} "
                 f"query heads of K/V head 0, positions 0..{S - 1}", cores, el)
+    if w.qkv_fp8:
+        S = 1024
+        q8, k8, v8 = W.make_qkv_e4m3(w, B=1, Sq=S, Sk=S)
+        q8, k8, v8 = q8[:, :, : w.G].contiguous(), k8[:, :, :1].contiguous(), \
+            v8[:, :, :1].contiguous()
+        sc = W.FP8_PREFILL_SCALE
+        flops = W.attention_flops(1, w.G, S, S, w.D, w.causal)
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.attention_e4m3(q8, k8, v8, q_scale=sc, k_scale=sc, v_scale=sc,
+                                  scale=w.scale, causal=w.causal)
+            el += time.perf_counter() - t0
+            n += 1
+        return (n * flops / 1e12 / el, f"{n} x the e4m3 forward of batch element 0, the "
+                f"{w.G} query heads of K/V head 0, positions 0..{S - 1}", cores, el)
+    if w.block_sparse and w.varlen:
+        lengths = W.varlen_lengths(w).tolist()
+        q, k, v, cu = W.make_varlen(w, lengths=lengths)
+        rp, col = W.bigbird_pattern_varlen(lengths, w.block_sparse, seed=w.seed + 101)
+        # sequence 0, the G query heads of K/V head 0, with its rows of the pattern
+        n0, nb = lengths[0], -(-lengths[0] // 128)
+        q, k, v = (t[: n0][None][:, :, : h].contiguous() for t, h in ((q, w.G), (k, 1), (v, 1)))
+        sub_rp, sub_col = rp[: nb + 1], col[: int(rp[nb])]
+        flops = W.blocksparse_varlen_flops([n0], sub_rp, sub_col, w.G, w.D)
+        n, el = 0, 0.0
+        while el < target_s and el < max_s:
+            t0 = time.perf_counter()
+            oracle.attention_blocksparse(q, k, v, sub_rp, sub_col, scale=w.scale, blk=128)
+            el += time.perf_counter() - t0
+            n += 1
+        return (n * flops / 1e12 / el, f"{n} x packed sequence 0 ({n0} positions), the "
+                f"{w.G} query heads of KV head 0", cores, el)
     if w.block_sparse:
         q, k, v = W.make_qkv(w, B=1)
         q, k, v = q[:, :, : w.G].contiguous(), k[:, :, :1].contiguous(), v[:, :, :1].contiguous()
@@ -491,6 +564,8 @@ def workload_config(w) -> dict:
            "D": w.D, "causal": w.causal}
     if w.kv_fp8:
         cfg["kv_cache"] = f"e4m3 codes, k_scale = v_scale = {W.FP8_SCALE}"
+    if w.qkv_fp8:
+        cfg["inputs"] = f"e4m3 codes, q_scale = k_scale = v_scale = {W.FP8_PREFILL_SCALE}"
     if w.backward:
         cfg["pass"] = "backward: dQ, dK, dV for a seeded dO (O and L from the forward)"
         cfg["flops"] = "2.5 x the forward's (five products against two)"
@@ -609,6 +684,27 @@ def run_ours(args, world, rank, local):
             for h, d in zip(hgrads, gd):
                 h.copy_(d, non_blocking=True)
             return
+        if w.qkv_fp8:
+            sc = W.FP8_PREFILL_SCALE
+            for d, h in ((dq, hq), (dk, hk), (dv, hv)):
+                d.copy_(h, non_blocking=True)
+            G.gqa_attn_fp8(dq, dk, dv, q_scale=sc, k_scale=sc, v_scale=sc, causal=w.causal,
+                           out=case.out, lse=case.lse)
+            ho.copy_(case.out, non_blocking=True)
+            hl.copy_(case.lse, non_blocking=True)
+            return
+        if w.block_sparse and case.varlen:
+            # the schedule from the host copies of the offsets and the pattern, then the
+            # inputs in, the attention, the results out
+            plan = G.gqa_attn_blocksparse_varlen_plan(cu_h, hrp, Hq=w.Hq, Hkv=w.Hkv,
+                                                      max_seqlen=case.max_len, device=dq.device)
+            for d, h in ((dq, hq), (dk, hk), (dv, hv), (dcu, cu_h), (drp, hrp), (dcol, hcol)):
+                d.copy_(h, non_blocking=True)
+            G.gqa_attn_blocksparse_varlen(dq, dk, dv, dcu, drp, dcol, max_seqlen=case.max_len,
+                                          plan=plan, out=case.out, lse=case.lse)
+            ho.copy_(case.out, non_blocking=True)
+            hl.copy_(case.lse, non_blocking=True)
+            return
         if w.block_sparse:
             for d, h in ((dq, hq), (dk, hk), (dv, hv), (drp, hrp), (dcol, hcol)):
                 d.copy_(h, non_blocking=True)
@@ -664,6 +760,8 @@ def run_ours(args, world, rank, local):
         ((ht.numel() + hs.numel()) * 4 if case.paged else 0) + \
         ((hrp.numel() + hcol.numel()) * 4 if w.block_sparse else 0)
     d2h = ho.numel() * 2 + hl.numel() * 4
+    if w.block_sparse and case.varlen:  # the plan's block offsets and tile order
+        h2d += case.plan.blk_off.numel() * 4 + case.plan.n_order * 4
     if w.backward:
         h2d += hout.numel() * 2 + hlse.numel() * 4 + hdo.numel() * 2
         d2h = sum(t.numel() * 2 for t in hgrads)
@@ -685,14 +783,18 @@ def run_ours(args, world, rank, local):
         sustained = ms_total >= 1000.0 and "bf16_tflops_sustained" in peaks
         key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
         achieved = case.flops / (kernel_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks[key],
-                "unit": "TFLOP/s", "frac_of_burst": achieved / peaks["bf16_tflops"]}
+        # an e4m3 contraction: the measured bf16 figure times the nominal 2x of fp8
+        ratio = 2.0 if w.qkv_fp8 else 1.0
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks[key] * ratio,
+                "unit": "TFLOP/s",
+                "frac_of_burst": achieved / (peaks["bf16_tflops"] * ratio)}
     roof["frac"] = roof["achieved"] / roof["peak"]
     if case.decode:
         roof["peak_source"] = f"{peak_kind} (hbm_gbs, copy)"
     else:
         roof["peak_source"] = (f"{peak_kind} ({key}: timed region {ms_total / 1e3:.1f} s, "
-                               f"{'sustained' if sustained else 'burst'})")
+                               f"{'sustained' if sustained else 'burst'})"
+                               + (" x 2, the nominal e4m3 / bf16 ratio" if w.qkv_fp8 else ""))
     roof["kernel"] = case.kernel
     tr = load_traffic(w.name, case.kernel)
     roof["traffic"] = tr
@@ -717,18 +819,31 @@ def run_ours(args, world, rank, local):
     if case.varlen:
         cfg["total_tokens"] = int(case.q.shape[0])
     if w.block_sparse:
+        every = (sum((-(-int(n) // 128)) ** 2 for n in case.lengths.tolist()) if case.varlen
+                 else (case.rp.numel() - 1) * -(-w.Sk // 128))
         cfg["block_pattern"] = dict(w.block_sparse, block=128, blocks=int(case.col.numel()),
-                                    of=int((case.rp.numel() - 1) * -(-w.Sk // 128)))
+                                    of=int(every))
+        if case.varlen:
+            cfg["padding"] = "each sequence to whole 128-position blocks (minimum padding)"
+            cfg["tile_order"] = "host schedule: longest first onto the least loaded CTA"
     line = {"metric": METRIC, "value": value, "unit": case.unit, "n_gpus": world,
             "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) bf16)", "config": cfg, "roofline": roof,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3" if w.qkv_fp8 else "bf16",
+            "data": "synthetic (seeded N(0,1) bf16)" + (", as e4m3 codes" if w.qkv_fp8 else ""),
+            "config": cfg, "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": case.units * world / (e2e_ms / 1e3), "unit": case.unit,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms,
                     "path": ("gqa_attn_backward after pinned host copies of q, k, v, O, L "
                              "and dO; dQ, dK, dV copied back" if w.backward else
+                             "gqa_attn_fp8 after pinned host copies of the e4m3 q, k, v; "
+                             "results copied back" if w.qkv_fp8 else
+                             "gqa_attn_blocksparse_varlen_plan on the host offsets and "
+                             "pattern, pinned host copies of q, k, v, cu_seqlens and the "
+                             "pattern, gqa_attn_blocksparse_varlen; results copied back"
+                             if w.block_sparse and case.varlen else
                              "gqa_attn_blocksparse after pinned host copies of q, k, v and "
                              "the block pattern; results copied back" if w.block_sparse else
                              "gqa_attn_kvcache on the e4m3 cache after pinned host copies "

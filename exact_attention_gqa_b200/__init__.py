@@ -26,7 +26,9 @@ __all__ = ["gqa_attn", "gqa_attn_host", "gqa_attn_kvcache", "gqa_attn_blockspars
            "gqa_attn_backward",
            "gqa_attn_fwd", "gqa_attn_fwd_f32", "gqa_attn_plan",
            "gqa_attn_workspace_bytes", "gqa_attn_set_workspace", "gqa_attn_get_device_error",
-           "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path"]
+           "GqaError", "STATUS", "STATUS_CODE", "strerror", "library_path",
+           "gqa_attn_blocksparse_varlen", "gqa_attn_blocksparse_varlen_plan",
+           "SparseVarlenPlan", "gqa_attn_fp8"]
 
 KERNEL_NAMES = {0: "none", 1: "prefill_sm100", 2: "decode_splitkv", 3: "zero_fill"}
 
@@ -179,6 +181,147 @@ def _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_sp
                               stream)
         if rc != 0:
             raise GqaError("gqa_attn_fwd_f32", rc)
+
+
+def gqa_attn_fp8(q8, k8, v8, *, q_scale: float, k_scale: float, v_scale: float,
+                 causal: bool = False, scale: float | None = None, cu_seqlens=None,
+                 max_seqlen: int | None = None, out=None, lse=None):
+    """Prefill on e4m3 codes (gqa_attn_fwd_fp8): q8 [B, Sq, Hq, 128], k8/v8 [B, Sk, Hkv,
+    128] as torch.float8_e4m3fn or uint8 on the GPU (or packed [total, H, 128] with
+    cu_seqlens and max_seqlen); element = value(code) * its tensor's scale.  Returns
+    (out bf16 like q8, lse)."""
+    import torch
+
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+            raise ValueError(f"{name} must hold e4m3 codes (uint8 or float8_e4m3fn)")
+    varlen = cu_seqlens is not None
+    if varlen:
+        if q8.dim() != 3 or k8.dim() != 3 or v8.shape != k8.shape or max_seqlen is None:
+            raise ValueError("packed q8 [total, Hq, D], k8/v8 [total, Hkv, D], max_seqlen")
+        total, Hq, D = q8.shape
+        Hkv = k8.shape[1]
+        B, Sq, Sk = cu_seqlens.numel() - 1, int(max_seqlen), total
+        lse_shape = (Hq, total)
+    else:
+        if q8.dim() != 4 or k8.dim() != 4 or v8.shape != k8.shape:
+            raise ValueError("q8 [B, Sq, Hq, D], k8/v8 [B, Sk, Hkv, D]")
+        B, Sq, Hq, D = q8.shape
+        _, Sk, Hkv, _ = k8.shape
+        lse_shape = (B, Hq, Sq)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out = torch.empty(q8.shape, dtype=torch.bfloat16, device=q8.device) if out is None else out
+    lse = torch.empty(lse_shape, dtype=torch.float32, device=q8.device) if lse is None else lse
+    lib = _capi.load()
+    with torch.cuda.device(q8.device):
+        rc = lib.gqa_attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(out), _ptr(lse), B, Hq,
+                                  Hkv, Sq, Sk, D, scale, float(q_scale), float(k_scale),
+                                  float(v_scale), int(bool(causal)),
+                                  _ptr(cu_seqlens) if varlen else None,
+                                  _stream_handle(torch, q8.device))
+    if rc != 0:
+        raise GqaError("gqa_attn_fwd_fp8", rc)
+    return out, lse
+
+
+class SparseVarlenPlan:
+    """Device metadata of one packed block-sparse problem: each sequence's first
+    pattern row (blk_off) and, when balanced, the tile order with its grid."""
+
+    def __init__(self, blk_off, order, n_order: int, grid: int, rows: int):
+        self.blk_off, self.order, self.n_order, self.grid, self.rows = \
+            blk_off, order, n_order, grid, rows
+
+
+def gqa_attn_blocksparse_varlen_plan(cu_seqlens, blk_row_ptr, *, Hq: int, Hkv: int,
+                                     max_seqlen: int, device, balance: bool = True):
+    """Build a SparseVarlenPlan with the library's host schedule
+    (gqa_attn_sparse_varlen_schedule): cu_seqlens and blk_row_ptr are read on the host
+    once, the plan's arrays live on `device`."""
+    import numpy as np
+    import torch
+
+    lib = _capi.load()
+    cu_h = np.ascontiguousarray(torch.as_tensor(cu_seqlens).cpu().numpy(), dtype=np.int32)
+    rp_h = np.ascontiguousarray(torch.as_tensor(blk_row_ptr).cpu().numpy(), dtype=np.int32)
+    B = cu_h.size - 1
+    off_h = np.zeros(B + 1, dtype=np.int32)
+    n_order, grid = ctypes.c_int(0), ctypes.c_int(0)
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    args = (cu_h.ctypes.data, rp_h.ctypes.data, B, int(Hq), int(Hkv), int(max_seqlen), sms,
+            off_h.ctypes.data)
+    rc = lib.gqa_attn_sparse_varlen_schedule(*args, None, 0, ctypes.byref(n_order),
+                                             ctypes.byref(grid))
+    if rc not in (0, STATUS_CODE["GQA_ERR_WORKSPACE"]):
+        raise GqaError("gqa_attn_sparse_varlen_schedule", rc)
+    order_h = np.zeros(max(n_order.value, 1), dtype=np.int32)
+    rc = lib.gqa_attn_sparse_varlen_schedule(*args, order_h.ctypes.data, order_h.size,
+                                             ctypes.byref(n_order), ctypes.byref(grid))
+    if rc != 0:
+        raise GqaError("gqa_attn_sparse_varlen_schedule", rc)
+    if int(off_h[-1]) + 1 != rp_h.size:
+        raise ValueError(f"blk_row_ptr must hold {int(off_h[-1]) + 1} entries (one row per "
+                         "128-position block of each sequence, plus one)")
+    order = torch.from_numpy(order_h).to(device) if balance else None
+    return SparseVarlenPlan(torch.from_numpy(off_h).to(device), order,
+                            n_order.value if balance else 0, grid.value if balance else 0,
+                            int(off_h[-1]))
+
+
+def gqa_attn_blocksparse_varlen(q, k, v, cu_seqlens, blk_row_ptr, blk_col, *,
+                                max_seqlen: int, plan=None, balance: bool = True,
+                                scale: float | None = None, out=None, lse=None):
+    """Block-sparse attention over packed sequences with minimum padding
+    (gqa_attn_fwd_blocksparse_varlen).
+
+    q [total, Hq, D], k/v [total, Hkv, D] bf16 on the GPU (Hq / Hkv >= 2 dividing 128);
+    cu_seqlens int32 [B + 1] on the GPU; blk_row_ptr / blk_col int32 on the GPU: one
+    pattern row per 128-position block of each sequence in order, col entries counting
+    the sequence's own key blocks.  `plan` (gqa_attn_blocksparse_varlen_plan) is built
+    here when not given; balance=True orders the tiles by the library's host schedule
+    (longest first onto the least loaded CTA).  Returns (out, lse [Hq, total])."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens", cu_seqlens),
+                    ("blk_row_ptr", blk_row_ptr), ("blk_col", blk_col)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype == torch.bfloat16):
+        raise ValueError("q, k, v must be bf16")
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or k.shape[0] != q.shape[0]:
+        raise ValueError("q [total, Hq, D], k/v [total, Hkv, D]")
+    for name, t in (("cu_seqlens", cu_seqlens), ("blk_row_ptr", blk_row_ptr),
+                    ("blk_col", blk_col)):
+        if t.dtype != torch.int32:
+            raise ValueError(f"{name} must be int32")
+    total, Hq, D = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if plan is None:
+        plan = gqa_attn_blocksparse_varlen_plan(cu_seqlens, blk_row_ptr, Hq=Hq, Hkv=Hkv,
+                                                max_seqlen=max_seqlen, device=q.device,
+                                                balance=balance)
+    if plan.rows + 1 != blk_row_ptr.numel():
+        raise ValueError("the plan was built for another pattern")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(Hq, total, dtype=torch.float32, device=q.device) if lse is None else lse
+    lib = _capi.load()
+    with torch.cuda.device(q.device):
+        rc = lib.gqa_attn_fwd_blocksparse_varlen(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
+            _ptr(plan.blk_off), B, Hq, Hkv, int(max_seqlen), total, D, scale,
+            _ptr(blk_row_ptr), _ptr(blk_col), None if plan.order is None else _ptr(plan.order),
+            plan.n_order, plan.grid, _stream_handle(torch, q.device))
+    if rc != 0:
+        raise GqaError("gqa_attn_fwd_blocksparse_varlen", rc)
+    return out, lse
 
 
 def gqa_attn_backward(q, k, v, out, lse, dout, *, causal: bool = False,

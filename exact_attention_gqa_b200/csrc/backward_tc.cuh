@@ -136,6 +136,10 @@ __global__ void __launch_bounds__(BwdTcCfg<HD, DQ, EW>::THREADS, 1)
     constexpr int CW = C::CW;
     constexpr int WP = EW;      // producer warp
     constexpr int WM = EW + 1;  // MMA warp
+    // the elementwise warps confirm block t + 2 has landed before they release block t
+    // (so the MMA thread skips that probe); the producer refills block t + 2's stage
+    // only after block t + 2 - ST is released, which needs ST >= 3
+    static_assert(ST >= 3, "block t + 2 must not wait on block t's release");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -289,7 +293,11 @@ __global__ void __launch_bounds__(BwdTcCfg<HD, DQ, EW>::THREADS, 1)
             for (int t = 0; t <= n; ++t) {
                 if (t < n) {
                     const int s = t % ST;
-                    if (!mbar_wait(bar_full + s, (t / ST) & 1, abort_flag)) goto mma_done;
+                    // blocks 0 and 1 are waited for here; block t >= 2 was confirmed by
+                    // the elementwise warps before they released block t - 2, whose
+                    // release this thread has already observed
+                    if (t < 2 && !mbar_wait(bar_full + s, (t / ST) & 1, abort_flag))
+                        goto mma_done;
                     tc_fence_after();
                     const uint32_t tb = tmem + C::BUF0 + (t & 1) * C::BUF;
                     const uint64_t da = dk0 + uint64_t((s * C::STAGE) >> 4);
@@ -441,6 +449,14 @@ __global__ void __launch_bounds__(BwdTcCfg<HD, DQ, EW>::THREADS, 1)
             }
             tmem_st_cols(tS, pp);
             tmem_st_cols(tS + N, dd);
+            if (t + 2 < n) {  // block t + 2 has landed (see the MMA thread)
+                const int s2 = (t + 2) % ST;
+                if (!mbar_wait_warp(bar_full + s2, ((t + 2) / ST) & 1, abort_flag)) {
+                    tmem_st_wait();
+                    ok = false;
+                    break;
+                }
+            }
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();

@@ -8,6 +8,8 @@
 #include <cstring>
 #include <algorithm>
 #include <mutex>
+#include <queue>
+#include <vector>
 
 #include "gqa_attn.h"
 #include "sm100_ptx.cuh"
@@ -126,6 +128,22 @@ bool make_map_u8(CUtensorMap* m, const void* base, long long rows, int heads, in
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 8-bit [rows, heads, D] view with 128-byte swizzle: boxes of {128 bytes, box_h,
+// box_rows} (e4m3 Q, K, V of the prefill; D = 128 is one swizzle atom)
+bool make_map_u8_sw128(CUtensorMap* m, const void* base, long long rows, int heads, int D,
+                       int box_h, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(heads), cuuint64_t(rows)};
+    cuuint64_t strides[2] = {cuuint64_t(D), cuuint64_t(heads) * D};
+    cuuint32_t box[3] = {128u, cuuint32_t(box_h), cuuint32_t(box_rows)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------- plan
 struct Plan {
     int kernel = kNone;
@@ -204,13 +222,16 @@ size_t ws_bytes(int B, int Hq, int Sq, int D, int n) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-template <int HD>
+template <int HD, bool FP8 = false>
 int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                    int Hq, int Hkv, int Sq, int Sk, float scale, int causal, int pack,
                    const int* cu, int sms, cudaStream_t stream,
-                   const int* blk_row_ptr = nullptr, const int* blk_col = nullptr) {
-    using C = PrefillCfg<HD>;
-    {
+                   const int* blk_row_ptr = nullptr, const int* blk_col = nullptr,
+                   const int* blk_off = nullptr, const int* tile_order = nullptr,
+                   int n_order = 0, int order_grid = 0, float qk_scale = 1.f,
+                   float o_scale = 1.f) {
+    using C = PrefillCfg<HD, FP8>;
+    if constexpr (!FP8) {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD>, HD == 64 ? 1 : 2,
                                          C::SMEM_BYTES);
         if (rc != GQA_OK) return rc;
@@ -248,10 +269,14 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
         if (hg > per_m) hg = per_m;
         p.hu_group = int(hg);
     }
-    p.scale_log2 = scale * kLog2e;
+    p.scale_log2 = scale * qk_scale * kLog2e;  // e4m3: the Q and K code units folded in
+    p.o_scale = o_scale;
     p.blk_row_ptr = blk_row_ptr;
     p.blk_col = blk_col;
     p.n_kblk = (Sk + C::BN - 1) / C::BN;
+    p.blk_off = blk_off;
+    p.tile_order = tile_order;
+    if (tile_order) p.n_units = n_order;  // the balanced order lists every step
     // Row extents of the 3-D views: exactly the rows the caller allocated
     // (packed variable length: Sk carries the packed row count).
     const long long rows_q = cu ? (long long)Sk : (long long)B * Sq;
@@ -259,12 +284,26 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     p.total_rows = cu ? Sk : 0;
     CUtensorMap tq, tk, tv, to;
     // the output leaves through the same box shape as Q arrives in (one sub-tile)
-    if (!make_map(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) ||
-        !make_map(&tk, k, rows_k, Hkv, HD, 1, C::BN) ||
-        !make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN) ||
-        !make_map(&to, out, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128))
+    bool maps_ok;
+    if constexpr (FP8)
+        maps_ok = make_map_u8_sw128(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) &&
+                  make_map_u8_sw128(&tk, k, rows_k, Hkv, HD, 1, C::BN) &&
+                  make_map_u8_sw128(&tv, v, rows_k, Hkv, HD, 1, C::BN);
+    else
+        maps_ok = make_map(&tq, q, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128) &&
+                  make_map(&tk, k, rows_k, Hkv, HD, 1, C::BN) &&
+                  make_map(&tv, v, rows_k, Hkv, HD, 1, C::BN);
+    if (!maps_ok || !make_map(&to, out, rows_q, Hq, HD, pack ? G : 1, pack ? 128 / G : 128))
         return GQA_ERR_CUDA;
-    const int grid = p.n_units < sms ? p.n_units : sms;
+    const int grid = tile_order ? order_grid : (p.n_units < sms ? p.n_units : sms);
+    if constexpr (FP8) {
+        const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD, false, true>, 65536,
+                                         C::SMEM_BYTES);
+        if (rc != GQA_OK) return rc;
+        gqa::prefill_fwd_sm100<HD, false, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
+            tq, tk, tv, to, p);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
     if (blk_row_ptr) {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD, true>, HD == 64 ? 1024 : 2048,
                                          C::SMEM_BYTES);
@@ -374,7 +413,10 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     const long long rows = kv.block_table ? (long long)kv.num_pages * kv.page_size
                                           : (long long)B * Sk;
     const int box = kv.block_table ? (kv.page_size < C::BN ? kv.page_size : C::BN) : C::BN;
-    const bool maps = kv.fp8 ? (make_map_u8(&tk, k, rows, Hkv, HD, box) &&
+    // e4m3 K at D = 128: 128-byte rows with the 128B swizzle (the QK^T fragments are read
+    // straight from the stage); V stays unswizzled for its conversion to f16
+    const bool maps = kv.fp8 ? ((HD == 128 ? make_map_u8_sw128(&tk, k, rows, Hkv, HD, 1, box)
+                                           : make_map_u8(&tk, k, rows, Hkv, HD, box)) &&
                                 make_map_u8(&tv, v, rows, Hkv, HD, box))
                              : (make_map(&tk, k, rows, Hkv, HD, 1, box) &&
                                 make_map(&tv, v, rows, Hkv, HD, 1, box));
@@ -987,6 +1029,133 @@ int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                                           nullptr, dev->sms, stream, blk_row_ptr, blk_col)
                     : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 0, 1,
                                          nullptr, dev->sms, stream, blk_row_ptr, blk_col);
+}
+
+int gqa_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* out, float* lse,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, float q_scale,
+                     float k_scale, float v_scale, int causal, const int* cu_seqlens,
+                     cudaStream_t stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, 1, -1, varlen, false);
+    if (rc != GQA_OK) return rc;
+    if (D != 128) return GQA_ERR_HEADDIM;
+    if (!(std::isfinite(q_scale) && q_scale > 0.f && std::isfinite(k_scale) && k_scale > 0.f &&
+          std::isfinite(v_scale) && v_scale > 0.f))
+        return GQA_ERR_SCALE;
+    if (B == 0 || Sq == 0 || (varlen && Sk == 0)) return GQA_OK;
+    const bool reads_kv = varlen || Sk > 0;
+    if (!q8 || !out || !lse || (reads_kv && (!k8 || !v8))) return GQA_ERR_NULL;
+    if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || (varlen && !aligned(cu_seqlens, 4)))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    if (!varlen && Sk == 0) {
+        gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(out), (long long)B * Sq * Hq * D, lse,
+            (long long)B * Hq * Sq);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
+    Plan pl;
+    make_plan(&pl, B, Hq, Hkv, Sq, Sk, 1, -1, varlen, dev->sms);
+    return launch_prefill<128, true>(q8, k8, v8, out, lse, B, Hq, Hkv, Sq, Sk, scale, causal,
+                                     pl.pack, cu_seqlens, dev->sms, stream, nullptr, nullptr,
+                                     nullptr, nullptr, 0, 0, q_scale * k_scale, v_scale);
+}
+
+int gqa_attn_sparse_varlen_schedule(const int* cu_seqlens, const int* blk_row_ptr, int B,
+                                    int Hq, int Hkv, int max_seqlen, int grid, int* blk_off,
+                                    int* order, int order_cap, int* n_order, int* order_grid) {
+    if (!cu_seqlens || !blk_row_ptr || !blk_off || !n_order || !order_grid || B < 0 ||
+        Hq <= 0 || Hkv <= 0 ||
+        Hq % Hkv != 0 || max_seqlen < 0 || grid <= 0 || order_cap < 0 || (order_cap && !order))
+        return GQA_ERR_NULL;
+    const int G = Hq / Hkv;
+    if (G < 2 || 128 % G != 0) return GQA_ERR_UNSUPPORTED;
+    // minimum padding: sequence b owns ceil(n_b / 128) pattern rows, after the earlier ones
+    blk_off[0] = 0;
+    for (int b = 0; b < B; ++b) {
+        const int n = cu_seqlens[b + 1] - cu_seqlens[b];
+        if (n < 0 || n > max_seqlen) return GQA_ERR_SHAPE;
+        blk_off[b + 1] = blk_off[b] + (n + 127) / 128;
+    }
+    // units (b, kv head, m) as the kernel linearises them; cost = key blocks of the row
+    // times the sub-tiles that hold positions, plus one block for the tile's fixed work
+    const int sub = 128 / G, n_mblk = (max_seqlen + 2 * sub - 1) / (2 * sub);
+    struct Unit { long long cost; int u; };
+    std::vector<Unit> units;
+    for (int b = 0; b < B; ++b) {
+        const int n = cu_seqlens[b + 1] - cu_seqlens[b];
+        for (int m = 0; m < n_mblk; ++m) {
+            const int p0 = m * 2 * sub;
+            if (p0 >= n) break;
+            const int qb = blk_off[b] + p0 / 128;
+            const int row = blk_row_ptr[qb + 1] - blk_row_ptr[qb];
+            if (row < 0) return GQA_ERR_SHAPE;
+            const int subs = 1 + (p0 + sub < n ? 1 : 0);
+            for (int h = 0; h < Hkv; ++h)
+                units.push_back({(long long)row * subs + 1, (b * Hkv + h) * n_mblk + m});
+        }
+    }
+    // longest processing time first: each unit goes to the CTA with the least work so far
+    std::stable_sort(units.begin(), units.end(),
+                     [](const Unit& a, const Unit& c) { return a.cost > c.cost; });
+    const int g = (int)std::min<size_t>((size_t)grid, std::max<size_t>(units.size(), 1));
+    std::vector<std::vector<int>> lists(g);
+    using Load = std::pair<long long, int>;
+    std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+    for (int c = 0; c < g; ++c) heap.push({0, c});
+    for (const Unit& x : units) {
+        Load top = heap.top();
+        heap.pop();
+        lists[top.second].push_back(x.u);
+        heap.push({top.first + x.cost, top.second});
+    }
+    size_t depth = 0;
+    for (const auto& l : lists) depth = std::max(depth, l.size());
+    const long long need = (long long)g * (long long)depth;
+    if (need > INT32_MAX) return GQA_ERR_SHAPE;
+    *n_order = (int)need;
+    *order_grid = g;
+    if (need > order_cap) return GQA_ERR_WORKSPACE;  // *n_order says how many entries
+    // CTA c takes steps c, c + g, c + 2 g, ... of the persistent loop
+    for (size_t k = 0; k < depth; ++k)
+        for (int c = 0; c < g; ++c)
+            order[k * g + c] = k < lists[c].size() ? lists[c][k] : -1;
+    return GQA_OK;
+}
+
+int gqa_attn_fwd_blocksparse_varlen(const void* q, const void* k, const void* v, void* out,
+                                    float* lse, const int* cu_seqlens, const int* blk_off,
+                                    int B, int Hq, int Hkv, int max_seqlen, int total, int D,
+                                    float scale, const int* blk_row_ptr, const int* blk_col,
+                                    const int* tile_order, int n_order, int order_grid,
+                                    cudaStream_t stream) {
+    int rc = check_shape(B, Hq, Hkv, max_seqlen, total, D, scale, 1, 1, true, false);
+    if (rc != GQA_OK) return rc;
+    const int G = Hq / Hkv;
+    if (G < 2 || 128 % G != 0) return GQA_ERR_UNSUPPORTED;
+    if (B == 0 || max_seqlen == 0 || total == 0) return GQA_OK;
+    if (!q || !k || !v || !out || !lse || !cu_seqlens || !blk_off || !blk_row_ptr || !blk_col)
+        return GQA_ERR_NULL;
+    if (tile_order && (n_order <= 0 || order_grid <= 0 || n_order % order_grid != 0))
+        return GQA_ERR_SHAPE;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || !aligned(blk_row_ptr, 4) || !aligned(blk_col, 4) ||
+        !aligned(cu_seqlens, 4) || !aligned(blk_off, 4) || !aligned(tile_order, 4))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, max_seqlen, total,
+                                          scale, 0, 1, cu_seqlens, dev->sms, stream,
+                                          blk_row_ptr, blk_col, blk_off, tile_order, n_order,
+                                          order_grid)
+                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, max_seqlen, total,
+                                         scale, 0, 1, cu_seqlens, dev->sms, stream,
+                                         blk_row_ptr, blk_col, blk_off, tile_order, n_order,
+                                         order_grid);
 }
 
 int gqa_attn_decode_kvcache(const void* q, const void* k_cache, const void* v_cache,

@@ -71,28 +71,42 @@ struct PrefillParams {
     const int* blk_row_ptr = nullptr;  // [ceil(Sq / 128) + 1]
     const int* blk_col = nullptr;      // [nnz], ascending within a row
     int n_kblk = 0;                    // ceil(Sk / 128): key blocks that exist
+    // block-sparse over packed sequences (minimum padding): first pattern row of each
+    // sequence, [B + 1] (prefix sum of ceil(n_b / 128)); nullptr: one dense pattern
+    const int* blk_off = nullptr;
+    // optional tile order (attention balancing): entry t is the unit the persistent
+    // loop's t-th step takes, as (b * n_hu + hu) * n_mblk + m, or -1 for no tile
+    const int* tile_order = nullptr;
+    // e4m3 Q/K/V: O = accumulator * o_scale / l (v_scale over P's range shift)
+    float o_scale = 1.f;
 };
 
-template <int HD>
+template <int HD, bool FP8 = false>
 struct PrefillCfg {
+    // FP8: Q, K, V are e4m3 (one byte per element); D = 128 only
+    static_assert(!FP8 || HD == 128, "e4m3 prefill: D = 128");
+    static constexpr int ES = FP8 ? 1 : 2;        // bytes per input element
     static constexpr int BM = 128;                // rows per sub-tile
     static constexpr int BN = 128;                // keys per K/V block
-    static constexpr int ATOMS = HD / 64;         // 128-byte swizzle atoms along D
+    static constexpr int ATOMS = HD * ES / 128;   // 128-byte swizzle atoms along D
+    static constexpr int ATOM_ELEMS = 128 / ES;   // elements of D per atom
     static constexpr int ATOM_Q = BM * 128;       // bytes of one Q atom
     static constexpr int ATOM_KV = BN * 128;      // bytes of one K or V atom
-    static constexpr int Q_SUB = BM * HD * 2;     // bytes of one Q sub-tile
+    static constexpr int Q_SUB = BM * HD * ES;    // bytes of one Q sub-tile
     static constexpr int Q_TILE = 2 * Q_SUB;      // both sub-tiles
-    static constexpr int KV_TILE = BN * HD * 2;   // bytes of one K or V block
-    static constexpr int STAGES = (HD == 128) ? 2 : 4;
+    static constexpr int KV_TILE = BN * HD * ES;  // bytes of one K or V block
+    static constexpr int STAGES = (HD == 128) ? (FP8 ? 4 : 2) : 4;
     static constexpr int Q_STAGES = (HD == 128) ? 1 : 2;
+    // MMA K-step: 32 bytes of the reduction dimension (16 bf16 or 32 e4m3 elements)
+    static constexpr int KSTEP = 32 / ES;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_STAGES * Q_TILE;
     static constexpr int OFF_V = OFF_K + STAGES * KV_TILE;
     // D = 64: full sub-tiles of O leave through a shared-memory box and one TMA store
     // (128B-swizzled rows, the same box as Q's); D = 128 has no room and stores rows.
-    static constexpr bool EPI_TMA = (HD == 64);
+    static constexpr bool EPI_TMA = (HD == 64) && !FP8;
     static constexpr int OFF_O = OFF_V + STAGES * KV_TILE;
-    static constexpr int O_SUB = BM * HD * 2;
+    static constexpr int O_SUB = BM * HD * 2;  // bf16 output
     static constexpr int OFF_BAR = OFF_O + (EPI_TMA ? 2 * O_SUB : 0);
     static constexpr int NUM_BARS = 2 * Q_STAGES + 4 * STAGES + 6 + 1 + 4;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -106,7 +120,11 @@ struct PrefillCfg {
     __device__ static constexpr uint32_t p_col(int i) {
         return P_OWN ? 384u + uint32_t(i) * 64u : s_col(i);
     }
-    static constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+    // e4m3 P: the running max moves when a block's max exceeds it by more than a factor
+    // 2, and P carries a factor 2^7 (folded into the exponent), so P <= 256 < 448 (the
+    // largest e4m3 value) while small probabilities keep 7 more bits of range
+    static constexpr float RESCALE_THRESHOLD = FP8 ? 1.0f : 8.0f;  // log2 units
+    static constexpr float P_SHIFT = FP8 ? 7.0f : 0.0f;            // log2 units
 };
 
 struct TileInfo {
@@ -123,7 +141,15 @@ struct TileInfo {
 template <int BN, bool SPARSE = false>
 __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
     TileInfo ti;
-    if (p.kv_major) {
+    bool none = false;
+    if constexpr (SPARSE) {
+        if (p.tile_order) {  // balanced order: unit index in the (b, hu, m) linearisation
+            const int u = __ldg(p.tile_order + t);
+            none = u < 0;
+            t = none ? 0 : u;
+        }
+    }
+    if (p.kv_major || (SPARSE && p.tile_order)) {
         const int bh = t / p.n_mblk;
         ti.m = t - bh * p.n_mblk;
         ti.b = bh / p.n_hu;
@@ -175,9 +201,15 @@ __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
     }
     ti.kb0 = 0;
     if constexpr (SPARSE) {
-        // both sub-tiles lie in query block qb and share its list of key blocks
-        const int qb = (ti.m * 2 * p.sub_pos) >> 7;
-        const int r0 = __ldg(p.blk_row_ptr + qb), r1 = __ldg(p.blk_row_ptr + qb + 1);
+        // both sub-tiles lie in query block qb (of this sequence) and share its list of
+        // key blocks; packed sequences start at their own first pattern row
+        const int qb = ((ti.m * 2 * p.sub_pos) >> 7) + (p.blk_off ? __ldg(p.blk_off + ti.b) : 0);
+        // an empty slot of the balanced order is no tile at all: no role may touch the
+        // unit it decoded to (the softmax warps key their epilogue on `valid`)
+        if (none) ti.valid[0] = ti.valid[1] = 0;
+        const bool any = ti.valid[0] || ti.valid[1];
+        const int r0 = any ? __ldg(p.blk_row_ptr + qb) : 0;
+        const int r1 = any ? __ldg(p.blk_row_ptr + qb + 1) : 0;
         ti.kb0 = r0;
 #pragma unroll
         for (int i = 0; i < 2; ++i) ti.nblk[i] = ti.valid[i] ? max(r1 - r0, 0) : 0;
@@ -191,7 +223,7 @@ template <bool SPARSE>
 __device__ __forceinline__ int sparse_block(const PrefillParams& p, const TileInfo& ti, int j) {
     if constexpr (!SPARSE) return j;
     int kb = __ldg(p.blk_col + ti.kb0 + j);
-    if (kb < 0 || kb >= p.n_kblk) {
+    if (kb < 0 || kb >= (ti.sk + 127) >> 7) {  // key blocks of this sequence
         raise_device_error(kDevBadTile);
         kb = 0;
     }
@@ -211,13 +243,13 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 // SPARSE = true walks the block pattern of p.blk_row_ptr / p.blk_col; the dense
 // instantiation carries none of that code.
-template <int HD, bool SPARSE = false>
+template <int HD, bool SPARSE = false, bool FP8 = false>
 __global__ void __launch_bounds__(320, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
-    using C = PrefillCfg<HD>;
+    using C = PrefillCfg<HD, FP8>;
     constexpr int BN = C::BN;
     constexpr int ST = C::STAGES;
     constexpr int QS = C::Q_STAGES;
@@ -303,7 +335,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                     for (int a = 0; a < C::ATOMS; ++a)
                         tma_load_3d(sQ + qs * C::Q_TILE + i * C::Q_SUB + a * C::ATOM_Q, &tm_q,
-                                    bar_q_full + qs, a * 64, y, z);
+                                    bar_q_full + qs, a * C::ATOM_ELEMS, y, z);
                 }
                 ++qc;
                 const int kvh = p.pack ? ti.hu : ti.hu / p.G;
@@ -317,7 +349,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                         for (int a = 0; a < C::ATOMS; ++a)
                             tma_load_3d(sK + s * C::KV_TILE + a * C::ATOM_KV, &tm_k,
-                                        bar_k_full + s, a * 64, kvh, z);
+                                        bar_k_full + s, a * C::ATOM_ELEMS, kvh, z);
                         ++kc;
                     }
                     {
@@ -328,7 +360,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                         for (int a = 0; a < C::ATOMS; ++a)
                             tma_load_3d(sV + s * C::KV_TILE + a * C::ATOM_KV, &tm_v,
-                                        bar_v_full + s, a * 64, kvh, z);
+                                        bar_v_full + s, a * C::ATOM_ELEMS, kvh, z);
                         ++vc;
                     }
                 }
@@ -349,8 +381,10 @@ __global__ void __launch_bounds__(320, 1)
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, 0, 0);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, 0, 1);
+            constexpr uint32_t idesc_s =
+                FP8 ? idesc_e4m3_f32(128, BN, 0, 0) : idesc_bf16_f32(128, BN, 0, 0);
+            constexpr uint32_t idesc_o =
+                FP8 ? idesc_e4m3_f32(128, HD, 0, 1) : idesc_bf16_f32(128, HD, 0, 1);
             const uint32_t sQ0 = smem_u32(smem + C::OFF_Q);
             const uint32_t sK = smem_u32(smem + C::OFF_K);
             const uint32_t sV = smem_u32(smem + C::OFF_V);
@@ -361,17 +395,24 @@ __global__ void __launch_bounds__(320, 1)
             const uint64_t dq0 = sw128_desc(sQ0, 16, 1024);
             const uint64_t dk0 = sw128_desc(sK, 16, 1024);
             const uint64_t dv0 = sw128_desc(sV, C::ATOM_KV, 1024);
-            constexpr int NS = HD / 16;   // k-steps of S = Q K^T
-            constexpr int NPV = BN / 16;  // k-steps of O += P V
+            constexpr int NS = HD / C::KSTEP;   // k-steps of S = Q K^T (32 bytes each)
+            constexpr int NPV = BN / C::KSTEP;  // k-steps of O += P V
             auto s_step = [&](uint64_t dq, uint64_t dk, int i, int kk) {
                 const uint32_t oq = ((kk >> 2) * C::ATOM_Q + (kk & 3) * 32) >> 4;
                 const uint32_t ok = ((kk >> 2) * C::ATOM_KV + (kk & 3) * 32) >> 4;
-                umma_ss(tmem + C::s_col(i), dq + oq, dk + ok, idesc_s, kk > 0 ? 1u : 0u);
+                if constexpr (FP8)
+                    umma_ss_f8(tmem + C::s_col(i), dq + oq, dk + ok, idesc_s, kk > 0 ? 1u : 0u);
+                else
+                    umma_ss(tmem + C::s_col(i), dq + oq, dk + ok, idesc_s, kk > 0 ? 1u : 0u);
             };
+            // P: 32 bytes of keys per k-step are 8 TMEM columns in either precision
             auto pv_step = [&](uint64_t dv, int i, int kk, bool accumulate) {
-                umma_ts(tmem + C::o_col(i), tmem + C::p_col(i) + kk * 8,
-                        dv + uint64_t((kk * 16 * 128) >> 4), idesc_o,
-                        (accumulate || kk > 0) ? 1u : 0u);
+                const uint64_t b = dv + uint64_t((kk * C::KSTEP * 128) >> 4);
+                const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
+                if constexpr (FP8)
+                    umma_ts_f8(tmem + C::o_col(i), tmem + C::p_col(i) + kk * 8, b, idesc_o, acc);
+                else
+                    umma_ts(tmem + C::o_col(i), tmem + C::p_col(i) + kk * 8, b, idesc_o, acc);
             };
             for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
                 const TileInfo ti = decode_tile<BN, SPARSE>(p, t);
@@ -540,7 +581,8 @@ __global__ void __launch_bounds__(320, 1)
                     m_run = mb;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                const uint64_t negm2 = f2_pack(-m_use, -m_use);
+                // FP8: p carries 2^P_SHIFT (cancels between O and l; L removes it)
+                const uint64_t negm2 = f2_pack(C::P_SHIFT - m_use, C::P_SHIFT - m_use);
                 // p = 2^(s*scale*log2e - m); two row sums in fp32: of the exact p (for L)
                 // and of the bf16 p the P.V MMA consumes (for O / l).  The second sum
                 // takes the bf16 halves either unpacked into paired adds (D = 64) or
@@ -550,6 +592,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t pk[16];
+                    float pprev0 = 0.f, pprev1 = 0.f;  // FP8: the pair before this one
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
                         const uint64_t a = ffma2(f2_pack(__uint_as_float(sr[c][2 * e]),
@@ -559,12 +602,19 @@ __global__ void __launch_bounds__(320, 1)
                         f2_unpack(a, a0, a1);
                         const float p0 = ex2_approx(a0);
                         const float p1 = ex2_approx(a1);
-                        pk[e] = pack_bf16x2(p0, p1);
                         const uint64_t pe = f2_pack(p0, p1);
                         if (e & 1)
                             se1 = fadd2(se1, pe);
                         else
                             se0 = fadd2(se0, pe);
+                        if constexpr (FP8) {
+                            // four keys per 32-bit column, key order = byte order
+                            if (e & 1) pk[e >> 1] = pack_e4m3x4(pprev0, pprev1, p0, p1);
+                            pprev0 = p0;
+                            pprev1 = p1;
+                            continue;
+                        }
+                        pk[e] = pack_bf16x2(p0, p1);
                         if constexpr (HD == 128) {
                             if (e & 1)
                                 add_bf16x2_to_f32(pk[e], rq2, rq3);
@@ -578,10 +628,15 @@ __global__ void __launch_bounds__(320, 1)
                                 sq0 = fadd2(sq0, pr);
                         }
                     }
+                    if constexpr (FP8) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) sr[c >> 1][(c & 1) * 16 + e] = pk[e];
+                        for (int e = 0; e < 8; ++e) sr[0][c * 8 + e] = pk[e];
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) sr[c >> 1][(c & 1) * 16 + e] = pk[e];
+                    }
                 }
-                if constexpr (HD == 128) sq0 = f2_pack(rq0 + rq2, rq1 + rq3);
+                if constexpr (HD == 128 && !FP8) sq0 = f2_pack(rq0 + rq2, rq1 + rq3);
                 // P.V(j-1) has finished: it no longer reads P's columns and O holds
                 // every block before j (needed before P is overwritten or O rescaled)
                 if (j > 0) {
@@ -589,16 +644,18 @@ __global__ void __launch_bounds__(320, 1)
                     o_phase ^= 1;
                     tc_fence_after();
                 }
-                // P (bf16 pairs): its own 64 columns, or the first 64 columns of S
+                // P (bf16 pairs: 64 columns, its own or the first 64 of S; e4m3 quads: the
+                // first 32 columns of S)
                 tmem_st32(tP, sr[0]);
-                tmem_st32(tP + 32, sr[1]);
+                if constexpr (!FP8) tmem_st32(tP + 32, sr[1]);
                 float lsum, lrnd;
                 {
                     float x0, x1, y0, y1;
                     f2_unpack(fadd2(se0, se1), x0, x1);
                     f2_unpack(fadd2(sq0, sq1), y0, y1);
                     lsum = x0 + x1;
-                    lrnd = y0 + y1;
+                    // FP8: O is normalised by the sum of the unrounded p
+                    lrnd = FP8 ? lsum : y0 + y1;
                 }
                 l_run = l_run * alpha + lsum;
                 l_rnd = l_rnd * alpha + lrnd;
@@ -635,7 +692,8 @@ __global__ void __launch_bounds__(320, 1)
                     o_phase ^= 1;
                     tc_fence_after();
                 }
-                const float inv_l = (l_rnd > 0.f) ? 1.f / l_rnd : 0.f;
+                // FP8: o_scale = v_scale (the V codes' unit)
+                const float inv_l = (l_rnd > 0.f) ? (FP8 ? p.o_scale : 1.f) / l_rnd : 0.f;
                 // a sub-tile whose 128 rows are all real leaves through one TMA store
                 const bool tma_out = C::EPI_TMA && (my_p0 + p.sub_pos <= ti.sq);
                 if constexpr (C::EPI_TMA) {
@@ -712,8 +770,10 @@ __global__ void __launch_bounds__(320, 1)
                     }
                 }
                 if (row_valid) {
-                    const float L = (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f
-                                                  : -INFINITY;
+                    const float L = (l_run > 0.f)
+                                        ? (m_run - C::P_SHIFT + __log2f(l_run)) *
+                                              0.69314718055994531f
+                                        : -INFINITY;
                     size_t li;
                     if (p.cu_seqlens)
                         li = size_t(head) * p.total_rows + ti.q_row0 + pos;

@@ -267,6 +267,65 @@ int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                              const int* blk_row_ptr, const int* blk_col, cudaStream_t stream);
 
 /*
+ * Prefill forward on e4m3 Q, K and V with one scale per tensor (the batch-size guide
+ * names FP8 as the precision that lowers memory-bandwidth pressure: hardware adaptation
+ * section, Hopper item; precision row of its production checklist).
+ *   element = value(code) * scale of its tensor; q8 [B, Sq, Hq, D], k8/v8 [B, Sk, Hkv,
+ *   D] bytes (or packed [total, H, D] with cu_seqlens as gqa_attn_fwd); D = 128;
+ *   out bf16 like q, lse fp32 as gqa_attn_fwd; causal as gqa_attn_fwd.
+ * S = Q K^T and O += P V run as 8-bit tensor-core products (kind::f8f6f4, fp32
+ * accumulation); P is rounded to e4m3 (relative to the running row max, times 2^7),
+ * O is normalised by the sum of the unrounded p.  Codes 0x7f / 0xff (NaN) are not
+ * supported.  Errors as gqa_attn_fwd, plus GQA_ERR_SCALE for a scale that is not
+ * finite and positive.
+ */
+int gqa_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* out, float* lse,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, float q_scale,
+                     float k_scale, float v_scale, int causal, const int* cu_seqlens,
+                     cudaStream_t stream);
+
+/*
+ * Block-sparse attention over packed variable-length sequences with minimum padding
+ * (Raptor-T abstract: BigBird's block-sparse attention; the minimum-padding algorithm
+ * pads each sequence only to whole blocks instead of to the longest sequence; the
+ * attention-balancing algorithm assigns thread-block work by its execution time).
+ *   q, out [total, Hq, D], k, v [total, Hkv, D] bf16 packed as gqa_attn_fwd's varlen
+ *   form; lse [Hq, total]; cu_seqlens device int32 [B + 1]; self attention within each
+ *   sequence, non-causal;
+ *   sequence b owns ceil(n_b / 128) query and key blocks (the last one partial);
+ *   blk_off device int32 [B + 1]: its first pattern row, the prefix sum of those counts;
+ *   blk_row_ptr device int32 [blk_off[B] + 1], blk_col device int32: the CSR pattern,
+ *   rows in sequence order, col entries counting the sequence's own key blocks (an
+ *   entry outside them raises device error 2 and block 0 is read in its place);
+ *   tile_order (optional, device int32 [n_order], n_order a multiple of order_grid):
+ *   the tile each step of the persistent grid of order_grid CTAs takes, as written by
+ *   gqa_attn_sparse_varlen_schedule; nullptr: the varlen longest-first order.
+ * PackGQA always; G = Hq / Hkv >= 2 dividing 128 (GQA_ERR_UNSUPPORTED otherwise); D 64
+ * or 128; errors as gqa_attn_fwd.
+ */
+int gqa_attn_fwd_blocksparse_varlen(const void* q, const void* k, const void* v, void* out,
+                                    float* lse, const int* cu_seqlens, const int* blk_off,
+                                    int B, int Hq, int Hkv, int max_seqlen, int total, int D,
+                                    float scale, const int* blk_row_ptr, const int* blk_col,
+                                    const int* tile_order, int n_order, int order_grid,
+                                    cudaStream_t stream);
+
+/*
+ * Host-side schedule for gqa_attn_fwd_blocksparse_varlen (no device work).  From host
+ * copies of cu_seqlens [B + 1] and blk_row_ptr, writes blk_off [B + 1] (host) and the
+ * tile order: every (sequence, KV head, position tile) with a cost of its row's key
+ * blocks times its occupied sub-tiles plus one, assigned longest first to the least
+ * loaded of `grid` CTAs (grid is capped at the number of tiles); CTA c's k-th tile goes
+ * to order[k * g + c], unused slots -1.  *order_grid receives g (grid capped at the
+ * number of tiles: the launch's order_grid) and *n_order the entries needed (g times
+ * the longest list); GQA_ERR_WORKSPACE if order_cap is smaller (call with
+ * order_cap = 0 to size it).
+ */
+int gqa_attn_sparse_varlen_schedule(const int* cu_seqlens, const int* blk_row_ptr, int B,
+                                    int Hq, int Hkv, int max_seqlen, int grid, int* blk_off,
+                                    int* order, int order_cap, int* n_order, int* order_grid);
+
+/*
  * Decode (one new query position per sequence) against a KV cache, with per-
  * sequence cache lengths and an optional sliding window.  Ultralytics glossary
  * "Grouped Query Attention (GQA)": during generation the model keeps the keys and

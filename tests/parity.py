@@ -7,6 +7,9 @@ output element whose reference magnitude is so large that one bf16 ulp exceeds
 can use half of it.  fp32 path: max |dO| <= 1e-4, max |dL| <= 1e-4.
 Rows with no visible key must give exactly O = 0 and L = -inf.
 
+e4m3 prefill (P rounded to e4m3 before P V): O within the larger of the bf16 bar and
+1.5 x the distance of a rounding model of that arithmetic from the oracle; L as bf16.
+
 Backward (bf16 gradients, P and dS rounded to bf16 before their products, outputs
 rounded to bf16: each about 2^-9 relative): the forward's bar scaled by the
 gradient's magnitude, max |d| <= 1e-2 * max(1, max |ref|) and
@@ -123,3 +126,54 @@ def compare_grad(g_gpu, ref, model=None):
     assert stats["max_abs"] <= max_bar, stats
     assert stats["mean_abs"] <= mean_bar, stats
     return stats
+
+
+def e4m3_prefill_model(q8, k8, v8, q_scale, k_scale, v_scale, scale, causal):
+    """Rounding model of the e4m3 prefill, for the tolerance only: exact products of the
+    decoded codes, p relative to the row max times 2^7 rounded to e4m3 (nearest even),
+    O normalised by the sum of the unrounded p and rounded to bf16.  Dense layouts;
+    returns O float64 like q8."""
+    import torch
+    f8 = torch.float8_e4m3fn
+
+    def dec(t, sc):
+        t = t.detach().cpu()
+        return (t.view(f8) if t.dtype == torch.uint8 else t).to(torch.float64) * sc
+
+    q, k, v = dec(q8, q_scale), dec(k8, k_scale), dec(v8, v_scale)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    qt = q.permute(0, 2, 1, 3)
+    kt = k.permute(0, 2, 1, 3).repeat_interleave(G, dim=1)
+    vt = v.permute(0, 2, 1, 3).repeat_interleave(G, dim=1)
+    s2 = (qt @ kt.transpose(-1, -2)) * (scale * 1.4426950408889634)
+    if causal:
+        vis = torch.ones(Sq, Sk, dtype=torch.bool).tril(diagonal=Sk - Sq)
+        s2 = s2.masked_fill(~vis, float("-inf"))
+    m = s2.amax(-1, keepdim=True)
+    p = torch.exp2(s2 - m + 7.0).nan_to_num(0.0)
+    p8 = p.float().to(f8).to(torch.float64)
+    l = p.sum(-1, keepdim=True)
+    o = torch.where(l > 0, (p8 @ vt) / l.clamp_min(1e-300), torch.zeros_like(qt))
+    return o.to(torch.bfloat16).to(torch.float64).permute(0, 2, 1, 3).numpy()
+
+
+def compare_e4m3(o_gpu, lse_gpu, o_ref, lse_ref, model):
+    """The e4m3 prefill bar: O within max(fixed bar, 1.5 x the rounding model's own
+    distance from the oracle), max and mean; L as the bf16 bar (L uses exact sums)."""
+    o = to_np(o_gpu)
+    lse = to_np(lse_gpu)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    lse_ref = np.asarray(lse_ref, dtype=np.float64)
+    merr = np.abs(np.asarray(model, dtype=np.float64) - o_ref)
+    err = np.abs(o - o_ref)
+    max_bar = max(BF16_MAX_ABS, GRAD_MODEL_FACTOR * float(merr.max()))
+    mean_bar = max(BF16_MEAN_ABS, GRAD_MODEL_FACTOR * float(merr.mean()))
+    assert float(err.max()) <= max_bar, (float(err.max()), max_bar)
+    assert float(err.mean()) <= mean_bar, (float(err.mean()), mean_bar)
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isneginf(lse), np.isneginf(lse_ref))
+    assert float(np.abs(lse[fin] - lse_ref[fin]).max(initial=0.0)) <= BF16_MAX_LSE
+    return {"max_abs": float(err.max()), "mean_abs": float(err.mean()), "max_bar": max_bar,
+            "mean_bar": mean_bar}

@@ -314,3 +314,123 @@ def test_backward_front_end_checks_shapes_first():
         G.gqa_attn_backward(q, k[..., :32], k[..., :32], q, lse, q)
     with pytest.raises(ValueError, match="CUDA tensor"):
         G.gqa_attn_backward(q, k, k, q, lse, q)
+
+
+# ---------------------------------------------------------------- varlen block-sparse
+def schedule(lib, lens, rows_per_block, Hq=8, Hkv=2, grid=148):
+    """Run the host schedule; rows_per_block(b, r) gives the row length of block r of
+    sequence b.  Returns (status, blk_off, order, g)."""
+    import numpy as np
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    nblk = [-(-n // 128) for n in lens]
+    rp = [0]
+    for b, nb in enumerate(nblk):
+        for r in range(nb):
+            rp.append(rp[-1] + rows_per_block(b, r))
+    rp = np.array(rp, dtype=np.int32)
+    off = np.zeros(len(lens) + 1, dtype=np.int32)
+    n, g = ctypes.c_int(0), ctypes.c_int(0)
+    args = (cu.ctypes.data, rp.ctypes.data, len(lens), Hq, Hkv, max(lens), grid, off.ctypes.data)
+    rc = lib.gqa_attn_sparse_varlen_schedule(*args, None, 0, ctypes.byref(n), ctypes.byref(g))
+    if rc not in (0, G.STATUS_CODE["GQA_ERR_WORKSPACE"]):
+        return rc, None, None, None
+    order = np.zeros(max(n.value, 1), dtype=np.int32)
+    rc = lib.gqa_attn_sparse_varlen_schedule(*args, order.ctypes.data, order.size,
+                                             ctypes.byref(n), ctypes.byref(g))
+    return rc, off, order[:n.value], g.value
+
+
+def test_schedule_lists_every_tile_once_with_minimum_padding(lib):
+    import numpy as np
+    lens = [300, 0, 128, 1000, 17, 4096]
+    Hq, Hkv = 8, 2
+    rc, off, order, g = schedule(lib, lens, lambda b, r: 1 + (b + r) % 5, Hq, Hkv)
+    assert rc == 0
+    assert off.tolist() == [0, 3, 3, 4, 12, 13, 45]  # ceil(n / 128) rows per sequence
+    sub = 128 // (Hq // Hkv)
+    n_mblk = -(-max(lens) // (2 * sub))
+    want = sorted((b * Hkv + h) * n_mblk + m for b, n in enumerate(lens)
+                  for m in range(-(-n // (2 * sub))) for h in range(Hkv))
+    assert sorted(order[order >= 0].tolist()) == want
+    assert len(order) % g == 0 and g == min(148, len(want))
+
+
+def test_schedule_balances_the_cost(lib):
+    import numpy as np
+    lens = [8192, 128, 4000, 2000, 640] * 4
+    Hq, Hkv, grid = 8, 2, 16
+    cost_of = lambda b, r: 40 if r < 2 else 6  # global rows are long, the rest short
+    rc, off, order, g = schedule(lib, lens, cost_of, Hq, Hkv, grid)
+    assert rc == 0 and g == grid
+    sub = 128 // (Hq // Hkv)
+    n_mblk = -(-max(lens) // (2 * sub))
+    loads = np.zeros(g)
+    for idx, u in enumerate(order.tolist()):
+        if u < 0:
+            continue
+        m = u % n_mblk
+        b = (u // n_mblk) // Hkv
+        p0 = m * 2 * sub
+        subs = 1 + (p0 + sub < lens[b])
+        loads[idx % g] += cost_of(b, p0 // 128) * subs + 1
+    # longest-first onto the least loaded CTA: no CTA exceeds another by more than the
+    # largest single tile
+    assert loads.max() - loads.min() <= 40 * 2 + 1
+
+
+def test_schedule_argument_errors(lib):
+    rc, *_ = schedule(lib, [100, 50], lambda b, r: 1, Hq=8, Hkv=8)  # G = 1
+    assert G.STATUS[rc] == "GQA_ERR_UNSUPPORTED"
+    import numpy as np
+    cu = np.array([0, 300], dtype=np.int32)
+    rp = np.array([0, 1, 2, 3], dtype=np.int32)
+    off = np.zeros(2, dtype=np.int32)
+    n, g = ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib.gqa_attn_sparse_varlen_schedule(cu.ctypes.data, rp.ctypes.data, 1, 8, 2, 200, 148,
+                                             off.ctypes.data, None, 0, ctypes.byref(n),
+                                             ctypes.byref(g))
+    assert G.STATUS[rc] == "GQA_ERR_SHAPE"  # a sequence longer than max_seqlen
+
+
+def test_blocksparse_varlen_argument_errors(lib):
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, cu=FAKE, off=FAKE, B=2, Hq=8,
+                 Hkv=2, S=256, total=300, D=128, scale=0.125, rp=FAKE, col=FAKE, order=None,
+                 n_order=0, grid=0)
+        a.update(kw)
+        return G.STATUS[lib.gqa_attn_fwd_blocksparse_varlen(
+            a["q"], a["k"], a["v"], a["out"], a["lse"], a["cu"], a["off"], a["B"], a["Hq"],
+            a["Hkv"], a["S"], a["total"], a["D"], a["scale"], a["rp"], a["col"], a["order"],
+            a["n_order"], a["grid"], None)]
+    assert call(Hq=8, Hkv=8) == "GQA_ERR_UNSUPPORTED"
+    assert call(off=None) == "GQA_ERR_NULL"
+    assert call(D=96) == "GQA_ERR_HEADDIM"
+    assert call(order=FAKE, n_order=10, grid=3) == "GQA_ERR_SHAPE"
+    assert call(cu=ctypes.c_void_p(0x1002)) == "GQA_ERR_ALIGN"
+    assert call(B=0) == "GQA_OK"
+
+
+# ---------------------------------------------------------------- e4m3 prefill
+def fp8_prefill_call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=8, Hkv=2, Sq=256,
+             Sk=256, D=128, scale=0.125, qs=1.0, ks=1.0, vs=1.0, causal=1, cu=None):
+    return lib.gqa_attn_fwd_fp8(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, qs, ks, vs,
+                                causal, cu, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(D=64), "GQA_ERR_HEADDIM"),
+    (dict(qs=0.0), "GQA_ERR_SCALE"),
+    (dict(vs=float("inf")), "GQA_ERR_SCALE"),
+    (dict(scale=-1.0), "GQA_ERR_SCALE"),
+    (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
+    (dict(q=None), "GQA_ERR_NULL"),
+    (dict(v=None), "GQA_ERR_NULL"),
+    (dict(k=ctypes.c_void_p(0x1004)), "GQA_ERR_ALIGN"),
+])
+def test_fp8_prefill_argument_errors(lib, kw, code):
+    assert G.STATUS[fp8_prefill_call(lib, **kw)] == code
+
+
+def test_fp8_prefill_empty_problems_are_noops(lib):
+    assert fp8_prefill_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert fp8_prefill_call(lib, Sq=0, q=None, k=None, v=None, out=None, lse=None) == 0

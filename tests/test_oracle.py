@@ -798,6 +798,20 @@ def test_bf16_backward_model_tracks_the_oracle():
         assert err.mean() <= 2e-3 * max(1.0, np.abs(r).mean())
 
 
+def test_e4m3_prefill_model_tracks_the_oracle():
+    # the tolerance model of the e4m3 prefill: P rounded to e4m3 costs a few percent of
+    # O, not more; without that rounding (p kept exact) it equals the oracle
+    from parity import e4m3_prefill_model
+    q8, k8, v8 = e4m3_tensors((1, 64, 4, 128), 110), e4m3_tensors((1, 80, 2, 128), 111), \
+        e4m3_tensors((1, 80, 2, 128), 112)
+    o, _ = oracle.attention_e4m3(q8, k8, v8, q_scale=0.5, k_scale=0.25, v_scale=2.0,
+                                 scale=0.088, causal=True)
+    m = e4m3_prefill_model(q8, k8, v8, 0.5, 0.25, 2.0, 0.088, True)
+    err = np.abs(m - o)
+    assert 0 < err.mean() <= 0.05 * np.abs(o).mean()
+    assert err.max() <= 0.1 * np.abs(o).max()
+
+
 # ---------------------------------------------------------------------------------
 # Pin strength: every planted mistake is caught by at least one pin above
 

@@ -46,6 +46,7 @@ class Workload:
     varlen: dict = field(default_factory=dict)  # {"n": 32, "lo": 128, "hi": 8192}
     page_size: int = 0  # > 0: decode against a paged KV cache of pages of this many keys
     kv_fp8: bool = False  # decode against an e4m3 KV cache (scale FP8_SCALE)
+    qkv_fp8: bool = False  # prefill on e4m3 Q, K, V (scale FP8_PREFILL_SCALE each)
     block_sparse: dict = field(default_factory=dict)  # {"window": 3, "global": 2, "random": 3}
     backward: bool = False  # time the backward pass (dQ, dK, dV) of this forward
 
@@ -74,6 +75,10 @@ LLAMA_BWD = Workload("llama8b_backward_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8
                      D=128, dtype="bf16", causal=True, seed=2, backward=True)
 LLAMA_BWD_B1 = Workload("llama8b_backward_b1_s8192_causal", B=1, Hq=32, Hkv=8, Sq=8192, Sk=8192,
                      D=128, dtype="bf16", causal=True, seed=2, backward=True)
+# the Llama prefill's inputs as e4m3 codes (value / FP8_PREFILL_SCALE, rounded)
+LLAMA_FP8 = Workload("llama8b_prefill_fp8_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8192,
+                     Sk=8192, D=128, dtype="bf16", causal=True, seed=2, qkv_fp8=True)
+FP8_PREFILL_SCALE = 1.0 / 16.0
 LLAMA_STRESS = Workload("llama8b_prefill_b4_s8192_causal_qx4", B=4, Hq=32, Hkv=8, Sq=8192,
                         Sk=8192, D=128, dtype="bf16", causal=True, seed=3, q_mult=4.0)
 DECODE_BATCHES = (1, 16, 64, 128, 256)
@@ -160,6 +165,18 @@ def bigbird_pattern_varlen(lengths, block_sparse: dict, seed: int, blk: int = 12
     return row_ptr, col
 
 
+def blocksparse_varlen_flops(lengths, row_ptr, col, Hq: int, D: int, blk: int = 128) -> int:
+    """4*D flops per visible (query, key) pair per head over packed sequences."""
+    rp, cl = row_ptr.tolist(), col.tolist()
+    pairs, r = 0, 0
+    for n in [int(x) for x in lengths]:
+        for qb in range(-(-n // blk)):
+            rows_in = min(blk, n - qb * blk)
+            pairs += rows_in * sum(min(blk, n - c * blk) for c in cl[rp[r]:rp[r + 1]])
+            r += 1
+    return 4 * D * pairs * Hq
+
+
 def blocksparse_flops(w: Workload, row_ptr, col) -> int:
     """4*D flops per visible (query, key) pair per head under the block pattern."""
     blk = 128
@@ -176,6 +193,11 @@ def blocksparse_flops(w: Workload, row_ptr, col) -> int:
 VARLEN = Workload("varlen32_len128to8192_causal", B=32, Hq=32, Hkv=8, Sq=0, Sk=0, D=128,
                   dtype="bf16", causal=True, seed=5,
                   varlen={"n": 32, "lo": 128, "hi": 8192})
+# the same 32 lengths (seed 5), non-causal, a BigBird-style pattern per sequence
+BIGBIRD_VARLEN = Workload("bigbird_varlen32_len128to8192_blk128", B=32, Hq=32, Hkv=8, Sq=0,
+                          Sk=0, D=128, dtype="bf16", causal=False, seed=5,
+                          varlen={"n": 32, "lo": 128, "hi": 8192},
+                          block_sparse={"window": 3, "global": 2, "random": 3})
 
 
 def _gen(device, seed: int) -> torch.Generator:
@@ -197,6 +219,13 @@ def make_qkv(w: Workload, device="cpu", *, B=None, Sq=None, Sk=None):
     if w.q_mult != 1.0:
         q = q * w.q_mult
     return tuple(t.transpose(1, 2).contiguous() for t in (q, k, v))
+
+
+def make_qkv_e4m3(w: Workload, device="cpu", **kw):
+    """make_qkv's values as e4m3 codes: value / FP8_PREFILL_SCALE rounded (nearest
+    even) by torch's float8_e4m3fn cast."""
+    q, k, v = make_qkv(w, device=device, **kw)
+    return tuple((t.float() / FP8_PREFILL_SCALE).to(torch.float8_e4m3fn) for t in (q, k, v))
 
 
 def make_dout(w: Workload, device="cpu"):
