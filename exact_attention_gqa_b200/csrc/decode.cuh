@@ -698,9 +698,24 @@ __global__ void __launch_bounds__(160, 2)
         }
     }
     __syncthreads();
-    if (*abort_flag) return;
+    const bool aborted = *abort_flag != 0;
     for (int idx = threadIdx.x; idx < rows * HD; idx += blockDim.x) {
         const int r = idx / HD, d = idx - r * HD;
+        if (aborted) {
+            // a wait gave up (device error word set): this CTA's rows become empty,
+            // O = 0 and L = -inf, so that neither the output nor the combine can pick
+            // up what an earlier call left in the output or the partials buffer
+            const int h = h0 + r;
+            if (p.n_splits == 1) {
+                p.out[(size_t(b) * p.Hq + h) * HD + d] = __float2bfloat16_rn(0.f);
+                if (d == 0) p.lse[size_t(b) * p.Hq + h] = -INFINITY;
+            } else {
+                const size_t base = (size_t(b) * p.Hq + h) * p.n_splits + split;
+                p.part_o[base * HD + d] = 0.f;
+                if (d == 0) p.part_l[base] = -INFINITY;
+            }
+            continue;
+        }
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * 16 + r]);

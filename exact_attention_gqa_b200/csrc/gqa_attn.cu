@@ -983,8 +983,9 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
     Plan pl;
     make_plan(&pl, B, Hq, Hkv, 1, Sk, num_splits, pack_gqa, false, dev->sms);
     if (num_splits == 0) {
-        // automatic choice: the largest split count, up to the planned one, whose
-        // partials fit the static scratch (one split needs none)
+        // automatic choice: the planned count puts at most one CTA on each SM, whose
+        // partials (at most SMs x 16 rows) fit the static scratch on a 148-SM part; this
+        // step-down is a guard for parts with more SMs (one split needs no scratch)
         while (pl.splits > 1 && ws_bytes(B, Hq, 1, D, pl.splits) > GQA_NOALLOC_SCRATCH_BYTES) {
             Plan smaller;
             make_plan(&smaller, B, Hq, Hkv, 1, Sk, pl.splits - 1, pack_gqa, false, dev->sms);

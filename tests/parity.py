@@ -63,6 +63,9 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, *, f32=False):
 GRAD_MAX_REL = 1e-2
 GRAD_MEAN_REL = 1e-3
 GRAD_MODEL_FACTOR = 1.5
+# every compare_grad call's errors and effective bars, printed at the end of the run
+# (tests/conftest.py) so that a kernel drifting toward the model-scaled bar shows
+GRAD_LOG: list = []
 
 
 def bf16_backward_model(q, k, v, do, scale, causal):
@@ -117,12 +120,17 @@ def compare_grad(g_gpu, ref, model=None):
     big = max(1.0, float(np.abs(ref).max(initial=0.0)))
     typ = max(1.0, float(np.abs(ref).mean())) if ref.size else 1.0
     max_bar, mean_bar = GRAD_MAX_REL * big, GRAD_MEAN_REL * typ
+    fixed = (max_bar, mean_bar)
+    model_err = (None, None)
     if model is not None and ref.size:
         merr = np.abs(np.asarray(model, dtype=np.float64) - ref)
-        max_bar = max(max_bar, GRAD_MODEL_FACTOR * float(merr.max()))
-        mean_bar = max(mean_bar, GRAD_MODEL_FACTOR * float(merr.mean()))
+        model_err = (float(merr.max()), float(merr.mean()))
+        max_bar = max(max_bar, GRAD_MODEL_FACTOR * model_err[0])
+        mean_bar = max(mean_bar, GRAD_MODEL_FACTOR * model_err[1])
     stats = {"max_abs": float(err.max(initial=0.0)), "mean_abs": float(err.mean()) if err.size else 0.0,
-             "max_bar": max_bar, "mean_bar": mean_bar}
+             "max_bar": max_bar, "mean_bar": mean_bar, "fixed_max_bar": fixed[0],
+             "fixed_mean_bar": fixed[1], "model_max": model_err[0], "model_mean": model_err[1]}
+    GRAD_LOG.append(stats)
     assert stats["max_abs"] <= max_bar, stats
     assert stats["mean_abs"] <= mean_bar, stats
     return stats

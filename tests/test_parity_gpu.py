@@ -362,8 +362,12 @@ def test_full_llama_prefill_workload(w):
                w.causal)
 
 
-@pytest.mark.parametrize("B", [1, 16, 64])
+@pytest.mark.parametrize("B", W.DECODE_BATCHES)
 def test_full_decode_workload(B):
+    """Every batch size of the decode sweep (B up to 256: a 34 GB cache, drawn on the
+    device one element at a time) at every split count the sweep times, the automatic
+    count (0) included, with and without PackGQA; sampled batch elements {0, B - 1, one
+    at random} are compared element-wise with the oracle on that element's cache."""
     w = W.decode(B)
     q = W.make_decode_q(w, device=DEV)
     k = torch.empty(B, w.Sk, w.Hkv, w.D, dtype=torch.bfloat16, device=DEV)
@@ -371,14 +375,17 @@ def test_full_decode_workload(B):
     W.fill_decode_kv(w, k, v)
     rng = np.random.default_rng(B)
     bs = sorted({0, B - 1, int(rng.integers(B))})
-    for splits in W.DECODE_SPLITS:
+    # the oracle's result for an element does not depend on the split count or packing
+    refs = {b: oracle.attention(q[b:b + 1].cpu(), k[b:b + 1].cpu(), v[b:b + 1].cpu(),
+                                scale=w.scale, causal=False) for b in bs}
+    for splits in W.DECODE_SPLITS + (0,):
         for pack in (1, 0):
             out, lse = gqa_attn(q, k, v, num_splits=splits, pack_gqa=pack)
             torch.cuda.synchronize()
             for b in bs:
-                o_ref, l_ref = oracle.attention(q[b:b + 1].cpu(), k[b:b + 1].cpu(),
-                                                v[b:b + 1].cpu(), scale=w.scale, causal=False)
-                compare(out[b:b + 1], lse[b:b + 1], o_ref, l_ref)
+                compare(out[b:b + 1], lse[b:b + 1], *refs[b])
+    del k, v
+    torch.cuda.empty_cache()
 
 
 def test_full_varlen_workload():
