@@ -170,26 +170,6 @@ __device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-// D += A(16x32, row) * B(32x8, col), e4m3 inputs, fp32 accumulate
-__device__ __forceinline__ void mma_e4m3_16832(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-// four fp32 -> four e4m3 bytes (element i in byte i), nearest even, saturating
-__device__ __forceinline__ uint32_t pack_e4m3x4_sat(float v0, float v1, float v2, float v3) {
-    uint32_t r;
-    asm("{\n\t.reg .b16 lo, hi;\n\t"
-        "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
-        "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
-        "mov.b32 %0, {lo, hi};\n\t}"
-        : "=r"(r)
-        : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
-    return r;
-}
 template <bool F16>
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                           uint32_t b1) {
@@ -382,70 +362,6 @@ __global__ void __launch_bounds__(160, 2)
                 }
             }
         }
-        // e4m3 K at D = 128 (K8): Q K^T runs on the 8-bit MMA straight from the stage.
-        // q enters as two e4m3 terms with a per-row power-of-two scale s, q s = hi + lo
-        // (lo the rounded residual; both products accumulate into the same registers).
-        // A bf16 q has 8 significant bits and each term carries 4, so the split loses
-        // only residuals below e4m3's normal range (about 1e-6 of the row's largest
-        // |q|); 1 / s joins the row's exponent multiplier.
-        constexpr bool K8 = KV8 && HD == 128;
-        uint32_t qhi[K8 ? 4 : 1][4], qlo[K8 ? 4 : 1][4];
-        float sl2r[2] = {sl2, sl2};
-        if constexpr (K8) {
-            const int t4 = lane & 3;
-            float qv[2][32];  // rows g, g + 8: dims kk*32 + {4t..4t+3, 16+4t..16+4t+3}
-            const bool v0 = g < rows, v1 = g + 8 < rows;
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const uint32_t* qr = reinterpret_cast<const uint32_t*>(
-                    p.q + (size_t(b) * p.Hq + h0 + g + 8 * hr) * HD);
-                const bool ok = hr ? v1 : v0;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int d0 = kk * 32 + half * 16 + 4 * t4;
-                        const uint32_t w0 = ok ? __ldg(qr + d0 / 2) : 0u;
-                        const uint32_t w1 = ok ? __ldg(qr + d0 / 2 + 1) : 0u;
-                        float* dst = qv[hr] + kk * 8 + half * 4;
-                        dst[0] = __uint_as_float(w0 << 16);
-                        dst[1] = __uint_as_float(w0 & 0xffff0000u);
-                        dst[2] = __uint_as_float(w1 << 16);
-                        dst[3] = __uint_as_float(w1 & 0xffff0000u);
-                    }
-            }
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                float amax = 0.f;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(qv[hr][e]));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-                // 2^floor(log2(224 / amax)), capped so that it stays finite for tiny rows
-                const float sc_row =
-                    amax > 0.f ? fminf(exp2f(floorf(log2f(224.f / amax))), 0x1p100f) : 1.f;
-                sl2r[hr] = sl2 / sc_row;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const float* v = qv[hr] + kk * 8 + half * 4;
-                        const float x0 = v[0] * sc_row, x1 = v[1] * sc_row, x2 = v[2] * sc_row,
-                                    x3 = v[3] * sc_row;
-                        const uint32_t h = pack_e4m3x4_sat(x0, x1, x2, x3);
-                        uint32_t f01, f23;  // the hi term's values (exact in f16)
-                        e4m3x4_to_f16x4(h, f01, f23);
-                        const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&f01));
-                        const float2 c2 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
-                        const uint32_t l =
-                            pack_e4m3x4_sat(x0 - a.x, x1 - a.y, x2 - c2.x, x3 - c2.y);
-                        // A of m16n8k32: a0 (row g, dims 4t..), a1 (row g + 8, dims 4t..),
-                        // a2 (row g, dims 16 + 4t..), a3 (row g + 8, dims 16 + 4t..)
-                        qhi[kk][half * 2 + hr] = h;
-                        qlo[kk][half * 2 + hr] = l;
-                    }
-            }
-        }
         const uint32_t sK0 = smem_u32(smem + C::OFF_K);
         const uint32_t sV0 = smem_u32(smem + C::OFF_V);
         // KV8: this warp's f16 copies of its 16 keys; ldmatrix rows count from the warp's
@@ -501,7 +417,7 @@ __global__ void __launch_bounds__(160, 2)
                 // once), so neither side has bank conflicts
                 const int r_keep = key_end - (blk0 + c) * C::BN - warp * 16;  // rows kept
 #pragma unroll
-                for (int kv = K8 ? 1 : 0; kv < 2; ++kv) {
+                for (int kv = 0; kv < 2; ++kv) {
                     const uint32_t src = (kv ? sV : sK) + uint32_t(warp * 16 * HD);
                     const uint32_t dst = kv ? wV : wK;
 #pragma unroll
@@ -524,10 +440,8 @@ __global__ void __launch_bounds__(160, 2)
                     }
                 }
                 __syncwarp();
-                if constexpr (!K8) {
-                    if (lane == 0) mbar_arrive(bar_empty + s);
-                    sK = wK;
-                }
+                if (lane == 0) mbar_arrive(bar_empty + s);
+                sK = wK;
                 sV = wV;
             }
             float sc[2][4];
@@ -535,39 +449,14 @@ __global__ void __launch_bounds__(160, 2)
             for (int t = 0; t < 2; ++t)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sc[t][e] = 0.f;
-            if constexpr (K8) {
-                // B of m16n8k32: b0 = K[key g][dims 4t..4t+3], b1 = K[key g][16 + 4t..];
-                // 16-byte chunk c of stage row r sits at c ^ (r % 8) (128B swizzle), so
-                // the 8 rows of a fragment load fall on distinct banks
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        const int row = warp * 16 + nt * 8 + g;
-                        const uint32_t rb = sK + uint32_t(row * 128 + 4 * (lane & 3));
-                        uint32_t b0, b1;
-                        asm volatile("ld.shared.u32 %0, [%1];"
-                                     : "=r"(b0)
-                                     : "r"(rb + uint32_t(((2 * kk) ^ (row & 7)) << 4)));
-                        asm volatile("ld.shared.u32 %0, [%1];"
-                                     : "=r"(b1)
-                                     : "r"(rb + uint32_t(((2 * kk + 1) ^ (row & 7)) << 4)));
-                        mma_e4m3_16832(sc[nt], qhi[kk], b0, b1);
-                        mma_e4m3_16832(sc[nt], qlo[kk], b0, b1);
-                    }
-                // K and V of this stage are read: hand it back to TMA
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar_empty + s);
-            } else {
-#pragma unroll
-                for (int kk = 0; kk < KSTEPS; ++kk) {
-                    const int chunk = kk * 2 + chunk_qk;
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(sK + (chunk >> 3) * ATOM_B + sw128_off(key_qk - row0, chunk), b0,
-                            b1, b2, b3);
-                    mma_16816<KV8>(sc[0], qa[kk], b0, b1);
-                    mma_16816<KV8>(sc[1], qa[kk], b2, b3);
-                }
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                const int chunk = kk * 2 + chunk_qk;
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(sK + (chunk >> 3) * ATOM_B + sw128_off(key_qk - row0, chunk), b0, b1, b2,
+                        b3);
+                mma_16816<KV8>(sc[0], qa[kk], b0, b1);
+                mma_16816<KV8>(sc[1], qa[kk], b2, b3);
             }
             // mask keys past the end of this split / of the sequence, and keys
             // before the window (only blocks that straddle one of those edges)
@@ -590,7 +479,7 @@ __global__ void __launch_bounds__(160, 2)
                                  fmaxf(sc[1][2 * hr], sc[1][2 * hr + 1]));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float mb = mx * sl2r[hr];
+                const float mb = mx * sl2;
                 alpha[hr] = 1.f;
                 if (mb > m_run[hr] + 8.0f) {
                     alpha[hr] = ex2_approx(m_run[hr] - mb);
@@ -606,7 +495,7 @@ __global__ void __launch_bounds__(160, 2)
                     for (int e = 0; e < 4; ++e) {
                         const int hr = e >> 1;
                         const float mu = (m_run[hr] == -INFINITY) ? 0.f : m_run[hr];
-                        pr[t][e] = ex2_approx(fmaf(sc[t][e], sl2r[hr], -mu));
+                        pr[t][e] = ex2_approx(fmaf(sc[t][e], sl2, -mu));
                     }
                 if constexpr (KV8) {
                     pa[0] = pack_f16x2(pr[0][0], pr[0][1]);

@@ -413,10 +413,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* out, float*
     const long long rows = kv.block_table ? (long long)kv.num_pages * kv.page_size
                                           : (long long)B * Sk;
     const int box = kv.block_table ? (kv.page_size < C::BN ? kv.page_size : C::BN) : C::BN;
-    // e4m3 K at D = 128: 128-byte rows with the 128B swizzle (the QK^T fragments are read
-    // straight from the stage); V stays unswizzled for its conversion to f16
-    const bool maps = kv.fp8 ? ((HD == 128 ? make_map_u8_sw128(&tk, k, rows, Hkv, HD, 1, box)
-                                           : make_map_u8(&tk, k, rows, Hkv, HD, box)) &&
+    const bool maps = kv.fp8 ? (make_map_u8(&tk, k, rows, Hkv, HD, box) &&
                                 make_map_u8(&tv, v, rows, Hkv, HD, box))
                              : (make_map(&tk, k, rows, Hkv, HD, 1, box) &&
                                 make_map(&tv, v, rows, Hkv, HD, 1, box));
