@@ -339,10 +339,16 @@ class Case:
 
     def in_bytes(self):
         k, v = self.kv[0]
-        return (self.q.numel() * self.q.element_size() + k.numel() * k.element_size() +
-                v.numel() * v.element_size())
+        b = (self.q.numel() * self.q.element_size() + k.numel() * k.element_size() +
+             v.numel() * v.element_size())
+        if self.w.backward:  # the forward's O and L, and dO
+            b += (self.fwd_out.numel() * 2 + self.fwd_lse.numel() * 4 +
+                  self.do.numel() * 2)
+        return b
 
     def out_bytes(self):
+        if self.w.backward:  # dQ, dK, dV
+            return sum(t.numel() * 2 for t in self.grads)
         return self.out.numel() * 2 + self.lse.numel() * 4
 
     def step(self):

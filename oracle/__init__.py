@@ -88,6 +88,9 @@ def _load():
         lib.oracle_attention.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, P, I]
         lib.oracle_attention_rows.argtypes = [P, P, P, I, I, I, I, I, I, Dbl, I, P, I, P, P,
                                               P, I]
+        lib.oracle_attention_window.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, P, I]
+        lib.oracle_attention_rows_window.argtypes = [P, P, P, I, I, I, I, I, I, Dbl, I, I, P, I,
+                                                     P, P, P, I]
         lib.oracle_attention_keyrange.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, I,
                                                   I, I]
         lib.oracle_combine.argtypes = [I, I, P, P, P, P]
@@ -104,10 +107,10 @@ def _load():
                                               Dbl, I, P, I]
         lib.oracle_attention_e4m3.restype = I
         lib.oracle_attention_blocksparse_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, Dbl,
-                                                            P, P, I, I]
+                                                            I, P, P, I, I]
         lib.oracle_attention_blocksparse_varlen.restype = I
-        lib.oracle_attention_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, P, P,
-                                                     I, I]
+        lib.oracle_attention_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dbl, I, P,
+                                                     P, I, I]
         lib.oracle_attention_blocksparse.restype = I
         lib.oracle_attention_backward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, Dbl, I,
                                                   I]
@@ -119,7 +122,8 @@ def _load():
         lib.oracle_get_flaw.restype = I
         lib.oracle_max_threads.restype = I
         for name in ("oracle_attention", "oracle_attention_rows", "oracle_attention_keyrange",
-                     "oracle_attention_tiled"):
+                     "oracle_attention_tiled", "oracle_attention_window",
+                     "oracle_attention_rows_window"):
             getattr(lib, name).restype = I
         _lib = lib
     return _lib
@@ -161,23 +165,32 @@ def set_flaw(name: str) -> None:
     _load().oracle_set_flaw(FLAWS[name])
 
 
-def attention(q, k, v, *, scale: float, causal: bool, cu_seqlens=None, threads: int = 0):
-    """Full forward.  Returns (O float64 like q, L float64 [B,Hq,Sq] or [Hq,total])."""
+def attention(q, k, v, *, scale: float, causal: bool, cu_seqlens=None, window: int = 0,
+              threads: int = 0):
+    """Full forward.  Returns (O float64 like q, L float64 [B,Hq,Sq] or [Hq,total]).
+    window > 0 (causal only): each query sees its `window` most recent keys."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
     B, Hq, Hkv, Sq, Sk, D = _dims(q, k, cu)
     o = np.zeros(q.shape, dtype=np.float64)
     lse = np.zeros((Hq, q.shape[0]) if cu is not None else (B, Hq, Sq), dtype=np.float64)
-    rc = _load().oracle_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv,
-                                  Sq, Sk, D, float(scale), int(bool(causal)),
-                                  None if cu is None else _ptr(cu), int(threads))
+    if window:
+        if not causal or window < 1:
+            raise ValueError("a sliding window needs causal=True and window >= 1")
+        rc = _load().oracle_attention_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
+                                             Hq, Hkv, Sq, Sk, D, float(scale), int(window),
+                                             None if cu is None else _ptr(cu), int(threads))
+    else:
+        rc = _load().oracle_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
+                                      Hkv, Sq, Sk, D, float(scale), int(bool(causal)),
+                                      None if cu is None else _ptr(cu), int(threads))
     if rc != 0:
         raise ValueError("oracle_attention: bad arguments")
     return o, lse
 
 
 def attention_rows(q, k, v, rows, *, scale: float, causal: bool, cu_seqlens=None,
-                   threads: int = 0):
+                   window: int = 0, threads: int = 0):
     """O and L for selected rows; rows is an int array [n, 3] of (b, h, i)."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
@@ -186,10 +199,10 @@ def attention_rows(q, k, v, rows, *, scale: float, causal: bool, cu_seqlens=None
     n = rows.shape[0]
     o = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
-    rc = _load().oracle_attention_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk, D,
-                                       float(scale), int(bool(causal)),
-                                       None if cu is None else _ptr(cu), n, _ptr(rows),
-                                       _ptr(o), _ptr(lse), int(threads))
+    rc = _load().oracle_attention_rows_window(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Sk,
+                                              D, float(scale), int(bool(causal)), int(window),
+                                              None if cu is None else _ptr(cu), n, _ptr(rows),
+                                              _ptr(o), _ptr(lse), int(threads))
     if rc != 0:
         raise ValueError("oracle_attention_rows: bad arguments")
     return o, lse
@@ -316,9 +329,10 @@ def _np_int(a):
 
 
 def attention_blocksparse(q, k, v, row_ptr, col, *, scale: float, blk: int = 128,
-                          threads: int = 0):
+                          causal: bool = False, threads: int = 0):
     """Dense-layout attention restricted to a block pattern (CSR rows of key blocks per
-    query block of blk positions).  Returns (O float64 like q, L float64 [B,Hq,Sq])."""
+    query block of blk positions), optionally also causal (bottom-right aligned).
+    Returns (O float64 like q, L float64 [B,Hq,Sq])."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     B, Hq, Hkv, Sq, Sk, D = _dims(q, k, None)
     rp = np.ascontiguousarray(_np_int(row_ptr), dtype=np.int32)
@@ -328,15 +342,16 @@ def attention_blocksparse(q, k, v, row_ptr, col, *, scale: float, blk: int = 128
     o = np.zeros(q.shape, dtype=np.float64)
     lse = np.zeros((B, Hq, Sq), dtype=np.float64)
     rc = _load().oracle_attention_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B,
-                                              Hq, Hkv, Sq, Sk, D, float(scale), _ptr(rp),
-                                              _ptr(cl), int(blk), int(threads))
+                                              Hq, Hkv, Sq, Sk, D, float(scale),
+                                              int(bool(causal)), _ptr(rp), _ptr(cl), int(blk),
+                                              int(threads))
     if rc != 0:
         raise ValueError("oracle_attention_blocksparse: bad arguments")
     return o, lse
 
 
 def attention_blocksparse_varlen(q, k, v, cu_seqlens, row_ptr, col, *, scale: float,
-                                 blk: int = 128, threads: int = 0):
+                                 blk: int = 128, causal: bool = False, threads: int = 0):
     """Packed sequences ([total, H, D]), each with its own block pattern: the pattern's
     rows are the query blocks of sequence 0, then of sequence 1, ... (ceil(n_b / blk)
     each), col entries are key blocks of the same sequence.  Returns (O float64 like q,
@@ -355,8 +370,8 @@ def attention_blocksparse_varlen(q, k, v, cu_seqlens, row_ptr, col, *, scale: fl
     lse = np.zeros((Hq, q.shape[0]), dtype=np.float64)
     rc = _load().oracle_attention_blocksparse_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                                      _ptr(lse), _ptr(cu), B, Hq, Hkv, D,
-                                                     float(scale), _ptr(rp), _ptr(cl),
-                                                     int(blk), int(threads))
+                                                     float(scale), int(bool(causal)), _ptr(rp),
+                                                     _ptr(cl), int(blk), int(threads))
     if rc != 0:
         raise ValueError("oracle_attention_blocksparse_varlen: bad arguments")
     return o, lse

@@ -111,6 +111,7 @@ typedef struct {
     int Sq, Sk, D;
     double scale;
     int causal;
+    int window; /* > 0 (causal only): key j visible to query i only if j > i + Sk - Sq - window */
 } head_view;
 
 /* Grouped-query mapping: query head h reads key/value head h / G. */
@@ -120,13 +121,32 @@ static int kv_head_of(int h, int Hq, int Hkv)
     return h / (Hq / Hkv);
 }
 
-/* Causal visibility of key j to query i (bottom-right aligned). */
-static int key_visible(int i, int j, int Sq, int Sk, int causal)
+/*
+ * Causal visibility of key j to query i (bottom-right aligned), optionally within a
+ * sliding window: query i, at key position i + Sk - Sq, sees its `window` most recent
+ * keys, (i + Sk - Sq - window, i + Sk - Sq] (Ultralytics GQA glossary, "GQA and
+ * related techniques": sliding-window attention caps the tokens attended to; the same
+ * reading as the decode window below).
+ */
+static int key_visible_w(int i, int j, int Sq, int Sk, int causal, int window)
 {
     if (!causal) return 1;
-    if (g_flaw == FLAW_TOP_LEFT_CAUSAL) return j <= i;
-    if (g_flaw == FLAW_DROP_DIAGONAL) return j < i + (Sk - Sq);
-    return j <= i + (Sk - Sq);
+    int vis;
+    if (g_flaw == FLAW_TOP_LEFT_CAUSAL)
+        vis = j <= i;
+    else if (g_flaw == FLAW_DROP_DIAGONAL)
+        vis = j < i + (Sk - Sq);
+    else
+        vis = j <= i + (Sk - Sq);
+    if (window > 0) {
+        const int w = (g_flaw == FLAW_WINDOW_SHORT) ? window - 1 : window;
+        vis = vis && j > i + (Sk - Sq) - w;
+    }
+    return vis;
+}
+static int key_visible(int i, int j, int Sq, int Sk, int causal)
+{
+    return key_visible_w(i, j, Sq, Sk, causal, 0);
 }
 
 static double dot(const float* a, const float* b, int D)
@@ -148,7 +168,7 @@ static void attend_row(const head_view* hv, int i, int j0, int j1, double* row,
     const double scale = (g_flaw == FLAW_NO_SCALE) ? 1.0 : hv->scale;
     double m = -INFINITY;
     for (int j = j0; j < j1; ++j) {
-        if (key_visible(i, j, hv->Sq, hv->Sk, hv->causal)) {
+        if (key_visible_w(i, j, hv->Sq, hv->Sk, hv->causal, hv->window)) {
             row[j] = scale * dot(qi, hv->k + (size_t)j * hv->kv_stride, hv->D);
             if (row[j] > m) m = row[j];
         } else {
@@ -210,6 +230,7 @@ static head_view make_view(const float* q, const float* k, const float* v, int B
     hv.D = D;
     hv.scale = scale;
     hv.causal = causal;
+    hv.window = 0;
     return hv;
 }
 
@@ -259,11 +280,13 @@ int oracle_max_threads(void)
  * Full attention forward: every (sequence, head, query row).
  * o has the layout of q; lse is [B, Hq, Sq] (dense) or [Hq, total] (varlen).
  */
-int oracle_attention(const float* q, const float* k, const float* v, double* o, double* lse,
-                     int B, int Hq, int Hkv, int Sq, int Sk, int D, double scale, int causal,
-                     const int32_t* cu_seqlens, int nthreads)
+static int attention_impl(const float* q, const float* k, const float* v, double* o,
+                          double* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                          double scale, int causal, int window, const int32_t* cu_seqlens,
+                          int nthreads)
 {
     if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, cu_seqlens) || !o || !lse) return -1;
+    if (window < 0 || (window > 0 && !causal)) return -1;
     set_threads(nthreads);
     const int kmax = max_keys(B, Sk, cu_seqlens);
     const int nbh = B * Hq;
@@ -282,6 +305,7 @@ int oracle_attention(const float* q, const float* k, const float* v, double* o, 
             size_t qrow0, lse_off, lse_step;
             head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, cu_seqlens,
                                      b, h, &qrow0, &lse_off, &lse_step);
+            hv.window = window;
             for (int i = 0; i < hv.Sq; ++i) {
                 double* orow = o + ((qrow0 + (size_t)i) * Hq + h) * (size_t)D;
                 attend_row(&hv, i, 0, hv.Sk, row, orow, lse + lse_off + (size_t)i * lse_step);
@@ -292,17 +316,37 @@ int oracle_attention(const float* q, const float* k, const float* v, double* o, 
     return err;
 }
 
+int oracle_attention(const float* q, const float* k, const float* v, double* o, double* lse,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D, double scale, int causal,
+                     const int32_t* cu_seqlens, int nthreads)
+{
+    return attention_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, 0,
+                          cu_seqlens, nthreads);
+}
+
+/* Causal attention within a sliding window of `window` >= 1 keys (key_visible_w). */
+int oracle_attention_window(const float* q, const float* k, const float* v, double* o,
+                            double* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                            double scale, int window, const int32_t* cu_seqlens, int nthreads)
+{
+    if (window < 1) return -1;
+    return attention_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, D, scale, 1, window,
+                          cu_seqlens, nthreads);
+}
+
 /*
  * Selected rows only: rows holds n_rows triples (b, h, i).  For each, O[i, :] of
  * query head h of sequence b goes to o_rows[r*D .. r*D+D) and L_i to lse_rows[r].
  * Used to check outputs of problems too large to evaluate in full.
  */
-int oracle_attention_rows(const float* q, const float* k, const float* v, int B, int Hq,
-                          int Hkv, int Sq, int Sk, int D, double scale, int causal,
-                          const int32_t* cu_seqlens, int n_rows, const int32_t* rows,
-                          double* o_rows, double* lse_rows, int nthreads)
+int oracle_attention_rows_window(const float* q, const float* k, const float* v, int B,
+                                 int Hq, int Hkv, int Sq, int Sk, int D, double scale,
+                                 int causal, int window, const int32_t* cu_seqlens, int n_rows,
+                                 const int32_t* rows, double* o_rows, double* lse_rows,
+                                 int nthreads)
 {
     if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, cu_seqlens) || n_rows < 0) return -1;
+    if (window < 0 || (window > 0 && !causal)) return -1;
     if (n_rows > 0 && (!rows || !o_rows || !lse_rows)) return -1;
     for (int r = 0; r < n_rows; ++r) {
         const int b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
@@ -326,12 +370,22 @@ int oracle_attention_rows(const float* q, const float* k, const float* v, int B,
             size_t qrow0, lse_off, lse_step;
             head_view hv = make_view(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, cu_seqlens,
                                      rows[3 * r], rows[3 * r + 1], &qrow0, &lse_off, &lse_step);
+            hv.window = window;
             attend_row(&hv, rows[3 * r + 2], 0, hv.Sk, row, o_rows + (size_t)r * D,
                        lse_rows + r);
         }
         free(row);
     }
     return err;
+}
+
+int oracle_attention_rows(const float* q, const float* k, const float* v, int B, int Hq,
+                          int Hkv, int Sq, int Sk, int D, double scale, int causal,
+                          const int32_t* cu_seqlens, int n_rows, const int32_t* rows,
+                          double* o_rows, double* lse_rows, int nthreads)
+{
+    return oracle_attention_rows_window(q, k, v, B, Hq, Hkv, Sq, Sk, D, scale, causal, 0,
+                                        cu_seqlens, n_rows, rows, o_rows, lse_rows, nthreads);
 }
 
 /*
@@ -500,15 +554,17 @@ int oracle_attention_backward(const float* q, const float* k, const float* v, co
 }
 
 /*
- * Exact attention restricted to a block pattern (dense layout, non-causal).
+ * Exact attention restricted to a block pattern (dense layout), optionally causal:
+ * key j is visible to query i when its block is listed in the row of i's query block
+ * and, with causal, when j <= i + Sk - Sq as well.
  * row_ptr[n_qblk + 1], col[nnz]: key blocks of each query block of `blk` positions;
  * n_qblk = ceil(Sq / blk).  o like q, lse [B, Hq, Sq].  A row whose blocks hold no
- * key gets O = 0, L = -inf.
+ * visible key gets O = 0, L = -inf.
  */
 int oracle_attention_blocksparse(const float* q, const float* k, const float* v, double* o,
                                  double* lse, int B, int Hq, int Hkv, int Sq, int Sk, int D,
-                                 double scale, const int32_t* row_ptr, const int32_t* col,
-                                 int blk, int nthreads)
+                                 double scale, int causal, const int32_t* row_ptr,
+                                 const int32_t* col, int blk, int nthreads)
 {
     if (check_args(q, k, v, B, Hq, Hkv, Sq, Sk, D, NULL) || !o || !lse || !row_ptr || !col ||
         blk <= 0)
@@ -541,7 +597,8 @@ int oracle_attention_blocksparse(const float* q, const float* k, const float* v,
                 if (g_flaw == FLAW_SPARSE_ROW && qb + 1 < n_qblk) qb += 1;
                 memset(vis, 0, (size_t)Sk);
                 for (int e = row_ptr[qb]; e < row_ptr[qb + 1]; ++e)
-                    for (int j = col[e] * blk; j < (col[e] + 1) * blk && j < Sk; ++j) vis[j] = 1;
+                    for (int j = col[e] * blk; j < (col[e] + 1) * blk && j < Sk; ++j)
+                        vis[j] = (unsigned char)key_visible(i, j, Sq, Sk, causal);
                 const float* qi = hv.q + (size_t)i * hv.q_stride;
                 double m = -INFINITY;
                 for (int j = 0; j < Sk; ++j) {
@@ -581,12 +638,13 @@ int oracle_attention_blocksparse(const float* q, const float* k, const float* v,
  * Sequence b holds n_b = cu[b+1] - cu[b] positions and ceil(n_b / blk) blocks; its
  * query blocks are rows blk_off[b] .. blk_off[b] + ceil(n_b / blk) - 1 of the pattern,
  * blk_off[b] = sum over earlier sequences of their block counts, and their col entries
- * are key blocks of the same sequence, 0 .. ceil(n_b / blk) - 1.  Non-causal, self
- * attention within each sequence.  q, k, v, o packed [total, H, D], lse [Hq, total].
+ * are key blocks of the same sequence, 0 .. ceil(n_b / blk) - 1.  Self attention
+ * within each sequence, optionally causal (key j visible to query i only if j <= i).
+ * q, k, v, o packed [total, H, D], lse [Hq, total].
  */
 int oracle_attention_blocksparse_varlen(const float* q, const float* k, const float* v,
                                         double* o, double* lse, const int32_t* cu, int B,
-                                        int Hq, int Hkv, int D, double scale,
+                                        int Hq, int Hkv, int D, double scale, int causal,
                                         const int32_t* row_ptr, const int32_t* col, int blk,
                                         int nthreads)
 {
@@ -639,7 +697,8 @@ int oracle_attention_blocksparse_varlen(const float* q, const float* k, const fl
                 }
                 memset(vis, 0, (size_t)n);
                 for (int e = row_ptr[r]; e < row_ptr[r + 1]; ++e)
-                    for (int j = col[e] * blk; j < (col[e] + 1) * blk && j < n; ++j) vis[j] = 1;
+                    for (int j = col[e] * blk; j < (col[e] + 1) * blk && j < n; ++j)
+                        vis[j] = (unsigned char)key_visible(i, j, n, n, causal);
                 const float* qi = hv.q + (size_t)i * hv.q_stride;
                 double m = -INFINITY;
                 for (int j = 0; j < n; ++j) {

@@ -530,6 +530,128 @@ def test_kvcache_e4m3_paged_matches_sdpa():
 # ---------------------------------------------------------------------------------
 # Block-sparse attention (Raptor-T abstract: BigBird's block pattern)
 
+# ---------------------------------------------------------------------------------
+# Prefill sliding window (causal): query i sees keys (i + Sk - Sq - W, i + Sk - Sq]
+
+def band_mask(Sq, Sk, window):
+    i = np.arange(Sq)[:, None] + (Sk - Sq)
+    j = np.arange(Sk)[None, :]
+    return (j <= i) & (j > i - window)
+
+
+@pytest.mark.parametrize("Sq,Sk,window", [(40, 40, 1), (40, 40, 7), (33, 70, 16), (50, 20, 5),
+                                          (25, 25, 25), (25, 25, 400)])
+def test_window_prefill_matches_sdpa_with_the_band_mask(Sq, Sk, window):
+    B, Hq, Hkv, D = 2, 6, 2, 16
+    q, k, v = rnd((B, Sq, Hq, D), 300 + Sq, 2.0), rnd((B, Sk, Hkv, D), 301 + Sk, 2.0), \
+        rnd((B, Sk, Hkv, D), 302)
+    O, L = oracle.attention(q, k, v, scale=0.3, causal=True, window=window)
+    Or, Lr = masked_sdpa(q, k, v, 0.3, band_mask(Sq, Sk, window))
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isneginf(L), np.isneginf(Lr))
+    fin = np.isfinite(Lr)
+    np.testing.assert_allclose(L[fin], Lr[fin], rtol=0, atol=1e-12)
+
+
+def test_window_of_one_returns_the_diagonal_value():
+    # one visible key per row: its value unchanged, L its logit (closed form)
+    B, Hq, Hkv, Sq, Sk, D = 2, 4, 2, 9, 13, 8
+    q, k, v = rnd((B, Sq, Hq, D), 310), rnd((B, Sk, Hkv, D), 311), rnd((B, Sk, Hkv, D), 312)
+    O, L = oracle.attention(q, k, v, scale=0.7, causal=True, window=1)
+    for b in range(B):
+        for h in range(Hq):
+            c = h // (Hq // Hkv)
+            for i in range(Sq):
+                j = i + Sk - Sq
+                np.testing.assert_array_equal(O[b, i, h], v[b, j, c].astype(np.float64))
+                expect = 0.7 * float(np.dot(q[b, i, h].astype(np.float64),
+                                            k[b, j, c].astype(np.float64)))
+                assert abs(L[b, h, i] - expect) < 1e-12
+
+
+def test_window_covering_every_key_is_causal_attention():
+    B, Hq, Hkv, Sq, Sk, D = 2, 8, 2, 30, 45, 16
+    q, k, v = rnd((B, Sq, Hq, D), 320), rnd((B, Sk, Hkv, D), 321), rnd((B, Sk, Hkv, D), 322)
+    O, L = oracle.attention(q, k, v, scale=0.25, causal=True, window=Sk)
+    Or, Lr = sdpa_ref(q, k, v, 0.25, True, bottom_right=True)
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, Lr, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", [1, 6, 31])
+def test_window_last_row_equals_the_decode_window(window):
+    # the newest query of a windowed prefill (Sq = Sk) is the decode step with that window
+    B, Hq, Hkv, S, D = 3, 8, 4, 31, 16
+    q, k, v = rnd((B, S, Hq, D), 330), rnd((B, S, Hkv, D), 331), rnd((B, S, Hkv, D), 332)
+    O, L = oracle.attention(q, k, v, scale=0.4, causal=True, window=window)
+    Od, Ld = oracle.decode_kvcache(np.ascontiguousarray(q[:, -1:]), k, v, scale=0.4,
+                                   window=window)
+    np.testing.assert_allclose(O[:, -1], Od, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(L[:, :, -1], Ld, rtol=0, atol=1e-13)
+
+
+def brute_force_window(q, k, v, scale, window):
+    mpmath.mp.dps = 50
+    B, Sq, Hq, D = q.shape
+    _, Sk, Hkv, _ = k.shape
+    O = np.zeros(q.shape)
+    L = np.zeros((B, Hq, Sq))
+    for b in range(B):
+        for h in range(Hq):
+            c = h // (Hq // Hkv)
+            for i in range(Sq):
+                top = i + Sk - Sq
+                vis = [j for j in range(Sk) if top - window < j <= top]
+                if not vis:
+                    L[b, h, i] = -np.inf
+                    continue
+                e = [mpmath.exp(mpmath.mpf(scale) * mpmath.fsum(
+                    mpmath.mpf(float(q[b, i, h, d])) * mpmath.mpf(float(k[b, j, c, d]))
+                    for d in range(D))) for j in vis]
+                z = mpmath.fsum(e)
+                for d in range(D):
+                    O[b, i, h, d] = float(mpmath.fsum(e[t] * mpmath.mpf(float(v[b, j, c, d]))
+                                                      for t, j in enumerate(vis)) / z)
+                L[b, h, i] = float(mpmath.log(z))
+    return O, L
+
+
+def test_window_brute_force_50_digits():
+    q, k, v = rnd((1, 6, 4, 3), 340, 3.0), rnd((1, 8, 2, 3), 341, 3.0), rnd((1, 8, 2, 3), 342)
+    O, L = oracle.attention(q, k, v, scale=1.1, causal=True, window=3)
+    Ob, Lb = brute_force_window(q, k, v, 1.1, 3)
+    assert np.max(np.abs(O - Ob)) < 1e-13
+    assert np.max(np.abs(L - Lb)) < 1e-13
+
+
+def test_window_varlen_and_rows_agree_with_the_dense_form():
+    lens = [9, 0, 23, 1, 40]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total, Hq, Hkv, D = int(cu[-1]), 4, 2, 8
+    q, k, v = rnd((total, Hq, D), 350), rnd((total, Hkv, D), 351), rnd((total, Hkv, D), 352)
+    O, L = oracle.attention(q, k, v, scale=0.5, causal=True, cu_seqlens=cu, window=6)
+    for b, n in enumerate(lens):
+        if n == 0:
+            continue
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        Ob, Lb = oracle.attention(q[sl][None], k[sl][None], v[sl][None], scale=0.5,
+                                  causal=True, window=6)
+        np.testing.assert_array_equal(O[sl], Ob[0])
+        np.testing.assert_array_equal(L[:, sl], Lb[0])
+    rows = np.array([[2, 1, 22], [4, 3, 0], [0, 0, 8], [4, 2, 39]], dtype=np.int32)
+    Or, Lr = oracle.attention_rows(q, k, v, rows, scale=0.5, causal=True, cu_seqlens=cu,
+                                   window=6)
+    for r, (b, h, i) in enumerate(rows):
+        np.testing.assert_array_equal(Or[r], O[cu[b] + i, h])
+        assert Lr[r] == L[h, cu[b] + i]
+
+
+def test_window_needs_causal():
+    q, k, v = rnd((1, 4, 2, 8), 360), rnd((1, 4, 1, 8), 361), rnd((1, 4, 1, 8), 362)
+    with pytest.raises(ValueError):
+        oracle.attention(q, k, v, scale=0.5, causal=False, window=2)
+
+
 def random_pattern(n_q, n_k, seed, density=0.35, empty_rows=()):
     rng = np.random.default_rng(seed)
     rows = []
@@ -598,6 +720,34 @@ def test_blocksparse_with_every_block_is_dense_attention():
     np.testing.assert_allclose(L, Lr, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("Sq,Sk,blk,seed", [(300, 300, 128, 4), (96, 120, 16, 5), (70, 40, 8, 6)])
+def test_causal_blocksparse_matches_sdpa_with_pattern_and_causal_mask(Sq, Sk, blk, seed):
+    B, Hq, Hkv, D = 2, 8, 2, 16
+    q, k, v = rnd((B, Sq, Hq, D), seed), rnd((B, Sk, Hkv, D), seed + 10), \
+        rnd((B, Sk, Hkv, D), seed + 20)
+    n_q, n_k = -(-Sq // blk), -(-Sk // blk)
+    row_ptr, col = random_pattern(n_q, n_k, seed, density=0.5)
+    O, L = oracle.attention_blocksparse(q, k, v, row_ptr, col, scale=0.3, blk=blk, causal=True)
+    mask = expand_pattern(row_ptr, col, Sq, Sk, blk) & band_mask(Sq, Sk, Sk + Sq)
+    Or, Lr = masked_sdpa(q, k, v, 0.3, mask)
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+    assert np.array_equal(np.isneginf(L), np.isneginf(Lr))
+    fin = np.isfinite(Lr)
+    np.testing.assert_allclose(L[fin], Lr[fin], rtol=0, atol=1e-12)
+
+
+def test_causal_blocksparse_with_every_block_is_causal_attention():
+    B, Hq, Hkv, Sq, Sk, D = 1, 4, 2, 70, 90, 8
+    q, k, v = rnd((B, Sq, Hq, D), 33), rnd((B, Sk, Hkv, D), 34), rnd((B, Sk, Hkv, D), 35)
+    n_q, n_k = -(-Sq // 16), -(-Sk // 16)
+    row_ptr = np.arange(n_q + 1, dtype=np.int32) * n_k
+    col = np.tile(np.arange(n_k, dtype=np.int32), n_q)
+    O, L = oracle.attention_blocksparse(q, k, v, row_ptr, col, scale=0.5, blk=16, causal=True)
+    Or, Lr = sdpa_ref(q, k, v, 0.5, True, bottom_right=True)
+    np.testing.assert_allclose(O, Or, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L, Lr, rtol=0, atol=1e-12)
+
+
 def test_blocksparse_rejects_bad_patterns():
     q, k, v = rnd((1, 20, 2, 4), 40), rnd((1, 20, 1, 4), 41), rnd((1, 20, 1, 4), 42)
     with pytest.raises(ValueError):  # key block 3 does not exist for 20 keys in blocks of 8
@@ -661,6 +811,37 @@ def test_blocksparse_varlen_equals_the_dense_form_per_sequence():
             np.testing.assert_allclose(O[sl], Od[0], rtol=0, atol=1e-13)
             np.testing.assert_allclose(L[:, sl], Ld[0], rtol=0, atol=1e-13)
         row0 += nb
+
+
+def test_causal_blocksparse_varlen_equals_the_causal_dense_form_per_sequence():
+    blk = 16
+    lens = [37, 0, 64, 5, 90]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total, Hq, Hkv, D = int(cu[-1]), 4, 2, 8
+    q, k, v = rnd((total, Hq, D), 370), rnd((total, Hkv, D), 371), rnd((total, Hkv, D), 372)
+    rps, cols, r0 = [np.zeros(1, dtype=np.int32)], [], 0
+    parts = []
+    for b, n in enumerate(lens):
+        nb = -(-n // blk)
+        rp, cl = random_pattern(nb, nb, 380 + b, density=0.6) if nb else \
+            (np.zeros(1, dtype=np.int32), np.zeros(0, dtype=np.int32))
+        parts.append((rp, cl))
+        rps.append(rp[1:] + r0)
+        cols.append(cl)
+        r0 += int(rp[-1])
+    row_ptr = np.concatenate(rps).astype(np.int32)
+    col = np.concatenate(cols).astype(np.int32)
+    O, L = oracle.attention_blocksparse_varlen(q, k, v, cu, row_ptr, col, scale=0.4, blk=blk,
+                                               causal=True)
+    for b, n in enumerate(lens):
+        if n == 0:
+            continue
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        rp, cl = parts[b]
+        Ob, Lb = oracle.attention_blocksparse(q[sl][None], k[sl][None], v[sl][None], rp, cl,
+                                              scale=0.4, blk=blk, causal=True)
+        np.testing.assert_array_equal(O[sl], Ob[0])
+        np.testing.assert_array_equal(L[:, sl], Lb[0])
 
 
 def test_blocksparse_varlen_rejects_blocks_of_other_sequences():
@@ -830,6 +1011,8 @@ PIN_BATTERY = [
     lambda: test_backward_matches_torch_autograd_float64(2, 8, 2, 33, 33, 16, True),
     lambda: test_e4m3_prefill_matches_sdpa_on_torch_decoded_values(2, 8, 2, 33, 33, 16, True),
     lambda: test_blocksparse_varlen_matches_sdpa_per_sequence(16, 90),
+    lambda: test_window_prefill_matches_sdpa_with_the_band_mask(33, 70, 16),
+    lambda: test_causal_blocksparse_matches_sdpa_with_pattern_and_causal_mask(96, 120, 16, 5),
 ]
 
 
