@@ -195,6 +195,8 @@ def workload_by_name(name: str):
         return W.LLAMA
     if name == "llama_stress":
         return W.LLAMA_STRESS
+    if name == "llama_window":
+        return W.LLAMA_WINDOW
     if name == "varlen":
         return W.VARLEN
     if name == "bigbird":
@@ -322,7 +324,7 @@ class Case:
         else:
             q, k, v = W.make_qkv(w, device=device)
             self.q, self.kv = q, [(k, v)]
-            self.flops = W.attention_flops(w.B, w.Hq, w.Sq, w.Sk, w.D, w.causal)
+            self.flops = W.attention_flops(w.B, w.Hq, w.Sq, w.Sk, w.D, w.causal, w.window)
             self.units, self.unit = self.flops / 1e12, "TFLOP/s"
             self.launches_per_step = 1
             self.kernel = "prefill_fwd_sm100"
@@ -385,6 +387,8 @@ class Case:
                                     pack_gqa=w.pack_gqa, out=self.out, lse=self.lse)
             return
         kw = dict(causal=w.causal, out=self.out, lse=self.lse, pack_gqa=w.pack_gqa)
+        if w.window:
+            kw["window"] = w.window
         if self.decode:
             kw["num_splits"] = w.num_splits
         if self.varlen:
@@ -554,12 +558,15 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
         def flops(rows):
             if not w.causal:
                 return len(rows) * 4 * w.D * w.Sk
-            return int(sum(4 * w.D * min(w.Sk, i + w.Sk - w.Sq + 1) for _, _, i in rows))
+            lim = w.window if w.window > 0 else w.Sk
+            return int(sum(4 * w.D * max(0, min(lim, i + w.Sk - w.Sq + 1))
+                           for _, _, i in rows))
     n, el, done, nrows = 64, 0.0, 0, 0
     while el < target_s and el < max_s:
         rows = rows_of(n)
         t0 = time.perf_counter()
-        oracle.attention_rows(q, k, v, rows, scale=w.scale, causal=w.causal, cu_seqlens=cu)
+        oracle.attention_rows(q, k, v, rows, scale=w.scale, causal=w.causal, cu_seqlens=cu,
+                              window=w.window)
         el += time.perf_counter() - t0
         done += flops(rows)
         nrows += n
@@ -582,6 +589,9 @@ def workload_config(w) -> dict:
     if w.page_size:
         cfg["page_size"] = w.page_size
         cfg["block_table"] = "seeded shuffle of the page pool"
+    if w.window:
+        cfg["window"] = w.window
+        cfg["flops"] = "4 D per (query, key) pair inside the causal window"
     return cfg
 
 
@@ -741,6 +751,13 @@ def run_ours(args, world, rank, local):
             ho.copy_(case.out, non_blocking=True)
             hl.copy_(case.lse, non_blocking=True)
             return
+        if w.window:
+            for d, h in ((dq, hq), (dk, hk), (dv, hv)):
+                d.copy_(h, non_blocking=True)
+            G.gqa_attn(dq, dk, dv, causal=True, window=w.window, out=case.out, lse=case.lse)
+            ho.copy_(case.out, non_blocking=True)
+            hl.copy_(case.lse, non_blocking=True)
+            return
         if not case.varlen:
             # the public host-buffer entry point: batch chunks with copy in, attention and
             # copy out overlapped on the library's streams
@@ -861,6 +878,8 @@ def run_ours(args, world, rank, local):
                              "the block pattern; results copied back" if w.block_sparse else
                              "gqa_attn_kvcache on the e4m3 cache after pinned host copies "
                              "of q and the caches; results copied back" if w.kv_fp8 else
+                             "gqa_attn(window=...) after pinned host copies of q, k, v; "
+                             "results copied back" if w.window else
                              "gqa_attn_kvcache on the paged cache after pinned host "
                              "copies of q, the page pools, the block table and the lengths; "
                              "results copied back" if case.paged else

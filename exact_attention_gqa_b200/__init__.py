@@ -114,11 +114,13 @@ def _workspace(torch, device, nbytes):
 
 def gqa_attn(q, k, v, *, causal: bool = False, scale: float | None = None,
              num_splits: int = 1, pack_gqa: int = -1, cu_seqlens=None, max_seqlen=None,
-             out=None, lse=None):
+             window: int = 0, out=None, lse=None):
     """Exact attention forward with grouped-query heads on the current CUDA stream.
 
     Returns (out, lse).  bf16 inputs run the sm_100a kernels, fp32 inputs the fp32
     path.  ``scale`` defaults to 1/sqrt(D) (FlashAttention's softmax_scale=None).
+    ``window`` > 0 (bf16, causal) limits each query to its `window` most recent keys
+    (gqa_attn_fwd_window).
     """
     import torch
 
@@ -157,6 +159,17 @@ def gqa_attn(q, k, v, *, causal: bool = False, scale: float | None = None,
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    if window:
+        if not causal or window < 1 or q.dtype != torch.bfloat16 or num_splits not in (0, 1):
+            raise ValueError("a sliding window needs causal=True, window >= 1, bf16 inputs "
+                             "and no split count")
+        with torch.cuda.device(q.device):
+            rc = _capi.load().gqa_attn_fwd_window(
+                _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
+                int(window), pack_gqa, _ptr(cu), _stream_handle(torch, q.device))
+        if rc != 0:
+            raise GqaError("gqa_attn_fwd_window", rc)
+        return out, lse
     with torch.cuda.device(q.device):  # the library works on the current device
         _call(torch, q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, num_splits,
               pack_gqa, varlen, cu)
@@ -274,7 +287,8 @@ def gqa_attn_blocksparse_varlen_plan(cu_seqlens, blk_row_ptr, *, Hq: int, Hkv: i
 
 def gqa_attn_blocksparse_varlen(q, k, v, cu_seqlens, blk_row_ptr, blk_col, *,
                                 max_seqlen: int, plan=None, balance: bool = True,
-                                scale: float | None = None, out=None, lse=None):
+                                causal: bool = False, scale: float | None = None, out=None,
+                                lse=None):
     """Block-sparse attention over packed sequences with minimum padding
     (gqa_attn_fwd_blocksparse_varlen).
 
@@ -283,7 +297,8 @@ def gqa_attn_blocksparse_varlen(q, k, v, cu_seqlens, blk_row_ptr, blk_col, *,
     pattern row per 128-position block of each sequence in order, col entries counting
     the sequence's own key blocks.  `plan` (gqa_attn_blocksparse_varlen_plan) is built
     here when not given; balance=True orders the tiles by the library's host schedule
-    (longest first onto the least loaded CTA).  Returns (out, lse [Hq, total])."""
+    (longest first onto the least loaded CTA); causal=True also masks keys after each
+    query within the listed blocks.  Returns (out, lse [Hq, total])."""
     import torch
 
     for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens", cu_seqlens),
@@ -317,7 +332,7 @@ def gqa_attn_blocksparse_varlen(q, k, v, cu_seqlens, blk_row_ptr, blk_col, *,
         rc = lib.gqa_attn_fwd_blocksparse_varlen(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
             _ptr(plan.blk_off), B, Hq, Hkv, int(max_seqlen), total, D, scale,
-            _ptr(blk_row_ptr), _ptr(blk_col), None if plan.order is None else _ptr(plan.order),
+            int(bool(causal)), _ptr(blk_row_ptr), _ptr(blk_col), None if plan.order is None else _ptr(plan.order),
             plan.n_order, plan.grid, _stream_handle(torch, q.device))
     if rc != 0:
         raise GqaError("gqa_attn_fwd_blocksparse_varlen", rc)
@@ -373,9 +388,10 @@ def gqa_attn_backward(q, k, v, out, lse, dout, *, causal: bool = False,
     return dq, dk, dv
 
 
-def gqa_attn_blocksparse(q, k, v, blk_row_ptr, blk_col, *, scale: float | None = None,
-                         out=None, lse=None):
-    """Non-causal attention restricted to a block pattern (gqa_attn_fwd_blocksparse).
+def gqa_attn_blocksparse(q, k, v, blk_row_ptr, blk_col, *, causal: bool = False,
+                         scale: float | None = None, out=None, lse=None):
+    """Attention restricted to a block pattern (gqa_attn_fwd_blocksparse), optionally
+    also causal.
 
     q [B, Sq, Hq, D], k/v [B, Sk, Hkv, D] bf16 (Hq / Hkv >= 2 and dividing 128);
     blk_row_ptr int32 [ceil(Sq / 128) + 1] and blk_col int32 [nnz] on the GPU: the
@@ -408,7 +424,7 @@ def gqa_attn_blocksparse(q, k, v, blk_row_ptr, blk_col, *, scale: float | None =
     with torch.cuda.device(q.device):
         rc = _capi.load().gqa_attn_fwd_blocksparse(
             _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, scale,
-            _ptr(blk_row_ptr), _ptr(col), _stream_handle(torch, q.device))
+            int(bool(causal)), _ptr(blk_row_ptr), _ptr(col), _stream_handle(torch, q.device))
     if rc != 0:
         raise GqaError("gqa_attn_fwd_blocksparse", rc)
     return out, lse

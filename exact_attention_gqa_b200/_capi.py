@@ -32,6 +32,7 @@ EXPORTS = (
     "gqa_attn_decode_paged",
     "gqa_attn_decode_fp8",
     "gqa_attn_selftest_timeout",
+    "gqa_attn_fwd_window",
 )
 
 STATUS = {
@@ -84,15 +85,17 @@ def load() -> ctypes.CDLL:
     lib.gqa_attn_bwd_workspace_bytes.restype = Z
     lib.gqa_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
     lib.gqa_attn_bwd.restype = I
-    lib.gqa_attn_fwd_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P]
+    lib.gqa_attn_fwd_blocksparse.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, P, P, P]
     lib.gqa_attn_fwd_blocksparse.restype = I
     lib.gqa_attn_fwd_blocksparse_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F,
-                                                    P, P, P, I, I, P]
+                                                    I, P, P, P, I, I, P]
     lib.gqa_attn_fwd_blocksparse_varlen.restype = I
     lib.gqa_attn_sparse_varlen_schedule.argtypes = [P, P, I, I, I, I, I, P, P, I, IP, IP]
     lib.gqa_attn_sparse_varlen_schedule.restype = I
     lib.gqa_attn_fwd_fp8.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, F, F, F, I, P, P]
     lib.gqa_attn_fwd_fp8.restype = I
+    lib.gqa_attn_fwd_window.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, P, P]
+    lib.gqa_attn_fwd_window.restype = I
     lib.gqa_attn_decode_kvcache.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, P]
     lib.gqa_attn_decode_kvcache.restype = I
     lib.gqa_attn_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, I,

@@ -229,7 +229,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
                    const int* blk_row_ptr = nullptr, const int* blk_col = nullptr,
                    const int* blk_off = nullptr, const int* tile_order = nullptr,
                    int n_order = 0, int order_grid = 0, float qk_scale = 1.f,
-                   float o_scale = 1.f) {
+                   float o_scale = 1.f, int window = 0) {
     using C = PrefillCfg<HD, FP8>;
     if constexpr (!FP8) {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD>, HD == 64 ? 1 : 2,
@@ -277,6 +277,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     p.blk_off = blk_off;
     p.tile_order = tile_order;
     if (tile_order) p.n_units = n_order;  // the balanced order lists every step
+    p.window = window;
     // Row extents of the 3-D views: exactly the rows the caller allocated
     // (packed variable length: Sk carries the packed row count).
     const long long rows_q = cu ? (long long)Sk : (long long)B * Sq;
@@ -302,6 +303,14 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
         if (rc != GQA_OK) return rc;
         gqa::prefill_fwd_sm100<HD, false, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
             tq, tk, tv, to, p);
+        return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+    }
+    if (window > 0) {
+        const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD, false, false, true>,
+                                         HD == 64 ? 1 << 17 : 1 << 18, C::SMEM_BYTES);
+        if (rc != GQA_OK) return rc;
+        gqa::prefill_fwd_sm100<HD, false, false, true>
+            <<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
         return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
     }
     if (blk_row_ptr) {
@@ -713,6 +722,43 @@ int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
                       pack_gqa, cu_seqlens, stream, false);
 }
 
+int gqa_attn_fwd_window(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int window,
+                        int pack_gqa, const int* cu_seqlens, cudaStream_t stream) {
+    const bool varlen = cu_seqlens != nullptr;
+    int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, 1, pack_gqa, varlen, false);
+    if (rc != GQA_OK) return rc;
+    if (window < 1) return GQA_ERR_SHAPE;
+    // a window that holds every key is plain causal attention
+    if (window >= (varlen ? Sq : Sk))
+        return fwd_common(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, 1, 1, pack_gqa,
+                          cu_seqlens, stream, false);
+    if (!varlen && Sq == 1) {
+        // one query: the decode kernel's window over a dense cache of Sk keys
+        KvCacheArgs kv;
+        kv.window = window;
+        return kvcache_common(q, k, v, out, lse, B, Hq, Hkv, Sk, D, Sk, scale, kv, 1, pack_gqa,
+                              stream);
+    }
+    if (B == 0 || Sq == 0) return GQA_OK;
+    if (!q || !k || !v || !out || !lse) return GQA_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        !aligned(lse, 4) || (varlen && !aligned(cu_seqlens, 4)))
+        return GQA_ERR_ALIGN;
+    DeviceInfo* dev = nullptr;
+    rc = device_info(&dev);
+    if (rc != GQA_OK) return rc;
+    Plan pl;
+    make_plan(&pl, B, Hq, Hkv, Sq, Sk, 1, pack_gqa, varlen, dev->sms);
+    if (pl.kernel == kNone) return GQA_OK;
+    return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 1,
+                                          pl.pack, cu_seqlens, dev->sms, stream, nullptr,
+                                          nullptr, nullptr, nullptr, 0, 0, 1.f, 1.f, window)
+                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 1,
+                                         pl.pack, cu_seqlens, dev->sms, stream, nullptr,
+                                         nullptr, nullptr, nullptr, 0, 0, 1.f, 1.f, window);
+}
+
 int gqa_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* out_h,
                       float* lse_h, void* q_d, void* k_d, void* v_d, void* out_d, float* lse_d,
                       int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
@@ -1002,7 +1048,8 @@ int gqa_attn_decode_noalloc(const void* q, const void* k, const void* v, void* o
 
 int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, float* lse,
                              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
-                             const int* blk_row_ptr, const int* blk_col, cudaStream_t stream) {
+                             int causal, const int* blk_row_ptr, const int* blk_col,
+                             cudaStream_t stream) {
     int rc = check_shape(B, Hq, Hkv, Sq, Sk, D, scale, 1, 1, false, false);
     if (rc != GQA_OK) return rc;
     const int G = Hq / Hkv;
@@ -1023,9 +1070,10 @@ int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
             (long long)B * Hq * Sq);
         return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
     }
-    return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 0, 1,
+    const int cz = causal ? 1 : 0;
+    return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, cz, 1,
                                           nullptr, dev->sms, stream, blk_row_ptr, blk_col)
-                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, 0, 1,
+                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, scale, cz, 1,
                                          nullptr, dev->sms, stream, blk_row_ptr, blk_col);
 }
 
@@ -1127,7 +1175,8 @@ int gqa_attn_sparse_varlen_schedule(const int* cu_seqlens, const int* blk_row_pt
 int gqa_attn_fwd_blocksparse_varlen(const void* q, const void* k, const void* v, void* out,
                                     float* lse, const int* cu_seqlens, const int* blk_off,
                                     int B, int Hq, int Hkv, int max_seqlen, int total, int D,
-                                    float scale, const int* blk_row_ptr, const int* blk_col,
+                                    float scale, int causal, const int* blk_row_ptr,
+                                    const int* blk_col,
                                     const int* tile_order, int n_order, int order_grid,
                                     cudaStream_t stream) {
     int rc = check_shape(B, Hq, Hkv, max_seqlen, total, D, scale, 1, 1, true, false);
@@ -1147,11 +1196,11 @@ int gqa_attn_fwd_blocksparse_varlen(const void* q, const void* k, const void* v,
     rc = device_info(&dev);
     if (rc != GQA_OK) return rc;
     return D == 128 ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, max_seqlen, total,
-                                          scale, 0, 1, cu_seqlens, dev->sms, stream,
+                                          scale, causal ? 1 : 0, 1, cu_seqlens, dev->sms, stream,
                                           blk_row_ptr, blk_col, blk_off, tile_order, n_order,
                                           order_grid)
                     : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, max_seqlen, total,
-                                         scale, 0, 1, cu_seqlens, dev->sms, stream,
+                                         scale, causal ? 1 : 0, 1, cu_seqlens, dev->sms, stream,
                                          blk_row_ptr, blk_col, blk_off, tile_order, n_order,
                                          order_grid);
 }

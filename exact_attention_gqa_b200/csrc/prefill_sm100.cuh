@@ -39,6 +39,13 @@
 // a fixed size, several patterns combined): blk_row_ptr / blk_col list, per query block
 // of 128 positions, the 128-key blocks it attends to; a CTA tile (at most 128 positions,
 // PackGQA with G >= 2) lies in one query block and walks that list instead of 0..n-1.
+// With causal set, keys past a row's diagonal are masked inside the listed blocks.
+//
+// Sliding-window form (WINDOW; Ultralytics GQA glossary, "GQA and related techniques":
+// sliding-window attention caps the tokens attended to): causal, and query position i
+// sees only keys (i + Sk - Sq - window, i + Sk - Sq].  Each sub-tile walks its own
+// blocks [jb0, nblk); the K/V stream covers their union, and only blocks that cross the
+// window's lower edge or the diagonal are masked element by element.
 //
 // Online softmax in the log2 domain: s2 = s * scale * log2(e).  The running
 // max used for the exponentials is only raised when a block's max exceeds it by
@@ -79,6 +86,8 @@ struct PrefillParams {
     const int* tile_order = nullptr;
     // e4m3 Q/K/V: O = accumulator * o_scale / l (v_scale over P's range shift)
     float o_scale = 1.f;
+    // sliding window (causal): keys per query, >= 1 (WINDOW instantiation only)
+    int window = 0;
 };
 
 template <int HD, bool FP8 = false>
@@ -136,9 +145,11 @@ struct TileInfo {
     int valid[2];         // sub-tile holds at least one real query row
     int full_blk[2];      // blocks [0, full_blk) need no mask for any row
     int kb0;              // block-sparse: first entry of this tile's row in blk_col
+    int jb0[2];           // sliding window: first block each sub-tile visits (else 0)
+    int lo_full[2];       // sliding window: blocks >= lo_full have no key below a row's window
 };
 
-template <int BN, bool SPARSE = false>
+template <int BN, bool SPARSE = false, bool WINDOW = false>
 __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
     TileInfo ti;
     bool none = false;
@@ -198,6 +209,15 @@ __device__ __forceinline__ TileInfo decode_tile(const PrefillParams& p, int t) {
         ti.nblk[i] = (ti.valid[i] && lim > 0) ? (lim + BN - 1) / BN : 0;
         int first_lim = p.causal ? min(ti.sk, p0 + ti.sk - ti.sq + 1) : ti.sk;
         ti.full_blk[i] = first_lim > 0 ? first_lim / BN : 0;
+        ti.jb0[i] = 0;
+        ti.lo_full[i] = 0;
+        if constexpr (WINDOW) {
+            // first visible key of the sub-tile's first and last rows
+            const int lo_first = p0 + ti.sk - ti.sq - p.window + 1;
+            const int lo_last = last + ti.sk - ti.sq - p.window + 1;
+            ti.jb0[i] = (ti.nblk[i] > 0 && lo_first > 0) ? min(lo_first / BN, ti.nblk[i]) : 0;
+            ti.lo_full[i] = lo_last > 0 ? (lo_last + BN - 1) / BN : 0;
+        }
     }
     ti.kb0 = 0;
     if constexpr (SPARSE) {
@@ -243,7 +263,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 
 // SPARSE = true walks the block pattern of p.blk_row_ptr / p.blk_col; the dense
 // instantiation carries none of that code.
-template <int HD, bool SPARSE = false, bool FP8 = false>
+template <int HD, bool SPARSE = false, bool FP8 = false, bool WINDOW = false>
 __global__ void __launch_bounds__(320, 1)
     prefill_fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -319,7 +339,7 @@ __global__ void __launch_bounds__(320, 1)
             uint8_t* sV = smem + C::OFF_V;
             int qc = 0, kc = 0, vc = 0;
             for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
-                const TileInfo ti = decode_tile<BN, SPARSE>(p, t);
+                const TileInfo ti = decode_tile<BN, SPARSE, WINDOW>(p, t);
                 const int n = max(ti.nblk[0], ti.nblk[1]);
                 if (n == 0) continue;
                 const int qs = qc % QS;
@@ -339,7 +359,10 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 ++qc;
                 const int kvh = p.pack ? ti.hu : ti.hu / p.G;
-                for (int j = 0; j < n; ++j) {
+                // the blocks the sub-tiles visit: [0, n), or with a window the union of
+                // their ranges (sub-tile 0 holds the earlier positions)
+                const int jmin = WINDOW ? (ti.nblk[0] > 0 ? ti.jb0[0] : ti.jb0[1]) : 0;
+                for (int j = jmin; j < n; ++j) {
                     const int z = ti.k_row0 + sparse_block<SPARSE>(p, ti, j) * BN;
                     {
                         const int s = kc % ST;
@@ -415,81 +438,161 @@ __global__ void __launch_bounds__(320, 1)
                     umma_ts(tmem + C::o_col(i), tmem + C::p_col(i) + kk * 8, b, idesc_o, acc);
             };
             for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
-                const TileInfo ti = decode_tile<BN, SPARSE>(p, t);
+                const TileInfo ti = decode_tile<BN, SPARSE, WINDOW>(p, t);
                 const int n = max(ti.nblk[0], ti.nblk[1]);
                 if (n == 0) continue;
                 const int qs = qc % QS;
                 if (!mbar_wait(bar_q_full + qs, (qc / QS) & 1, abort_flag)) goto mma_done;
                 ++qc;
                 const uint64_t dq = dq0 + uint64_t((qs * C::Q_TILE) >> 4);
-                {
-                    const int s = kc % ST;
-                    if (!mbar_wait(bar_k_full + s, (kc / ST) & 1, abort_flag)) goto mma_done;
-                    tc_fence_after();
-                    const uint64_t dk = dk0 + uint64_t((s * C::KV_TILE) >> 4);
+                if constexpr (WINDOW) {
+                    // sub-tile i visits blocks [jb0[i], nblk[i]); the stream covers their
+                    // union [jmin, n), and every streamed block is released (a block in a
+                    // gap between the two ranges is waited for and handed back unused)
+                    const int jmin = ti.nblk[0] > 0 ? ti.jb0[0] : ti.jb0[1];
+                    {
+                        const int s = kc % ST;
+                        if (!mbar_wait(bar_k_full + s, (kc / ST) & 1, abort_flag)) goto mma_done;
+                        tc_fence_after();
+                        const uint64_t dk = dk0 + uint64_t((s * C::KV_TILE) >> 4);
 #pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        if (ti.nblk[i] > 0) {
-                            const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
+                        for (int i = 0; i < 2; ++i)
+                            if (ti.nblk[i] > jmin && ti.jb0[i] == jmin) {
+                                const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
 #pragma unroll
-                            for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
-                            umma_commit(bar_s_full + i);
-                        }
-                    umma_commit(bar_k_empty + s);
-                    ++kc;
-                }
-                for (int j = 0; j < n; ++j) {
-                    const int sv = vc % ST;
-                    if (!mbar_wait(bar_v_full + sv, (vc / ST) & 1, abort_flag)) goto mma_done;
-                    tc_fence_after();
-                    const uint64_t dv = dv0 + uint64_t((sv * C::KV_TILE) >> 4);
-                    int sk_next = -1;
-                    uint64_t dk = 0;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        if (j >= ti.nblk[i]) continue;
-                        const bool more = j + 1 < ti.nblk[i];
-                        if (more && sk_next < 0) {
+                                for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                umma_commit(bar_s_full + i);
+                            }
+                        umma_commit(bar_k_empty + s);
+                        ++kc;
+                    }
+                    for (int j = jmin; j < n; ++j) {
+                        const int sv = vc % ST;
+                        if (!mbar_wait(bar_v_full + sv, (vc / ST) & 1, abort_flag)) goto mma_done;
+                        tc_fence_after();
+                        const uint64_t dv = dv0 + uint64_t((sv * C::KV_TILE) >> 4);
+                        int sk_next = -1;
+                        uint64_t dk = 0;
+                        if (j + 1 < n) {
                             sk_next = kc % ST;
                             if (!mbar_wait(bar_k_full + sk_next, (kc / ST) & 1, abort_flag))
                                 goto mma_done;
                             dk = dk0 + uint64_t((sk_next * C::KV_TILE) >> 4);
                         }
-                        if (!mbar_wait(bar_p_full + i, p_phase[i], abort_flag)) goto mma_done;
-                        p_phase[i] ^= 1;
-                        tc_fence_after();
-                        // When P has its own columns (D = 64), S_i(j+1) = Q_i K_{j+1}^T is
-                        // issued before O_i += P_i(j) V_j, since the softmax needs it first;
-                        // when P overlays S, every P.V step must come before S(j+1)
-                        // overwrites those columns.  o_done_i is committed after every P.V:
-                        // the softmax waits for it before it writes P_i(j+1) or rescales O_i.
-                        const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
-                        if constexpr (C::P_OWN) {
-                            // S(j+1) first: the softmax needs it next, P.V(j) only later
-                            if (more) {
 #pragma unroll
-                                for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
-                                umma_commit(bar_s_full + i);
+                        for (int i = 0; i < 2; ++i) {
+                            const bool act = ti.jb0[i] <= j && j < ti.nblk[i];
+                            const bool nxt = ti.jb0[i] <= j + 1 && j + 1 < ti.nblk[i];
+                            if (!act && !nxt) continue;
+                            if (act) {
+                                if (!mbar_wait(bar_p_full + i, p_phase[i], abort_flag))
+                                    goto mma_done;
+                                p_phase[i] ^= 1;
+                                tc_fence_after();
                             }
+                            const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
+                            const bool acc = j > ti.jb0[i];
+                            if constexpr (C::P_OWN) {
+                                if (nxt) {
 #pragma unroll
-                            for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
-                            umma_commit(bar_o_done + i);
-                        } else {
+                                    for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                    umma_commit(bar_s_full + i);
+                                }
+                                if (act) {
 #pragma unroll
-                            for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
-                            umma_commit(bar_o_done + i);
-                            if (more) {
+                                    for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, acc);
+                                    umma_commit(bar_o_done + i);
+                                }
+                            } else {
+                                if (act) {
 #pragma unroll
-                                for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
-                                umma_commit(bar_s_full + i);
+                                    for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, acc);
+                                    umma_commit(bar_o_done + i);
+                                }
+                                if (nxt) {
+#pragma unroll
+                                    for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                    umma_commit(bar_s_full + i);
+                                }
                             }
                         }
+                        umma_commit(bar_v_empty + sv);
+                        ++vc;
+                        if (sk_next >= 0) {
+                            umma_commit(bar_k_empty + sk_next);
+                            ++kc;
+                        }
                     }
-                    umma_commit(bar_v_empty + sv);
-                    ++vc;
-                    if (sk_next >= 0) {
-                        umma_commit(bar_k_empty + sk_next);
+                } else {
+                    {
+                        const int s = kc % ST;
+                        if (!mbar_wait(bar_k_full + s, (kc / ST) & 1, abort_flag)) goto mma_done;
+                        tc_fence_after();
+                        const uint64_t dk = dk0 + uint64_t((s * C::KV_TILE) >> 4);
+    #pragma unroll
+                        for (int i = 0; i < 2; ++i)
+                            if (ti.nblk[i] > 0) {
+                                const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
+    #pragma unroll
+                                for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                umma_commit(bar_s_full + i);
+                            }
+                        umma_commit(bar_k_empty + s);
                         ++kc;
+                    }
+                    for (int j = 0; j < n; ++j) {
+                        const int sv = vc % ST;
+                        if (!mbar_wait(bar_v_full + sv, (vc / ST) & 1, abort_flag)) goto mma_done;
+                        tc_fence_after();
+                        const uint64_t dv = dv0 + uint64_t((sv * C::KV_TILE) >> 4);
+                        int sk_next = -1;
+                        uint64_t dk = 0;
+    #pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            if (j >= ti.nblk[i]) continue;
+                            const bool more = j + 1 < ti.nblk[i];
+                            if (more && sk_next < 0) {
+                                sk_next = kc % ST;
+                                if (!mbar_wait(bar_k_full + sk_next, (kc / ST) & 1, abort_flag))
+                                    goto mma_done;
+                                dk = dk0 + uint64_t((sk_next * C::KV_TILE) >> 4);
+                            }
+                            if (!mbar_wait(bar_p_full + i, p_phase[i], abort_flag)) goto mma_done;
+                            p_phase[i] ^= 1;
+                            tc_fence_after();
+                            // When P has its own columns (D = 64), S_i(j+1) = Q_i K_{j+1}^T is
+                            // issued before O_i += P_i(j) V_j, since the softmax needs it first;
+                            // when P overlays S, every P.V step must come before S(j+1)
+                            // overwrites those columns.  o_done_i is committed after every P.V:
+                            // the softmax waits for it before it writes P_i(j+1) or rescales O_i.
+                            const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
+                            if constexpr (C::P_OWN) {
+                                // S(j+1) first: the softmax needs it next, P.V(j) only later
+                                if (more) {
+    #pragma unroll
+                                    for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                    umma_commit(bar_s_full + i);
+                                }
+    #pragma unroll
+                                for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
+                                umma_commit(bar_o_done + i);
+                            } else {
+    #pragma unroll
+                                for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
+                                umma_commit(bar_o_done + i);
+                                if (more) {
+    #pragma unroll
+                                    for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
+                                    umma_commit(bar_s_full + i);
+                                }
+                            }
+                        }
+                        umma_commit(bar_v_empty + sv);
+                        ++vc;
+                        if (sk_next >= 0) {
+                            umma_commit(bar_k_empty + sk_next);
+                            ++kc;
+                        }
                     }
                 }
                 umma_commit(bar_q_empty + qs);
@@ -512,12 +615,16 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t s_phase = 0, o_phase = 0;
         uint32_t ec = 0;  // O stores issued through the shared-memory box
         for (int t = blockIdx.x; t < p.n_units; t += gridDim.x) {
-            const TileInfo ti = decode_tile<BN, SPARSE>(p, t);
+            const TileInfo ti = decode_tile<BN, SPARSE, WINDOW>(p, t);
             // this warp's sub-tile, selected without runtime array indexing
             const int my_valid = i ? ti.valid[1] : ti.valid[0];
             const int my_p0 = i ? ti.p0[1] : ti.p0[0];
             const int nb = i ? ti.nblk[1] : ti.nblk[0];
             const int my_full = i ? ti.full_blk[1] : ti.full_blk[0];
+            // sliding window: this sub-tile's first block, and the blocks below lo_full
+            // that hold keys under some row's window
+            const int my_jb0 = WINDOW ? (i ? ti.jb0[1] : ti.jb0[0]) : 0;
+            const int my_lo_full = WINDOW ? (i ? ti.lo_full[1] : ti.lo_full[0]) : 0;
             if (!my_valid) continue;
             int pos, head;
             if (p.pack) {
@@ -533,8 +640,10 @@ __global__ void __launch_bounds__(320, 1)
                 raise_device_error(kDevBadTile);
             int key_lim = p.causal ? pos + ti.sk - ti.sq + 1 : ti.sk;
             key_lim = min(key_lim, ti.sk);
+            // sliding window: the row's first visible key
+            const int key_lo = WINDOW ? pos + ti.sk - ti.sq - p.window + 1 : 0;
             float m_run = -INFINITY, l_run = 0.f, l_rnd = 0.f;
-            for (int j = 0; j < nb; ++j) {
+            for (int j = my_jb0; j < nb; ++j) {
                 if (!mbar_wait_warp(bar_s_full + i, s_phase, abort_flag)) goto softmax_done;
                 s_phase ^= 1;
                 tc_fence_after();
@@ -551,13 +660,27 @@ __global__ void __launch_bounds__(320, 1)
                     kbj = sparse_block<SPARSE>(p, ti, j);
                     need_mask = (kbj + 1) * BN > key_lim;
                 }
+                if constexpr (WINDOW) {
+                    if (j < my_lo_full) need_mask = true;
+                }
                 if (need_mask) {
                     const int lim = key_lim - kbj * BN;
+                    if constexpr (WINDOW) {
+                        // keys before the row's window as well
+                        const int lo = key_lo - kbj * BN;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c)
+                        for (int c = 0; c < 4; ++c)
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (c * 32 + e >= lim) sr[c][e] = __float_as_uint(-INFINITY);
+                            for (int e = 0; e < 32; ++e)
+                                if (c * 32 + e >= lim || c * 32 + e < lo)
+                                    sr[c][e] = __float_as_uint(-INFINITY);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (c * 32 + e >= lim) sr[c][e] = __float_as_uint(-INFINITY);
+                    }
                 }
                 // block row max: four independent three-input max chains
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
@@ -639,7 +762,7 @@ __global__ void __launch_bounds__(320, 1)
                 if constexpr (HD == 128 && !FP8) sq0 = f2_pack(rq0 + rq2, rq1 + rq3);
                 // P.V(j-1) has finished: it no longer reads P's columns and O holds
                 // every block before j (needed before P is overwritten or O rescaled)
-                if (j > 0) {
+                if (j > my_jb0) {
                     if (!mbar_wait_warp(bar_o_done + i, o_phase, abort_flag)) goto softmax_done;
                     o_phase ^= 1;
                     tc_fence_after();
@@ -659,7 +782,7 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 l_run = l_run * alpha + lsum;
                 l_rnd = l_rnd * alpha + lrnd;
-                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (j > my_jb0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                     const uint64_t al2 = f2_pack(alpha, alpha);
 #pragma unroll 1
                     for (int c = 0; c < HD / 32; ++c) {
@@ -687,7 +810,7 @@ __global__ void __launch_bounds__(320, 1)
             // ---------------------------------------------------------- epilogue
             {
                 const size_t row = size_t(ti.q_row0 + pos) * p.Hq + head;
-                if (nb > 0) {
+                if (nb > my_jb0) {
                     if (!mbar_wait_warp(bar_o_done + i, o_phase, abort_flag)) goto softmax_done;
                     o_phase ^= 1;
                     tc_fence_after();
@@ -711,7 +834,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll 1
                         for (int c = 0; c < HD / 32; ++c) {
                             uint32_t o[32];
-                            if (nb > 0) {
+                            if (nb > my_jb0) {
                                 tmem_ld32(tO + c * 32, o);
                                 tmem_ld_wait();
                                 reg_fence(o);
@@ -749,7 +872,7 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll 1
                 for (int c = 0; c < HD / 32 && !tma_out; ++c) {
                     uint32_t o[32];
-                    if (nb > 0) {
+                    if (nb > my_jb0) {
                         tmem_ld32(tO + c * 32, o);
                         tmem_ld_wait();
                         reg_fence(o);

@@ -247,11 +247,12 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
                  int Sk, int D, float scale, int causal, cudaStream_t stream);
 
 /*
- * Block-sparse attention: gqa_attn_fwd's dense, non-causal forward restricted to a
- * pattern of (query block, key block) pairs with blocks of 128 positions and 128 keys
- * (Raptor-T abstract: BigBird divides the input into blocks of a block size and
- * computes attention between blocks, several patterns combined into one).
- *   key j is visible to query i iff j / 128 is in row i / 128 of the pattern;
+ * Block-sparse attention: gqa_attn_fwd's dense forward restricted to a pattern of
+ * (query block, key block) pairs with blocks of 128 positions and 128 keys (Raptor-T
+ * abstract: BigBird divides the input into blocks of a block size and computes
+ * attention between blocks, several patterns combined into one).
+ *   key j is visible to query i iff j / 128 is in row i / 128 of the pattern and, when
+ *   causal != 0, j <= i + (Sk - Sq) as well (gqa_attn_fwd's causal mask);
  *   blk_row_ptr: device int32 [ceil(Sq / 128) + 1], blk_row_ptr[0] = 0, non-
  *     decreasing; blk_col: device int32 [blk_row_ptr[last]], the key blocks of each
  *     row, in [0, ceil(Sk / 128)) (an entry outside raises device error 2 and block 0
@@ -264,7 +265,24 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
  */
 int gqa_attn_fwd_blocksparse(const void* q, const void* k, const void* v, void* out, float* lse,
                              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale,
-                             const int* blk_row_ptr, const int* blk_col, cudaStream_t stream);
+                             int causal, const int* blk_row_ptr, const int* blk_col,
+                             cudaStream_t stream);
+
+/*
+ * Causal forward within a sliding window (Ultralytics glossary, "GQA and related
+ * techniques": sliding-window attention caps the tokens each token attends to, paired
+ * there with GQA).  Reading taken where the page gives no formula: query i, at key
+ * position i + (Sk - Sq), sees its `window` most recent keys,
+ *   key j visible to query i iff i + (Sk - Sq) - window < j <= i + (Sk - Sq),
+ * the same window as the decode entry points' (the newest query sees the last
+ * `window` keys).  window >= 1 (GQA_ERR_SHAPE otherwise); a window holding every key
+ * is gqa_attn_fwd with causal = 1.  Arguments, layouts (dense or packed with
+ * cu_seqlens), dtypes (bf16), D, pack_gqa and errors as gqa_attn_fwd; one query
+ * (Sq = 1, dense) runs the decode kernel without splits.
+ */
+int gqa_attn_fwd_window(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int window,
+                        int pack_gqa, const int* cu_seqlens, cudaStream_t stream);
 
 /*
  * Prefill forward on e4m3 Q, K and V with one scale per tensor (the batch-size guide
@@ -291,7 +309,7 @@ int gqa_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* out, 
  * attention-balancing algorithm assigns thread-block work by its execution time).
  *   q, out [total, Hq, D], k, v [total, Hkv, D] bf16 packed as gqa_attn_fwd's varlen
  *   form; lse [Hq, total]; cu_seqlens device int32 [B + 1]; self attention within each
- *   sequence, non-causal;
+ *   sequence, causal (key j visible to query i only if j <= i) when causal != 0;
  *   sequence b owns ceil(n_b / 128) query and key blocks (the last one partial);
  *   blk_off device int32 [B + 1]: its first pattern row, the prefix sum of those counts;
  *   blk_row_ptr device int32 [blk_off[B] + 1], blk_col device int32: the CSR pattern,
@@ -306,9 +324,9 @@ int gqa_attn_fwd_fp8(const void* q8, const void* k8, const void* v8, void* out, 
 int gqa_attn_fwd_blocksparse_varlen(const void* q, const void* k, const void* v, void* out,
                                     float* lse, const int* cu_seqlens, const int* blk_off,
                                     int B, int Hq, int Hkv, int max_seqlen, int total, int D,
-                                    float scale, const int* blk_row_ptr, const int* blk_col,
-                                    const int* tile_order, int n_order, int order_grid,
-                                    cudaStream_t stream);
+                                    float scale, int causal, const int* blk_row_ptr,
+                                    const int* blk_col, const int* tile_order, int n_order,
+                                    int order_grid, cudaStream_t stream);
 
 /*
  * Host-side schedule for gqa_attn_fwd_blocksparse_varlen (no device work).  From host

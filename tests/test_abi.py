@@ -240,9 +240,9 @@ def test_fp8_empty_batch_is_a_noop(lib):
 
 
 def sparse_call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=8, Hkv=2, Sq=256,
-                Sk=256, D=128, scale=0.125, rp=FAKE, col=FAKE):
-    return lib.gqa_attn_fwd_blocksparse(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, rp,
-                                        col, None)
+                Sk=256, D=128, scale=0.125, causal=0, rp=FAKE, col=FAKE):
+    return lib.gqa_attn_fwd_blocksparse(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale,
+                                        causal, rp, col, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -262,6 +262,34 @@ def test_blocksparse_argument_errors(lib, kw, code):
 
 def test_blocksparse_empty_batch_is_a_noop(lib):
     assert sparse_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert sparse_call(lib, B=0, causal=1, q=None, k=None, v=None, out=None, lse=None) == 0
+
+
+# ---------------------------------------------------------------- sliding window
+def window_call(lib, *, q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=8, Hkv=2, Sq=256,
+                Sk=256, D=128, scale=0.125, window=64, pack=-1, cu=None):
+    return lib.gqa_attn_fwd_window(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, window,
+                                   pack, cu, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(window=0), "GQA_ERR_SHAPE"),
+    (dict(window=-3), "GQA_ERR_SHAPE"),
+    (dict(Hq=6, Hkv=4), "GQA_ERR_SHAPE"),
+    (dict(D=96), "GQA_ERR_HEADDIM"),
+    (dict(scale=0.0), "GQA_ERR_SCALE"),
+    (dict(pack=2), "GQA_ERR_UNSUPPORTED"),
+    (dict(q=None), "GQA_ERR_NULL"),
+    (dict(k=None), "GQA_ERR_NULL"),
+    (dict(out=ctypes.c_void_p(0x1008)), "GQA_ERR_ALIGN"),
+])
+def test_window_argument_errors(lib, kw, code):
+    assert G.STATUS[window_call(lib, **kw)] == code
+
+
+def test_window_empty_problems_are_noops(lib):
+    assert window_call(lib, B=0, q=None, k=None, v=None, out=None, lse=None) == 0
+    assert window_call(lib, Sq=0, q=None, k=None, v=None, out=None, lse=None) == 0
 
 
 # ---------------------------------------------------------------------------- backward
@@ -400,7 +428,7 @@ def test_blocksparse_varlen_argument_errors(lib):
         a.update(kw)
         return G.STATUS[lib.gqa_attn_fwd_blocksparse_varlen(
             a["q"], a["k"], a["v"], a["out"], a["lse"], a["cu"], a["off"], a["B"], a["Hq"],
-            a["Hkv"], a["S"], a["total"], a["D"], a["scale"], a["rp"], a["col"], a["order"],
+            a["Hkv"], a["S"], a["total"], a["D"], a["scale"], 0, a["rp"], a["col"], a["order"],
             a["n_order"], a["grid"], None)]
     assert call(Hq=8, Hkv=8) == "GQA_ERR_UNSUPPORTED"
     assert call(off=None) == "GQA_ERR_NULL"

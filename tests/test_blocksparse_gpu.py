@@ -104,3 +104,33 @@ def test_full_bigbird_workload():
                                            v[b:b + 1, :, c:c + 1], rp, col, scale=w.scale,
                                            blk=128)
         compare(out[b:b + 1, :, hs], lse[b:b + 1, hs], *ref)
+
+
+# ------------------------------------------------------------------ causal patterns
+@pytest.mark.parametrize("B,Hq,Hkv,Sq,Sk,D", [
+    (2, 8, 2, 700, 700, 128),    # blocks above the diagonal in the pattern: fully masked
+    (1, 16, 2, 500, 900, 64),    # Sq < Sk: the diagonal is shifted (bottom-right)
+    (1, 8, 4, 640, 300, 128),    # Sq > Sk: the first rows see no key at all
+])
+def test_causal_blocksparse_matches_oracle(B, Hq, Hkv, Sq, Sk, D):
+    q, k, v = rand_qkv(B, Hq, Hkv, Sq, Sk, D, seed=Sq + 3 * Sk + D)
+    n_q, n_k = -(-Sq // 128), -(-Sk // 128)
+    rp, col = pattern(n_q, n_k, seed=Sq + 1, density=0.5, empty=(2,))
+    out, lse = gqa_attn_blocksparse(q.to(DEV), k.to(DEV), v.to(DEV), rp.to(DEV), col.to(DEV),
+                                    causal=True)
+    torch.cuda.synchronize()
+    ref = oracle.attention_blocksparse(q, k, v, rp, col, scale=1 / math.sqrt(D), blk=128,
+                                       causal=True)
+    compare(out, lse, *ref)
+
+
+def test_causal_full_pattern_equals_the_causal_dense_kernel():
+    q, k, v = rand_qkv(2, 16, 4, 600, 777, 128, seed=13)
+    n_q, n_k = -(-600 // 128), -(-777 // 128)
+    rp = torch.arange(n_q + 1, dtype=torch.int32) * n_k
+    col = torch.arange(n_k, dtype=torch.int32).repeat(n_q)
+    qd, kd, vd = q.to(DEV), k.to(DEV), v.to(DEV)
+    out, lse = gqa_attn_blocksparse(qd, kd, vd, rp.to(DEV), col.to(DEV), causal=True)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, scale=1 / math.sqrt(128), causal=True)
+    compare(out, lse, *ref)

@@ -86,3 +86,19 @@ def test_full_size_varlen_bigbird_sampled():
         o_ref, l_ref = oracle.attention_blocksparse(q[sl][None], k[sl][None], v[sl][None],
                                                     sub_rp, sub_cl, scale=w.scale)
         compare(out[sl][None], lse[:, sl][None], o_ref, l_ref)
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D", [
+    ([300, 0, 128, 1000, 17, 513], 8, 2, 128),
+    ([129, 256, 700], 8, 4, 64),
+])
+def test_causal_blocksparse_varlen_matches_oracle(lens, Hq, Hkv, D):
+    q, k, v, cu = packed(lens, Hq, Hkv, D, seed=sum(lens) + D + 1)
+    rp, cl = W.bigbird_pattern_varlen(lens, PATTERN, seed=len(lens) + 1)
+    out, lse = gqa_attn_blocksparse_varlen(q.to(DEV), k.to(DEV), v.to(DEV), cu.to(DEV),
+                                           rp.to(DEV), cl.to(DEV), max_seqlen=max(lens),
+                                           causal=True)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle.attention_blocksparse_varlen(q, k, v, cu, rp, cl,
+                                                       scale=1 / math.sqrt(D), causal=True)
+    compare(out, lse, o_ref, l_ref)

@@ -49,6 +49,7 @@ class Workload:
     qkv_fp8: bool = False  # prefill on e4m3 Q, K, V (scale FP8_PREFILL_SCALE each)
     block_sparse: dict = field(default_factory=dict)  # {"window": 3, "global": 2, "random": 3}
     backward: bool = False  # time the backward pass (dQ, dK, dV) of this forward
+    window: int = 0  # > 0: causal attention within a sliding window of this many keys
 
     @property
     def scale(self) -> float:
@@ -79,6 +80,10 @@ LLAMA_BWD_B1 = Workload("llama8b_backward_b1_s8192_causal", B=1, Hq=32, Hkv=8, S
 LLAMA_FP8 = Workload("llama8b_prefill_fp8_b4_s8192_causal", B=4, Hq=32, Hkv=8, Sq=8192,
                      Sk=8192, D=128, dtype="bf16", causal=True, seed=2, qkv_fp8=True)
 FP8_PREFILL_SCALE = 1.0 / 16.0
+# the Llama prefill shape with a 4096-key sliding window (Ultralytics GQA glossary, "GQA
+# and related techniques": sliding-window attention, paired there with GQA in Mistral 7B)
+LLAMA_WINDOW = Workload("llama8b_prefill_b4_s8192_window4096", B=4, Hq=32, Hkv=8, Sq=8192,
+                        Sk=8192, D=128, dtype="bf16", causal=True, seed=2, window=4096)
 LLAMA_STRESS = Workload("llama8b_prefill_b4_s8192_causal_qx4", B=4, Hq=32, Hkv=8, Sq=8192,
                         Sk=8192, D=128, dtype="bf16", causal=True, seed=3, q_mult=4.0)
 DECODE_BATCHES = (1, 16, 64, 128, 256)
@@ -322,9 +327,15 @@ def causal_pairs(Sq: int, Sk: int) -> int:
     return sum(min(max(i + off + 1, 0), Sk) for i in range(Sq))
 
 
-def attention_flops(B: int, Hq: int, Sq: int, Sk: int, D: int, causal: bool) -> int:
-    """4*D flops per visible (query, key) pair per head: 2*D for QK^T, 2*D for PV."""
-    pairs = causal_pairs(Sq, Sk) if causal else Sq * Sk
+def attention_flops(B: int, Hq: int, Sq: int, Sk: int, D: int, causal: bool,
+                    window: int = 0) -> int:
+    """4*D flops per visible (query, key) pair per head: 2*D for QK^T, 2*D for PV.  With a
+    window, query i sees keys (i + Sk - Sq - window, i + Sk - Sq] that exist."""
+    if window > 0:
+        # row i: keys max(0, t - window + 1) .. t with t = i + Sk - Sq (none when t < 0)
+        pairs = sum(max(0, min(i + Sk - Sq + 1, window)) for i in range(Sq))
+    else:
+        pairs = causal_pairs(Sq, Sk) if causal else Sq * Sk
     return 4 * D * pairs * B * Hq
 
 
