@@ -546,7 +546,7 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
             return np.stack([b, rng.integers(0, w.Hq, n), i], axis=1).astype(np.int32)
 
         def flops(rows):
-            return int(sum(4 * w.D * (i + 1) for _, _, i in rows))
+            return sum(4 * w.D * (int(i) + 1) for _, _, i in rows)
     else:
         q, k, v = W.make_qkv(w)
         cu = None
@@ -559,8 +559,11 @@ def oracle_sample(w: W.Workload, target_s: float, max_s: float, seed: int = 0):
             if not w.causal:
                 return len(rows) * 4 * w.D * w.Sk
             lim = w.window if w.window > 0 else w.Sk
-            return int(sum(4 * w.D * max(0, min(lim, i + w.Sk - w.Sq + 1))
-                           for _, _, i in rows))
+            return sum(4 * w.D * max(0, min(lim, int(i) + w.Sk - w.Sq + 1))
+                       for _, _, i in rows)
+    # the inputs widened to float32 once, outside the timed calls (the oracle's own entry
+    # widens a torch tensor on every call, which would dominate the sample's time)
+    q, k, v = (t.float().numpy() for t in (q, k, v))
     n, el, done, nrows = 64, 0.0, 0, 0
     while el < target_s and el < max_s:
         rows = rows_of(n)
