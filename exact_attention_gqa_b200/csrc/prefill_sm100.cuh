@@ -529,11 +529,11 @@ __global__ void __launch_bounds__(320, 1)
                         if (!mbar_wait(bar_k_full + s, (kc / ST) & 1, abort_flag)) goto mma_done;
                         tc_fence_after();
                         const uint64_t dk = dk0 + uint64_t((s * C::KV_TILE) >> 4);
-    #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 2; ++i)
                             if (ti.nblk[i] > 0) {
                                 const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
-    #pragma unroll
+#pragma unroll
                                 for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
                                 umma_commit(bar_s_full + i);
                             }
@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(320, 1)
                         const uint64_t dv = dv0 + uint64_t((sv * C::KV_TILE) >> 4);
                         int sk_next = -1;
                         uint64_t dk = 0;
-    #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 2; ++i) {
                             if (j >= ti.nblk[i]) continue;
                             const bool more = j + 1 < ti.nblk[i];
@@ -569,19 +569,19 @@ __global__ void __launch_bounds__(320, 1)
                             if constexpr (C::P_OWN) {
                                 // S(j+1) first: the softmax needs it next, P.V(j) only later
                                 if (more) {
-    #pragma unroll
+#pragma unroll
                                     for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
                                     umma_commit(bar_s_full + i);
                                 }
-    #pragma unroll
+#pragma unroll
                                 for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
                                 umma_commit(bar_o_done + i);
                             } else {
-    #pragma unroll
+#pragma unroll
                                 for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
                                 umma_commit(bar_o_done + i);
                                 if (more) {
-    #pragma unroll
+#pragma unroll
                                     for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
                                     umma_commit(bar_s_full + i);
                                 }

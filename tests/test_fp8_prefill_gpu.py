@@ -77,3 +77,31 @@ def test_fp8_prefill_uint8_codes_equal_float8_codes():
     b = gqa_attn_fp8(q8.view(torch.uint8).to(DEV), k8.view(torch.uint8).to(DEV),
                      v8.view(torch.uint8).to(DEV), causal=True, **SCALES)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_full_llama_fp8_workload_prefix_and_suffix_rows():
+    """The benchmark's e4m3 workload (Llama shape B=4, Hq=32, Hkv=8, S=8192, causal), whole
+    on the GPU.  Causal rows depend only on the keys up to their own position, so the
+    first 2048 positions of a (batch, KV head) group are exactly the problem cut to 2048
+    positions, and the last 16 positions are the problem of those 16 queries against all
+    8192 keys with bottom-right alignment: both are compared with the oracle, for two
+    groups."""
+    import workloads as W
+    w = W.LLAMA_FP8
+    sc = W.FP8_PREFILL_SCALE
+    q8, k8, v8 = W.make_qkv_e4m3(w)
+    out, lse = gqa_attn_fp8(q8.to(DEV), k8.to(DEV), v8.to(DEV), causal=True, q_scale=sc,
+                            k_scale=sc, v_scale=sc)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    for b, c in ((0, 0), (3, 7)):
+        hs = slice(c * w.G, (c + 1) * w.G)
+        kc, vc = k8[b:b + 1, :, c:c + 1].contiguous(), v8[b:b + 1, :, c:c + 1].contiguous()
+        for rows in (slice(0, 2048), slice(w.Sq - 16, w.Sq)):
+            qs = q8[b:b + 1, rows, hs].contiguous()
+            ks, vs = (kc, vc) if rows.start > 0 else (kc[:, :2048].contiguous(),
+                                                      vc[:, :2048].contiguous())
+            o_ref, l_ref = oracle.attention_e4m3(qs, ks, vs, q_scale=sc, k_scale=sc,
+                                                 v_scale=sc, scale=w.scale, causal=True)
+            model = e4m3_prefill_model(qs, ks, vs, sc, sc, sc, w.scale, True)
+            compare_e4m3(out[b:b + 1, rows, hs], lse[b:b + 1, hs, rows], o_ref, l_ref, model)
