@@ -112,6 +112,12 @@ def test_flop_accounting_counts_visible_pairs():
         assert W.causal_pairs(Sq, Sk) == brute
     assert W.causal_pairs(8192, 8192) == 8192 * 8193 // 2
     assert W.attention_flops(2, 3, 5, 7, 8, False) == 4 * 8 * 5 * 7 * 2 * 3
+    # sliding window: the pairs the oracle's window mask keeps, counted one by one
+    for Sq, Sk, win in [(9, 9, 1), (9, 9, 4), (6, 11, 3), (11, 6, 2), (16, 16, 40)]:
+        brute = int(band_mask(Sq, Sk, win).sum())
+        assert W.attention_flops(1, 1, Sq, Sk, 1, True, window=win) == 4 * brute
+    assert W.attention_flops(1, 1, 64, 64, 1, True, window=64) == \
+        W.attention_flops(1, 1, 64, 64, 1, True)
 
 
 # ---------------------------------------------------------------------------------
