@@ -900,7 +900,9 @@ def run_ours(args, world, rank, local):
                              "copies of q, the page pools, the block table and the lengths; "
                              "results copied back" if case.paged else
                              "gqa_attn_fwd_host" + ("_varlen: 8 chunks of whole sequences"
-                                                    if case.varlen else ": 8 batch chunks")
+                                                    if case.varlen else
+                                                    ": 8 chunks (batch elements, or ranges of "
+                                                    "positions when the batch is smaller)")
                              + ", pinned host buffers, copy in / attention / copy out "
                                "overlapped")},
             "gpu_launches": steps * case.launches_per_step,

@@ -229,7 +229,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
                    const int* blk_row_ptr = nullptr, const int* blk_col = nullptr,
                    const int* blk_off = nullptr, const int* tile_order = nullptr,
                    int n_order = 0, int order_grid = 0, float qk_scale = 1.f,
-                   float o_scale = 1.f, int window = 0) {
+                   float o_scale = 1.f, int window = 0, int lse_ld = 0) {
     using C = PrefillCfg<HD, FP8>;
     if constexpr (!FP8) {
         const int rc = ensure_smem_limit(gqa::prefill_fwd_sm100<HD>, HD == 64 ? 1 : 2,
@@ -278,6 +278,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     p.tile_order = tile_order;
     if (tile_order) p.n_units = n_order;  // the balanced order lists every step
     p.window = window;
+    p.lse_ld = lse_ld > 0 ? lse_ld : Sq;
     // Row extents of the 3-D views: exactly the rows the caller allocated
     // (packed variable length: Sk carries the packed row count).
     const long long rows_q = cu ? (long long)Sk : (long long)B * Sq;
@@ -778,22 +779,90 @@ int gqa_attn_fwd_host(const void* q_h, const void* k_h, const void* v_h, void* o
     Pipe* pp = nullptr;
     rc = pipe_for_device(&pp);
     if (rc != GQA_OK) return rc;
-    // chunks of whole batch elements: [B, S, H, D] and [B, H, S] are batch-major
-    int n = chunks == 0 ? 8 : chunks;
-    if (n > B) n = B;
-    const int per = (B + n - 1) / n;
-    n = (B + per - 1) / per;
+    const int want = chunks == 0 ? 8 : chunks;
     const size_t qb = size_t(Sq) * Hq * D * 2, kb = size_t(Sk) * Hkv * D * 2;
     const size_t lb = size_t(Hq) * Sq * 4;
     auto at = [](const void* base, size_t off) {
         return static_cast<void*>(static_cast<char*>(const_cast<void*>(base)) + off);
     };
+    // Fewer batch elements than chunks: a prefill (not a decode step, keys at least as
+    // many as queries when causal) is cut into ranges of query positions of each batch
+    // element instead.  Queries [s0, s1) see the key prefix [0, e(s1)) (e(s) = s + Sk - Sq
+    // when causal, Sk otherwise), so a chunk copies in only the keys the previous
+    // chunks of its batch element did not, and runs as a problem of its own with
+    // bottom-right alignment: every row computes what the whole launch computes.
+    int per_b = B < want ? (want + B - 1) / B : 1;
+    if (per_b > kMaxChunks / B) per_b = kMaxChunks / B;
+    const bool by_pos = per_b > 1 && Sq >= 512 && Sk > 0 && (!causal || Sq <= Sk);
+    if (by_pos && (!aligned(q_d, 16) || !aligned(k_d, 16) || !aligned(v_d, 16) ||
+                   !aligned(out_d, 16) || !aligned(lse_d, 4)))
+        return GQA_ERR_ALIGN;
     if (cudaEventRecord(pp->start, stream) != cudaSuccess ||
         cudaStreamWaitEvent(pp->s_in, pp->start, 0) != cudaSuccess ||
         cudaStreamWaitEvent(pp->s_c, pp->start, 0) != cudaSuccess ||
         cudaStreamWaitEvent(pp->s_out, pp->start, 0) != cudaSuccess)
         return GQA_ERR_CUDA;
     int status = GQA_OK;
+    if (by_pos) {
+        int len = (Sq + per_b - 1) / per_b;
+        len = (len + 255) / 256 * 256;  // whole 256-row tiles for every group size
+        const int cpb = (Sq + len - 1) / len;  // <= per_b, so B * cpb <= kMaxChunks
+        const size_t qrow = size_t(Hq) * D * 2, krow = size_t(Hkv) * D * 2;
+        for (int b = 0; b < B && status == GQA_OK; ++b) {
+            int kdone = 0;  // keys of batch element b already copied in
+            for (int j = 0; j < cpb && status == GQA_OK; ++j) {
+                const int c = b * cpb + j;
+                const int s0 = j * len, s1 = (s0 + len < Sq) ? s0 + len : Sq;
+                const int kend = causal ? s1 + (Sk - Sq) : Sk;
+                const size_t oq = size_t(b) * qb + size_t(s0) * qrow;
+                const size_t okb = size_t(b) * kb;
+                const size_t ok = okb + size_t(kdone) * krow;
+                const size_t nk = size_t(kend - kdone) * krow;
+                if (cudaMemcpyAsync(at(q_d, oq), at(q_h, oq), size_t(s1 - s0) * qrow,
+                                    cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess ||
+                    (nk && (cudaMemcpyAsync(at(k_d, ok), at(k_h, ok), nk,
+                                            cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess ||
+                            cudaMemcpyAsync(at(v_d, ok), at(v_h, ok), nk,
+                                            cudaMemcpyHostToDevice, pp->s_in) != cudaSuccess)) ||
+                    cudaEventRecord(pp->in_done[c], pp->s_in) != cudaSuccess ||
+                    cudaStreamWaitEvent(pp->s_c, pp->in_done[c], 0) != cudaSuccess) {
+                    status = GQA_ERR_CUDA;
+                    break;
+                }
+                kdone = kend;
+                Plan pl;
+                make_plan(&pl, 1, Hq, Hkv, s1 - s0, kend, 1, pack_gqa, false, dev->sms);
+                float* lse_c = lse_d + size_t(b) * Hq * Sq + s0;
+                status = D == 128
+                             ? launch_prefill<128>(at(q_d, oq), at(k_d, okb), at(v_d, okb),
+                                                   at(out_d, oq), lse_c, 1, Hq, Hkv, s1 - s0,
+                                                   kend, scale, causal, pl.pack, nullptr,
+                                                   dev->sms, pp->s_c, nullptr, nullptr,
+                                                   nullptr, nullptr, 0, 0, 1.f, 1.f, 0, Sq)
+                             : launch_prefill<64>(at(q_d, oq), at(k_d, okb), at(v_d, okb),
+                                                  at(out_d, oq), lse_c, 1, Hq, Hkv, s1 - s0,
+                                                  kend, scale, causal, pl.pack, nullptr,
+                                                  dev->sms, pp->s_c, nullptr, nullptr, nullptr,
+                                                  nullptr, 0, 0, 1.f, 1.f, 0, Sq);
+                if (status != GQA_OK) break;
+                // O rows of the range are contiguous; L is Hq rows of s1 - s0 values
+                float* lse_hc = lse_h + size_t(b) * Hq * Sq + s0;
+                if (cudaEventRecord(pp->c_done[c], pp->s_c) != cudaSuccess ||
+                    cudaStreamWaitEvent(pp->s_out, pp->c_done[c], 0) != cudaSuccess ||
+                    cudaMemcpyAsync(at(out_h, oq), at(out_d, oq), size_t(s1 - s0) * qrow,
+                                    cudaMemcpyDeviceToHost, pp->s_out) != cudaSuccess ||
+                    cudaMemcpy2DAsync(lse_hc, size_t(Sq) * 4, lse_c, size_t(Sq) * 4,
+                                      size_t(s1 - s0) * 4, Hq, cudaMemcpyDeviceToHost,
+                                      pp->s_out) != cudaSuccess)
+                    status = GQA_ERR_CUDA;
+            }
+        }
+    }
+    // otherwise chunks of whole batch elements: [B, S, H, D] and [B, H, S] are batch-major
+    int n = want;
+    if (n > B) n = B;
+    const int per = (B + n - 1) / n;
+    n = by_pos ? 0 : (B + per - 1) / per;
     for (int c = 0; c < n && status == GQA_OK; ++c) {
         const int b0 = c * per, nb = (B - b0 < per) ? B - b0 : per;
         const size_t oq = size_t(b0) * qb, ok = size_t(b0) * kb, ol = size_t(b0) * lb;

@@ -88,6 +88,9 @@ struct PrefillParams {
     float o_scale = 1.f;
     // sliding window (causal): keys per query, >= 1 (WINDOW instantiation only)
     int window = 0;
+    // dense layout: elements between consecutive (batch, head) rows of lse (Sq, or the
+    // full problem's length when a range of positions is computed on its own)
+    int lse_ld = 0;
 };
 
 template <int HD, bool FP8 = false>
@@ -901,7 +904,7 @@ __global__ void __launch_bounds__(320, 1)
                     if (p.cu_seqlens)
                         li = size_t(head) * p.total_rows + ti.q_row0 + pos;
                     else
-                        li = (size_t(ti.b) * p.Hq + head) * p.Sq + pos;
+                        li = (size_t(ti.b) * p.Hq + head) * p.lse_ld + pos;
                     p.lse[li] = L;
                 }
             }

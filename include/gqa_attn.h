@@ -109,10 +109,13 @@ int gqa_attn_fwd_f32(const void* q, const void* k, const void* v, void* out, flo
 
 /*
  * gqa_attn_fwd on inputs and outputs in host memory, with the transfers overlapped:
- * the batch is cut into `chunks` groups of whole batch elements (0 = 8; at most 64,
- * at most B) and, on three streams the library creates once per device, the copy of
- * chunk c+1 to the device, the attention of chunk c and the copy of chunk c-1's
- * results back run at the same time.  Dense only (no cu_seqlens), bf16.
+ * the problem is cut into `chunks` pieces (0 = 8; at most 64) and, on three streams the
+ * library creates once per device, the copy of piece c+1 to the device, the attention
+ * of piece c and the copy of piece c-1's results back run at the same time.  Pieces are
+ * groups of whole batch elements; when the batch has fewer elements than `chunks`, a
+ * prefill (Sq >= 512; causal only with Sq <= Sk) is cut into ranges of query positions
+ * of each batch element instead, each copying in the keys its queries newly see (the
+ * results are those of gqa_attn_fwd, bit for bit).  Dense only (no cu_seqlens), bf16.
  *   q_h, k_h, v_h, out_h, lse_h : host buffers in gqa_attn_fwd's layouts; page-locked
  *                  (cudaHostAlloc / cudaHostRegister) for the copies to overlap
  *   q_d ... lse_d : caller-owned device buffers of the same sizes (the staging area;

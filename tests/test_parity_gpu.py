@@ -128,6 +128,13 @@ def test_decode_sixteen_heads_per_kv_head(splits):
     (4, 16, 4, 257, 513, 128, True, 1, 0),    # default chunking, Sq < Sk
     (6, 32, 8, 1, 3000, 128, False, 4, 4),    # decode, explicit splits per chunk
     (3, 8, 2, 64, 0, 64, True, 1, 2),         # no keys: zeros and -inf come back
+    # fewer batch elements than chunks: ranges of query positions, keys copied as the
+    # causal prefix grows (or all at once without the mask)
+    (1, 8, 2, 2000, 2000, 128, True, 1, 0),   # 8 ranges of 256 positions, ragged last
+    (2, 16, 4, 1100, 1500, 64, True, 1, 6),   # Sq < Sk: the prefix is shifted
+    (3, 8, 8, 700, 900, 128, False, 1, 0),    # non-causal, MHA (no packing)
+    (1, 32, 8, 4096, 4096, 128, True, 1, 64), # 16 ranges
+    (2, 8, 2, 800, 600, 64, True, 1, 8),      # causal Sq > Sk: whole batch elements
 ])
 def test_host_pipeline_equals_device_path(B, Hq, Hkv, Sq, Sk, D, causal, splits, chunks):
     """gqa_attn_fwd_host (inputs and outputs in pinned host memory, chunked and
