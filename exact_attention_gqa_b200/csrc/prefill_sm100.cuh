@@ -273,6 +273,8 @@ __global__ void __launch_bounds__(320, 1)
                       const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
     using C = PrefillCfg<HD, FP8>;
+    // e4m3 P is stored chunk by chunk over S (no wait for P.V(j-1) in the block loop)
+    static_assert(!(FP8 && C::P_OWN), "e4m3 P overlays S");
     constexpr int BN = C::BN;
     constexpr int ST = C::STAGES;
     constexpr int QS = C::Q_STAGES;
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(320, 1)
                                 if (act) {
 #pragma unroll
                                     for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, acc);
-                                    umma_commit(bar_o_done + i);
+                                    if (!nxt) umma_commit(bar_o_done + i);
                                 }
                                 if (nxt) {
 #pragma unroll
@@ -564,10 +566,13 @@ __global__ void __launch_bounds__(320, 1)
                             p_phase[i] ^= 1;
                             tc_fence_after();
                             // When P has its own columns (D = 64), S_i(j+1) = Q_i K_{j+1}^T is
-                            // issued before O_i += P_i(j) V_j, since the softmax needs it first;
-                            // when P overlays S, every P.V step must come before S(j+1)
-                            // overwrites those columns.  o_done_i is committed after every P.V:
-                            // the softmax waits for it before it writes P_i(j+1) or rescales O_i.
+                            // issued before O_i += P_i(j) V_j, since the softmax needs it first,
+                            // and o_done_i is committed after every P.V: the softmax waits for
+                            // it before it writes P_i(j+1) or rescales O_i.  When P overlays S,
+                            // every P.V step must come before S(j+1) overwrites those columns;
+                            // the commit of S(j+1) then also covers P.V(j) (a commit tracks all
+                            // earlier MMAs of this thread), so o_done_i is committed only after
+                            // the sub-tile's last P.V, for the epilogue.
                             const uint64_t dqi = dq + uint64_t((i * C::Q_SUB) >> 4);
                             if constexpr (C::P_OWN) {
                                 // S(j+1) first: the softmax needs it next, P.V(j) only later
@@ -582,7 +587,7 @@ __global__ void __launch_bounds__(320, 1)
                             } else {
 #pragma unroll
                                 for (int kk = 0; kk < NPV; ++kk) pv_step(dv, i, kk, j > 0);
-                                umma_commit(bar_o_done + i);
+                                if (!more) umma_commit(bar_o_done + i);
                                 if (more) {
 #pragma unroll
                                     for (int kk = 0; kk < NS; ++kk) s_step(dqi, dk, i, kk);
@@ -713,6 +718,9 @@ __global__ void __launch_bounds__(320, 1)
                 // and of the bf16 p the P.V MMA consumes (for O / l).  The second sum
                 // takes the bf16 halves either unpacked into paired adds (D = 64) or
                 // through the mixed bf16 + f32 add (D = 128), whichever measured faster.
+                // When P overlays S, each 32-key chunk of P goes to TMEM as soon as it is
+                // packed: S(j) is complete, so P.V(j-1), issued before it, no longer reads
+                // those columns.
                 uint64_t se0 = 0, se1 = 0, sq0 = 0, sq1 = 0;
                 float rq0 = 0.f, rq1 = 0.f, rq2 = 0.f, rq3 = 0.f;
 #pragma unroll
@@ -755,25 +763,27 @@ __global__ void __launch_bounds__(320, 1)
                         }
                     }
                     if constexpr (FP8) {
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) sr[0][c * 8 + e] = pk[e];
+                        tmem_st8(tP + c * 8, *reinterpret_cast<const uint32_t(*)[8]>(pk));
+                    } else if constexpr (!C::P_OWN) {
+                        tmem_st16(tP + c * 16, pk);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 16; ++e) sr[c >> 1][(c & 1) * 16 + e] = pk[e];
                     }
                 }
                 if constexpr (HD == 128 && !FP8) sq0 = f2_pack(rq0 + rq2, rq1 + rq3);
-                // P.V(j-1) has finished: it no longer reads P's columns and O holds
-                // every block before j (needed before P is overwritten or O rescaled)
-                if (j > my_jb0) {
-                    if (!mbar_wait_warp(bar_o_done + i, o_phase, abort_flag)) goto softmax_done;
-                    o_phase ^= 1;
-                    tc_fence_after();
+                if constexpr (C::P_OWN) {
+                    // P in its own 64 columns: P.V(j-1), issued after S(j), has to finish
+                    // before P is overwritten or O rescaled
+                    if (j > my_jb0) {
+                        if (!mbar_wait_warp(bar_o_done + i, o_phase, abort_flag))
+                            goto softmax_done;
+                        o_phase ^= 1;
+                        tc_fence_after();
+                    }
+                    tmem_st32(tP, sr[0]);
+                    tmem_st32(tP + 32, sr[1]);
                 }
-                // P (bf16 pairs: 64 columns, its own or the first 64 of S; e4m3 quads: the
-                // first 32 columns of S)
-                tmem_st32(tP, sr[0]);
-                if constexpr (!FP8) tmem_st32(tP + 32, sr[1]);
                 float lsum, lrnd;
                 {
                     float x0, x1, y0, y1;
