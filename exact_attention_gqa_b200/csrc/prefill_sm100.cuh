@@ -656,11 +656,14 @@ __global__ void __launch_bounds__(320, 1)
                 s_phase ^= 1;
                 tc_fence_after();
                 uint32_t sr[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
+                // S in two halves: the row max of keys 0..63 runs while 64..127 load
+                tmem_ld32(tS, sr[0]);
+                tmem_ld32(tS + 32, sr[1]);
                 tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+                reg_fence(sr[0]);
+                reg_fence(sr[1]);
+                tmem_ld32(tS + 64, sr[2]);
+                tmem_ld32(tS + 96, sr[3]);
                 // keys of this block past the row's limit (causal diagonal, sequence end)
                 int kbj = j;
                 bool need_mask = j >= my_full;
@@ -670,6 +673,13 @@ __global__ void __launch_bounds__(320, 1)
                 }
                 if constexpr (WINDOW) {
                     if (j < my_lo_full) need_mask = true;
+                }
+                // the mask reads all four chunks; need_mask can differ between the rows of
+                // a warp (block-sparse), and the wait is a warp-wide (.sync.aligned) step
+                if (__any_sync(0xffffffffu, need_mask)) {
+                    tmem_ld_wait();
+                    reg_fence(sr[2]);
+                    reg_fence(sr[3]);
                 }
                 if (need_mask) {
                     const int lim = key_lim - kbj * BN;
@@ -693,7 +703,12 @@ __global__ void __launch_bounds__(320, 1)
                 // block row max: four independent three-input max chains
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 4; ++c)
+                for (int c = 0; c < 4; ++c) {
+                    if (c == 2) {
+                        tmem_ld_wait();
+                        reg_fence(sr[2]);
+                        reg_fence(sr[3]);
+                    }
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
                         mx0 = fmax3(mx0, __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
@@ -704,6 +719,7 @@ __global__ void __launch_bounds__(320, 1)
                         mx3 = fmax3(mx3, __uint_as_float(sr[c][e + 6]),
                                     __uint_as_float(sr[c][e + 7]));
                     }
+                }
                 const float mx = fmax3(fmaxf(mx0, mx1), mx2, mx3);
                 const float mb = mx * sl2;
                 float alpha = 1.f;
