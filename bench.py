@@ -62,6 +62,20 @@ def kernel_source_hash(kernel: str = "") -> str:
     return h.hexdigest()[:12]
 
 
+def fp8_decode_splits(units: int, nblk: int, slots: int) -> int:
+    """Split count the library picks for the e4m3 decode: the n in [1, min(64, nblk / 4)]
+    with the shortest estimated makespan, ceil(units * pieces / slots) * (blocks per
+    split + 3), over two resident CTAs per SM (ties: fewer splits)."""
+    best_n, best = 1, None
+    for n in range(1, max(1, min(64, nblk // 4)) + 1):
+        bps = -(-nblk // n)
+        pieces = -(-nblk // bps)
+        cost = -(-(units * pieces) // slots) * (bps + 3)
+        if best is None or cost < best:
+            best_n, best = n, cost
+    return best_n
+
+
 def load_peaks():
     p = ROOT / "MEASURED_PEAKS.json"
     if p.exists():
@@ -252,10 +266,10 @@ class Case:
                                                      num_splits=w.num_splits,
                                                      pack_gqa=w.pack_gqa)
             if w.kv_fp8 and w.num_splits == 0:
-                # the e4m3 path's own automatic count: two CTAs per SM (whole waves)
+                # the e4m3 path's own automatic count (the library's rule, restated)
                 sms = torch.cuda.get_device_properties(device).multi_processor_count
-                ctas = w.B * w.Hkv * (1 if pack else w.G)
-                splits = max(1, min(64, (2 * sms) // ctas, max(1, (w.Sk // 64) // 4)))
+                splits = fp8_decode_splits(w.B * w.Hkv * (1 if pack else w.G),
+                                           (w.Sk + 63) // 64, 2 * sms)
             self.splits, self.pack = splits, pack
             self.bytes = W.decode_bytes(w.B, w.Hq, w.Hkv, w.Sk, w.D,
                                         kv_elt=1 if w.kv_fp8 else 2)

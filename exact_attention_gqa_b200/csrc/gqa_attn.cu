@@ -174,6 +174,26 @@ int check_shape(int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int 
     return GQA_OK;
 }
 
+// Split count of the e4m3 decode for `units` CTAs' worth of (batch, head unit) work of
+// `nblk` 64-key blocks each over `slots` resident CTAs: the n in [1, min(64, nblk / 4)]
+// minimising ceil(units * pieces / slots) * (ceil(nblk / n) + 3).
+int fp8_decode_splits(long long units, int nblk, long long slots) {
+    const int n_max = std::max(1, std::min(64, nblk / 4));
+    int best_n = 1;
+    long long best = -1;
+    for (int n = 1; n <= n_max; ++n) {
+        const long long bps = (nblk + n - 1) / n;
+        const long long pieces = (nblk + bps - 1) / bps;
+        const long long waves = (units * pieces + slots - 1) / slots;
+        const long long cost = waves * (bps + 3);
+        if (best < 0 || cost < best) {
+            best = cost;
+            best_n = n;
+        }
+    }
+    return best_n;
+}
+
 void make_plan(Plan* pl, int B, int Hq, int Hkv, int Sq, int Sk, int num_splits, int pack_gqa,
                bool varlen, int sms) {
     const int G = Hq / Hkv;
@@ -494,16 +514,14 @@ int kvcache_common(const void* q, const void* k, const void* v, void* out, float
     Plan pl;
     make_plan(&pl, B, Hq, Hkv, 1, keys, num_splits, pack_gqa, false, dev->sms);
     if (kv.fp8 && num_splits == 0 && pl.kernel == kDecode) {
-        // the e4m3 kernel converts every element, so one CTA per SM leaves each SM
-        // sub-partition a single warp; two resident CTAs per SM (they fit) measured
-        // faster at every batch size
-        const long long ctas = (long long)B * Hkv * pl.decode_units;
-        const int nblk = (keys + 63) / 64;
-        long long n = (2LL * dev->sms) / ctas;  // whole waves: at most two CTAs per SM
-        if (n < 1) n = 1;
-        if (n > 64) n = 64;
-        if (n > nblk / 4) n = nblk / 4 > 0 ? nblk / 4 : 1;
-        make_plan(&pl, B, Hq, Hkv, 1, keys, int(n), pack_gqa, false, dev->sms);
+        // The e4m3 kernel converts every element, so its rate is set by each SM, not by
+        // HBM: two CTAs per SM (they fit) measured faster at every batch size, and the
+        // split count is the one with the shortest estimated makespan over those slots:
+        // whole waves of equal splits, each split costing its 64-key blocks plus about
+        // three blocks of pipeline fill and drain (ties: fewer splits).
+        const int n = fp8_decode_splits((long long)B * Hkv * pl.decode_units,
+                                        (keys + 63) / 64, 2LL * dev->sms);
+        make_plan(&pl, B, Hq, Hkv, 1, keys, n, pack_gqa, false, dev->sms);
     }
     if (pl.kernel == kZeroFill) {
         gqa::fill_no_keys<__nv_bfloat16><<<256, 256, 0, stream>>>(
