@@ -419,9 +419,11 @@ int gqa_attn_decode_paged(const void* q, const void* k_pages, const void* v_page
  *   q bf16 [B, 1, Hq, D] (rounded to f16 for the products: |q| must stay below
  *     65504), out bf16 [B, 1, Hq, D], lse fp32 [B, Hq, 1]; k_scale, v_scale finite
  *     and > 0 (GQA_ERR_SCALE otherwise).
- * num_splits = 0 chooses up to 64 splits so that two CTAs share each SM (the 8-bit
- * path converts every element and needs the extra warps); a registered workspace of
- * gqa_attn_workspace_bytes(B, Hq, 1, D, 64) always suffices.  Status codes, window,
+ * num_splits = 0 chooses up to 64 splits for two resident CTAs per SM (the 8-bit path
+ * converts every element and needs the extra warps): the count with the shortest
+ * estimated makespan, whole waves of equal splits each costing its 64-key blocks plus
+ * about three; a registered workspace of gqa_attn_workspace_bytes(B, Hq, 1, D, 64)
+ * always suffices.  Status codes, window,
  * explicit splits and pack_gqa as gqa_attn_decode_kvcache.
  */
 int gqa_attn_decode_fp8(const void* q, const void* k8, const void* v8, float k_scale,
